@@ -1,0 +1,455 @@
+#!/usr/bin/env python
+"""Benchmark of the Prefix Sliding attention hot path on B200.
+
+Default workload: steady-state batched decode on one layer (batch 64, 16 query / 2 KV
+heads, head_dim 128, bf16, L_prefix = 100, W = 4096, positions drawn in [8192, 131072],
+KV prefilled with RoPE at every absolute position).  One step = one decode step of the
+whole batch: ps_kv_append_rope (new token, Continue-PE RoPE, ring write) + ps_decode_attn
+(split-K decode + merge).  Prints ONE JSON line on rank 0.
+
+  python bench.py [--gpus N --steps K --warmup W] [--impl reference]
+
+Under torchrun every rank decodes its own batch (weak scaling, no data-path collective);
+the step time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import synth  # noqa: E402
+
+D = 128
+METRIC = "decode attn tokens/s and HBM GB/s (% roofline) vs position; prefill TFLOP/s"
+UNIT = "tok/s"
+WORKLOAD = "decode_b64_w4096"
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            j = json.load(f)
+        return {"hbm_gbs": float(j["hbm_gbs"]), "bf16_tflops": float(j["bf16_tflops"]),
+                "bf16_tflops_sustained": float(j["bf16_tflops_sustained"]), "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "source": "fallback"}
+
+
+# --------------------------------------------------------------------- clocks
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML on a background thread."""
+
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x2: "applications_clocks_setting", 0x1: "gpu_idle"}
+
+    def __init__(self, device_index: int, period_s: float = 0.002):
+        self.samples = []
+        self.reasons = 0
+        self.max_mhz = None
+        self.ok = False
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            uuid = "GPU-" + str(torch.cuda.get_device_properties(device_index).uuid)
+            self.h = pynvml.nvmlDeviceGetHandleByUUID(uuid.encode())
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.nv = pynvml
+            self.ok = True
+        except Exception:
+            self.ok = False
+        self.period = period_s
+        self._t = None
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append((time.perf_counter(), mhz, r))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self.ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+
+    def stop(self):
+        if self._t is not None:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self, t0=None, t1=None):
+        if not self.ok or not self.samples:
+            return None
+        inside = [s for s in self.samples if t0 is None or (t0 <= s[0] <= t1)]
+        window = "timed"
+        if len(inside) < 3:
+            inside = self.samples
+            window = "warmup+timed"
+        mhz = [s[1] for s in inside]
+        bits = 0
+        for s in inside:
+            bits |= s[2]
+        reasons = [name for bit, name in self.REASONS.items() if bits & bit and name != "gpu_idle"]
+        return {"sm_mhz": float(statistics.median(mhz)), "sm_max_mhz": float(self.max_mhz),
+                "reasons": reasons, "samples": len(inside), "window": window}
+
+
+# ------------------------------------------------------------- distributed
+def _dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def _barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def _max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def _sum_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+# ------------------------------------------------------------- decode setup
+class DecodeWorkload:
+    """Prefix Sliding decode workload resident in HBM (one layer)."""
+
+    def __init__(self, wl: synth.Workload, dev, rank: int, max_steps: int):
+        from prefix_sliding_window_b200 import binding as B
+        from prefix_sliding_window_b200.cache import PrefixSlidingCache
+        self.B = B
+        self.wl = wl
+        self.dev = dev
+        Bn, hq, hkv, lp, w = wl.batch, wl.n_q_heads, wl.n_kv_heads, wl.l_prefix, wl.window
+        self.params = B.make_params(hq, hkv, D, lp, w, wl.rope_theta)
+        s = lambda k: synth.seed_for(wl.index, 10 * rank + k)  # noqa: E731
+        self.pos_start = synth.uniform_positions(Bn, wl.pos_lo, wl.pos_hi, s(0), dev)
+        self.cache = PrefixSlidingCache(Bn, hkv, lp, w, D, dev, fill=None)
+        st = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.status = st
+        # prefix [0, lp) and window history [p - W + 1, p - 1], RoPE at absolute positions
+        k_pre = synth.normal_bf16((Bn, lp, hkv, D), s(1), dev)
+        v_pre = synth.normal_bf16((Bn, lp, hkv, D), s(2), dev)
+        B.ps_kv_append_rope(self.params, self.cache.struct, k_pre, v_pre, None,
+                            torch.zeros(Bn, dtype=torch.int64, device=dev), lp, st)
+        del k_pre, v_pre
+        chunk = 1024
+        for c0 in range(0, w - 1, chunk):
+            T = min(chunk, w - 1 - c0)
+            k = synth.normal_bf16((Bn, T, hkv, D), s(3) + c0, dev)
+            v = synth.normal_bf16((Bn, T, hkv, D), s(4) + c0, dev)
+            B.ps_kv_append_rope(self.params, self.cache.struct, k, v, None,
+                                self.pos_start - (w - 1) + c0, T, st)
+        # per-step new tokens (distinct buffers per step, so no step reuses another's input)
+        n = max_steps
+        self.k_new = synth.normal_bf16((n, Bn, 1, hkv, D), s(5), dev)
+        self.v_new = synth.normal_bf16((n, Bn, 1, hkv, D), s(6), dev)
+        self.q_raw = synth.normal_bf16((n, Bn, hq, D), s(7), dev)
+        self.q = self.q_raw.clone()
+        self.pos = torch.stack([self.pos_start + i for i in range(n)])
+        self.out = torch.empty((n, Bn, hq, D), dtype=torch.bfloat16, device=dev)
+        nb = B.ps_decode_workspace_bytes(self.params, Bn)
+        self.ws = torch.empty(max(nb, 1), dtype=torch.uint8, device=dev)
+        self.splits_used = nb > 0
+        torch.cuda.synchronize()
+
+    def kernels_per_step(self) -> int:
+        return 2 + (1 if self.splits_used else 0)
+
+    def append(self, i):
+        B = self.B
+        B.ps_kv_append_rope(self.params, self.cache.struct, self.k_new[i], self.v_new[i],
+                            self.q[i], self.pos[i], 1, self.status)
+
+    def decode(self, i):
+        self.B.ps_decode_attn(self.params, self.cache.struct, self.q[i], self.pos[i], self.out[i],
+                              None, self.ws, self.status)
+
+    def algorithmic_bytes_per_decode(self) -> int:
+        """K+V of every visible key plus q and out: 1024 B per visible token per sequence
+        (2 KV heads x 128 x 2 B x 2) + 2 x Hq x D x 2 B."""
+        wl = self.wl
+        n = self.pos_start + 1
+        vis = torch.clamp(n, max=wl.l_prefix + wl.window)
+        kv = int(vis.sum().item()) * 2 * wl.n_kv_heads * D * 2
+        return kv + wl.batch * 2 * wl.n_q_heads * D * 2
+
+
+def run_decode(args, world, rank, dev):
+    wl = synth.WORKLOADS[WORKLOAD]
+    K, W = args.steps, args.warmup
+    work = DecodeWorkload(wl, dev, rank, K + W)
+    stream = torch.cuda.current_stream()
+
+    def step(i):
+        work.append(i)
+        work.decode(i)
+
+    for i in range(W):
+        step(i)
+    torch.cuda.synchronize()
+    sampler = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
+    if sampler:
+        sampler.start()
+    # soak: a few more untimed steps so the clocks are sampled under this load
+    for _ in range(3):
+        for i in range(W):
+            step(i)
+    ev_dec = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(K)]
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    _barrier(world)
+    torch.cuda.synchronize()
+    t_host0 = time.perf_counter()
+    ev0.record(stream)
+    for j in range(K):
+        i = W + j
+        work.append(i)
+        ev_dec[j][0].record(stream)
+        work.decode(i)
+        ev_dec[j][1].record(stream)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    t_host1 = time.perf_counter()
+    _barrier(world)
+    if sampler:
+        sampler.stop()
+    ms_local = ev0.elapsed_time(ev1)
+    ms = _max_over_ranks(ms_local, world)
+    dec_ms = [a.elapsed_time(b) for a, b in ev_dec]
+    assert work.status.item() == 0, f"device status {work.status.item()}"
+    tokens = _sum_over_ranks(float(wl.batch * K), world)
+    value = tokens / (ms / 1e3)
+
+    peaks = _peaks()
+    alg = work.algorithmic_bytes_per_decode()
+    dec_avg_s = statistics.mean(dec_ms) / 1e3
+    achieved = alg / dec_avg_s / 1e9
+    roof = {"bound": "hbm", "kernel": "ps_decode_attn (decode_kernel + merge_kernel)",
+            "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": args.traffic,
+            "peak_source": peaks["source"], "algorithmic_bytes_per_launch": alg,
+            "decode_us_median": round(statistics.median(dec_ms) * 1e3, 2),
+            "decode_us_p10": round(float(np.percentile(dec_ms, 10)) * 1e3, 2),
+            "decode_us_p90": round(float(np.percentile(dec_ms, 90)) * 1e3, 2),
+            "frac_of_8tbs_spec": round(achieved / 8000.0, 4)}
+    e2e = run_decode_e2e(work, K, W, world)
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": K,
+        "warmup": W, "ms_per_step": round(ms / K, 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "batch_per_gpu": wl.batch, "global_batch": wl.batch * world,
+                   "n_q_heads": wl.n_q_heads, "n_kv_heads": wl.n_kv_heads, "head_dim": D,
+                   "l_prefix": wl.l_prefix, "window": wl.window,
+                   "positions": f"U[{wl.pos_lo},{wl.pos_hi}]", "layers": 1,
+                   "step": "ps_kv_append_rope + ps_decode_attn",
+                   "l2": "inputs larger than L2 (275 MB of K/V read per step vs 126 MB L2)",
+                   "parallelism": f"dp{world} (independent sequences, no collective)"},
+        "roofline": roof,
+        "e2e": e2e,
+        "gpu_launches": work.kernels_per_step() * K,
+    }
+    if sampler:
+        line["clocks"] = sampler.summary(t_host0, t_host1)
+    return line, work
+
+
+def run_decode_e2e(work: DecodeWorkload, K: int, W: int, world: int):
+    """Same metric through the C ABI with host buffers: every step copies its inputs
+    (q, k_new, v_new, pos) host->device from pinned memory and reads out device->host."""
+    B = work.B
+    dev = work.dev
+    stream = torch.cuda.current_stream()
+    n = K + W
+    h_k = work.k_new.cpu().pin_memory()
+    h_v = work.v_new.cpu().pin_memory()
+    h_q = work.q_raw.cpu().pin_memory()
+    h_pos = work.pos.cpu().pin_memory()
+    h_out = torch.empty((n,) + tuple(work.out.shape[1:]), dtype=torch.bfloat16).pin_memory()
+    d_k = torch.empty_like(work.k_new[0])
+    d_v = torch.empty_like(work.v_new[0])
+    d_q = torch.empty_like(work.q[0])
+    d_pos = torch.empty_like(work.pos[0])
+    d_out = torch.empty_like(work.out[0])
+
+    def step(i):
+        d_k.copy_(h_k[i], non_blocking=True)
+        d_v.copy_(h_v[i], non_blocking=True)
+        d_q.copy_(h_q[i], non_blocking=True)
+        d_pos.copy_(h_pos[i], non_blocking=True)
+        B.ps_kv_append_rope(work.params, work.cache.struct, d_k, d_v, d_q, d_pos, 1, work.status)
+        B.ps_decode_attn(work.params, work.cache.struct, d_q, d_pos, d_out, None, work.ws,
+                         work.status)
+        h_out[i].copy_(d_out, non_blocking=True)
+
+    for i in range(W):
+        step(i)
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    _barrier(world)
+    ev0.record(stream)
+    for j in range(K):
+        step(W + j)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    ms = _max_over_ranks(ev0.elapsed_time(ev1), world)
+    tokens = _sum_over_ranks(float(work.wl.batch * K), world)
+    bi = (d_k.numel() + d_v.numel() + d_q.numel()) * 2 + d_pos.numel() * 8
+    bo = d_out.numel() * 2
+    return {"value": round(tokens / (ms / 1e3), 1), "unit": UNIT, "h2d_bytes_per_step": bi,
+            "d2h_bytes_per_step": bo}
+
+
+# ----------------------------------------------------------- CPU oracle leg
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        return max([i.get("num_threads", 1) for i in info] or [1])
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def oracle_decode_sample(wl: synth.Workload, n_seq: int, seed_stream: int = 0):
+    """Oracle decode of ``n_seq`` sequences of the workload (fresh CPU inputs with the
+    workload's shapes).  Returns (sequences decoded, seconds)."""
+    import oracle as O
+    hq, hkv, lp, w = wl.n_q_heads, wl.n_kv_heads, wl.l_prefix, wl.window
+    pos = synth.uniform_positions(n_seq, wl.pos_lo, wl.pos_hi, synth.seed_for(wl.index, 900 + seed_stream))
+    scale = 1.0 / math.sqrt(D)
+    data = []
+    for b in range(n_seq):
+        p = int(pos[b])
+        vis = O.visible_positions(p, lp, w)
+        k = synth.normal_bf16((len(vis), hkv, D), 7000 + b + 97 * seed_stream).double().numpy()
+        v = synth.normal_bf16((len(vis), hkv, D), 8000 + b + 97 * seed_stream).double().numpy()
+        q = synth.normal_bf16((hq, D), 9000 + b + 97 * seed_stream).double().numpy()
+        data.append((p, vis, k, v, q))
+    t0 = time.perf_counter()
+    for p, vis, k, v, q in data:
+        k_rot = O.rope_rotate(k, vis[:, None], wl.rope_theta)
+        O.attend_gqa(O.rope_rotate(q, p, wl.rope_theta), k_rot, v, scale)
+    return n_seq, time.perf_counter() - t0
+
+
+def cpu_baseline(wl: synth.Workload, budget_s: float = 12.0):
+    done, spent, calls = 0, 0.0, 0
+    while spent < budget_s:
+        n, t = oracle_decode_sample(wl, 8, calls)
+        done += n
+        spent += t
+        calls += 1
+    return {"value": round(done / spent, 2), "unit": UNIT, "cores": _blas_threads(),
+            "kind": "oracle",
+            "sample": f"{done} sequences of {wl.name} (one decode step each: all {wl.n_q_heads} "
+                      f"heads over {wl.l_prefix + wl.window} visible keys), float64 numpy, "
+                      f"{spent:.1f} s"}
+
+
+def run_reference(args, world, rank):
+    """Reference arm: the float64 oracle on the host cores, same metric and config."""
+    if rank != 0:
+        return None
+    wl = synth.WORKLOADS[WORKLOAD]
+    per_step = 1  # sequences per step: a bounded sample of the workload's batch
+    for i in range(args.warmup):
+        oracle_decode_sample(wl, per_step, 1000 + i)
+    total_t, total_n = 0.0, 0
+    for i in range(args.steps):
+        n, t = oracle_decode_sample(wl, per_step, 2000 + i)
+        total_t += t
+        total_n += n
+    value = total_n / total_t
+    return {
+        "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total_t / args.steps * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "impl": "reference",
+        "config": {"workload": WORKLOAD, "batch_per_gpu": wl.batch, "n_q_heads": wl.n_q_heads,
+                   "n_kv_heads": wl.n_kv_heads, "head_dim": D, "l_prefix": wl.l_prefix,
+                   "window": wl.window, "positions": f"U[{wl.pos_lo},{wl.pos_hi}]"},
+        "cpu_baseline": {"value": round(value, 3), "unit": UNIT, "cores": _blas_threads(),
+                         "kind": "oracle",
+                         "sample": f"{per_step} sequence per step of {WORKLOAD}, float64 numpy"},
+        "e2e": {"value": round(value, 3), "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=256)
+    ap.add_argument("--warmup", type=int, default=8)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--traffic", type=float, default=None,
+                    help="ncu dram bytes per decode launch, when known for this kernel")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+    if args.impl == "reference":
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        line = run_reference(args, world, rank)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+    world, rank, local = _dist_setup()
+    dev = torch.device("cuda", local)
+    line, _ = run_decode(args, world, rank, dev)
+    if rank == 0:
+        if not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(synth.WORKLOADS[WORKLOAD])
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,191 @@
+/*
+ * ps.h -- C ABI of libps.so, the Prefix Sliding attention hot path for NVIDIA B200 (sm_100a).
+ *
+ * Prefix Sliding ("Prefix Sliding 完全拆解", pinghaoyang blog, §核心机制, eq. A(i)): the
+ * query at (1-indexed) position i may attend key j iff j <= L_prefix or i - W < j <= i.
+ * Every other key is evicted.  At most L_prefix + W keys are visible (same section,
+ * eq. L_total), so decode cost per token is constant once the window is full.
+ *
+ * This library uses 0-based absolute positions.  The query at position p sees
+ *     V(p) = { k : 0 <= k <= p  and  (k < l_prefix  or  k > p - window) }.
+ * The window holds the W positions ending at, and including, the query.
+ *
+ * Conventions for every call:
+ *   - The caller owns every buffer.  The library never allocates, frees or synchronises.
+ *     Every call is asynchronous on the given stream.
+ *   - "device" pointers live in GPU global memory; "host" pointers in CPU memory.
+ *   - bf16 = IEEE bfloat16 stored as uint16.  All device buffers must be 16-byte aligned.
+ *   - Host-detectable problems (null pointer, unsupported shape, n_q_heads % n_kv_heads
+ *     != 0, workspace too small, misaligned pointer) return a negative ps_status and
+ *     launch nothing.  ps_last_error() then describes the failure.
+ *   - Conditions only the device can see (a position < 0, or past the end of a linear
+ *     cache) set a bit in the optional device word *dev_status (atomic OR).  The kernel
+ *     then skips that sequence: its output rows are written as zeros and its lse as
+ *     -inf.  No kernel traps.
+ *   - Every wait inside a kernel is bounded (about one second).  A wait that runs out
+ *     sets PS_DEV_TIMEOUT in *dev_status and the kernel returns.
+ */
+#ifndef PS_H_
+#define PS_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t; declared here so callers need no CUDA headers.
+ * NULL selects the legacy default stream. */
+typedef struct CUstream_st* ps_stream_t;
+
+typedef enum {
+  PS_OK = 0,
+  PS_ERR_INVALID_ARG = -1, /* null pointer, bad size, misaligned pointer            */
+  PS_ERR_UNSUPPORTED = -2, /* shape outside what this build implements              */
+  PS_ERR_WORKSPACE = -3,   /* workspace null or smaller than the *_workspace_bytes  */
+  PS_ERR_CUDA = -4         /* a CUDA runtime call or kernel launch failed           */
+} ps_status;
+
+/* Bits of *dev_status (device int32, OR-ed by kernels; the caller clears it). */
+#define PS_DEV_BAD_POS 1   /* a position < 0: that sequence was skipped            */
+#define PS_DEV_POS_RANGE 2 /* a position past the end of a linear (full) cache      */
+#define PS_DEV_TIMEOUT 4   /* a bounded in-kernel wait ran out; output is invalid   */
+
+/* Tile flags of the prefill plan ("Prefix Sliding 完全拆解", §Kernel 实现, two-level
+ * filtering: SKIP tiles are neither loaded nor computed and never appear in a plan;
+ * PARTIAL tiles get an element-wise mask; FULL tiles need none). */
+#define PS_TILE_FULL 1
+#define PS_TILE_PARTIAL 2
+
+/* Attention geometry, shared by every call. */
+typedef struct {
+  int32_t n_q_heads;   /* Hq; Hq % Hkv == 0                                          */
+  int32_t n_kv_heads;  /* Hkv; GQA: query head h reads KV head h / (Hq / Hkv)        */
+  int32_t head_dim;    /* D; this build supports D == 128 only                       */
+  int32_t l_prefix;    /* L_prefix >= 0; 0 gives the pure sliding window            */
+  int32_t window;      /* W >= 1                                                    */
+  int32_t reserved;    /* must be 0                                                 */
+  double rope_theta;   /* RoPE base (rotate-half form), e.g. 1e6; > 0               */
+  float softmax_scale; /* 0 selects 1/sqrt(head_dim)                                 */
+  int32_t reserved2;   /* must be 0                                                 */
+} ps_params;
+
+/* Per-sequence bounded KV store: a pinned prefix region plus a W-slot ring.
+ * Position p < l_prefix lives in prefix row p; position p >= l_prefix lives in ring slot
+ * (p - l_prefix) mod W.  Writing a slot evicts the position it held (hard eviction,
+ * §核心机制); cached keys are never rotated again (Continue PE, §位置编码).
+ * Layouts (device, bf16, contiguous):
+ *   k_prefix, v_prefix : [batch, Hkv, l_prefix, D]   (may be NULL when l_prefix == 0)
+ *   k_ring,   v_ring   : [batch, Hkv, W, D]
+ * A linear full-attention cache is the same struct with l_prefix = Lmax, window = 1 and
+ * the ring pointers NULL; every position must then be < Lmax. */
+typedef struct {
+  void* k_prefix;
+  void* v_prefix;
+  void* k_ring;
+  void* v_ring;
+  int64_t batch;
+} ps_kv_cache;
+
+/* Append T tokens per sequence and apply Continue-PE RoPE exactly once.
+ * Source: §位置编码 (Continue PE: absolute position ids, rotated K reused as cached),
+ * §核心机制 (hard eviction, bounded per-sequence store).
+ *   k_new, v_new : device bf16 [batch, T, Hkv, D], raw (un-rotated) keys and values.
+ *   q_inout      : device bf16 [batch, T, Hq, D] or NULL; rotated in place when given.
+ *   pos0         : device int64 [batch]; token t of sequence b has absolute position
+ *                  pos0[b] + t.  RoPE angles are position * theta^(-2i/D), formed and
+ *                  reduced in float64.
+ *   T            : tokens per sequence, >= 1.
+ * When several of the T tokens map to one ring slot, only the latest is written (only
+ * the last W positions beyond the prefix survive).  A token whose position is < 0 is
+ * skipped (PS_DEV_BAD_POS); in a linear cache (ring NULL) a position >= l_prefix is
+ * skipped (PS_DEV_POS_RANGE).  Its q rows are left as they were. */
+int ps_kv_append_rope(const ps_params* params, const ps_kv_cache* cache, const void* k_new,
+                      const void* v_new, void* q_inout, const int64_t* pos0, int32_t T,
+                      int32_t* dev_status, ps_stream_t stream);
+
+/* Bytes of device workspace ps_decode_attn needs for this geometry and batch (split-K
+ * partial outputs).  Returns 0 on invalid arguments. */
+size_t ps_decode_workspace_bytes(const ps_params* params, int64_t batch);
+
+/* One decode step: attention of one query token per sequence over its visible keys.
+ * Source: eq. A(i) and eq. L_total (§核心机制); §Kernel 实现 (only prefix and window
+ * ranges are read; everything else is skipped).
+ *   q     : device bf16 [batch, Hq, D], already rotated at pos[b] (ps_kv_append_rope).
+ *   pos   : device int64 [batch], absolute position of the query; its own K/V must
+ *           already be in the cache (append first, then decode).
+ *   out   : device bf16 [batch, Hq, D].
+ *   lse   : device fp32 [batch, Hq] or NULL; natural-log softmax denominator
+ *           (max included) of scores q.k * scale.
+ *   workspace, ws_bytes : device scratch of at least ps_decode_workspace_bytes(); its
+ *           contents on entry do not matter.
+ * Requires 1 <= Hq / Hkv <= 8. */
+int ps_decode_attn(const ps_params* params, const ps_kv_cache* cache, const void* q,
+                   const int64_t* pos, void* out, float* lse, void* workspace, size_t ws_bytes,
+                   int32_t* dev_status, ps_stream_t stream);
+
+/* Bytes of device workspace ps_full_attn_ref needs (same split-K layout as decode). */
+size_t ps_full_attn_workspace_bytes(const ps_params* params, int64_t batch, int64_t lmax);
+
+/* Full causal attention comparator (the baseline the pages compare against, §Kernel 实现
+ * and Table 1 full-attention row): the query at pos[b] attends every key in [0, pos[b]].
+ *   k_full, v_full : device bf16 [batch, Hkv, lmax, D], keys already rotated (fill it with
+ *                    ps_kv_append_rope on a cache with l_prefix = lmax, ring NULL).
+ *   pos[b] >= lmax sets PS_DEV_POS_RANGE and skips sequence b.
+ * params->l_prefix and params->window are ignored. Other arguments as ps_decode_attn. */
+int ps_full_attn_ref(const ps_params* params, const void* k_full, const void* v_full,
+                     int64_t lmax, const void* q, const int64_t* pos, int64_t batch, void* out,
+                     float* lse, void* workspace, size_t ws_bytes, int32_t* dev_status,
+                     ps_stream_t stream);
+
+/* Prefill tile geometry (query rows Bq, key rows Bk) the masked prefill kernel uses. */
+int ps_prefill_tile_geometry(int32_t* bq, int32_t* bk);
+
+/* Number of non-SKIP tiles of the prefill plan for one (batch, head), host-computed from
+ * the same closed forms the device planner uses.  Returns < 0 on invalid arguments. */
+int64_t ps_prefill_plan_tiles(const ps_params* params, int64_t seq);
+
+/* Bytes of device workspace ps_masked_prefill_attn needs. */
+size_t ps_prefill_workspace_bytes(const ps_params* params, int64_t batch, int64_t seq);
+
+/* Masked prefill / truncated-backprop context forward over sequence indices [0, seq).
+ * Source: eq. A(i) (§核心机制); §Kernel 实现 (two-level filtering); §截断回传 (the trainer
+ * runs the forward over the last 4W tokens of a rollout).
+ * Row i attends V(i) with positions taken as sequence indices: the first l_prefix
+ * indices are the prefix.  With window >= seq this is dense causal attention.
+ *   q      : device bf16 [batch, seq, Hq, D], already rotated.
+ *   k, v   : device bf16 [batch, seq, Hkv, D], k already rotated.
+ *   out    : device bf16 [batch, seq, Hq, D].
+ *   lse    : device fp32 [batch, Hq, seq] or NULL (natural log).
+ *   tile_plan : device int32 [tile_plan_cap, 3] or NULL.  When given, receives the plan
+ *           the kernel ran: rows (q_tile, k_tile, flag), q-tile-major, ascending k_tile,
+ *           SKIP tiles omitted (flag PS_TILE_FULL or PS_TILE_PARTIAL).
+ *   n_tiles : host int64 or NULL; receives the number of plan rows.
+ *   workspace, ws_bytes : device scratch of at least ps_prefill_workspace_bytes().
+ * Requires seq >= 1 and Hq / Hkv integral.  tile_plan_cap smaller than the plan is
+ * PS_ERR_INVALID_ARG. */
+int ps_masked_prefill_attn(const ps_params* params, const void* q, const void* k, const void* v,
+                           int64_t batch, int64_t seq, void* out, float* lse, int32_t* tile_plan,
+                           int64_t tile_plan_cap, int64_t* n_tiles, void* workspace,
+                           size_t ws_bytes, ps_stream_t stream);
+
+/* Introspection for bit-exact checks: the visible-range descriptor the decode kernel
+ * uses, computed by the same device code.  ranges_out: device int32 [batch, 4] =
+ * (pre_len, seg0_start, seg0_len, seg1_len): the prefix rows [0, pre_len) and the ring
+ * slots [seg0_start, seg0_start + seg0_len) then [0, seg1_len).  An empty window reports
+ * (.., 0, 0, 0).  A position < 0 reports (0, 0, 0, 0). */
+int ps_decode_visible_ranges(const ps_params* params, const int64_t* pos, int64_t batch,
+                             int32_t* ranges_out, ps_stream_t stream);
+
+/* Thread-local description of the last host-side failure of this thread ("" if none). */
+const char* ps_last_error(void);
+
+/* Library version string. */
+const char* ps_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PS_H_ */

@@ -1,0 +1,378 @@
+// C-ABI entry points of libps: argument validation, status codes, tensor-map encoding and
+// kernel launches.  The declarations and their contracts are in include/ps.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdio.h>
+
+#include <mutex>
+#include <string>
+
+#include "../../include/ps.h"
+#include "ps_internal.h"
+#include "ps_ranges.cuh"
+
+namespace ps {
+
+namespace {
+thread_local std::string g_last_error;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// Validates the geometry shared by every call.
+int check_params(const ps_params* prm, bool need_window) {
+  if (!prm) return fail(PS_ERR_INVALID_ARG, "params is NULL");
+  if (prm->reserved != 0 || prm->reserved2 != 0)
+    return fail(PS_ERR_INVALID_ARG, "params reserved fields must be 0");
+  if (prm->head_dim != kHeadDim)
+    return fail(PS_ERR_UNSUPPORTED, "head_dim must be 128 in this build");
+  if (prm->n_q_heads < 1 || prm->n_kv_heads < 1)
+    return fail(PS_ERR_INVALID_ARG, "n_q_heads and n_kv_heads must be >= 1");
+  if (prm->n_q_heads % prm->n_kv_heads != 0)
+    return fail(PS_ERR_INVALID_ARG, "n_q_heads must be a multiple of n_kv_heads");
+  if (need_window) {
+    if (prm->l_prefix < 0) return fail(PS_ERR_INVALID_ARG, "l_prefix must be >= 0");
+    if (prm->window < 1) return fail(PS_ERR_INVALID_ARG, "window must be >= 1");
+  }
+  if (!(prm->rope_theta > 0.0) || !isfinite(prm->rope_theta))
+    return fail(PS_ERR_INVALID_ARG, "rope_theta must be finite and > 0");
+  if (!(prm->softmax_scale >= 0.f) || !isfinite(prm->softmax_scale))
+    return fail(PS_ERR_INVALID_ARG, "softmax_scale must be finite and >= 0");
+  return PS_OK;
+}
+
+float resolve_scale(const ps_params* prm) {
+  return prm->softmax_scale > 0.f ? prm->softmax_scale
+                                  : static_cast<float>(1.0 / sqrt(double(prm->head_dim)));
+}
+
+int check_ptr(const void* p, const char* name, bool nullable = false) {
+  if (!p) {
+    if (nullable) return PS_OK;
+    return fail(PS_ERR_INVALID_ARG, std::string(name) + " is NULL");
+  }
+  if (!aligned16(p)) return fail(PS_ERR_INVALID_ARG, std::string(name) + " is not 16-byte aligned");
+  return PS_OK;
+}
+
+#define PS_TRY(expr)             \
+  do {                           \
+    const int rc_ = (expr);      \
+    if (rc_ != PS_OK) return rc_; \
+  } while (0)
+
+}  // namespace
+
+int fail(int code, const std::string& msg) {
+  g_last_error = msg;
+  return code;
+}
+
+int check_cuda(cudaError_t e, const char* what) {
+  if (e == cudaSuccess) return PS_OK;
+  return fail(PS_ERR_CUDA, std::string(what) + ": " + cudaGetErrorString(e));
+}
+
+bool make_map_3d(CUtensorMap* map, const void* base, uint64_t x, uint64_t y, uint64_t z,
+                 uint32_t box_x, uint32_t box_y) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) {
+    fail(PS_ERR_CUDA, "cuTensorMapEncodeTiled unavailable (no CUDA driver?)");
+    return false;
+  }
+  const cuuint64_t dims[3] = {x, y, z};
+  const cuuint64_t strides[2] = {x * 2, x * y * 2};
+  const cuuint32_t box[3] = {box_x, box_y, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    char buf[160];
+    snprintf(buf, sizeof(buf), "cuTensorMapEncodeTiled failed (%d) dims %llu x %llu x %llu",
+             int(r), (unsigned long long)x, (unsigned long long)y, (unsigned long long)z);
+    fail(PS_ERR_CUDA, buf);
+    return false;
+  }
+  return true;
+}
+
+int sm_count() {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (cached[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1)
+      n = 148;
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
+}  // namespace ps
+
+using namespace ps;
+
+extern "C" {
+
+const char* ps_last_error(void) { return g_last_error.c_str(); }
+
+const char* ps_version(void) { return "libps 0.1 (sm_100a)"; }
+
+int ps_kv_append_rope(const ps_params* params, const ps_kv_cache* cache, const void* k_new,
+                      const void* v_new, void* q_inout, const int64_t* pos0, int32_t T,
+                      int32_t* dev_status, ps_stream_t stream) {
+  g_last_error.clear();
+  PS_TRY(check_params(params, true));
+  if (!cache) return fail(PS_ERR_INVALID_ARG, "cache is NULL");
+  if (cache->batch < 0) return fail(PS_ERR_INVALID_ARG, "cache->batch must be >= 0");
+  if (T < 1) return fail(PS_ERR_INVALID_ARG, "T must be >= 1");
+  if (cache->batch == 0) return PS_OK;
+  const bool linear = cache->k_ring == nullptr && cache->v_ring == nullptr;
+  if (!linear) {
+    PS_TRY(check_ptr(cache->k_ring, "cache->k_ring"));
+    PS_TRY(check_ptr(cache->v_ring, "cache->v_ring"));
+  }
+  if (params->l_prefix > 0 || linear) {
+    PS_TRY(check_ptr(cache->k_prefix, "cache->k_prefix"));
+    PS_TRY(check_ptr(cache->v_prefix, "cache->v_prefix"));
+  }
+  if (linear && params->l_prefix < 1)
+    return fail(PS_ERR_INVALID_ARG, "a linear cache (ring NULL) needs l_prefix = Lmax >= 1");
+  PS_TRY(check_ptr(k_new, "k_new"));
+  PS_TRY(check_ptr(v_new, "v_new"));
+  PS_TRY(check_ptr(q_inout, "q_inout", true));
+  if (!pos0) return fail(PS_ERR_INVALID_ARG, "pos0 is NULL");
+  if ((reinterpret_cast<uintptr_t>(pos0) & 7u) != 0)
+    return fail(PS_ERR_INVALID_ARG, "pos0 is not 8-byte aligned");
+  if ((reinterpret_cast<uintptr_t>(dev_status) & 3u) != 0)
+    return fail(PS_ERR_INVALID_ARG, "dev_status is not 4-byte aligned");
+  AppendArgs a;
+  a.k_new = k_new;
+  a.v_new = v_new;
+  a.q = q_inout;
+  a.pos0 = pos0;
+  a.k_pre = cache->k_prefix;
+  a.v_pre = cache->v_prefix;
+  a.k_ring = linear ? nullptr : cache->k_ring;
+  a.v_ring = linear ? nullptr : cache->v_ring;
+  a.status = dev_status;
+  a.batch = cache->batch;
+  a.T = T;
+  a.hq = params->n_q_heads;
+  a.hkv = params->n_kv_heads;
+  a.lp = params->l_prefix;
+  a.w = params->window;
+  a.theta = params->rope_theta;
+  return check_cuda(launch_append(a, reinterpret_cast<cudaStream_t>(stream)),
+                    "append_rope_kernel launch");
+}
+
+size_t ps_decode_workspace_bytes(const ps_params* params, int64_t batch) {
+  if (check_params(params, true) != PS_OK || batch < 0) return 0;
+  return decode_workspace_bytes(batch, params->n_kv_heads,
+                                (int64_t)params->l_prefix + params->window);
+}
+
+int ps_decode_attn(const ps_params* params, const ps_kv_cache* cache, const void* q,
+                   const int64_t* pos, void* out, float* lse, void* workspace, size_t ws_bytes,
+                   int32_t* dev_status, ps_stream_t stream) {
+  g_last_error.clear();
+  PS_TRY(check_params(params, true));
+  if (params->n_q_heads / params->n_kv_heads > kMaxGroup)
+    return fail(PS_ERR_UNSUPPORTED, "decode supports at most 8 query heads per KV head");
+  if (!cache) return fail(PS_ERR_INVALID_ARG, "cache is NULL");
+  if (cache->batch < 0) return fail(PS_ERR_INVALID_ARG, "cache->batch must be >= 0");
+  if (cache->batch == 0) return PS_OK;
+  PS_TRY(check_ptr(cache->k_ring, "cache->k_ring"));
+  PS_TRY(check_ptr(cache->v_ring, "cache->v_ring"));
+  if (params->l_prefix > 0) {
+    PS_TRY(check_ptr(cache->k_prefix, "cache->k_prefix"));
+    PS_TRY(check_ptr(cache->v_prefix, "cache->v_prefix"));
+  }
+  PS_TRY(check_ptr(q, "q"));
+  PS_TRY(check_ptr(out, "out"));
+  PS_TRY(check_ptr(lse, "lse", true));
+  if (!pos) return fail(PS_ERR_INVALID_ARG, "pos is NULL");
+  if ((reinterpret_cast<uintptr_t>(pos) & 7u) != 0)
+    return fail(PS_ERR_INVALID_ARG, "pos is not 8-byte aligned");
+  if ((reinterpret_cast<uintptr_t>(dev_status) & 3u) != 0)
+    return fail(PS_ERR_INVALID_ARG, "dev_status is not 4-byte aligned");
+  const size_t need = decode_workspace_bytes(cache->batch, params->n_kv_heads,
+                                             (int64_t)params->l_prefix + params->window);
+  if (need > 0) {
+    if (!workspace || ws_bytes < need)
+      return fail(PS_ERR_WORKSPACE, "workspace smaller than ps_decode_workspace_bytes()");
+    PS_TRY(check_ptr(workspace, "workspace"));
+  }
+  DecodeLaunch l{};
+  l.q = q;
+  l.pos = pos;
+  l.out = out;
+  l.lse = lse;
+  l.workspace = workspace;
+  l.status = dev_status;
+  l.batch = cache->batch;
+  l.hq = params->n_q_heads;
+  l.hkv = params->n_kv_heads;
+  l.lp = params->l_prefix;
+  l.w = params->window;
+  l.lmax = 0;
+  l.full_mode = 0;
+  l.scale = resolve_scale(params);
+  l.k0 = cache->k_prefix;
+  l.v0 = cache->v_prefix;
+  l.k1 = cache->k_ring;
+  l.v1 = cache->v_ring;
+  return launch_decode(l, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t ps_full_attn_workspace_bytes(const ps_params* params, int64_t batch, int64_t lmax) {
+  if (check_params(params, false) != PS_OK || batch < 0 || lmax < 1) return 0;
+  return decode_workspace_bytes(batch, params->n_kv_heads, lmax);
+}
+
+int ps_full_attn_ref(const ps_params* params, const void* k_full, const void* v_full,
+                     int64_t lmax, const void* q, const int64_t* pos, int64_t batch, void* out,
+                     float* lse, void* workspace, size_t ws_bytes, int32_t* dev_status,
+                     ps_stream_t stream) {
+  g_last_error.clear();
+  PS_TRY(check_params(params, false));
+  if (params->n_q_heads / params->n_kv_heads > kMaxGroup)
+    return fail(PS_ERR_UNSUPPORTED, "decode supports at most 8 query heads per KV head");
+  if (batch < 0) return fail(PS_ERR_INVALID_ARG, "batch must be >= 0");
+  if (lmax < 1 || lmax > 0x7fffffffLL) return fail(PS_ERR_INVALID_ARG, "lmax out of range");
+  if (batch == 0) return PS_OK;
+  PS_TRY(check_ptr(k_full, "k_full"));
+  PS_TRY(check_ptr(v_full, "v_full"));
+  PS_TRY(check_ptr(q, "q"));
+  PS_TRY(check_ptr(out, "out"));
+  PS_TRY(check_ptr(lse, "lse", true));
+  if (!pos) return fail(PS_ERR_INVALID_ARG, "pos is NULL");
+  if ((reinterpret_cast<uintptr_t>(pos) & 7u) != 0)
+    return fail(PS_ERR_INVALID_ARG, "pos is not 8-byte aligned");
+  const size_t need = decode_workspace_bytes(batch, params->n_kv_heads, lmax);
+  if (need > 0) {
+    if (!workspace || ws_bytes < need)
+      return fail(PS_ERR_WORKSPACE, "workspace smaller than ps_full_attn_workspace_bytes()");
+    PS_TRY(check_ptr(workspace, "workspace"));
+  }
+  DecodeLaunch l{};
+  l.q = q;
+  l.pos = pos;
+  l.out = out;
+  l.lse = lse;
+  l.workspace = workspace;
+  l.status = dev_status;
+  l.batch = batch;
+  l.hq = params->n_q_heads;
+  l.hkv = params->n_kv_heads;
+  l.lp = 0;
+  l.w = 1;
+  l.lmax = lmax;
+  l.full_mode = 1;
+  l.scale = resolve_scale(params);
+  l.k0 = k_full;
+  l.v0 = v_full;
+  l.k1 = nullptr;
+  l.v1 = nullptr;
+  return launch_decode(l, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int ps_decode_visible_ranges(const ps_params* params, const int64_t* pos, int64_t batch,
+                             int32_t* ranges_out, ps_stream_t stream) {
+  g_last_error.clear();
+  PS_TRY(check_params(params, true));
+  if (batch < 0) return fail(PS_ERR_INVALID_ARG, "batch must be >= 0");
+  if (batch == 0) return PS_OK;
+  if (!pos || !ranges_out) return fail(PS_ERR_INVALID_ARG, "pos / ranges_out is NULL");
+  return check_cuda(launch_visible_ranges(pos, batch, params->l_prefix, params->window,
+                                          ranges_out, reinterpret_cast<cudaStream_t>(stream)),
+                    "visible_ranges_kernel launch");
+}
+
+int ps_prefill_tile_geometry(int32_t* bq, int32_t* bk) {
+  if (!bq || !bk) return fail(PS_ERR_INVALID_ARG, "bq / bk is NULL");
+  *bq = kPrefillBq;
+  *bk = kPrefillBk;
+  return PS_OK;
+}
+
+int64_t ps_prefill_plan_tiles(const ps_params* params, int64_t seq) {
+  if (check_params(params, true) != PS_OK) return PS_ERR_INVALID_ARG;
+  if (seq < 1) return fail(PS_ERR_INVALID_ARG, "seq must be >= 1");
+  return prefill_plan_tiles(seq, params->l_prefix, params->window);
+}
+
+size_t ps_prefill_workspace_bytes(const ps_params* params, int64_t batch, int64_t seq) {
+  if (check_params(params, true) != PS_OK || batch < 0 || seq < 1) return 0;
+  return prefill_workspace_bytes(batch, seq, params->n_q_heads);
+}
+
+int ps_masked_prefill_attn(const ps_params* params, const void* q, const void* k, const void* v,
+                           int64_t batch, int64_t seq, void* out, float* lse, int32_t* tile_plan,
+                           int64_t tile_plan_cap, int64_t* n_tiles, void* workspace,
+                           size_t ws_bytes, ps_stream_t stream) {
+  g_last_error.clear();
+  PS_TRY(check_params(params, true));
+  if (batch < 0) return fail(PS_ERR_INVALID_ARG, "batch must be >= 0");
+  if (seq < 1 || seq > (1LL << 30)) return fail(PS_ERR_INVALID_ARG, "seq out of range");
+  const int64_t nt = prefill_plan_tiles(seq, params->l_prefix, params->window);
+  if (n_tiles) *n_tiles = nt;
+  if (tile_plan) {
+    PS_TRY(check_ptr(tile_plan, "tile_plan"));
+    if (tile_plan_cap < nt) return fail(PS_ERR_INVALID_ARG, "tile_plan_cap smaller than the plan");
+  }
+  if (batch == 0) return PS_OK;
+  PS_TRY(check_ptr(q, "q"));
+  PS_TRY(check_ptr(k, "k"));
+  PS_TRY(check_ptr(v, "v"));
+  PS_TRY(check_ptr(out, "out"));
+  PS_TRY(check_ptr(lse, "lse", true));
+  const size_t need = prefill_workspace_bytes(batch, seq, params->n_q_heads);
+  if (need > 0) {
+    if (!workspace || ws_bytes < need)
+      return fail(PS_ERR_WORKSPACE, "workspace smaller than ps_prefill_workspace_bytes()");
+    PS_TRY(check_ptr(workspace, "workspace"));
+  }
+  PrefillLaunch l{};
+  l.q = q;
+  l.k = k;
+  l.v = v;
+  l.out = out;
+  l.lse = lse;
+  l.plan_out = tile_plan;
+  l.workspace = workspace;
+  l.batch = batch;
+  l.seq = seq;
+  l.hq = params->n_q_heads;
+  l.hkv = params->n_kv_heads;
+  l.lp = params->l_prefix;
+  l.w = params->window;
+  l.scale = resolve_scale(params);
+  l.n_tiles = nt;
+  return launch_prefill(l, reinterpret_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,143 @@
+// KV append with Continue-PE RoPE into the Prefix Sliding store, sm_100a.
+//
+// "Prefix Sliding 完全拆解", §位置编码 (Continue PE): every token keeps its absolute position
+// id, so a key is rotated exactly once, when it is cached, and reused as is afterwards.
+// §核心机制: the store per sequence is bounded by L_prefix + W; a token past the prefix
+// overwrites the ring slot (pos - L_prefix) mod W, evicting the position it held.
+//
+// One CTA per appended token (sequence b, token t, position p = pos0[b] + t):
+//  * threads 0..63 form the 64 RoPE angles p * theta^(-2i/128) and reduce them in float64
+//    (at p ~ 2^18 an fp32 product would already be off by ~0.03 rad), then keep cos/sin in
+//    fp32 in shared memory;
+//  * every thread rotates 8 rotate-half pairs at a time (16-byte loads of x1 and x2),
+//    writes rotated K and the V row to the prefix row or ring slot, and rotates q in place.
+// When several of the T tokens fall on one ring slot only the latest is written, so the
+// result does not depend on thread scheduling.
+#include <cuda_bf16.h>
+#include <math.h>
+
+#include "ps_device.cuh"
+#include "ps_internal.h"
+
+namespace ps {
+namespace {
+
+constexpr int kAppendThreads = 256;
+constexpr int kHalf = kHeadDim / 2;  // rotate-half pairs per head
+constexpr int kChunks = kHalf / 8;   // 16-byte chunks per half
+
+__device__ __forceinline__ void rotate8(const uint4& x1, const uint4& x2, const float* cs,
+                                        const float* sn, uint4& y1, uint4& y2) {
+  const __nv_bfloat162* a = reinterpret_cast<const __nv_bfloat162*>(&x1);
+  const __nv_bfloat162* bb = reinterpret_cast<const __nv_bfloat162*>(&x2);
+  __nv_bfloat162* o1 = reinterpret_cast<__nv_bfloat162*>(&y1);
+  __nv_bfloat162* o2 = reinterpret_cast<__nv_bfloat162*>(&y2);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float2 u = __bfloat1622float2(a[e]);
+    const float2 v = __bfloat1622float2(bb[e]);
+    const float c0 = cs[2 * e], c1 = cs[2 * e + 1];
+    const float s0 = sn[2 * e], s1 = sn[2 * e + 1];
+    o1[e] = __floats2bfloat162_rn(u.x * c0 - v.x * s0, u.y * c1 - v.y * s1);
+    o2[e] = __floats2bfloat162_rn(v.x * c0 + u.x * s0, v.y * c1 + u.y * s1);
+  }
+}
+
+__global__ void __launch_bounds__(kAppendThreads) append_rope_kernel(const AppendArgs a) {
+  __shared__ float s_cos[kHalf];
+  __shared__ float s_sin[kHalf];
+  const int64_t tok = blockIdx.x;
+  const int64_t b = tok / a.T;
+  const int t = static_cast<int>(tok % a.T);
+  const int64_t p0 = a.pos0[b];
+  const int64_t p = p0 + t;
+  const int64_t p_last = p0 + a.T - 1;
+
+  if (p < 0) {
+    if (threadIdx.x == 0 && a.status) atomicOr(a.status, PS_DEV_BAD_POS);
+    return;
+  }
+  const bool linear = (a.k_ring == nullptr);
+  if (linear && p >= a.lp) {
+    if (threadIdx.x == 0 && a.status) atomicOr(a.status, PS_DEV_POS_RANGE);
+    return;
+  }
+  if (threadIdx.x < kHalf) {
+    const int i = threadIdx.x;
+    const double inv_f = pow(a.theta, -2.0 * i / double(kHeadDim));
+    double sd, cd;
+    sincos(double(p) * inv_f, &sd, &cd);
+    s_cos[i] = static_cast<float>(cd);
+    s_sin[i] = static_cast<float>(sd);
+  }
+  __syncthreads();
+
+  // where this token's K/V row goes (or nowhere, if a later token of this call owns it)
+  const __nv_bfloat16* k_src = static_cast<const __nv_bfloat16*>(a.k_new) + tok * a.hkv * kHeadDim;
+  const __nv_bfloat16* v_src = static_cast<const __nv_bfloat16*>(a.v_new) + tok * a.hkv * kHeadDim;
+  __nv_bfloat16* k_dst_base = nullptr;
+  __nv_bfloat16* v_dst_base = nullptr;
+  int64_t row_stride_rows = 0, row = 0;
+  if (p < a.lp) {
+    k_dst_base = static_cast<__nv_bfloat16*>(a.k_pre);
+    v_dst_base = static_cast<__nv_bfloat16*>(a.v_pre);
+    row_stride_rows = a.lp;
+    row = p;
+  } else if (p > p_last - a.w) {
+    k_dst_base = static_cast<__nv_bfloat16*>(a.k_ring);
+    v_dst_base = static_cast<__nv_bfloat16*>(a.v_ring);
+    row_stride_rows = a.w;
+    row = (p - a.lp) % a.w;
+  }
+
+  // K: rotate; V: copy.  Items: hkv heads x kChunks rotate items, hkv x 16 copy items.
+  const int n_k = a.hkv * kChunks;
+  const int n_v = a.hkv * (kHeadDim / 8);
+  if (k_dst_base != nullptr) {
+    for (int it = threadIdx.x; it < n_k + n_v; it += blockDim.x) {
+      if (it < n_k) {
+        const int h = it / kChunks, c = it % kChunks;
+        const __nv_bfloat16* src = k_src + h * kHeadDim;
+        const uint4 x1 = *reinterpret_cast<const uint4*>(src + 8 * c);
+        const uint4 x2 = *reinterpret_cast<const uint4*>(src + kHalf + 8 * c);
+        uint4 y1, y2;
+        rotate8(x1, x2, s_cos + 8 * c, s_sin + 8 * c, y1, y2);
+        __nv_bfloat16* dst = k_dst_base + ((b * a.hkv + h) * row_stride_rows + row) * kHeadDim;
+        *reinterpret_cast<uint4*>(dst + 8 * c) = y1;
+        *reinterpret_cast<uint4*>(dst + kHalf + 8 * c) = y2;
+      } else {
+        const int j = it - n_k;
+        const int h = j / (kHeadDim / 8), c = j % (kHeadDim / 8);
+        const uint4 x = *reinterpret_cast<const uint4*>(v_src + h * kHeadDim + 8 * c);
+        __nv_bfloat16* dst = v_dst_base + ((b * a.hkv + h) * row_stride_rows + row) * kHeadDim;
+        *reinterpret_cast<uint4*>(dst + 8 * c) = x;
+      }
+    }
+  }
+  // q rotated in place at the token's own absolute position
+  if (a.q != nullptr) {
+    __nv_bfloat16* qb = static_cast<__nv_bfloat16*>(a.q) + tok * a.hq * kHeadDim;
+    for (int it = threadIdx.x; it < a.hq * kChunks; it += blockDim.x) {
+      const int h = it / kChunks, c = it % kChunks;
+      __nv_bfloat16* src = qb + h * kHeadDim;
+      const uint4 x1 = *reinterpret_cast<const uint4*>(src + 8 * c);
+      const uint4 x2 = *reinterpret_cast<const uint4*>(src + kHalf + 8 * c);
+      uint4 y1, y2;
+      rotate8(x1, x2, s_cos + 8 * c, s_sin + 8 * c, y1, y2);
+      *reinterpret_cast<uint4*>(src + 8 * c) = y1;
+      *reinterpret_cast<uint4*>(src + kHalf + 8 * c) = y2;
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_append(const AppendArgs& a, cudaStream_t stream) {
+  const int64_t tokens = a.batch * a.T;
+  if (tokens <= 0) return cudaSuccess;
+  if (tokens > 0x7fffffff) return cudaErrorInvalidConfiguration;
+  append_rope_kernel<<<static_cast<unsigned>(tokens), kAppendThreads, 0, stream>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace ps

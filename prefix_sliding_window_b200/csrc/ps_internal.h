@@ -1,0 +1,94 @@
+// Internal declarations shared by the libps translation units (not part of the C ABI).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <string>
+
+#include "../../include/ps.h"
+
+namespace ps {
+
+constexpr int kHeadDim = 128;
+constexpr int kMaxGroup = 8;  // query heads per KV head handled by one decode CTA
+
+// Records a host-side failure message for ps_last_error() and returns `code`.
+int fail(int code, const std::string& msg);
+// Maps a CUDA runtime error to PS_ERR_CUDA with its message (PS_OK if no error).
+int check_cuda(cudaError_t e, const char* what);
+
+// Encodes a 3-D bf16 tensor map [z][y][x] with a box of {box_x, box_y, 1} and 128-byte
+// swizzle.  Returns false (with a message recorded) on failure.
+bool make_map_3d(CUtensorMap* map, const void* base, uint64_t x, uint64_t y, uint64_t z,
+                 uint32_t box_x, uint32_t box_y);
+
+// Streaming multiprocessor count of the current device.
+int sm_count();
+
+// ---------------------------------------------------------------- append
+struct AppendArgs {
+  const void* k_new;
+  const void* v_new;
+  void* q;
+  const int64_t* pos0;
+  void* k_pre;
+  void* v_pre;
+  void* k_ring;
+  void* v_ring;
+  int32_t* status;
+  int64_t batch;
+  int32_t T, hq, hkv, lp, w;
+  double theta;
+};
+cudaError_t launch_append(const AppendArgs& a, cudaStream_t stream);
+
+// ---------------------------------------------------------------- decode
+struct DecodeLaunch {
+  const void* q;
+  const int64_t* pos;
+  void* out;
+  float* lse;
+  void* workspace;
+  int32_t* status;
+  int64_t batch;
+  int32_t hq, hkv;
+  int32_t lp, w;
+  int64_t lmax;        // full-attention mode: rows of the linear cache
+  int32_t full_mode;   // 1: attend [0, pos] of a linear cache
+  float scale;
+  const void *k0, *v0;  // prefix (or linear) cache
+  const void *k1, *v1;  // ring (unused in full mode)
+};
+// Split count and workspace bytes for a decode of this shape on the current device.
+int decode_splits(int64_t batch, int32_t hkv, int64_t max_keys);
+size_t decode_workspace_bytes(int64_t batch, int32_t hkv, int64_t max_keys);
+int launch_decode(const DecodeLaunch& a, cudaStream_t stream);
+cudaError_t launch_visible_ranges(const int64_t* pos, int64_t batch, int32_t lp, int32_t w,
+                                  int32_t* out, cudaStream_t stream);
+
+// ---------------------------------------------------------------- prefill
+constexpr int kPrefillBq = 128;
+constexpr int kPrefillBk = 128;
+struct PrefillLaunch {
+  const void* q;
+  const void* k;
+  const void* v;
+  void* out;
+  float* lse;
+  int32_t* plan_out;  // optional copy of the plan
+  void* workspace;
+  int64_t batch, seq;
+  int32_t hq, hkv, lp, w;
+  float scale;
+  int64_t n_tiles;  // plan rows per (batch, head)
+};
+size_t prefill_workspace_bytes(int64_t batch, int64_t seq, int32_t hq);
+size_t prefill_plan_bytes(int64_t seq, int64_t n_tiles);
+cudaError_t launch_plan(int64_t seq, int32_t lp, int32_t w, int64_t n_tiles, void* workspace,
+                        int32_t* plan_out, cudaStream_t stream);
+int64_t prefill_plan_tiles(int64_t seq, int32_t lp, int32_t w);
+int launch_prefill(const PrefillLaunch& a, cudaStream_t stream);
+
+}  // namespace ps

@@ -1,0 +1,135 @@
+"""Host-side checks of libps.so that need no GPU: it loads, it exports every function
+include/ps.h declares, host validation returns the documented status codes before
+touching the device, and the host tile-plan count matches the oracle's brute force."""
+import ctypes
+import os
+
+import pytest
+
+import oracle as O
+from prefix_sliding_window_b200 import binding as B
+from prefix_sliding_window_b200 import build as BLD
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(B.LIB_PATH):
+        BLD.build(quiet=True)
+    return B.load()
+
+
+def test_library_exports_every_header_function(lib):
+    names = B.header_functions()
+    assert "ps_kv_append_rope" in names and "ps_decode_attn" in names
+    assert "ps_masked_prefill_attn" in names and "ps_full_attn_ref" in names
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) <= set(B._SIGS), set(names) - set(B._SIGS)
+
+
+def test_version_string(lib):
+    assert "sm_100a" in B.ps_version()
+
+
+def test_struct_layout_matches_header():
+    assert ctypes.sizeof(B.PsParams) == 40
+    assert B.PsParams.rope_theta.offset == 24
+    assert ctypes.sizeof(B.PsKVCache) == 40
+
+
+def _params(**kw):
+    base = dict(n_q_heads=16, n_kv_heads=2, head_dim=128, l_prefix=100, window=512)
+    base.update(kw)
+    return B.make_params(**base)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(head_dim=64), B.PS_ERR_UNSUPPORTED),
+    (dict(n_q_heads=15), B.PS_ERR_INVALID_ARG),
+    (dict(window=0), B.PS_ERR_INVALID_ARG),
+    (dict(l_prefix=-1), B.PS_ERR_INVALID_ARG),
+    (dict(n_kv_heads=0), B.PS_ERR_INVALID_ARG),
+    (dict(rope_theta=-1.0), B.PS_ERR_INVALID_ARG),
+])
+def test_bad_params_rejected_on_host(lib, kw, code):
+    p = _params(**kw)
+    cache = B.PsKVCache(None, None, None, None, 1)
+    rc = lib.ps_decode_attn(ctypes.byref(p), ctypes.byref(cache), None, None, None, None, None, 0,
+                            None, None)
+    assert rc == code
+    assert B.last_error() != ""
+
+
+def test_group_above_eight_unsupported_for_decode(lib):
+    p = _params(n_q_heads=32, n_kv_heads=2)
+    cache = B.PsKVCache(16, 16, 16, 16, 1)
+    rc = lib.ps_decode_attn(ctypes.byref(p), ctypes.byref(cache), 16, 16, 16, None, None, 0, None,
+                            None)
+    assert rc == B.PS_ERR_UNSUPPORTED
+
+
+def test_null_and_misaligned_pointers_rejected(lib):
+    p = _params()
+    cache = B.PsKVCache(16, 16, 16, 16, 2)
+    # q misaligned
+    rc = lib.ps_decode_attn(ctypes.byref(p), ctypes.byref(cache), 18, 16, 32, None, None, 0, None,
+                            None)
+    assert rc == B.PS_ERR_INVALID_ARG and "aligned" in B.last_error()
+    # ring NULL
+    cache2 = B.PsKVCache(16, 16, None, 16, 2)
+    rc = lib.ps_decode_attn(ctypes.byref(p), ctypes.byref(cache2), 16, 16, 32, None, None, 0,
+                            None, None)
+    assert rc == B.PS_ERR_INVALID_ARG
+    # pos misaligned (needs 8 bytes)
+    rc = lib.ps_kv_append_rope(ctypes.byref(p), ctypes.byref(cache), 16, 16, None, 20, 1, None,
+                               None)
+    assert rc == B.PS_ERR_INVALID_ARG
+    # T < 1
+    rc = lib.ps_kv_append_rope(ctypes.byref(p), ctypes.byref(cache), 16, 16, None, 16, 0, None,
+                               None)
+    assert rc == B.PS_ERR_INVALID_ARG
+
+
+def test_zero_batch_is_a_no_op(lib):
+    p = _params()
+    cache = B.PsKVCache(None, None, None, None, 0)
+    rc = lib.ps_kv_append_rope(ctypes.byref(p), ctypes.byref(cache), None, None, None, None, 1,
+                               None, None)
+    assert rc == B.PS_OK
+
+
+def test_tile_geometry(lib):
+    assert B.ps_prefill_tile_geometry() == (128, 128)
+
+
+@pytest.mark.parametrize("seq,lp,w", [(8192, 256, 2048), (300, 0, 300), (1000, 33, 100),
+                                     (129, 5, 1), (4096, 4096, 1), (1, 0, 1), (777, 100, 4096)])
+def test_host_plan_count_matches_oracle(lib, seq, lp, w):
+    bq, bk = B.ps_prefill_tile_geometry()
+    n = B.ps_prefill_plan_tiles(_params(l_prefix=lp, window=w), seq)
+    want = O.tile_plan(seq, lp, w, bq, bk).shape[0]
+    assert n == want
+
+
+def test_prefill_plan_rejects_bad_seq(lib):
+    with pytest.raises(B.PsError) as e:
+        B.ps_prefill_plan_tiles(_params(), 0)
+    assert e.value.code == B.PS_ERR_INVALID_ARG
+
+
+def test_prefill_small_plan_capacity_rejected(lib):
+    p = _params(l_prefix=256, window=2048)
+    n_tiles = ctypes.c_int64(-1)
+    rc = lib.ps_masked_prefill_attn(ctypes.byref(p), 16, 16, 16, 1, 8192, 16, None, 16, 10,
+                                    ctypes.byref(n_tiles), None, 0, None)
+    assert rc == B.PS_ERR_INVALID_ARG
+    assert n_tiles.value == O.tile_plan(8192, 256, 2048, 128, 128).shape[0]
+
+
+def test_workspace_too_small_rejected(lib):
+    p = _params(l_prefix=256, window=2048)
+    need = B.ps_prefill_workspace_bytes(p, 1, 8192)
+    assert need > 0
+    rc = lib.ps_masked_prefill_attn(ctypes.byref(p), 16, 16, 16, 1, 8192, 16, None, None, 0, None,
+                                    16, need - 1, None)
+    assert rc == B.PS_ERR_WORKSPACE
