@@ -125,6 +125,24 @@ int ps_decode_attn(const ps_params* params, const ps_kv_cache* cache, const void
                    const int64_t* pos, void* out, float* lse, void* workspace, size_t ws_bytes,
                    int32_t* dev_status, ps_stream_t stream);
 
+/* ps_decode_attn without a workspace argument, for callers that cannot allocate device
+ * memory: for example a plugin that its host framework hands only the input and output
+ * buffers, or a fixed-memory serving loop where a cudaMalloc (or a caching allocator
+ * growing) is not allowed between steps.  The paper has no counterpart; this is a
+ * convenience of this library.
+ * The split-K scratch lives in a device array built into libps (4 MiB = 4194304 bytes,
+ * held on every GPU that loads the library until the process exits).  A shape whose
+ * ps_decode_workspace_bytes() exceeds that returns PS_ERR_WORKSPACE and launches nothing.
+ * This call never allocates or frees memory (no cudaMalloc, no cudaFree).  The first call on
+ * each device looks up the array's device address with cudaGetSymbolAddress (with that
+ * device current); make that first call before any stream capture.  Every call shares the
+ * array and it keeps the last call's contents (nothing in it needs to start at zero); calls
+ * that overlap on the GPU, e.g. on two streams, race on it and must be serialised by the
+ * caller.  Arguments, results and errors are otherwise exactly those of ps_decode_attn. */
+int ps_decode_attn_noalloc(const ps_params* params, const ps_kv_cache* cache, const void* q,
+                           const int64_t* pos, void* out, float* lse, int32_t* dev_status,
+                           ps_stream_t stream);
+
 /* Bytes of device workspace ps_full_attn_ref needs (same split-K layout as decode). */
 size_t ps_full_attn_workspace_bytes(const ps_params* params, int64_t batch, int64_t lmax);
 

@@ -69,6 +69,8 @@ _SIGS = {
     "ps_decode_workspace_bytes": (c_size_t, [POINTER(PsParams), c_int64]),
     "ps_decode_attn": (c_int32, [POINTER(PsParams), POINTER(PsKVCache), c_void_p, c_void_p,
                                  c_void_p, c_void_p, c_void_p, c_size_t, c_void_p, c_void_p]),
+    "ps_decode_attn_noalloc": (c_int32, [POINTER(PsParams), POINTER(PsKVCache), c_void_p,
+                                         c_void_p, c_void_p, c_void_p, c_void_p, c_void_p]),
     "ps_full_attn_workspace_bytes": (c_size_t, [POINTER(PsParams), c_int64, c_int64]),
     "ps_full_attn_ref": (c_int32, [POINTER(PsParams), c_void_p, c_void_p, c_int64, c_void_p,
                                    c_void_p, c_int64, c_void_p, c_void_p, c_void_p, c_size_t,
@@ -163,6 +165,15 @@ def ps_decode_attn(params: PsParams, cache: PsKVCache, q, pos, out, lse=None, wo
                                _ptr(out), _ptr(lse), _ptr(workspace), ws_bytes, _ptr(dev_status),
                                _stream(stream))
     _check(rc, "ps_decode_attn")
+
+
+def ps_decode_attn_noalloc(params: PsParams, cache: PsKVCache, q, pos, out, lse=None,
+                           dev_status=None, stream=None) -> None:
+    """ps_decode_attn whose split-K scratch is the library's built-in device array."""
+    rc = load().ps_decode_attn_noalloc(ctypes.byref(params), ctypes.byref(cache), _ptr(q),
+                                       _ptr(pos), _ptr(out), _ptr(lse), _ptr(dev_status),
+                                       _stream(stream))
+    _check(rc, "ps_decode_attn_noalloc")
 
 
 def ps_full_attn_workspace_bytes(params: PsParams, batch: int, lmax: int) -> int:

@@ -248,6 +248,52 @@ int ps_decode_attn(const ps_params* params, const ps_kv_cache* cache, const void
   return launch_decode(l, reinterpret_cast<cudaStream_t>(stream));
 }
 
+int ps_decode_attn_noalloc(const ps_params* params, const ps_kv_cache* cache, const void* q,
+                           const int64_t* pos, void* out, float* lse, int32_t* dev_status,
+                           ps_stream_t stream) {
+  g_last_error.clear();
+  PS_TRY(check_params(params, true));
+  if (params->n_q_heads / params->n_kv_heads > kMaxGroup)
+    return fail(PS_ERR_UNSUPPORTED, "decode supports at most 8 query heads per KV head");
+  if (!cache) return fail(PS_ERR_INVALID_ARG, "cache is NULL");
+  if (cache->batch < 0) return fail(PS_ERR_INVALID_ARG, "cache->batch must be >= 0");
+  if (cache->batch == 0) return PS_OK;
+  PS_TRY(check_ptr(cache->k_ring, "cache->k_ring"));
+  PS_TRY(check_ptr(cache->v_ring, "cache->v_ring"));
+  if (params->l_prefix > 0) {
+    PS_TRY(check_ptr(cache->k_prefix, "cache->k_prefix"));
+    PS_TRY(check_ptr(cache->v_prefix, "cache->v_prefix"));
+  }
+  PS_TRY(check_ptr(q, "q"));
+  PS_TRY(check_ptr(out, "out"));
+  PS_TRY(check_ptr(lse, "lse", true));
+  if (!pos) return fail(PS_ERR_INVALID_ARG, "pos is NULL");
+  if ((reinterpret_cast<uintptr_t>(pos) & 7u) != 0)
+    return fail(PS_ERR_INVALID_ARG, "pos is not 8-byte aligned");
+  if ((reinterpret_cast<uintptr_t>(dev_status) & 3u) != 0)
+    return fail(PS_ERR_INVALID_ARG, "dev_status is not 4-byte aligned");
+  DecodeLaunch l{};
+  l.q = q;
+  l.pos = pos;
+  l.out = out;
+  l.lse = lse;
+  l.workspace = nullptr;
+  l.status = dev_status;
+  l.batch = cache->batch;
+  l.hq = params->n_q_heads;
+  l.hkv = params->n_kv_heads;
+  l.lp = params->l_prefix;
+  l.w = params->window;
+  l.lmax = 0;
+  l.full_mode = 0;
+  l.scale = resolve_scale(params);
+  l.k0 = cache->k_prefix;
+  l.v0 = cache->v_prefix;
+  l.k1 = cache->k_ring;
+  l.v1 = cache->v_ring;
+  return launch_decode_static_scratch(l, reinterpret_cast<cudaStream_t>(stream));
+}
+
 size_t ps_full_attn_workspace_bytes(const ps_params* params, int64_t batch, int64_t lmax) {
   if (check_params(params, false) != PS_OK || batch < 0 || lmax < 1) return 0;
   return decode_workspace_bytes(batch, params->n_kv_heads, lmax);

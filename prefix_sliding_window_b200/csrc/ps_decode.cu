@@ -28,6 +28,9 @@
 #include "ps_internal.h"
 #include "ps_ranges.cuh"
 
+#include <mutex>
+#include <string>
+
 namespace ps {
 namespace {
 
@@ -440,6 +443,48 @@ cudaError_t launch_visible_ranges(const int64_t* pos, int64_t batch, int32_t lp,
   const unsigned blocks = static_cast<unsigned>((batch + 127) / 128);
   visible_ranges_kernel<<<blocks, 128, 0, stream>>>(pos, batch, lp, w, out);
   return cudaGetLastError();
+}
+
+// ------------------------------------------------- decode with built-in scratch
+// Scratch for callers that cannot allocate device memory: the split-K partials of
+// launch_decode_static_scratch live in this file-scope array.  It is part of the loaded
+// module, so every GPU that loads the library holds it until the process exits.  All calls
+// share it; it keeps the last call's contents (nothing in it has to start at zero), and
+// calls that overlap on the GPU (for example on two streams) race on it.
+static __device__ __align__(256) unsigned char g_decode_scratch[kDecodeScratchBytes];
+
+namespace {
+std::mutex g_scratch_mu;
+void* g_scratch_ptr[64] = {nullptr};
+}  // namespace
+
+int launch_decode_static_scratch(const DecodeLaunch& l, cudaStream_t stream) {
+  const int64_t max_keys = l.full_mode ? l.lmax : (int64_t)l.lp + l.w;
+  const size_t need = decode_workspace_bytes(l.batch, l.hkv, max_keys);
+  if (need > kDecodeScratchBytes)
+    return fail(PS_ERR_WORKSPACE,
+                "decode needs " + std::to_string(need) + " bytes of scratch; the built-in array "
+                "holds " + std::to_string(kDecodeScratchBytes) + " (use ps_decode_attn)");
+  int dev = 0;
+  int rc = check_cuda(cudaGetDevice(&dev), "cudaGetDevice");
+  if (rc != PS_OK) return rc;
+  if (dev < 0 || dev >= 64) return fail(PS_ERR_UNSUPPORTED, "device index above 63");
+  void* ptr = nullptr;
+  {
+    // Host code cannot use g_decode_scratch's address directly: on the host the name is a
+    // stand-in.  Ask the runtime once per device, with that device current.
+    std::lock_guard<std::mutex> lock(g_scratch_mu);
+    if (g_scratch_ptr[dev] == nullptr) {
+      void* p = nullptr;
+      rc = check_cuda(cudaGetSymbolAddress(&p, g_decode_scratch), "cudaGetSymbolAddress");
+      if (rc != PS_OK) return rc;
+      g_scratch_ptr[dev] = p;
+    }
+    ptr = g_scratch_ptr[dev];
+  }
+  DecodeLaunch l2 = l;
+  l2.workspace = ptr;
+  return launch_decode(l2, stream);
 }
 
 }  // namespace ps

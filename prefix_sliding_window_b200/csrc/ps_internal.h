@@ -65,6 +65,9 @@ struct DecodeLaunch {
 int decode_splits(int64_t batch, int32_t hkv, int64_t max_keys);
 size_t decode_workspace_bytes(int64_t batch, int32_t hkv, int64_t max_keys);
 int launch_decode(const DecodeLaunch& a, cudaStream_t stream);
+// Decode whose split-K scratch is the library's file-scope device array (no allocation).
+constexpr size_t kDecodeScratchBytes = size_t(4) << 20;
+int launch_decode_static_scratch(const DecodeLaunch& a, cudaStream_t stream);
 cudaError_t launch_visible_ranges(const int64_t* pos, int64_t batch, int32_t lp, int32_t w,
                                   int32_t* out, cudaStream_t stream);
 
