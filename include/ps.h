@@ -180,13 +180,15 @@ size_t ps_prefill_workspace_bytes(const ps_params* params, int64_t batch, int64_
  *           the kernel ran: rows (q_tile, k_tile, flag), q-tile-major, ascending k_tile,
  *           SKIP tiles omitted (flag PS_TILE_FULL or PS_TILE_PARTIAL).
  *   n_tiles : host int64 or NULL; receives the number of plan rows.
- *   workspace, ws_bytes : device scratch of at least ps_prefill_workspace_bytes().
+ *   workspace, ws_bytes : device scratch of at least ps_prefill_workspace_bytes() (it holds
+ *           the tile plan the kernel walks).
+ *   dev_status : device int32 or NULL (PS_DEV_TIMEOUT only).
  * Requires seq >= 1 and Hq / Hkv integral.  tile_plan_cap smaller than the plan is
  * PS_ERR_INVALID_ARG. */
 int ps_masked_prefill_attn(const ps_params* params, const void* q, const void* k, const void* v,
                            int64_t batch, int64_t seq, void* out, float* lse, int32_t* tile_plan,
                            int64_t tile_plan_cap, int64_t* n_tiles, void* workspace,
-                           size_t ws_bytes, ps_stream_t stream);
+                           size_t ws_bytes, int32_t* dev_status, ps_stream_t stream);
 
 /* Introspection for bit-exact checks: the visible-range descriptor the decode kernel
  * uses, computed by the same device code.  ranges_out: device int32 [batch, 4] =

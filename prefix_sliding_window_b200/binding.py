@@ -80,7 +80,8 @@ _SIGS = {
     "ps_prefill_workspace_bytes": (c_size_t, [POINTER(PsParams), c_int64, c_int64]),
     "ps_masked_prefill_attn": (c_int32, [POINTER(PsParams), c_void_p, c_void_p, c_void_p, c_int64,
                                          c_int64, c_void_p, c_void_p, c_void_p, c_int64,
-                                         POINTER(c_int64), c_void_p, c_size_t, c_void_p]),
+                                         POINTER(c_int64), c_void_p, c_size_t, c_void_p,
+                                         c_void_p]),
     "ps_decode_visible_ranges": (c_int32, [POINTER(PsParams), c_void_p, c_int64, c_void_p,
                                            c_void_p]),
     "ps_last_error": (c_char_p, []),
@@ -208,7 +209,7 @@ def ps_prefill_workspace_bytes(params: PsParams, batch: int, seq: int) -> int:
 
 
 def ps_masked_prefill_attn(params: PsParams, q, k, v, batch: int, seq: int, out, lse=None,
-                           tile_plan=None, workspace=None, stream=None) -> int:
+                           tile_plan=None, workspace=None, dev_status=None, stream=None) -> int:
     """Returns the number of plan rows (tiles per (batch, head))."""
     n_tiles = c_int64(-1)
     cap = 0 if tile_plan is None else tile_plan.shape[0]
@@ -216,7 +217,7 @@ def ps_masked_prefill_attn(params: PsParams, q, k, v, batch: int, seq: int, out,
     rc = load().ps_masked_prefill_attn(ctypes.byref(params), _ptr(q), _ptr(k), _ptr(v), int(batch),
                                        int(seq), _ptr(out), _ptr(lse), _ptr(tile_plan), int(cap),
                                        ctypes.byref(n_tiles), _ptr(workspace), ws_bytes,
-                                       _stream(stream))
+                                       _ptr(dev_status), _stream(stream))
     _check(rc, "ps_masked_prefill_attn")
     return n_tiles.value
 

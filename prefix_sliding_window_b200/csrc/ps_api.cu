@@ -117,6 +117,29 @@ bool make_map_3d(CUtensorMap* map, const void* base, uint64_t x, uint64_t y, uin
   return true;
 }
 
+bool make_map_4d(CUtensorMap* map, const void* base, const uint64_t dims[4],
+                 const uint32_t box[4]) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) {
+    fail(PS_ERR_CUDA, "cuTensorMapEncodeTiled unavailable (no CUDA driver?)");
+    return false;
+  }
+  const cuuint64_t d[4] = {dims[0], dims[1], dims[2], dims[3]};
+  const cuuint64_t strides[3] = {dims[0] * 2, dims[0] * dims[1] * 2,
+                                 dims[0] * dims[1] * dims[2] * 2};
+  const cuuint32_t bx[4] = {box[0], box[1], box[2], box[3]};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), d,
+                        strides, bx, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    fail(PS_ERR_CUDA, "cuTensorMapEncodeTiled (4-D) failed (" + std::to_string(int(r)) + ")");
+    return false;
+  }
+  return true;
+}
+
 int sm_count() {
   static int cached[64] = {0};
   int dev = 0;
@@ -373,13 +396,13 @@ int64_t ps_prefill_plan_tiles(const ps_params* params, int64_t seq) {
 
 size_t ps_prefill_workspace_bytes(const ps_params* params, int64_t batch, int64_t seq) {
   if (check_params(params, true) != PS_OK || batch < 0 || seq < 1) return 0;
-  return prefill_workspace_bytes(batch, seq, params->n_q_heads);
+  return prefill_workspace_bytes(seq, params->l_prefix, params->window);
 }
 
 int ps_masked_prefill_attn(const ps_params* params, const void* q, const void* k, const void* v,
                            int64_t batch, int64_t seq, void* out, float* lse, int32_t* tile_plan,
                            int64_t tile_plan_cap, int64_t* n_tiles, void* workspace,
-                           size_t ws_bytes, ps_stream_t stream) {
+                           size_t ws_bytes, int32_t* dev_status, ps_stream_t stream) {
   g_last_error.clear();
   PS_TRY(check_params(params, true));
   if (batch < 0) return fail(PS_ERR_INVALID_ARG, "batch must be >= 0");
@@ -396,7 +419,10 @@ int ps_masked_prefill_attn(const ps_params* params, const void* q, const void* k
   PS_TRY(check_ptr(v, "v"));
   PS_TRY(check_ptr(out, "out"));
   PS_TRY(check_ptr(lse, "lse", true));
-  const size_t need = prefill_workspace_bytes(batch, seq, params->n_q_heads);
+  if ((reinterpret_cast<uintptr_t>(dev_status) & 3u) != 0)
+    return fail(PS_ERR_INVALID_ARG, "dev_status is not 4-byte aligned");
+  if (batch > 0x7fffffffLL) return fail(PS_ERR_UNSUPPORTED, "batch too large");
+  const size_t need = prefill_workspace_bytes(seq, params->l_prefix, params->window);
   if (need > 0) {
     if (!workspace || ws_bytes < need)
       return fail(PS_ERR_WORKSPACE, "workspace smaller than ps_prefill_workspace_bytes()");
@@ -418,6 +444,7 @@ int ps_masked_prefill_attn(const ps_params* params, const void* q, const void* k
   l.w = params->window;
   l.scale = resolve_scale(params);
   l.n_tiles = nt;
+  l.status = dev_status;
   return launch_prefill(l, reinterpret_cast<cudaStream_t>(stream));
 }
 

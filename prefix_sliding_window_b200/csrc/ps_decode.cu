@@ -172,7 +172,8 @@ __global__ void __launch_bounds__(kThreads)
 
     for (int i = 0; i < ntiles; ++i) {
       const int s = i % STAGES;
-      if (!mbar_wait(&full[s], (i / STAGES) & 1, a.status)) break;
+      // warp-uniform outcome: ldmatrix / mma.sync below are warp-collective
+      if (!__all_sync(0xffffffffu, mbar_wait(&full[s], (i / STAGES) & 1, a.status))) break;
       const DecodeTile d = tiling_tile(t, t_begin + i);
       const uint32_t kbase = smem_u32(smem + s * kStageBytes);
       const uint32_t vbase = kbase + kTileBytes;

@@ -24,6 +24,10 @@ int check_cuda(cudaError_t e, const char* what);
 bool make_map_3d(CUtensorMap* map, const void* base, uint64_t x, uint64_t y, uint64_t z,
                  uint32_t box_x, uint32_t box_y);
 
+// Encodes a 4-D bf16 tensor map (dims innermost first, dense strides) with 128-byte swizzle.
+bool make_map_4d(CUtensorMap* map, const void* base, const uint64_t dims[4],
+                 const uint32_t box[4]);
+
 // Streaming multiprocessor count of the current device.
 int sm_count();
 
@@ -86,8 +90,9 @@ struct PrefillLaunch {
   int32_t hq, hkv, lp, w;
   float scale;
   int64_t n_tiles;  // plan rows per (batch, head)
+  int32_t* status;
 };
-size_t prefill_workspace_bytes(int64_t batch, int64_t seq, int32_t hq);
+size_t prefill_workspace_bytes(int64_t seq, int32_t lp, int32_t w);
 size_t prefill_plan_bytes(int64_t seq, int64_t n_tiles);
 cudaError_t launch_plan(int64_t seq, int32_t lp, int32_t w, int64_t n_tiles, void* workspace,
                         int32_t* plan_out, cudaStream_t stream);

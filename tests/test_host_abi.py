@@ -121,7 +121,7 @@ def test_prefill_small_plan_capacity_rejected(lib):
     p = _params(l_prefix=256, window=2048)
     n_tiles = ctypes.c_int64(-1)
     rc = lib.ps_masked_prefill_attn(ctypes.byref(p), 16, 16, 16, 1, 8192, 16, None, 16, 10,
-                                    ctypes.byref(n_tiles), None, 0, None)
+                                    ctypes.byref(n_tiles), None, 0, None, None)
     assert rc == B.PS_ERR_INVALID_ARG
     assert n_tiles.value == O.tile_plan(8192, 256, 2048, 128, 128).shape[0]
 
@@ -131,5 +131,5 @@ def test_workspace_too_small_rejected(lib):
     need = B.ps_prefill_workspace_bytes(p, 1, 8192)
     assert need > 0
     rc = lib.ps_masked_prefill_attn(ctypes.byref(p), 16, 16, 16, 1, 8192, 16, None, None, 0, None,
-                                    16, need - 1, None)
+                                    16, need - 1, None, None)
     assert rc == B.PS_ERR_WORKSPACE
