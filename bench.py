@@ -345,6 +345,276 @@ def run_decode_e2e(work: DecodeWorkload, K: int, W: int, world: int):
             "d2h_bytes_per_step": bo}
 
 
+# ------------------------------------------------------------- prefill leg
+def prefill_visible_pairs(S: int, lp: int, w: int) -> int:
+    """Visible (row, key) pairs of one (batch, head): sum over rows of min(i + 1, Lp + W)."""
+    cap = lp + w
+    n1 = min(S, cap)
+    return n1 * (n1 + 1) // 2 + (S - n1) * cap
+
+
+def run_prefill(dev, steps: int = 10, warmup: int = 3):
+    """Masked prefill / truncated-backprop context forward: batch 4, 8192 tokens,
+    28/4/128, L_prefix 256, W 2048.  TFLOP/s counts unmasked FLOPs only
+    (4 * D per visible pair per query head)."""
+    from prefix_sliding_window_b200 import binding as B
+    wl = synth.WORKLOADS["prefill_b4_s8192_w2048"]
+    Bn, S, hq, hkv, lp, w = wl.batch, wl.seq, wl.n_q_heads, wl.n_kv_heads, wl.l_prefix, wl.window
+    params = B.make_params(hq, hkv, D, lp, w, wl.rope_theta)
+    q = synth.normal_bf16((Bn, S, hq, D), synth.seed_for(3, 1), dev)
+    k = synth.normal_bf16((Bn, S, hkv, D), synth.seed_for(3, 2), dev)
+    v = synth.normal_bf16((Bn, S, hkv, D), synth.seed_for(3, 3), dev)
+    out = torch.empty_like(q)
+    lse = torch.empty((Bn, hq, S), dtype=torch.float32, device=dev)
+    n = B.ps_prefill_plan_tiles(params, S)
+    plan = torch.empty((n, 3), dtype=torch.int32, device=dev)
+    ws = torch.empty(B.ps_prefill_workspace_bytes(params, Bn, S), dtype=torch.uint8, device=dev)
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        B.ps_masked_prefill_attn(params, q, k, v, Bn, S, out, lse, plan, ws, st)
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(steps)]
+    for a, b in evs:
+        a.record(stream)
+        B.ps_masked_prefill_attn(params, q, k, v, Bn, S, out, lse, None, ws, st)
+        b.record(stream)
+    torch.cuda.synchronize()
+    assert st.item() == 0, f"device status {st.item()}"
+    ms = [a.elapsed_time(b) for a, b in evs]
+    flags = plan[:, 2].cpu()
+    n_full = int((flags == B.PS_TILE_FULL).sum())
+    n_part = int((flags == B.PS_TILE_PARTIAL).sum())
+    nq = -(-S // 128)
+    pairs = prefill_visible_pairs(S, lp, w)
+    flops = 4 * D * pairs * hq * Bn
+    computed = 4 * D * 128 * 128 * n * hq * Bn
+    med = statistics.median(ms) / 1e3
+    tflops = flops / med / 1e12
+    peaks = _peaks()
+    return {"workload": wl.name, "ms": round(med * 1e3, 4),
+            "ms_p10": round(float(np.percentile(ms, 10)), 4),
+            "ms_p90": round(float(np.percentile(ms, 90)), 4),
+            "tflops_unmasked": round(tflops, 1), "unit": "TFLOP/s",
+            "peak": peaks["bf16_tflops"], "frac": round(tflops / peaks["bf16_tflops"], 4),
+            "frac_of_2250_spec": round(tflops / 2250.0, 4),
+            "tflops_computed_tiles": round(computed / med / 1e12, 1),
+            "unmasked_gflop": round(flops / 1e9, 1), "computed_gflop": round(computed / 1e9, 1),
+            "tiles_per_head": {"full": n_full, "partial": n_part, "skip": nq * nq - n},
+            "launches_per_call": 2, "inputs": "Q 235 MB + K,V 67 MB per call (> L2)"}
+
+
+# -------------------------------------------------------- full attention leg
+def run_full_attention(work: DecodeWorkload, steps: int = 16, warmup: int = 3):
+    """Full causal attention over the same positions as the decode workload (every key in
+    [0, pos] of a linear cache), one append + ps_full_attn_ref per step."""
+    from prefix_sliding_window_b200 import binding as B
+    from prefix_sliding_window_b200.cache import LinearCache
+    wl, dev = work.wl, work.dev
+    Bn, hq, hkv = wl.batch, wl.n_q_heads, wl.n_kv_heads
+    n_steps = min(steps + warmup, work.k_new.shape[0])
+    steps = n_steps - warmup
+    lmax = int(work.pos_start.max().item()) + n_steps + 1
+    lin = LinearCache(Bn, hkv, lmax, D, dev, fill=None)
+    lp_params = lin.params(hq, wl.rope_theta)
+    st = work.status
+    chunk = 4096
+    for c0 in range(0, lmax, chunk):
+        T = min(chunk, lmax - c0)
+        kk = synth.normal_bf16((Bn, T, hkv, D), 50_000 + c0, dev)
+        vv = synth.normal_bf16((Bn, T, hkv, D), 90_000 + c0, dev)
+        B.ps_kv_append_rope(lp_params, lin.struct, kk, vv, None,
+                            torch.full((Bn,), c0, dtype=torch.int64, device=dev), T, st)
+        del kk, vv
+    params = B.make_params(hq, hkv, D, 0, 1, wl.rope_theta)
+    ws = torch.empty(max(1, B.ps_full_attn_workspace_bytes(params, Bn, lmax)), dtype=torch.uint8,
+                     device=dev)
+    q = work.q_raw[:n_steps].clone()
+    out = torch.empty_like(work.out[0])
+    stream = torch.cuda.current_stream()
+
+    def step(i):
+        B.ps_kv_append_rope(lp_params, lin.struct, work.k_new[i], work.v_new[i], q[i], work.pos[i],
+                            1, st)
+        B.ps_full_attn_ref(params, lin.k, lin.v, lmax, q[i], work.pos[i], Bn, out, None, ws, st)
+
+    for i in range(warmup):
+        step(i)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(warmup, n_steps):
+        step(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    ms = e0.elapsed_time(e1) / steps
+    mean_pos = float(work.pos_start.double().mean().item()) + warmup + steps / 2
+    kv_bytes = Bn * (mean_pos + 1) * 2 * hkv * D * 2
+    del lin
+    return {"workload": wl.name + " (full causal attention over [0, pos])",
+            "ms_per_step": round(ms, 4), "tok_per_s": round(Bn / (ms / 1e3), 1),
+            "kv_gb_per_step": round(kv_bytes / 1e9, 3),
+            "gbs": round(kv_bytes / (ms / 1e3) / 1e9, 1)}
+
+
+# ------------------------------------------------------ long-trace sweep leg
+def _fill_cache(B, params, cache_struct, Bn, hkv, ranges, dev, seed, st, chunk=2048):
+    """Append N(0,1) tokens at absolute positions [lo, hi) for every sequence."""
+    for lo, hi in ranges:
+        for c0 in range(lo, hi, chunk):
+            T = min(chunk, hi - c0)
+            k = synth.normal_bf16((Bn, T, hkv, D), seed + c0, dev)
+            v = synth.normal_bf16((Bn, T, hkv, D), seed + 7 * c0 + 1, dev)
+            B.ps_kv_append_rope(params, cache_struct, k, v, None,
+                                torch.full((Bn,), c0, dtype=torch.int64, device=dev), T, st)
+            del k, v
+
+
+def run_sweep(dev, steps: int = 20, warmup: int = 3):
+    """Long-trace decode sweep: batch 256, 16/2/128, W = 8192; every sequence at the same
+    position P in {4K, ..., 128K}; prefix sliding (L_prefix = 100) vs pure sliding window
+    (L_prefix = 0) vs full attention.  Per-step latency of append + attention and the
+    attention kernel's HBM GB/s."""
+    from prefix_sliding_window_b200 import binding as B
+    from prefix_sliding_window_b200.cache import LinearCache, PrefixSlidingCache
+    wl = synth.WORKLOADS["decode_sweep_b256_w8192"]
+    Bn, hq, hkv, w = wl.batch, wl.n_q_heads, wl.n_kv_heads, wl.window
+    peaks = _peaks()
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    n = steps + warmup
+    k_new = synth.normal_bf16((n, Bn, 1, hkv, D), 11, dev)
+    v_new = synth.normal_bf16((n, Bn, 1, hkv, D), 12, dev)
+    q_raw = synth.normal_bf16((n, Bn, hq, D), 13, dev)
+    out = torch.empty((Bn, hq, D), dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream()
+    points = []
+    for P in (4096, 8192, 16384, 32768, 65536, 131072):
+        pos = torch.stack([torch.full((Bn,), P + i, dtype=torch.int64, device=dev)
+                           for i in range(n)])
+        res = {"position": P}
+        for mode in ("prefix_sliding", "sliding_window", "full"):
+            if mode == "full":
+                lmax = P + n + 1
+                cache = LinearCache(Bn, hkv, lmax, D, dev, fill=None)
+                aparams = cache.params(hq, wl.rope_theta)
+                _fill_cache(B, aparams, cache.struct, Bn, hkv, [(0, P)], dev, 1000, st)
+                dparams = B.make_params(hq, hkv, D, 0, 1, wl.rope_theta)
+                ws = torch.empty(max(1, B.ps_full_attn_workspace_bytes(dparams, Bn, lmax)),
+                                 dtype=torch.uint8, device=dev)
+
+                def attn(i, cache=cache, dparams=dparams, ws=ws, lmax=lmax):
+                    B.ps_full_attn_ref(dparams, cache.k, cache.v, lmax, q[i], pos[i], Bn, out,
+                                       None, ws, st)
+            else:
+                lp = wl.l_prefix if mode == "prefix_sliding" else 0
+                cache = PrefixSlidingCache(Bn, hkv, lp, w, D, dev, fill=None)
+                aparams = dparams = B.make_params(hq, hkv, D, lp, w, wl.rope_theta)
+                _fill_cache(B, aparams, cache.struct, Bn, hkv,
+                            [(0, min(lp, P)), (max(lp, P - w + 1), P)], dev, 1000, st)
+                ws = torch.empty(max(1, B.ps_decode_workspace_bytes(dparams, Bn)),
+                                 dtype=torch.uint8, device=dev)
+
+                def attn(i, cache=cache, dparams=dparams, ws=ws):
+                    B.ps_decode_attn(dparams, cache.struct, q[i], pos[i], out, None, ws, st)
+            q = q_raw.clone()
+            evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+                    torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+            for i in range(n):
+                evs[i][0].record(stream)
+                B.ps_kv_append_rope(aparams, cache.struct, k_new[i], v_new[i], q[i], pos[i], 1, st)
+                evs[i][1].record(stream)
+                attn(i)
+                evs[i][2].record(stream)
+            torch.cuda.synchronize()
+            assert st.item() == 0
+            step_ms = statistics.median([a.elapsed_time(c) for a, _, c in evs[warmup:]])
+            attn_ms = statistics.median([b.elapsed_time(c) for _, b, c in evs[warmup:]])
+            if mode == "full":
+                keys = P + warmup + steps / 2 + 1
+            else:
+                keys = min(P + 1, (wl.l_prefix if mode == "prefix_sliding" else 0) + w)
+            kv_bytes = Bn * keys * 2 * hkv * D * 2 + 2 * Bn * hq * D * 2
+            gbs = kv_bytes / (attn_ms / 1e3) / 1e9
+            res[mode] = {"step_us": round(step_ms * 1e3, 1), "attn_us": round(attn_ms * 1e3, 1),
+                         "attn_gbs": round(gbs, 1), "frac": round(gbs / peaks["hbm_gbs"], 4),
+                         "tok_per_s": round(Bn / (step_ms / 1e3), 1)}
+            del cache, ws
+            torch.cuda.empty_cache()
+        points.append(res)
+    return {"leg": "sweep", "workload": wl.name, "steps": steps, "points": points,
+            "peak_hbm_gbs": peaks["hbm_gbs"]}
+
+
+# ------------------------------------------------------- full-stack decode leg
+def run_stack(dev, batch: int, distinct: int, steps: int = 3, warmup: int = 1):
+    """Full-stack decode step: 28 layers x (append + decode), 16/2/128, L_prefix 2000,
+    W 16384, positions in [32768, 262144].  The 28 logical layers are mapped round-robin
+    onto `distinct` resident layer caches (all 28 caches of 1024 sequences, 540 GB, do not
+    fit in one GPU's 180 GB); each layer's working set is far larger than L2, so every
+    layer reads its K/V from HBM."""
+    from prefix_sliding_window_b200 import binding as B
+    from prefix_sliding_window_b200.cache import PrefixSlidingCache
+    wl = synth.WORKLOADS["decode_stack_l28_b1024_w16384"]
+    Bn, hq, hkv, lp, w, L = batch, wl.n_q_heads, wl.n_kv_heads, wl.l_prefix, wl.window, wl.n_layers
+    params = B.make_params(hq, hkv, D, lp, w, wl.rope_theta)
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    pos0 = synth.uniform_positions(Bn, wl.pos_lo, wl.pos_hi, synth.seed_for(5), dev)
+    caches = []
+    for li in range(distinct):
+        c = PrefixSlidingCache(Bn, hkv, lp, w, D, dev, fill=None)
+        # prefix, then the window history [p - W + 1, p - 1] of every sequence
+        B.ps_kv_append_rope(params, c.struct, synth.normal_bf16((Bn, lp, hkv, D), 3 * li, dev),
+                            synth.normal_bf16((Bn, lp, hkv, D), 3 * li + 1, dev), None,
+                            torch.zeros(Bn, dtype=torch.int64, device=dev), lp, st)
+        chunk = 1024
+        for c0 in range(0, w - 1, chunk):
+            T = min(chunk, w - 1 - c0)
+            B.ps_kv_append_rope(params, c.struct,
+                                synth.normal_bf16((Bn, T, hkv, D), 100 * li + c0, dev),
+                                synth.normal_bf16((Bn, T, hkv, D), 100 * li + c0 + 1, dev), None,
+                                pos0 - (w - 1) + c0, T, st)
+        caches.append(c)
+    torch.cuda.synchronize()
+    k_new = synth.normal_bf16((L, Bn, 1, hkv, D), 21, dev)
+    v_new = synth.normal_bf16((L, Bn, 1, hkv, D), 22, dev)
+    q_raw = synth.normal_bf16((L, Bn, hq, D), 23, dev)
+    q = q_raw.clone()
+    out = torch.empty((Bn, hq, D), dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(max(1, B.ps_decode_workspace_bytes(params, Bn)), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(i):
+        pos = pos0 + i
+        for layer in range(L):
+            c = caches[layer % distinct]
+            q[layer].copy_(q_raw[layer])
+            B.ps_kv_append_rope(params, c.struct, k_new[layer], v_new[layer], q[layer], pos, 1, st)
+            B.ps_decode_attn(params, c.struct, q[layer], pos, out, None, ws, st)
+
+    for i in range(warmup):
+        step(i)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(warmup, warmup + steps):
+        step(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    ms = e0.elapsed_time(e1) / steps
+    kv_bytes = L * Bn * (lp + w) * 2 * hkv * D * 2
+    gbs = kv_bytes / (ms / 1e3) / 1e9
+    peaks = _peaks()
+    return {"leg": "stack", "workload": wl.name, "batch": Bn, "layers": L,
+            "distinct_layer_caches": distinct,
+            "resident_kv_gb": round(distinct * caches[0].nbytes() / 1e9, 1),
+            "ms_per_step": round(ms, 3), "tok_per_s": round(Bn / (ms / 1e3), 1),
+            "kv_gb_per_step": round(kv_bytes / 1e9, 1), "gbs": round(gbs, 1),
+            "frac": round(gbs / peaks["hbm_gbs"], 4)}
+
+
 # ----------------------------------------------------------- CPU oracle leg
 def _blas_threads():
     try:
@@ -428,6 +698,12 @@ def main():
     ap.add_argument("--warmup", type=int, default=8)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--leg", default="main", choices=["main", "prefill", "sweep", "stack"],
+                    help="main: the driver's line; prefill/sweep/stack: one extra workload")
+    ap.add_argument("--stack-batch", type=int, default=1024)
+    ap.add_argument("--stack-distinct", type=int, default=6)
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the full-attention comparator and the prefill leg")
     ap.add_argument("--traffic", type=float, default=None,
                     help="ncu dram bytes per decode launch, when known for this kernel")
     args = ap.parse_args()
@@ -441,7 +717,24 @@ def main():
         return
     world, rank, local = _dist_setup()
     dev = torch.device("cuda", local)
-    line, _ = run_decode(args, world, rank, dev)
+    if args.leg != "main":
+        if args.leg == "prefill":
+            res = {"leg": "prefill", **run_prefill(dev, steps=args.steps, warmup=args.warmup)}
+        elif args.leg == "sweep":
+            res = run_sweep(dev)
+        else:
+            res = run_stack(dev, args.stack_batch, args.stack_distinct)
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+        return
+    line, work = run_decode(args, world, rank, dev)
+    if not args.no_extras:
+        full = run_full_attention(work)
+        full["ps_speedup"] = round(line["value"] / full["tok_per_s"], 2)
+        line["full_attention"] = full
+        del work
+        torch.cuda.empty_cache()
+        line["prefill"] = run_prefill(dev)
     if rank == 0:
         if not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(synth.WORKLOADS[WORKLOAD])

@@ -207,7 +207,8 @@ int ps_kv_append_rope(const ps_params* params, const ps_kv_cache* cache, const v
   a.hkv = params->n_kv_heads;
   a.lp = params->l_prefix;
   a.w = params->window;
-  a.theta = params->rope_theta;
+  for (int i = 0; i < kHeadDim / 2; ++i)
+    a.inv_freq[i] = pow(params->rope_theta, -2.0 * i / double(kHeadDim));
   return check_cuda(launch_append(a, reinterpret_cast<cudaStream_t>(stream)),
                     "append_rope_kernel launch");
 }

@@ -6,9 +6,9 @@
 // overwrites the ring slot (pos - L_prefix) mod W, evicting the position it held.
 //
 // One CTA per appended token (sequence b, token t, position p = pos0[b] + t):
-//  * threads 0..63 form the 64 RoPE angles p * theta^(-2i/128) and reduce them in float64
-//    (at p ~ 2^18 an fp32 product would already be off by ~0.03 rad), then keep cos/sin in
-//    fp32 in shared memory;
+//  * threads 0..63 form the 64 RoPE angles p * theta^(-2i/128) in float64 (at p ~ 2^18 an
+//    fp32 product would already be off by ~0.03 rad; the host supplies theta^(-2i/128) in
+//    float64), reduce them modulo 2*pi in float64 and keep cos/sin in fp32 in shared memory;
 //  * every thread rotates 8 rotate-half pairs at a time (16-byte loads of x1 and x2),
 //    writes rotated K and the V row to the prefix row or ring slot, and rotates q in place.
 // When several of the T tokens fall on one ring slot only the latest is written, so the
@@ -44,6 +44,9 @@ __device__ __forceinline__ void rotate8(const uint4& x1, const uint4& x2, const 
 }
 
 __global__ void __launch_bounds__(kAppendThreads) append_rope_kernel(const AppendArgs a) {
+  // the decode that usually follows may start its prologue now (it waits for this grid
+  // to complete before reading anything)
+  pdl_trigger();
   __shared__ float s_cos[kHalf];
   __shared__ float s_sin[kHalf];
   const int64_t tok = blockIdx.x;
@@ -63,12 +66,18 @@ __global__ void __launch_bounds__(kAppendThreads) append_rope_kernel(const Appen
     return;
   }
   if (threadIdx.x < kHalf) {
-    const int i = threadIdx.x;
-    const double inv_f = pow(a.theta, -2.0 * i / double(kHeadDim));
-    double sd, cd;
-    sincos(double(p) * inv_f, &sd, &cd);
-    s_cos[i] = static_cast<float>(cd);
-    s_sin[i] = static_cast<float>(sd);
+    // angle = p * inv_f[i] in float64, reduced to [-pi, pi] by subtracting k * 2*pi with
+    // 2*pi split in two parts (Cody-Waite): the first has 24 significant bits, so k * part1
+    // is exact for |k| < 2^29; the second carries the rest of 2*pi in double precision.
+    // The remainder is small, so the fp32 sincosf of it is accurate to ~1e-7.
+    const double ang = double(p) * a.inv_freq[threadIdx.x];
+    const double k = rint(ang * 0.15915494309189535);
+    double red = fma(-k, 6.2831854820251465, ang);
+    red = fma(-k, -1.748455600074497e-07, red);
+    float sf, cf;
+    sincosf(static_cast<float>(red), &sf, &cf);
+    s_cos[threadIdx.x] = cf;
+    s_sin[threadIdx.x] = sf;
   }
   __syncthreads();
 

@@ -7,20 +7,24 @@
 // those rows are read ("§Kernel 实现": evicted keys are never loaded), so the bytes read per
 // step stop growing once the window is full (eq. L_total).
 //
-// Design:
-//  * One CTA per (sequence, KV head, split).  The visible keys are cut into 64-row TMA
-//    tiles (see make_tiling); a split owns a contiguous run of tiles.
-//  * Warp 4 is the producer: one lane issues four 3-D TMA loads per tile (K and V, two
-//    64-column halves each, 128-byte swizzle) into a STAGES-deep mbarrier ring.
-//  * Warps 0-3 consume 16 keys each per tile with warp-level bf16 tensor-core MMAs in fp32:
+// Work units are (sequence, KV head) pairs; a unit's visible keys are cut into 64-row TMA
+// tiles (make_tiling).  Two schedules:
+//  * per-unit: when there are at least as many units as CTA slots (148 SMs x 2), one CTA
+//    per unit, written straight to `out`;
+//  * stream-K: otherwise exactly one wave of CTAs (2 per SM) takes equal contiguous shares
+//    of the global tile sequence (all units' tiles back to back), so every SM streams the
+//    same number of bytes whatever the positions are.  A CTA whose share crosses a unit
+//    boundary flushes a partial (o, lse) per unit piece; merge_kernel combines the pieces.
+// Inside a CTA:
+//  * warp 4 is the producer: one lane issues four 3-D TMA loads per tile (K and V, two
+//    64-column halves each, 128-byte swizzle) into a 3-stage mbarrier ring;
+//  * warps 0-3 consume 16 keys each per tile with warp-level bf16 tensor-core MMAs in fp32:
 //      S^T[16 keys x 8 heads] = K[16 x 128] . Q^T       (GQA: the 8 query heads of the
 //                                                          KV head share every K/V load)
 //      O^T[128 x 8 heads]    += V^T[128 x 16] . P^T
-//    P^T is moved from the accumulator layout to the operand layout with movmatrix.
-//    Softmax runs online in base 2 with warp-shuffle max reductions.
-//  * The four warps' (m, l, O) states are merged in shared memory; with one split the CTA
-//    writes bf16 out (and lse) directly, otherwise normalised fp32 partials plus their
-//    base-2 lse go to the workspace and merge_kernel combines them.
+//    P^T goes from the accumulator layout to the operand layout with movmatrix; softmax is
+//    online, in base 2, with warp-shuffle max reductions;
+//  * the four warps' (m, l, O) states are merged through shared memory.
 #include <cuda_bf16.h>
 #include <math.h>
 
@@ -35,29 +39,38 @@ namespace ps {
 namespace {
 
 constexpr int kConsumerWarps = 4;
+constexpr int kConsumerThreads = kConsumerWarps * 32;
 constexpr int kThreads = (kConsumerWarps + 1) * 32;
 constexpr int kBoxBytes = kDecodeTile * 128;  // 64 rows x 64 bf16
 constexpr int kTileBytes = 2 * kBoxBytes;     // one K (or V) tile: two column halves
 constexpr int kStageBytes = 2 * kTileBytes;   // K + V
 constexpr int kStages = 3;
-constexpr int kMaxSplits = 64;
-constexpr int kMinTilesPerSplit = 4;
+constexpr int kCtasPerSm = 2;
+constexpr int kMaxStreamKSeqs = 1024;  // stream-K runs only when units < CTA slots
+constexpr int kMinTilesPerCta = 4;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
-constexpr size_t smem_bytes(int stages) { return 1024 + size_t(stages) * kStageBytes + 256; }
+// shared memory: stages | barriers (2 x STAGES) | flush area [2][32 lanes][36] | prefix
+constexpr size_t kFlushFloats = 2 * 32 * 36;
+constexpr size_t smem_bytes(int stages) {
+  return 1024 + size_t(stages) * kStageBytes + 64 + kFlushFloats * 4 +
+         (kMaxStreamKSeqs + 1) * 4;
+}
 
 struct DecodeArgs {
   const __nv_bfloat16* q;
   const int64_t* pos;
   __nv_bfloat16* out;
   float* lse;
-  float* ws_o;    // [units, splits, 8, D] normalised partial outputs
-  float* ws_lse;  // [units, splits, 8] base-2 lse of each partial
+  float* ws_o;      // stream-K: [slots, 8, D] normalised partial outputs
+  float* ws_lse;    // stream-K: [slots, 8] base-2 lse of each partial
+  int32_t* ws_pref; // stream-K: [batch + 1] tiles-per-sequence prefix
+  int32_t* ws_span; // stream-K: [units][2] first and last CTA holding a piece of the unit
   int32_t* status;
-  int32_t hq, hkv, group;
+  int32_t batch, hq, hkv, group;
   int32_t lp, w, dim0;
-  int32_t splits, full_mode;
+  int32_t streamk, full_mode;
   int64_t lmax;
   float scale_log2;
 };
@@ -66,6 +79,106 @@ struct DecodeArgs {
 // TMA applies (chunk index XOR row mod 8; boxes start 1024-byte aligned).
 __device__ __forceinline__ uint32_t swz(int row, int chunk) {
   return uint32_t(row) * 128u + (uint32_t(chunk ^ (row & 7)) << 4);
+}
+
+__device__ __forceinline__ bool bad_position(const DecodeArgs& a, int64_t p) {
+  return (p < 0) || (a.full_mode && p >= a.lmax);
+}
+
+__device__ __forceinline__ DecodeTiling tiling_of(const DecodeArgs& a, int64_t p) {
+  VisibleRanges r{0, 0, 0, 0};
+  if (!bad_position(a, p)) {
+    if (a.full_mode)
+      r.pre_len = static_cast<int32_t>(p + 1);
+    else
+      r = visible_ranges(p, a.lp, a.w);
+  }
+  return make_tiling(r, a.dim0, a.w);
+}
+
+// Walks a contiguous range of the global tile sequence: unit u = b * hkv + h owns tiles
+// [hkv * pref[b] + h * cnt_b, ... + cnt_b), cnt_b = pref[b+1] - pref[b].
+struct TileWalker {
+  int64_t t, t_end;      // global tile cursor and end
+  int64_t pu, pu1;       // tile range of the current unit
+  int32_t b, h;          // current unit
+  DecodeTiling tiling;   // tiling of sequence b
+
+  __device__ void enter_unit(const DecodeArgs& a, const int32_t* pref) {
+    const int64_t cnt = pref[b + 1] - pref[b];
+    pu = (int64_t)a.hkv * pref[b] + h * cnt;
+    pu1 = pu + cnt;
+    tiling = tiling_of(a, a.pos[b]);
+  }
+  // position the walker on global tile t0 (t0 < total)
+  __device__ void seek(const DecodeArgs& a, const int32_t* pref, int64_t t0) {
+    int lo = 0, hi = a.batch - 1;  // largest b with hkv * pref[b] <= t0
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if ((int64_t)a.hkv * pref[mid] <= t0) lo = mid; else hi = mid - 1;
+    }
+    b = lo;
+    const int64_t cnt = pref[b + 1] - pref[b];
+    h = static_cast<int32_t>((t0 - (int64_t)a.hkv * pref[b]) / cnt);
+    t = t0;
+    enter_unit(a, pref);
+  }
+  // move to the next unit that owns tiles, without its tiling (for a look-ahead)
+  __device__ void next_unit_light(const DecodeArgs& a, const int32_t* pref) {
+    do {
+      if (++h == a.hkv) {
+        h = 0;
+        ++b;
+      }
+    } while (pref[b + 1] == pref[b]);
+  }
+  // move to the next unit that owns tiles
+  __device__ void next_unit(const DecodeArgs& a, const int32_t* pref) {
+    do {
+      if (++h == a.hkv) {
+        h = 0;
+        ++b;
+      }
+    } while (pref[b + 1] == pref[b]);
+    enter_unit(a, pref);
+  }
+};
+
+// Merges another (m, l, O) state into the registers of this lane (same fragment layout).
+__device__ __forceinline__ void merge_state(float& m0, float& m1, float& l0, float& l1,
+                                            float (&o)[8][4], const float* other) {
+  const float om0 = other[32], om1 = other[33], ol0 = other[34], ol1 = other[35];
+  const float M0 = fmaxf(m0, om0), M1 = fmaxf(m1, om1);
+  const float fa0 = (m0 == -INFINITY) ? 0.f : fast_exp2(m0 - M0);
+  const float fb0 = (om0 == -INFINITY) ? 0.f : fast_exp2(om0 - M0);
+  const float fa1 = (m1 == -INFINITY) ? 0.f : fast_exp2(m1 - M1);
+  const float fb1 = (om1 == -INFINITY) ? 0.f : fast_exp2(om1 - M1);
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    o[j][0] = fa0 * o[j][0] + fb0 * other[4 * j + 0];
+    o[j][1] = fa1 * o[j][1] + fb1 * other[4 * j + 1];
+    o[j][2] = fa0 * o[j][2] + fb0 * other[4 * j + 2];
+    o[j][3] = fa1 * o[j][3] + fb1 * other[4 * j + 3];
+  }
+  l0 = fa0 * l0 + fb0 * ol0;
+  l1 = fa1 * l1 + fb1 * ol1;
+  m0 = M0;
+  m1 = M1;
+}
+
+__device__ __forceinline__ void store_state(float* dst, float m0, float m1, float l0, float l1,
+                                            const float (&o)[8][4]) {
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    dst[4 * j + 0] = o[j][0];
+    dst[4 * j + 1] = o[j][1];
+    dst[4 * j + 2] = o[j][2];
+    dst[4 * j + 3] = o[j][3];
+  }
+  dst[32] = m0;
+  dst[33] = m1;
+  dst[34] = l0;
+  dst[35] = l1;
 }
 
 template <int STAGES>
@@ -78,31 +191,10 @@ __global__ void __launch_bounds__(kThreads)
                                              ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * kStageBytes);
   uint64_t* empty = full + STAGES;
-
-  const int split = blockIdx.x % a.splits;
-  const int unit = blockIdx.x / a.splits;  // b * hkv + h
-  const int b = unit / a.hkv;
-  const int h = unit % a.hkv;
+  float* flush = reinterpret_cast<float*>(smem + STAGES * kStageBytes + 64);  // [2][32][36]
+  int32_t* pref = reinterpret_cast<int32_t*>(flush + kFlushFloats);            // [batch + 1]
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-
-  const int64_t p = a.pos[b];
-  const bool bad = (p < 0) || (a.full_mode && p >= a.lmax);
-  if (bad && threadIdx.x == 0 && split == 0 && a.status)
-    atomicOr(a.status, p < 0 ? PS_DEV_BAD_POS : PS_DEV_POS_RANGE);
-
-  VisibleRanges r{0, 0, 0, 0};
-  if (!bad) {
-    if (a.full_mode) {
-      r.pre_len = static_cast<int32_t>(p + 1);
-    } else {
-      r = visible_ranges(p, a.lp, a.w);
-    }
-  }
-  const DecodeTiling t = make_tiling(r, a.dim0, a.w);
-  const int t_begin = static_cast<int>((int64_t)t.total * split / a.splits);
-  const int t_end = static_cast<int>((int64_t)t.total * (split + 1) / a.splits);
-  const int ntiles = t_end - t_begin;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -111,29 +203,93 @@ __global__ void __launch_bounds__(kThreads)
     }
     fence_mbar_init();
   }
-  __syncthreads();
+  if (warp == kConsumerWarps && lane == 0) {
+    prefetch_tensormap(&mk0);
+    prefetch_tensormap(&mv0);
+    prefetch_tensormap(&mk1);
+    prefetch_tensormap(&mv1);
+  }
+  // launched with programmatic serialization: everything above overlapped the previous
+  // kernel (usually the append); positions, q and the cache are read only after this
+  pdl_wait();
+  pdl_trigger();  // the merge may be scheduled now; it waits for this grid to finish
 
-  float o[8][4];
-  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+  // ---------------------------------------------------------------- work range
+  TileWalker wk;
+  if (a.streamk) {
+    // tiles per sequence, then an inclusive scan (batch <= kMaxStreamKSeqs)
+    for (int b = threadIdx.x; b < a.batch; b += kThreads) {
+      const int64_t p = a.pos[b];
+      const int32_t cnt = tiling_of(a, p).total;
+      pref[b + 1] = cnt;
+      if (blockIdx.x == 0 && cnt == 0) {
+        if (bad_position(a, p) && a.status)
+          atomicOr(a.status, p < 0 ? PS_DEV_BAD_POS : PS_DEV_POS_RANGE);
+        for (int h = 0; h < a.hkv; ++h) {  // an empty span: no pieces to merge
+          a.ws_span[2 * (b * a.hkv + h)] = 1;
+          a.ws_span[2 * (b * a.hkv + h) + 1] = 0;
+        }
+      }
+    }
+    if (threadIdx.x == 0) pref[0] = 0;
+    __syncthreads();
+    if (warp == 0) {
+      int32_t carry = 0;
+      for (int base = 1; base <= a.batch; base += 32) {
+        const int i = base + lane;
+        int32_t v = i <= a.batch ? pref[i] : 0;
 #pragma unroll
-  for (int i = 0; i < 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+        for (int off = 1; off < 32; off <<= 1) {
+          const int32_t u = __shfl_up_sync(0xffffffffu, v, off);
+          if (lane >= off) v += u;
+        }
+        if (i <= a.batch) pref[i] = v + carry;
+        carry += __shfl_sync(0xffffffffu, v, 31);
+      }
+    }
+    __syncthreads();
+    if (blockIdx.x == 0)
+      for (int i = threadIdx.x; i <= a.batch; i += kThreads) a.ws_pref[i] = pref[i];
+    const int64_t total = (int64_t)a.hkv * pref[a.batch];
+    const int64_t t0 = total * blockIdx.x / gridDim.x;
+    const int64_t t1 = total * (blockIdx.x + 1) / gridDim.x;
+    wk.t_end = t1;
+    if (t0 < t1) {
+      wk.seek(a, pref, t0);
+    } else {
+      wk.t = t0;
+    }
+  } else {
+    __syncthreads();
+    const int unit = blockIdx.x;
+    wk.b = unit / a.hkv;
+    wk.h = unit % a.hkv;
+    const int64_t p = a.pos[wk.b];
+    if (bad_position(a, p) && threadIdx.x == 0 && wk.h == 0 && a.status)
+      atomicOr(a.status, p < 0 ? PS_DEV_BAD_POS : PS_DEV_POS_RANGE);
+    wk.tiling = tiling_of(a, p);
+    wk.t = 0;
+    wk.t_end = wk.tiling.total;
+    wk.pu = 0;
+    wk.pu1 = wk.t_end;
+  }
+  const int ntiles = static_cast<int>(wk.t_end - wk.t);
 
   if (warp == kConsumerWarps) {
     // ------------------------------------------------------------ producer
     if (lane == 0 && ntiles > 0) {
-      prefetch_tensormap(&mk0);
-      prefetch_tensormap(&mv0);
-      prefetch_tensormap(&mk1);
-      prefetch_tensormap(&mv1);
       const uint64_t pol = l2_policy_evict_first();
       int issued = 0;
-      for (int i = 0; i < ntiles; ++i) {
+      TileWalker pw = wk;
+      for (int i = 0; i < ntiles; ++i, ++pw.t) {
+        if (pw.t >= pw.pu1) pw.next_unit(a, pref);
         const int s = i % STAGES;
         const uint32_t ph = (i / STAGES) & 1;
         if (i >= STAGES && !mbar_wait(&empty[s], ph ^ 1, a.status)) break;
-        const DecodeTile d = tiling_tile(t, t_begin + i);
+        const DecodeTile d = tiling_tile(pw.tiling, static_cast<int32_t>(pw.t - pw.pu));
         const CUtensorMap* mk = d.map_id ? &mk1 : &mk0;
         const CUtensorMap* mv = d.map_id ? &mv1 : &mv0;
+        const int unit = pw.b * a.hkv + pw.h;
         uint8_t* st = smem + s * kStageBytes;
         mbar_arrive_expect_tx(&full[s], kStageBytes);
         tma_load_3d_hint(st, mk, 0, d.row0, unit, &full[s], pol);
@@ -150,31 +306,144 @@ __global__ void __launch_bounds__(kThreads)
     // ------------------------------------------------------------ consumers
     const int qh = lane >> 2;  // query head within the group (MMA column)
     const int qq = lane & 3;
-    uint32_t qf[8][2];
-    if (qh < a.group) {
-      const __nv_bfloat16* qrow = a.q + ((int64_t)b * a.hq + h * a.group + qh) * kHeadDim;
-#pragma unroll
-      for (int ks = 0; ks < 8; ++ks) {
-        qf[ks][0] = *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 2 * qq);
-        qf[ks][1] = *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 8 + 2 * qq);
-      }
-    } else {
-#pragma unroll
-      for (int ks = 0; ks < 8; ++ks) qf[ks][0] = qf[ks][1] = 0u;
-    }
     const float sl2 = a.scale_log2;
-    const int arow = 16 * warp + (lane & 15);        // ldmatrix row for K
-    const int achunk = lane >> 4;                    // 0/1: k 0-7 or 8-15
+    const int arow = 16 * warp + (lane & 15);  // ldmatrix row for K
+    const int achunk = lane >> 4;              // 0/1: k 0-7 or 8-15
     const int vkey = 16 * warp + (lane & 7) + ((lane >> 4) << 3);
     const int vdoff = ((lane >> 3) & 1) << 3;
     const int r0 = 16 * warp + (lane >> 2);
     const int r1 = r0 + 8;
 
-    for (int i = 0; i < ntiles; ++i) {
+    float o[8][4];
+    float m0, m1, l0, l1;
+    uint32_t qf[8][2];
+    auto reset = [&]() {
+      m0 = m1 = -INFINITY;
+      l0 = l1 = 0.f;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+    };
+    auto load_q = [&](int b, int h) {
+      if (qh < a.group) {
+        const __nv_bfloat16* qrow = a.q + ((int64_t)b * a.hq + h * a.group + qh) * kHeadDim;
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+          qf[ks][0] = *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 2 * qq);
+          qf[ks][1] = *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 8 + 2 * qq);
+        }
+      } else {
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) qf[ks][0] = qf[ks][1] = 0u;
+      }
+    };
+    // Folds the four warps' states of the current unit into warp 0 (two rounds through
+    // shared memory) and writes the result: to `out` for a whole unit, to the workspace
+    // for a stream-K piece.
+    auto flush_unit = [&](int b, int h) {
+#pragma unroll
+      for (int off = 4; off < 32; off <<= 1) {
+        l0 += __shfl_xor_sync(0xffffffffu, l0, off);
+        l1 += __shfl_xor_sync(0xffffffffu, l1, off);
+      }
+      if (warp >= 2) store_state(flush + ((warp - 2) * 32 + lane) * 36, m0, m1, l0, l1, o);
+      named_bar_sync(1, kConsumerThreads);
+      if (warp < 2) merge_state(m0, m1, l0, l1, o, flush + (warp * 32 + lane) * 36);
+      named_bar_sync(1, kConsumerThreads);
+      if (warp == 1) store_state(flush + lane * 36, m0, m1, l0, l1, o);
+      named_bar_sync(1, kConsumerThreads);
+      if (warp == 0) {
+        merge_state(m0, m1, l0, l1, o, flush + lane * 36);
+        const int unit = b * a.hkv + h;
+        const int64_t slot = (int64_t)unit + blockIdx.x;  // unique per (unit, CTA) piece
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int hh = 2 * qq + e;
+          const float m = e ? m1 : m0;
+          const float l = e ? l1 : l0;
+          const float inv = l > 0.f ? 1.f / l : 0.f;
+          const float lse2 = l > 0.f ? m + log2f(l) : -INFINITY;
+          if (hh < a.group) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const int d0 = 16 * j + (lane >> 2);
+              const float v0 = o[j][e] * inv, v1 = o[j][2 + e] * inv;
+              if (a.streamk) {
+                float* dst = a.ws_o + (slot * 8 + hh) * kHeadDim;
+                dst[d0] = v0;
+                dst[d0 + 8] = v1;
+              } else {
+                __nv_bfloat16* dst = a.out + ((int64_t)b * a.hq + h * a.group + hh) * kHeadDim;
+                dst[d0] = __float2bfloat16_rn(v0);
+                dst[d0 + 8] = __float2bfloat16_rn(v1);
+              }
+            }
+            if (lane < 4) {
+              if (a.streamk)
+                a.ws_lse[slot * 8 + hh] = lse2;
+              else if (a.lse)
+                a.lse[(int64_t)b * a.hq + h * a.group + hh] = lse2 * kLn2;
+            }
+          }
+        }
+      }
+      named_bar_sync(1, kConsumerThreads);  // the flush area is free again
+    };
+
+    // A unit's first tile is owned by exactly one CTA and so is its last: those CTAs
+    // record themselves, so the merge finds the pieces without any division.
+    auto note_span = [&](const TileWalker& w, int64_t t_first, int64_t t_last) {
+      if (a.streamk && threadIdx.x == 0) {
+        const int unit = w.b * a.hkv + w.h;
+        if (t_first == w.pu) a.ws_span[2 * unit] = blockIdx.x;
+        if (t_last == w.pu1 - 1) a.ws_span[2 * unit + 1] = blockIdx.x;
+      }
+    };
+    reset();
+    TileWalker cw = wk;
+    uint32_t qn[8][2];  // q of the next unit, prefetched
+    auto prefetch_next_q = [&](const TileWalker& w) {
+      if (w.pu1 < w.t_end) {
+        TileWalker nx = w;
+        nx.next_unit_light(a, pref);
+        if (qh < a.group) {
+          const __nv_bfloat16* qrow =
+              a.q + ((int64_t)nx.b * a.hq + nx.h * a.group + qh) * kHeadDim;
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks) {
+            qn[ks][0] = *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 2 * qq);
+            qn[ks][1] = *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 8 + 2 * qq);
+          }
+        } else {
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks) qn[ks][0] = qn[ks][1] = 0u;
+        }
+      }
+    };
+    if (ntiles > 0) {
+      load_q(cw.b, cw.h);
+      note_span(cw, cw.t, (cw.pu1 < wk.t_end ? cw.pu1 : wk.t_end) - 1);
+      prefetch_next_q(cw);
+    }
+    bool alive = true;
+    for (int i = 0; i < ntiles; ++i, ++cw.t) {
+      if (cw.t >= cw.pu1) {
+        flush_unit(cw.b, cw.h);
+        cw.next_unit(a, pref);
+        reset();
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+          qf[ks][0] = qn[ks][0];
+          qf[ks][1] = qn[ks][1];
+        }
+        note_span(cw, cw.t, (cw.pu1 < wk.t_end ? cw.pu1 : wk.t_end) - 1);
+        prefetch_next_q(cw);
+      }
       const int s = i % STAGES;
       // warp-uniform outcome: ldmatrix / mma.sync below are warp-collective
-      if (!__all_sync(0xffffffffu, mbar_wait(&full[s], (i / STAGES) & 1, a.status))) break;
-      const DecodeTile d = tiling_tile(t, t_begin + i);
+      if (alive && !__all_sync(0xffffffffu, mbar_wait(&full[s], (i / STAGES) & 1, a.status)))
+        alive = false;
+      if (!alive) continue;  // keep the flush barriers in step with the other warps
+      const DecodeTile d = tiling_tile(cw.tiling, static_cast<int32_t>(cw.t - cw.pu));
       const uint32_t kbase = smem_u32(smem + s * kStageBytes);
       const uint32_t vbase = kbase + kTileBytes;
 
@@ -229,94 +498,71 @@ __global__ void __launch_bounds__(kThreads)
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[s]);
     }
-#pragma unroll
-    for (int off = 4; off < 32; off <<= 1) {
-      l0 += __shfl_xor_sync(0xffffffffu, l0, off);
-      l1 += __shfl_xor_sync(0xffffffffu, l1, off);
-    }
-  }
-  __syncthreads();  // every tile consumed and every copy landed: stages are free
-
-  // ---------------------------------------------- merge the four warps' states
-  float* red_m = reinterpret_cast<float*>(smem);         // [4][8]
-  float* red_l = red_m + kConsumerWarps * 8;             // [4][8]
-  float* red_o = red_l + kConsumerWarps * 8;             // [4][8][D]
-  if (warp < kConsumerWarps) {
-    const int qq = lane & 3;
-    if (lane < 4) {
-      red_m[warp * 8 + 2 * qq] = m0;
-      red_m[warp * 8 + 2 * qq + 1] = m1;
-      red_l[warp * 8 + 2 * qq] = l0;
-      red_l[warp * 8 + 2 * qq + 1] = l1;
-    }
-    float* ow = red_o + warp * 8 * kHeadDim;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int dlo = 16 * j + (lane >> 2);
-      ow[(2 * qq) * kHeadDim + dlo] = o[j][0];
-      ow[(2 * qq + 1) * kHeadDim + dlo] = o[j][1];
-      ow[(2 * qq) * kHeadDim + dlo + 8] = o[j][2];
-      ow[(2 * qq + 1) * kHeadDim + dlo + 8] = o[j][3];
+    if (ntiles > 0) {
+      flush_unit(cw.b, cw.h);
+    } else if (!a.streamk) {
+      // a unit without visible keys (skipped position): zeros and lse = -inf
+      flush_unit(wk.b, wk.h);
     }
   }
   __syncthreads();
-  if (threadIdx.x < kHeadDim) {
-    const int dcol = threadIdx.x;
-    for (int hh = 0; hh < a.group; ++hh) {
-      float M = -INFINITY;
-#pragma unroll
-      for (int wv = 0; wv < kConsumerWarps; ++wv) M = fmaxf(M, red_m[wv * 8 + hh]);
-      float oval = 0.f, lse2 = -INFINITY;
-      if (M != -INFINITY) {
-        float wsum = 0.f, osum = 0.f;
-#pragma unroll
-        for (int wv = 0; wv < kConsumerWarps; ++wv) {
-          const float f = fast_exp2(red_m[wv * 8 + hh] - M);
-          wsum += f * red_l[wv * 8 + hh];
-          osum += f * red_o[(wv * 8 + hh) * kHeadDim + dcol];
-        }
-        oval = osum / wsum;
-        lse2 = M + log2f(wsum);
-      }
-      const int head = h * a.group + hh;
-      if (a.splits == 1) {
-        a.out[((int64_t)b * a.hq + head) * kHeadDim + dcol] = __float2bfloat16_rn(oval);
-        if (a.lse && dcol == 0) a.lse[(int64_t)b * a.hq + head] = lse2 * kLn2;
-      } else {
-        const int64_t slot = ((int64_t)unit * a.splits + split) * 8 + hh;
-        a.ws_o[slot * kHeadDim + dcol] = oval;
-        if (dcol == 0) a.ws_lse[slot] = lse2;
-      }
-    }
-  }
 }
 
-// Combines the splits of one (sequence, query head): weights 2^(lse_s - max).
+// Combines the stream-K pieces of one (sequence, query head): weights 2^(lse_s - max).
+// Pieces of unit u are the CTAs c in [first, last] recorded by the decode kernel, stored at
+// slot u + c.  One warp per (sequence, query head); lane i owns d = 4i .. 4i+3.
 __global__ void __launch_bounds__(128)
     merge_kernel(const float* __restrict__ ws_o, const float* __restrict__ ws_lse,
-                 __nv_bfloat16* __restrict__ out, float* __restrict__ lse, int32_t hq,
-                 int32_t hkv, int32_t group, int32_t splits) {
-  const int bh = blockIdx.x;
-  const int b = bh / hq, head = bh % hq;
+                 const int32_t* __restrict__ pref, const int32_t* __restrict__ span,
+                 __nv_bfloat16* __restrict__ out, float* __restrict__ lse, int32_t batch,
+                 int32_t hq, int32_t hkv, int32_t group, int32_t grid) {
+  const int64_t bh = (int64_t)blockIdx.x * 4 + (threadIdx.x >> 5);
+  if (bh >= (int64_t)batch * hq) return;
+  const int lane = threadIdx.x & 31;
+  const int b = static_cast<int>(bh / hq), head = static_cast<int>(bh % hq);
   const int h = head / group, hh = head % group;
   const int64_t unit = (int64_t)b * hkv + h;
-  const int dcol = threadIdx.x;
-  float M = -INFINITY;
-  for (int s = 0; s < splits; ++s) M = fmaxf(M, ws_lse[(unit * splits + s) * 8 + hh]);
-  float oval = 0.f, lse2 = -INFINITY;
-  if (M != -INFINITY) {
-    float wsum = 0.f, osum = 0.f;
-    for (int s = 0; s < splits; ++s) {
-      const int64_t slot = (unit * splits + s) * 8 + hh;
-      const float f = fast_exp2(ws_lse[slot] - M);
-      wsum += f;
-      osum += f * ws_o[slot * kHeadDim + dcol];
+  pdl_wait();  // the decode kernel's pieces and spans must be complete
+  const int2 sp = reinterpret_cast<const int2*>(span)[unit];
+  const int64_t total = (int64_t)hkv * pref[batch];
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  float lse2 = -INFINITY;
+  if (sp.x <= sp.y) {
+    const int c_lo = sp.x, c_hi = sp.y;
+    // with fewer tiles than CTAs some CTAs own nothing and wrote no piece
+    const bool maybe_empty = total < grid;
+    auto empty_cta = [&](int c) {
+      return maybe_empty && total * c / grid == total * (c + 1) / grid;
+    };
+    float M = -INFINITY;
+    for (int c = c_lo; c <= c_hi; ++c)
+      if (!empty_cta(c)) M = fmaxf(M, ws_lse[(unit + c) * 8 + hh]);
+    if (M != -INFINITY) {
+      float wsum = 0.f;
+      for (int c = c_lo; c <= c_hi; ++c) {
+        if (empty_cta(c)) continue;
+        const int64_t slot = (unit + c) * 8 + hh;
+        const float f = fast_exp2(ws_lse[slot] - M);
+        const float4 v = reinterpret_cast<const float4*>(ws_o + slot * kHeadDim)[lane];
+        wsum += f;
+        acc.x += f * v.x;
+        acc.y += f * v.y;
+        acc.z += f * v.z;
+        acc.w += f * v.w;
+      }
+      const float inv = 1.f / wsum;
+      acc.x *= inv;
+      acc.y *= inv;
+      acc.z *= inv;
+      acc.w *= inv;
+      lse2 = M + log2f(wsum);
     }
-    oval = osum / wsum;
-    lse2 = M + log2f(wsum);
   }
-  out[(int64_t)bh * kHeadDim + dcol] = __float2bfloat16_rn(oval);
-  if (lse && dcol == 0) lse[bh] = lse2 * kLn2;
+  uint2 pk;
+  pk.x = pack_bf16x2(acc.x, acc.y);
+  pk.y = pack_bf16x2(acc.z, acc.w);
+  reinterpret_cast<uint2*>(out + bh * kHeadDim)[lane] = pk;
+  if (lse && lane == 0) lse[bh] = lse2 * kLn2;
 }
 
 __global__ void visible_ranges_kernel(const int64_t* __restrict__ pos, int64_t batch, int32_t lp,
@@ -345,37 +591,44 @@ int occupancy_per_sm() {
             cudaSuccess ||
         occ < 1)
       occ = 1;
-    cached[dev] = occ;
+    cached[dev] = occ < kCtasPerSm ? occ : kCtasPerSm;
   }
   return cached[dev];
+}
+
+// Stream-K grid size for this shape, or 0 for the per-unit schedule.
+int64_t streamk_grid(int64_t batch, int32_t hkv, int64_t max_keys) {
+  const int64_t units = batch * hkv;
+  const int64_t slots = (int64_t)sm_count() * occupancy_per_sm();
+  if (units >= slots || batch > kMaxStreamKSeqs) return 0;
+  const int64_t max_tiles = units * ((max_keys + kDecodeTile - 1) / kDecodeTile + 2);
+  int64_t g = max_tiles / kMinTilesPerCta;
+  if (g > slots) g = slots;
+  if (g < 1) g = 1;
+  return g;
 }
 
 }  // namespace
 
 int decode_splits(int64_t batch, int32_t hkv, int64_t max_keys) {
-  const int64_t units = batch * hkv;
-  const int64_t slots = (int64_t)sm_count() * occupancy_per_sm();
-  // enough CTAs to keep every SM streaming, never fewer than kMinTilesPerSplit tiles each
-  const int64_t max_tiles = (max_keys + kDecodeTile - 1) / kDecodeTile + 2;
-  int64_t s = units >= slots ? 1 : slots / units;
-  const int64_t cap = max_tiles / kMinTilesPerSplit;
-  if (s > cap) s = cap;
-  if (s > kMaxSplits) s = kMaxSplits;
-  if (s < 1) s = 1;
-  return static_cast<int>(s);
+  const int64_t g = streamk_grid(batch, hkv, max_keys);
+  return g > 0 ? static_cast<int>(g) : 1;
 }
 
 size_t decode_workspace_bytes(int64_t batch, int32_t hkv, int64_t max_keys) {
-  const int s = decode_splits(batch, hkv, max_keys);
-  if (s <= 1) return 0;
-  const size_t slots = size_t(batch) * hkv * s * 8;
-  return slots * (kHeadDim + 1) * sizeof(float);
+  const int64_t g = streamk_grid(batch, hkv, max_keys);
+  if (g == 0) return 0;
+  const size_t slots = size_t(batch * hkv + g) * 8;
+  const size_t o_bytes = slots * kHeadDim * sizeof(float);
+  const size_t lse_bytes = (slots * sizeof(float) + 255) & ~size_t(255);
+  const size_t pref_bytes = (size_t(batch + 1) * sizeof(int32_t) + 255) & ~size_t(255);
+  return o_bytes + lse_bytes + pref_bytes + size_t(batch * hkv) * 2 * sizeof(int32_t);
 }
 
 int launch_decode(const DecodeLaunch& l, cudaStream_t stream) {
   const int group = l.hq / l.hkv;
   const int64_t max_keys = l.full_mode ? l.lmax : (int64_t)l.lp + l.w;
-  const int splits = decode_splits(l.batch, l.hkv, max_keys);
+  const int64_t g = streamk_grid(l.batch, l.hkv, max_keys);
   const int64_t units = l.batch * l.hkv;
   const int32_t dim0 = l.full_mode ? static_cast<int32_t>(l.lmax) : l.lp;
 
@@ -406,34 +659,46 @@ int launch_decode(const DecodeLaunch& l, cudaStream_t stream) {
   a.pos = l.pos;
   a.out = static_cast<__nv_bfloat16*>(l.out);
   a.lse = l.lse;
-  const size_t nslots = size_t(units) * splits * 8;
-  a.ws_o = static_cast<float*>(l.workspace);
-  a.ws_lse = a.ws_o ? a.ws_o + nslots * kHeadDim : nullptr;
+  const size_t nslots = size_t(units + g) * 8;
+  a.ws_o = g ? static_cast<float*>(l.workspace) : nullptr;
+  a.ws_lse = g ? a.ws_o + nslots * kHeadDim : nullptr;
+  a.ws_pref = g ? reinterpret_cast<int32_t*>(
+                      reinterpret_cast<char*>(a.ws_lse) +
+                      ((nslots * sizeof(float) + 255) & ~size_t(255)))
+                : nullptr;
+  a.ws_span = g ? a.ws_pref + (((size_t(l.batch + 1) * sizeof(int32_t) + 255) & ~size_t(255)) /
+                                sizeof(int32_t))
+                : nullptr;
   a.status = l.status;
+  a.batch = static_cast<int32_t>(l.batch);
   a.hq = l.hq;
   a.hkv = l.hkv;
   a.group = group;
   a.lp = l.full_mode ? static_cast<int32_t>(l.lmax) : l.lp;
   a.w = l.full_mode ? 1 : l.w;
   a.dim0 = dim0;
-  a.splits = splits;
+  a.streamk = g > 0 ? 1 : 0;
   a.full_mode = l.full_mode;
   a.lmax = l.lmax;
   a.scale_log2 = l.scale * kLog2e;
 
   const size_t sb = smem_bytes(kStages);
   occupancy_per_sm();  // sets the shared-memory attribute once per device
-  const int64_t grid = units * splits;
+  const int64_t grid = g > 0 ? g : units;
   if (grid <= 0) return PS_OK;
-  if (grid > 0x7fffffff) return fail(PS_ERR_UNSUPPORTED, "decode grid too large");
-  decode_kernel<kStages><<<static_cast<unsigned>(grid), kThreads, sb, stream>>>(mk0, mv0, mk1, mv1,
-                                                                             a);
-  int rc = check_cuda(cudaGetLastError(), "decode_kernel launch");
+  if (grid > 0x7fffffff || l.batch > 0x7fffffff)
+    return fail(PS_ERR_UNSUPPORTED, "decode grid too large");
+  int rc = check_cuda(launch_pdl(decode_kernel<kStages>, dim3(static_cast<unsigned>(grid)),
+                                 dim3(kThreads), sb, stream, mk0, mv0, mk1, mv1, a),
+                      "decode_kernel launch");
   if (rc != PS_OK) return rc;
-  if (splits > 1) {
-    merge_kernel<<<static_cast<unsigned>(l.batch * l.hq), kHeadDim, 0, stream>>>(
-        a.ws_o, a.ws_lse, a.out, a.lse, l.hq, l.hkv, group, splits);
-    rc = check_cuda(cudaGetLastError(), "merge_kernel launch");
+  if (g > 0) {
+    rc = check_cuda(
+        launch_pdl(merge_kernel, dim3(static_cast<unsigned>((l.batch * l.hq + 3) / 4)), dim3(128),
+                   0, stream, static_cast<const float*>(a.ws_o), static_cast<const float*>(a.ws_lse),
+                   static_cast<const int32_t*>(a.ws_pref), static_cast<const int32_t*>(a.ws_span),
+                   a.out, a.lse, a.batch, l.hq, l.hkv, group, static_cast<int32_t>(g)),
+        "merge_kernel launch");
   }
   return rc;
 }

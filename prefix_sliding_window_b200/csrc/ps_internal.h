@@ -6,6 +6,7 @@
 #include <stdint.h>
 
 #include <string>
+#include <utility>
 
 #include "../../include/ps.h"
 
@@ -28,6 +29,25 @@ bool make_map_3d(CUtensorMap* map, const void* base, uint64_t x, uint64_t y, uin
 bool make_map_4d(CUtensorMap* map, const void* base, const uint64_t dims[4],
                  const uint32_t box[4]);
 
+// Launches `kernel` with programmatic stream serialization: it may begin while the previous
+// kernel of the stream finishes, and must call pdl_wait() before touching data that kernel
+// (or anything before it) produced.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t stream, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 // Streaming multiprocessor count of the current device.
 int sm_count();
 
@@ -44,7 +64,7 @@ struct AppendArgs {
   int32_t* status;
   int64_t batch;
   int32_t T, hq, hkv, lp, w;
-  double theta;
+  double inv_freq[kHeadDim / 2];  // theta^(-2i/D), float64, filled by the host
 };
 cudaError_t launch_append(const AppendArgs& a, cudaStream_t stream);
 

@@ -9,23 +9,31 @@
 // unmasked; PARTIAL tiles (the diagonal, the window's lower edge, the prefix's end and the
 // ragged tail) get an element-wise mask.
 //
-// One CTA per (batch, query head, query tile), heaviest query tiles first, 6 warps:
-//   warp 4  - TMA producer: the Q tile once, then K and V tiles of the plan into a
-//             two-stage mbarrier ring (4-D tensor maps, 128-byte swizzle).
-//   warp 5  - allocates 512 TMEM columns; one lane issues the MMAs:
-//               S[buf] = Q K^T           (tcgen05.mma kind::f16, A and B from smem)
-//               O     += P V             (A = P from TMEM, B = V from smem, MN-major)
+// One CTA per (batch, query head, query tile), heaviest query tiles first, 11 warps:
+//   warps 8, 9 - TMA producers: warp 8 loads the Q tile once and the K tiles of the plan
+//             into a 3-stage ring, warp 9 the V tiles into a 2-stage ring (4-D tensor
+//             maps, 128-byte swizzle).  A K stage is released when its QK^T completes, a V
+//             stage when its PV completes.
+//   warp 10 - allocates 512 TMEM columns; one lane issues the MMAs:
+//               S[buf] = Q K^T             (tcgen05.mma kind::f16, A and B from smem)
+//               O_g   += P_g V_g, g = 0, 1 (A = P from TMEM, B = V from smem, MN-major;
+//                                           P_g, V_g: keys [64g, 64g+64) of the tile)
 //             and commits them to mbarriers.  S of tile j+1 is issued before PV of tile j,
 //             so the tensor pipe computes the next scores while softmax runs.
-//   warps 0-3 - softmax: thread r owns row r (TMEM lane r).  It reads its S row, masks it
-//             on PARTIAL tiles, keeps the running max m and sum l in fp32 (base 2), writes
-//             P as bf16 over the first 64 columns of the same S buffer, and signals the
-//             MMA warp.  O is rescaled in TMEM only when the max of some row of the warp
-//             grows by more than 8 (log2 units); otherwise P stays below 2^8 and the
-//             stale max keeps fp32 sums exact enough.  The decision is warp-uniform
-//             because tcgen05.ld/st are warp-collective.
-//   Epilogue: the softmax warps read O, divide by l, store bf16 out and the natural-log lse.
-// TMEM columns: S0 [0,128), S1 [128,256), O [256,384).
+//   warps 0-7 - softmax, two warpgroups: row r lives in TMEM lane r; group g handles the
+//             64 score columns [64g, 64g+64) of every row as an independent online softmax
+//             (its own max m_g, sum l_g and accumulator O_g), so the groups never wait for
+//             each other inside the loop.  Each thread masks its slice on PARTIAL tiles,
+//             writes P as bf16 over its columns of the same S buffer (packed fp32x2
+//             FMA/add, one ex2 per element) and signals the MMA warp.  O_g is rescaled in
+//             TMEM only when the max of some row of the warp grows by more than 8 (log2
+//             units); otherwise P stays below 2^8 and the stale max keeps fp32 sums exact
+//             enough.  The decision is warp-uniform because tcgen05.ld/st are
+//             warp-collective.
+//   Epilogue: O = (2^(m_0-M) O_0 + 2^(m_1-M) O_1) / (2^(m_0-M) l_0 + 2^(m_1-M) l_1),
+//             each group stores half of the columns as bf16; group 0 stores the lse.
+// TMEM columns: S0 [0,128), S1 [128,256), O_0 [256,384), O_1 [384,512).
+
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <math.h>
@@ -39,21 +47,26 @@ namespace {
 
 constexpr int kBq = kPrefillBq;
 constexpr int kBk = kPrefillBk;
-constexpr int kSoftmaxWarps = 4;
-constexpr int kProducerWarp = 4;
-constexpr int kMmaWarp = 5;
-constexpr int kThreads = 6 * 32;
-constexpr int kKVStages = 2;
+constexpr int kGroups = 2;                // softmax warpgroups, one column slice each
+constexpr int kCols = 128 / kGroups;       // score columns per group
+constexpr int kSoftmaxWarps = 4 * kGroups;
+constexpr int kSoftmaxThreads = kSoftmaxWarps * 32;
+constexpr int kKProducerWarp = kSoftmaxWarps;
+constexpr int kVProducerWarp = kSoftmaxWarps + 1;
+constexpr int kMmaWarp = kSoftmaxWarps + 2;
+constexpr int kThreads = (kSoftmaxWarps + 3) * 32;
+constexpr int kKStages = 3;
+constexpr int kVStages = 2;
 constexpr int kBoxBytes = 128 * 128;        // [128 rows][64 bf16]
 constexpr int kTileBytes = 2 * kBoxBytes;   // [128 rows][128 bf16]
 constexpr uint32_t kTmemCols = 512;
 __device__ __forceinline__ uint32_t col_s(int s) { return s ? 128u : 0u; }
-constexpr uint32_t kColO = 256;
+constexpr uint32_t kColO = 256;  // O_g at kColO + 128 g
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
-constexpr size_t kSmemBytes = 1024 + kTileBytes * (1 + 2 * kKVStages) + 256;
+constexpr size_t kSmemBytes = 1024 + kTileBytes * (1 + kKStages + kVStages) + 256 + 2 * kGroups * 128 * 4;
 
 struct PrefillArgs {
   const int32_t* off;  // [nq + 1] plan offsets
@@ -80,16 +93,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                                              ~uintptr_t(1023));
   uint8_t* sQ = smem;
   uint8_t* sK = sQ + kTileBytes;
-  uint8_t* sV = sK + kKVStages * kTileBytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + kKVStages * kTileBytes);
+  uint8_t* sV = sK + kKStages * kTileBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + kVStages * kTileBytes);
   uint64_t* q_full = bars + 0;
-  uint64_t* kv_full = bars + 1;   // [2]
-  uint64_t* kv_empty = bars + 3;  // [2]
-  uint64_t* s_full = bars + 5;    // [2]
-  uint64_t* p_ready = bars + 7;   // [2]
-  uint64_t* pv_done = bars + 9;
-  uint64_t* mma_done = bars + 10;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 11);
+  uint64_t* k_full = bars + 1;    // [kKStages]
+  uint64_t* k_empty = bars + 4;   // [kKStages]
+  uint64_t* v_full = bars + 7;    // [kVStages]
+  uint64_t* v_empty = bars + 9;   // [kVStages]
+  uint64_t* s_full = bars + 11;   // [2]
+  uint64_t* p_ready = bars + 13;  // [2 buffers][kGroups]
+  uint64_t* pv_done = bars + 13 + 2 * kGroups;
+  uint64_t* mma_done = pv_done + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
 
   const int64_t bh = (int64_t)a.batch * a.hq;
   const int qt = a.nq - 1 - static_cast<int>(blockIdx.x / bh);
@@ -104,11 +119,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
+    for (int s = 0; s < kKStages; ++s) {
+      mbar_init(&k_full[s], 1);
+      mbar_init(&k_empty[s], 1);
+    }
+    for (int s = 0; s < kVStages; ++s) {
+      mbar_init(&v_full[s], 1);
+      mbar_init(&v_empty[s], 1);
+    }
     for (int s = 0; s < 2; ++s) {
-      mbar_init(&kv_full[s], 1);
-      mbar_init(&kv_empty[s], 1);
       mbar_init(&s_full[s], 1);
-      mbar_init(&p_ready[s], kSoftmaxWarps);
+      for (int g = 0; g < kGroups; ++g) mbar_init(&p_ready[s * kGroups + g], 4);
     }
     mbar_init(pv_done, 1);
     mbar_init(mma_done, 1);
@@ -123,33 +144,40 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == kProducerWarp) {
-    // ------------------------------------------------------------ TMA producer
+  if (warp == kKProducerWarp || warp == kVProducerWarp) {
+    // ------------------------------------------------------------ TMA producers
+    // One warp streams Q and the K tiles, the other the V tiles; K and V have their own rings,
+    // so a K tile can be refilled as soon as its QK^T finished, independent of PV.
     if (lane == 0) {
-      prefetch_tensormap(&mq);
-      prefetch_tensormap(&mk);
-      prefetch_tensormap(&mv);
-      mbar_arrive_expect_tx(q_full, kTileBytes);
-      tma_load_4d(sQ, &mq, 0, head, qt * kBq, b, q_full);
-      tma_load_4d(sQ + kBoxBytes, &mq, 64, head, qt * kBq, b, q_full);
+      const bool is_k = (warp == kKProducerWarp);
+      const CUtensorMap* map = is_k ? &mk : &mv;
+      uint8_t* ring = is_k ? sK : sV;
+      uint64_t* full = is_k ? k_full : v_full;
+      uint64_t* empty = is_k ? k_empty : v_empty;
+      const int stages = is_k ? kKStages : kVStages;
+      prefetch_tensormap(map);
+      if (is_k) {
+        prefetch_tensormap(&mq);
+        mbar_arrive_expect_tx(q_full, kTileBytes);
+        tma_load_4d(sQ, &mq, 0, head, qt * kBq, b, q_full);
+        tma_load_4d(sQ + kBoxBytes, &mq, 64, head, qt * kBq, b, q_full);
+      }
       int issued = 0;
       for (int j = 0; j < n; ++j) {
-        const int s = j & 1;
-        if (j >= 2 && !mbar_wait(&kv_empty[s], ((j >> 1) & 1) ^ 1, a.status)) break;
+        const int s = j % stages;
+        const uint32_t ph = (j / stages) & 1;
+        if (j >= stages && !mbar_wait(&empty[s], ph ^ 1, a.status)) break;
         const int kt = a.ent[2 * (e0 + j)];
-        mbar_arrive_expect_tx(&kv_full[s], 2 * kTileBytes);
-        uint8_t* k_dst = sK + s * kTileBytes;
-        uint8_t* v_dst = sV + s * kTileBytes;
-        tma_load_4d(k_dst, &mk, 0, kvh, kt * kBk, b, &kv_full[s]);
-        tma_load_4d(k_dst + kBoxBytes, &mk, 64, kvh, kt * kBk, b, &kv_full[s]);
-        tma_load_4d(v_dst, &mv, 0, kvh, kt * kBk, b, &kv_full[s]);
-        tma_load_4d(v_dst + kBoxBytes, &mv, 64, kvh, kt * kBk, b, &kv_full[s]);
+        uint8_t* dst = ring + s * kTileBytes;
+        mbar_arrive_expect_tx(&full[s], kTileBytes);
+        tma_load_4d(dst, map, 0, kvh, kt * kBk, b, &full[s]);
+        tma_load_4d(dst + kBoxBytes, map, 64, kvh, kt * kBk, b, &full[s]);
         issued = j + 1;
       }
       // every issued copy lands before the CTA may exit
-      mbar_wait(q_full, 0, a.status);
-      for (int j = (issued > 2 ? issued - 2 : 0); j < issued; ++j)
-        mbar_wait(&kv_full[j & 1], (j >> 1) & 1, a.status);
+      if (is_k) mbar_wait(q_full, 0, a.status);
+      for (int j = (issued > stages ? issued - stages : 0); j < issued; ++j)
+        mbar_wait(&full[j % stages], (j / stages) & 1, a.status);
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
@@ -162,24 +190,31 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = mbar_wait(q_full, 0, a.status);
       auto issue_pv = [&](int i) -> bool {
         const int s = i & 1;
-        if (!mbar_wait(&p_ready[s], (i >> 1) & 1, a.status)) return false;
-        tc_fence_after();
-        const uint32_t vb = v_addr + s * kTileBytes;
+        const int vs = i % kVStages;
+        if (!mbar_wait(&v_full[vs], (i / kVStages) & 1, a.status)) return false;
+        const uint32_t vb = v_addr + vs * kTileBytes;
+        // group g's keys [64g, 64g+64) accumulate into its own O_g, as soon as its P is in
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          // B = V[16 keys][128 d]: MN-major, 64-column halves 16 KB apart (LBO), 8-key
-          // groups 1024 B apart (SBO); 16 keys = 2048 B per step.
-          const uint64_t bdesc = umma_desc_sw128(vb + kk * 2048, kBoxBytes, 1024);
-          umma_ts(tmem + kColO, tmem + col_s(s) + kk * 8, bdesc, idesc_pv,
-                  (i > 0 || kk > 0) ? 1u : 0u);
+        for (int g = 0; g < kGroups; ++g) {
+          if (!mbar_wait(&p_ready[s * kGroups + g], (i >> 1) & 1, a.status)) return false;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 4 * g; kk < 4 * g + 4; ++kk) {
+            // B = V[16 keys][128 d]: MN-major, 64-column halves 16 KB apart (LBO), 8-key
+            // groups 1024 B apart (SBO); 16 keys = 2048 B per step.
+            const uint64_t bdesc = umma_desc_sw128(vb + kk * 2048, kBoxBytes, 1024);
+            umma_ts(tmem + kColO + 128 * g, tmem + col_s(s) + kk * 8, bdesc, idesc_pv,
+                    (i > 0 || kk > 4 * g) ? 1u : 0u);
+          }
         }
-        umma_commit(&kv_empty[s]);
+        umma_commit(&v_empty[vs]);
         umma_commit(pv_done);
         return true;
       };
       for (int j = 0; ok && j < n; ++j) {
         const int s = j & 1;
-        if (!mbar_wait(&kv_full[s], (j >> 1) & 1, a.status)) {
+        const int ks = j % kKStages;
+        if (!mbar_wait(&k_full[ks], (j / kKStages) & 1, a.status)) {
           ok = false;
           break;
         }
@@ -189,7 +224,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         tc_fence_after();
-        const uint32_t kb = k_addr + s * kTileBytes;
+        const uint32_t kb = k_addr + ks * kTileBytes;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           // A = Q, B = K: K-major, 128-byte rows, 8-row groups 1024 B apart; 16 columns =
@@ -199,6 +234,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                   umma_desc_sw128(kb + off, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
         }
         umma_commit(&s_full[s]);
+        umma_commit(&k_empty[ks]);
         if (j >= 1 && !issue_pv(j - 1)) {
           ok = false;
           break;
@@ -209,12 +245,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_wait(mma_done, 0, a.status);
     }
   } else {
-    // ------------------------------------------------------------ softmax warpgroup
-    const int r = threadIdx.x;  // row within the tile == TMEM lane
+    // ------------------------------------------------------------ softmax warpgroups
+    // Two warpgroups share the 128 rows: warp w reads TMEM lanes 32*(w%4).., group g owns
+    // the 64 score columns [64g, 64g+64) of every row with its own running max m_g, sum
+    // l_g and accumulator O_g (= P[:, 64g:64g+64] V[64g:64g+64, :]), so the groups never
+    // wait for each other inside the loop; the epilogue combines the two halves once.
+    const int wg = threadIdx.x >> 7;
+    const int r = threadIdx.x & 127;  // row within the tile == TMEM lane
     const int64_t row = (int64_t)qt * kBq + r;
-    const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+    const uint32_t cs0 = static_cast<uint32_t>(kCols * wg);  // S column offset
+    const uint32_t og = kColO + 128u * wg;                    // this group's O_g
+    float* red = reinterpret_cast<float*>(tmem_slot + 4);     // [kGroups][2][128]
     const float sl2 = a.scale_log2;
-    float m = -INFINITY;
+    const uint64_t sl2x2 = pack_f32x2(sl2, sl2);
+    float m = -INFINITY;  // running max of raw scores (softmax scale > 0 keeps the order)
     float l = 0.f;
     bool ok = true;
     for (int j = 0; j < n; ++j) {
@@ -222,93 +267,120 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int kt = a.ent[2 * (e0 + j)];
       const int flag = a.ent[2 * (e0 + j) + 1];
       // warp-uniform outcome: the tcgen05.ld/st below are warp-collective
-      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[s], (j >> 1) & 1, a.status))) {
-        ok = false;
-        break;
-      }
+      ok = ok && __all_sync(0xffffffffu, mbar_wait(&s_full[s], (j >> 1) & 1, a.status));
+      if (!ok) continue;  // keep iterating: every warp must reach the epilogue barrier
       tc_fence_after();
-      float x[128];
+      float x[kCols];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < kCols / 32; ++c) {
         uint32_t raw[32];
-        tmem_ld32(lane_base + col_s(s) + 32 * c, raw);
+        tmem_ld32(lane_base + col_s(s) + cs0 + 32 * c, raw);
         tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 32; ++i) x[32 * c + i] = __uint_as_float(raw[i]) * sl2;
+        for (int i = 0; i < 32; ++i) x[32 * c + i] = __uint_as_float(raw[i]);
       }
       if (flag == PS_TILE_PARTIAL) {
-        const int64_t k0 = (int64_t)kt * kBk;
+        const int64_t k0 = (int64_t)kt * kBk + cs0;
 #pragma unroll
-        for (int i = 0; i < 128; ++i)
+        for (int i = 0; i < kCols; ++i)
           if (!visible(row, k0 + i, a.seq, a.lp, a.w)) x[i] = -INFINITY;
       }
-      float mt = x[0];
+      float t8[kCols / 4];
 #pragma unroll
-      for (int i = 1; i < 128; ++i) mt = fmaxf(mt, x[i]);
-      const float m_new = fmaxf(m, mt);
-      // The rescale touches TMEM with warp-collective tcgen05.ld/st, so the decision is
-      // taken per warp: if any row of the warp needs it, every row of the warp rescales
-      // (exact for every row, since m_new >= m).
-      if (__any_sync(0xffffffffu, m_new > m + kRescaleThreshold)) {
+      for (int i = 0; i < kCols / 4; ++i)
+        t8[i] = max3f(x[4 * i], x[4 * i + 1], fmaxf(x[4 * i + 2], x[4 * i + 3]));
+#pragma unroll
+      for (int n2 = kCols / 4; n2 > 1; n2 = (n2 + 1) / 2) {
+#pragma unroll
+        for (int i = 0; i < n2 / 2; ++i) t8[i] = fmaxf(t8[2 * i], t8[2 * i + 1]);
+        if (n2 & 1) t8[n2 / 2] = t8[n2 - 1];
+      }
+      const float m_new = fmaxf(m, t8[0]);
+      // Rescale O_g (and l) when the max of some row of this warp grew by more than 2^8.
+      if (__any_sync(0xffffffffu, (m_new - m) * sl2 > kRescaleThreshold)) {
         float f = 1.f;
-        if (m_new != -INFINITY) f = (m == -INFINITY) ? 0.f : fast_exp2(m - m_new);
+        if (m_new != -INFINITY) f = (m == -INFINITY) ? 0.f : fast_exp2((m - m_new) * sl2);
         if (j > 0) {
-          // O holds PV_0..PV_{j-1}; wait for the last of them, then scale in place
-          if (!__all_sync(0xffffffffu, mbar_wait(pv_done, (j - 1) & 1, a.status))) {
+          // O_g holds PV_0..PV_{j-1}: wait for the last one, then scale it in place
+          if (__all_sync(0xffffffffu, mbar_wait(pv_done, (j - 1) & 1, a.status))) {
+            tc_fence_after();
+            const uint64_t f2 = pack_f32x2(f, f);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              uint32_t o[32];
+              tmem_ld32(lane_base + og + 32 * c, o);
+              tmem_wait_ld();
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                const uint64_t v = fmul2(pack_f32x2(__uint_as_float(o[2 * i]),
+                                                    __uint_as_float(o[2 * i + 1])), f2);
+                const float2 w2 = unpack_f32x2(v);
+                o[2 * i] = __float_as_uint(w2.x);
+                o[2 * i + 1] = __float_as_uint(w2.y);
+              }
+              tmem_st32(lane_base + og + 32 * c, o);
+            }
+            tmem_wait_st();
+          } else {
             ok = false;
-            break;
+            continue;
           }
-          tc_fence_after();
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            uint32_t o[32];
-            tmem_ld32(lane_base + kColO + 32 * c, o);
-            tmem_wait_ld();
-#pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * f);
-            tmem_st32(lane_base + kColO + 32 * c, o);
-          }
-          tmem_wait_st();
         }
         l *= f;
         if (m_new != -INFINITY) m = m_new;
       }
-      const float mref = (m == -INFINITY) ? 0.f : m;
-      float sum = 0.f;
+      // p = 2^(x * scale*log2e - m * scale*log2e), two lanes per instruction
+      const float ms = (m == -INFINITY) ? 0.f : m * sl2;
+      const uint64_t nms2 = pack_f32x2(-ms, -ms);
+      uint64_t acc0 = pack_f32x2(0.f, 0.f), acc1 = acc0;
+      uint32_t pk[kCols / 2];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t pk[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float p0 = fast_exp2(x[32 * c + 2 * i] - mref);
-          const float p1 = fast_exp2(x[32 * c + 2 * i + 1] - mref);
-          sum += p0 + p1;
-          pk[i] = pack_bf16x2(p0, p1);
-        }
-        tmem_st16(lane_base + col_s(s) + 16 * c, pk);
+      for (int i = 0; i < kCols / 2; ++i) {
+        const float2 e = unpack_f32x2(ffma2(pack_f32x2(x[2 * i], x[2 * i + 1]), sl2x2, nms2));
+        const float p0 = fast_exp2(e.x), p1 = fast_exp2(e.y);
+        if (i & 1)
+          acc1 = fadd2(acc1, pack_f32x2(p0, p1));
+        else
+          acc0 = fadd2(acc0, pack_f32x2(p0, p1));
+        pk[i] = cvt_bf16x2(p0, p1);
       }
-      l += sum;
+      tmem_st32(lane_base + col_s(s) + cs0 / 2, pk);
+      const float2 a0 = unpack_f32x2(acc0), a1 = unpack_f32x2(acc1);
+      l += (a0.x + a0.y) + (a1.x + a1.y);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&p_ready[s]);
+      if (lane == 0) mbar_arrive(&p_ready[s * kGroups + wg]);
     }
     // ------------------------------------------------------------ epilogue
-    if (ok && n > 0 && __all_sync(0xffffffffu, mbar_wait(pv_done, (n - 1) & 1, a.status))) {
+    // O = (2^(m_0 - M) O_0 + 2^(m_1 - M) O_1) / (2^(m_0 - M) l_0 + 2^(m_1 - M) l_1)
+    const bool fin = ok && n > 0 && mbar_wait(pv_done, (n - 1) & 1, a.status);
+    red[(wg * 2 + 0) * 128 + r] = m;
+    red[(wg * 2 + 1) * 128 + r] = l;
+    const bool all_fin = named_bar_and(1, kSoftmaxThreads, fin);
+    if (all_fin) {
       tc_fence_after();
-      const float inv_l = l > 0.f ? 1.f / l : 0.f;
+      const float m0 = red[0 * 128 + r], l0 = red[1 * 128 + r];
+      const float m1 = red[2 * 128 + r], l1 = red[3 * 128 + r];
+      const float M = fmaxf(m0, m1);
+      const float f0 = (m0 == -INFINITY) ? 0.f : fast_exp2((m0 - M) * sl2);
+      const float f1 = (m1 == -INFINITY) ? 0.f : fast_exp2((m1 - M) * sl2);
+      const float lt = f0 * l0 + f1 * l1;
+      const float inv_l = lt > 0.f ? 1.f / lt : 0.f;
+      const float g0 = f0 * inv_l, g1 = f1 * inv_l;
       const bool store = row < a.seq;
-      __nv_bfloat16* orow = a.out + (((int64_t)b * a.seq + row) * a.hq + head) * kHeadDim;
+      __nv_bfloat16* orow = a.out + (((int64_t)b * a.seq + row) * a.hq + head) * kHeadDim + cs0;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t o[32];
-        tmem_ld32(lane_base + kColO + 32 * c, o);
+      for (int c = 0; c < kCols / 32; ++c) {
+        uint32_t oa[32], ob[32];
+        tmem_ld32(lane_base + kColO + cs0 + 32 * c, oa);
+        tmem_ld32(lane_base + kColO + 128 + cs0 + 32 * c, ob);
         tmem_wait_ld();
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i)
-          pk[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv_l,
-                              __uint_as_float(o[2 * i + 1]) * inv_l);
+          pk[i] = cvt_bf16x2(g0 * __uint_as_float(oa[2 * i]) + g1 * __uint_as_float(ob[2 * i]),
+                             g0 * __uint_as_float(oa[2 * i + 1]) + g1 * __uint_as_float(ob[2 * i + 1]));
         if (store) {
           uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
 #pragma unroll
@@ -316,9 +388,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
         }
       }
-      if (store && a.lse)
+      if (store && wg == 0 && a.lse)
         a.lse[((int64_t)b * a.hq + head) * a.seq + row] =
-            l > 0.f ? (m + log2f(l)) * kLn2 : -INFINITY;
+            lt > 0.f ? (M * sl2 + log2f(lt)) * kLn2 : -INFINITY;
     }
   }
   tc_fence_before();

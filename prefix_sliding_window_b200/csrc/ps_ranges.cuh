@@ -105,21 +105,27 @@ PS_HD DecodeTiling make_tiling(const VisibleRanges& r, int32_t dim_prefix, int32
 }
 
 PS_HD DecodeTile tiling_tile(const DecodeTiling& t, int32_t idx) {
-  int s = 0;
-  while (s < 2 && idx >= t.nt[s]) {
-    idx -= t.nt[s];
-    ++s;
+  // segment selection with constant indices only (keeps the tiling in registers)
+  int32_t begin, end, fwd, map_id, nt;
+  if (idx < t.nt[0]) {
+    begin = t.begin[0]; end = t.end[0]; fwd = t.forward[0]; map_id = t.map_id[0]; nt = t.nt[0];
+  } else if (idx < t.nt[0] + t.nt[1]) {
+    idx -= t.nt[0];
+    begin = t.begin[1]; end = t.end[1]; fwd = t.forward[1]; map_id = t.map_id[1]; nt = t.nt[1];
+  } else {
+    idx -= t.nt[0] + t.nt[1];
+    begin = t.begin[2]; end = t.end[2]; fwd = t.forward[2]; map_id = t.map_id[2]; nt = t.nt[2];
   }
   DecodeTile d;
-  d.map_id = t.map_id[s];
-  if (t.forward[s]) {
-    d.row0 = t.begin[s] + idx * kDecodeTile;
+  d.map_id = map_id;
+  if (fwd) {
+    d.row0 = begin + idx * kDecodeTile;
     d.lo = 0;
-    const int32_t left = t.end[s] - d.row0;
+    const int32_t left = end - d.row0;
     d.hi = left < kDecodeTile ? left : kDecodeTile;
   } else {
-    d.row0 = t.end[s] - (t.nt[s] - idx) * kDecodeTile;
-    d.lo = d.row0 < t.begin[s] ? t.begin[s] - d.row0 : 0;
+    d.row0 = end - (nt - idx) * kDecodeTile;
+    d.lo = d.row0 < begin ? begin - d.row0 : 0;
     d.hi = kDecodeTile;
   }
   return d;
