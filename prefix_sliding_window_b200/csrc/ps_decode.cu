@@ -695,9 +695,10 @@ int launch_decode(const DecodeLaunch& l, cudaStream_t stream) {
   if (g > 0) {
     rc = check_cuda(
         launch_pdl(merge_kernel, dim3(static_cast<unsigned>((l.batch * l.hq + 3) / 4)), dim3(128),
-                   0, stream, static_cast<const float*>(a.ws_o), static_cast<const float*>(a.ws_lse),
-                   static_cast<const int32_t*>(a.ws_pref), static_cast<const int32_t*>(a.ws_span),
-                   a.out, a.lse, a.batch, l.hq, l.hkv, group, static_cast<int32_t>(g)),
+                   0, stream, static_cast<const float*>(a.ws_o),
+                   static_cast<const float*>(a.ws_lse), static_cast<const int32_t*>(a.ws_pref),
+                   static_cast<const int32_t*>(a.ws_span), a.out, a.lse, a.batch, l.hq, l.hkv,
+                   group, static_cast<int32_t>(g)),
         "merge_kernel launch");
   }
   return rc;

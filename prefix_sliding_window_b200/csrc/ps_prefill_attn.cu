@@ -11,7 +11,7 @@
 //
 // One CTA per (batch, query head, query tile), heaviest query tiles first, 11 warps:
 //   warps 8, 9 - TMA producers: warp 8 loads the Q tile once and the K tiles of the plan
-//             into a 3-stage ring, warp 9 the V tiles into a 2-stage ring (4-D tensor
+//             into a 2-stage ring, warp 9 the V tiles into a 3-stage ring (4-D tensor
 //             maps, 128-byte swizzle).  A K stage is released when its QK^T completes, a V
 //             stage when its PV completes.
 //   warp 10 - allocates 512 TMEM columns; one lane issues the MMAs:
@@ -23,13 +23,13 @@
 //   warps 0-7 - softmax, two warpgroups: row r lives in TMEM lane r; group g handles the
 //             64 score columns [64g, 64g+64) of every row as an independent online softmax
 //             (its own max m_g, sum l_g and accumulator O_g), so the groups never wait for
-//             each other inside the loop.  Each thread masks its slice on PARTIAL tiles,
-//             writes P as bf16 over its columns of the same S buffer (packed fp32x2
-//             FMA/add, one ex2 per element) and signals the MMA warp.  O_g is rescaled in
-//             TMEM only when the max of some row of the warp grows by more than 8 (log2
-//             units); otherwise P stays below 2^8 and the stale max keeps fp32 sums exact
-//             enough.  The decision is warp-uniform because tcgen05.ld/st are
-//             warp-collective.
+//             each other inside the loop.  On PARTIAL tiles each thread masks its slice with
+//             a 64-bit interval mask built once per row; it then writes P as bf16 over its
+//             columns of the same S buffer (packed fp32x2 FMA/add, one ex2 per element) and
+//             signals the MMA warp.  O_g is rescaled in TMEM only when the max of some row
+//             of the warp grows by more than 8 (log2 units); otherwise P stays below 2^8
+//             and the stale max keeps fp32 sums exact enough.  The decision is warp-uniform
+//             because tcgen05.ld/st are warp-collective.
 //   Epilogue: O = (2^(m_0-M) O_0 + 2^(m_1-M) O_1) / (2^(m_0-M) l_0 + 2^(m_1-M) l_1),
 //             each group stores half of the columns as bf16; group 0 stores the lse.
 // TMEM columns: S0 [0,128), S1 [128,256), O_0 [256,384), O_1 [384,512).
@@ -55,8 +55,8 @@ constexpr int kKProducerWarp = kSoftmaxWarps;
 constexpr int kVProducerWarp = kSoftmaxWarps + 1;
 constexpr int kMmaWarp = kSoftmaxWarps + 2;
 constexpr int kThreads = (kSoftmaxWarps + 3) * 32;
-constexpr int kKStages = 3;
-constexpr int kVStages = 2;
+constexpr int kKStages = 2;
+constexpr int kVStages = 3;
 constexpr int kBoxBytes = 128 * 128;        // [128 rows][64 bf16]
 constexpr int kTileBytes = 2 * kBoxBytes;   // [128 rows][128 bf16]
 constexpr uint32_t kTmemCols = 512;
@@ -66,7 +66,8 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
-constexpr size_t kSmemBytes = 1024 + kTileBytes * (1 + kKStages + kVStages) + 256 + 2 * kGroups * 128 * 4;
+constexpr size_t kSmemBytes =
+    1024 + kTileBytes * (1 + kKStages + kVStages) + 256 + 2 * kGroups * 128 * 4;
 
 struct PrefillArgs {
   const int32_t* off;  // [nq + 1] plan offsets
@@ -80,9 +81,25 @@ struct PrefillArgs {
   float scale_log2;
 };
 
-__device__ __forceinline__ bool visible(int64_t row, int64_t col, int64_t seq, int32_t lp,
-                                        int32_t w) {
-  return col <= row && col < seq && (col < lp || col > row - w);
+// Bit c of the result is set iff key k0 + c (c < 64) is visible from query `row`: the keys
+// row can see are [0, min(lp, row+1)) and [max(lp, row-w+1), row+1), both cut at seq.
+__device__ __forceinline__ uint64_t interval_bits(int64_t lo, int64_t hi, int64_t k0) {
+  lo -= k0;
+  hi -= k0;
+  if (lo < 0) lo = 0;
+  if (hi > 64) hi = 64;
+  if (hi <= lo) return 0ull;
+  const uint64_t len = static_cast<uint64_t>(hi - lo);
+  const uint64_t ones = len >= 64 ? ~0ull : ((1ull << len) - 1ull);
+  return ones << lo;
+}
+__device__ __forceinline__ uint64_t visible_bits(int64_t row, int64_t k0, int64_t seq, int32_t lp,
+                                                 int32_t w) {
+  const int64_t end = row + 1 < seq ? row + 1 : seq;
+  const int64_t pre_end = lp < end ? lp : end;
+  int64_t win_lo = row - w + 1;
+  if (win_lo < lp) win_lo = lp;
+  return interval_bits(0, pre_end, k0) | interval_bits(win_lo, end, k0);
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -96,13 +113,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sV = sK + kKStages * kTileBytes;
   uint64_t* bars = reinterpret_cast<uint64_t*>(sV + kVStages * kTileBytes);
   uint64_t* q_full = bars + 0;
-  uint64_t* k_full = bars + 1;    // [kKStages]
-  uint64_t* k_empty = bars + 4;   // [kKStages]
-  uint64_t* v_full = bars + 7;    // [kVStages]
-  uint64_t* v_empty = bars + 9;   // [kVStages]
-  uint64_t* s_full = bars + 11;   // [2]
-  uint64_t* p_ready = bars + 13;  // [2 buffers][kGroups]
-  uint64_t* pv_done = bars + 13 + 2 * kGroups;
+  uint64_t* k_full = bars + 1;                       // [kKStages]
+  uint64_t* k_empty = k_full + kKStages;             // [kKStages]
+  uint64_t* v_full = k_empty + kKStages;             // [kVStages]
+  uint64_t* v_empty = v_full + kVStages;             // [kVStages]
+  uint64_t* s_full = v_empty + kVStages;             // [2]
+  uint64_t* p_ready = s_full + 2;                    // [2 buffers][kGroups]
+  uint64_t* pv_done = p_ready + 2 * kGroups;
   uint64_t* mma_done = pv_done + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
 
@@ -280,10 +297,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < 32; ++i) x[32 * c + i] = __uint_as_float(raw[i]);
       }
       if (flag == PS_TILE_PARTIAL) {
-        const int64_t k0 = (int64_t)kt * kBk + cs0;
+        // visible keys of this row inside the slice: two intervals, as a 64-bit mask
+        const uint64_t vis = visible_bits(row, (int64_t)kt * kBk + cs0, a.seq, a.lp, a.w);
+        const uint32_t vlo = static_cast<uint32_t>(vis), vhi = static_cast<uint32_t>(vis >> 32);
 #pragma unroll
-        for (int i = 0; i < kCols; ++i)
-          if (!visible(row, k0 + i, a.seq, a.lp, a.w)) x[i] = -INFINITY;
+        for (int i = 0; i < kCols; ++i) {
+          const uint32_t word = i < 32 ? vlo : vhi;
+          if (!(word & (1u << (i & 31)))) x[i] = -INFINITY;
+        }
       }
       float t8[kCols / 4];
 #pragma unroll
