@@ -8,6 +8,7 @@
 // then the window tiles.
 #include <cuda_runtime.h>
 
+#include "ps_device.cuh"
 #include "ps_internal.h"
 #include "ps_ranges.cuh"
 
@@ -24,6 +25,7 @@ __global__ void __launch_bounds__(kPlanThreads)
                 int32_t* __restrict__ ws_ent, int32_t* __restrict__ plan_out) {
   __shared__ int32_t s_scan[kPlanThreads];
   __shared__ int32_t s_base;
+  pdl_trigger();  // the attention kernel may start its prologue; it waits for this plan
   const int64_t nq = (seq + kPrefillBq - 1) / kPrefillBq;
   if (threadIdx.x == 0) s_base = 0;
   __syncthreads();

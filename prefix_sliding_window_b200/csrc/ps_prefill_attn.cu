@@ -9,11 +9,14 @@
 // unmasked; PARTIAL tiles (the diagonal, the window's lower edge, the prefix's end and the
 // ragged tail) get an element-wise mask.
 //
-// One CTA per (batch, query head, query tile), heaviest query tiles first, 11 warps:
-//   warps 8, 9 - TMA producers: warp 8 loads the Q tile once and the K tiles of the plan
-//             into a 2-stage ring, warp 9 the V tiles into a 3-stage ring (4-D tensor
-//             maps, 128-byte swizzle).  A K stage is released when its QK^T completes, a V
-//             stage when its PV completes.
+// Persistent: one CTA per SM walks the (batch, query head, 128-row query tile) items
+// blockIdx.x, blockIdx.x + gridDim.x, ... (heaviest query tiles first); TMEM, barriers and
+// the TMA rings live across items, so the next item's Q tile and first QK^T overlap the
+// previous item's tail.  11 warps:
+//   warps 8, 9 - TMA producers: warp 8 loads the query tiles (two buffers) and the K tiles
+//             of the plan into a 2-stage ring, warp 9 the V tiles into a 2-stage ring (4-D
+//             tensor maps, 128-byte swizzle).  A query buffer is released after its item's
+//             last QK^T, a K stage when its QK^T completes, a V stage when its PV completes.
 //   warp 10 - allocates 512 TMEM columns; one lane issues the MMAs:
 //               S[buf] = Q K^T             (tcgen05.mma kind::f16, A and B from smem)
 //               O_g   += P_g V_g, g = 0, 1 (A = P from TMEM, B = V from smem, MN-major;
@@ -30,8 +33,10 @@
 //             of the warp grows by more than 8 (log2 units); otherwise P stays below 2^8
 //             and the stale max keeps fp32 sums exact enough.  The decision is warp-uniform
 //             because tcgen05.ld/st are warp-collective.
-//   Epilogue: O = (2^(m_0-M) O_0 + 2^(m_1-M) O_1) / (2^(m_0-M) l_0 + 2^(m_1-M) l_1),
-//             each group stores half of the columns as bf16; group 0 stores the lse.
+//   Epilogue (per item): O = (2^(m_0-M) O_0 + 2^(m_1-M) O_1) / (2^(m_0-M) l_0 + 2^(m_1-M) l_1);
+//             once O is in registers the warps release it (o_free) so the next item's first
+//             PV may overwrite it; each group stores half of the columns as bf16, group 0
+//             the lse.
 // TMEM columns: S0 [0,128), S1 [128,256), O_0 [256,384), O_1 [384,512).
 
 #include <cuda_bf16.h>
@@ -55,8 +60,9 @@ constexpr int kKProducerWarp = kSoftmaxWarps;
 constexpr int kVProducerWarp = kSoftmaxWarps + 1;
 constexpr int kMmaWarp = kSoftmaxWarps + 2;
 constexpr int kThreads = (kSoftmaxWarps + 3) * 32;
+constexpr int kQStages = 2;
 constexpr int kKStages = 2;
-constexpr int kVStages = 3;
+constexpr int kVStages = 2;
 constexpr int kBoxBytes = 128 * 128;        // [128 rows][64 bf16]
 constexpr int kTileBytes = 2 * kBoxBytes;   // [128 rows][128 bf16]
 constexpr uint32_t kTmemCols = 512;
@@ -67,7 +73,7 @@ constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
 constexpr size_t kSmemBytes =
-    1024 + kTileBytes * (1 + kKStages + kVStages) + 256 + 2 * kGroups * 128 * 4;
+    1024 + kTileBytes * (kQStages + kKStages + kVStages) + 256 + 2 * 2 * kGroups * 128 * 4;
 
 struct PrefillArgs {
   const int32_t* off;  // [nq + 1] plan offsets
@@ -108,34 +114,40 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  uint8_t* sQ = smem;
-  uint8_t* sK = sQ + kTileBytes;
-  uint8_t* sV = sK + kKStages * kTileBytes;
+  uint8_t* sQ = smem;                       // [kQStages] query tiles
+  uint8_t* sK = sQ + kQStages * kTileBytes;  // [kKStages]
+  uint8_t* sV = sK + kKStages * kTileBytes;  // [kVStages]
   uint64_t* bars = reinterpret_cast<uint64_t*>(sV + kVStages * kTileBytes);
-  uint64_t* q_full = bars + 0;
-  uint64_t* k_full = bars + 1;                       // [kKStages]
+  uint64_t* q_full = bars;                           // [kQStages]
+  uint64_t* q_empty = q_full + kQStages;             // [kQStages]
+  uint64_t* k_full = q_empty + kQStages;             // [kKStages]
   uint64_t* k_empty = k_full + kKStages;             // [kKStages]
   uint64_t* v_full = k_empty + kKStages;             // [kVStages]
   uint64_t* v_empty = v_full + kVStages;             // [kVStages]
   uint64_t* s_full = v_empty + kVStages;             // [2]
   uint64_t* p_ready = s_full + 2;                    // [2 buffers][kGroups]
   uint64_t* pv_done = p_ready + 2 * kGroups;
-  uint64_t* mma_done = pv_done + 1;
+  uint64_t* o_free = pv_done + 1;
+  uint64_t* mma_done = o_free + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
 
   const int64_t bh = (int64_t)a.batch * a.hq;
-  const int qt = a.nq - 1 - static_cast<int>(blockIdx.x / bh);
-  const int rem = static_cast<int>(blockIdx.x % bh);
-  const int head = rem % a.hq;
-  const int b = rem / a.hq;
-  const int kvh = head / a.group;
-  const int e0 = a.off[qt];
-  const int n = a.off[qt + 1] - e0;
+  const int64_t n_items = bh * a.nq;
+  // item it (heaviest query tiles first): qt = nq-1 - it / (batch*hq), then (b, head)
+  auto item_of = [&](int64_t it, int& qt, int& b, int& head) {
+    qt = a.nq - 1 - static_cast<int>(it / bh);
+    const int rem = static_cast<int>(it % bh);
+    head = rem % a.hq;
+    b = rem / a.hq;
+  };
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    mbar_init(q_full, 1);
+    for (int s = 0; s < kQStages; ++s) {
+      mbar_init(&q_full[s], 1);
+      mbar_init(&q_empty[s], 1);
+    }
     for (int s = 0; s < kKStages; ++s) {
       mbar_init(&k_full[s], 1);
       mbar_init(&k_empty[s], 1);
@@ -149,6 +161,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int g = 0; g < kGroups; ++g) mbar_init(&p_ready[s * kGroups + g], 4);
     }
     mbar_init(pv_done, 1);
+    mbar_init(o_free, kSoftmaxWarps);
     mbar_init(mma_done, 1);
     fence_mbar_init();
   }
@@ -156,15 +169,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
   }
+  if (warp == kKProducerWarp && lane == 0) {
+    prefetch_tensormap(&mq);
+    prefetch_tensormap(&mk);
+    prefetch_tensormap(&mv);
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_wait();  // the plan comes from the kernel launched just before
 
   if (warp == kKProducerWarp || warp == kVProducerWarp) {
     // ------------------------------------------------------------ TMA producers
-    // One warp streams Q and the K tiles, the other the V tiles; K and V have their own rings,
-    // so a K tile can be refilled as soon as its QK^T finished, independent of PV.
+    // Warp 8 streams the query tiles (double-buffered, one per item) and the K tiles, warp 9
+    // the V tiles; both walk this CTA's items and their planned tiles in order.
     if (lane == 0) {
       const bool is_k = (warp == kKProducerWarp);
       const CUtensorMap* map = is_k ? &mk : &mv;
@@ -172,48 +191,73 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint64_t* full = is_k ? k_full : v_full;
       uint64_t* empty = is_k ? k_empty : v_empty;
       const int stages = is_k ? kKStages : kVStages;
-      prefetch_tensormap(map);
-      if (is_k) {
-        prefetch_tensormap(&mq);
-        mbar_arrive_expect_tx(q_full, kTileBytes);
-        tma_load_4d(sQ, &mq, 0, head, qt * kBq, b, q_full);
-        tma_load_4d(sQ + kBoxBytes, &mq, 64, head, qt * kBq, b, q_full);
-      }
-      int issued = 0;
-      for (int j = 0; j < n; ++j) {
-        const int s = j % stages;
-        const uint32_t ph = (j / stages) & 1;
-        if (j >= stages && !mbar_wait(&empty[s], ph ^ 1, a.status)) break;
-        const int kt = a.ent[2 * (e0 + j)];
-        uint8_t* dst = ring + s * kTileBytes;
-        mbar_arrive_expect_tx(&full[s], kTileBytes);
-        tma_load_4d(dst, map, 0, kvh, kt * kBk, b, &full[s]);
-        tma_load_4d(dst + kBoxBytes, map, 64, kvh, kt * kBk, b, &full[s]);
-        issued = j + 1;
+      int64_t g = 0;
+      int li = 0;
+      int q_issued = 0;
+      bool alive = true;
+      for (int64_t it = blockIdx.x; alive && it < n_items; it += gridDim.x, ++li) {
+        int qt, b, head;
+        item_of(it, qt, b, head);
+        const int kvh = head / a.group;
+        const int e0 = a.off[qt];
+        const int n = a.off[qt + 1] - e0;
+        if (is_k) {
+          const int qb = li % kQStages;
+          // the buffer's previous query tile must be done with (its item's last QK^T)
+          if (li >= kQStages &&
+              !mbar_wait(&q_empty[qb], ((li / kQStages) - 1) & 1, a.status)) {
+            alive = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&q_full[qb], kTileBytes);
+          tma_load_4d(sQ + qb * kTileBytes, &mq, 0, head, qt * kBq, b, &q_full[qb]);
+          tma_load_4d(sQ + qb * kTileBytes + kBoxBytes, &mq, 64, head, qt * kBq, b, &q_full[qb]);
+          ++q_issued;
+        }
+        for (int j = 0; j < n; ++j, ++g) {
+          const int s = static_cast<int>(g % stages);
+          const uint32_t ph = static_cast<uint32_t>((g / stages) & 1);
+          if (g >= stages && !mbar_wait(&empty[s], ph ^ 1, a.status)) {
+            alive = false;
+            break;
+          }
+          const int kt = a.ent[2 * (e0 + j)];
+          uint8_t* dst = ring + s * kTileBytes;
+          mbar_arrive_expect_tx(&full[s], kTileBytes);
+          tma_load_4d(dst, map, 0, kvh, kt * kBk, b, &full[s]);
+          tma_load_4d(dst + kBoxBytes, map, 64, kvh, kt * kBk, b, &full[s]);
+        }
       }
       // every issued copy lands before the CTA may exit
-      if (is_k) mbar_wait(q_full, 0, a.status);
-      for (int j = (issued > stages ? issued - stages : 0); j < issued; ++j)
-        mbar_wait(&full[j % stages], (j / stages) & 1, a.status);
+      for (int64_t j = (g > stages ? g - stages : 0); j < g; ++j)
+        mbar_wait(&full[j % stages], static_cast<uint32_t>((j / stages) & 1), a.status);
+      if (is_k)
+        for (int j = (q_issued > kQStages ? q_issued - kQStages : 0); j < q_issued; ++j)
+          mbar_wait(&q_full[j % kQStages], (j / kQStages) & 1, a.status);
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc_qk = umma_idesc_bf16(128, 128, false);
       constexpr uint32_t idesc_pv = umma_idesc_bf16(128, 128, true);
-      const uint32_t q_addr = smem_u32(sQ);
       const uint32_t k_addr = smem_u32(sK);
       const uint32_t v_addr = smem_u32(sV);
-      bool ok = mbar_wait(q_full, 0, a.status);
-      auto issue_pv = [&](int i) -> bool {
-        const int s = i & 1;
-        const int vs = i % kVStages;
-        if (!mbar_wait(&v_full[vs], (i / kVStages) & 1, a.status)) return false;
+      // PV of global tile gg; the first PV of an item zero-initialises O_0 / O_1, after the
+      // previous item's epilogue has read them (o_free)
+      auto issue_pv = [&](int64_t gg, bool first_of_item, int item_li) -> bool {
+        const int s = static_cast<int>(gg & 1);
+        const int vs = static_cast<int>(gg % kVStages);
+        if (!mbar_wait(&v_full[vs], static_cast<uint32_t>((gg / kVStages) & 1), a.status))
+          return false;
+        if (first_of_item && item_li > 0 && !mbar_wait(o_free, (item_li - 1) & 1, a.status))
+          return false;
         const uint32_t vb = v_addr + vs * kTileBytes;
         // group g's keys [64g, 64g+64) accumulate into its own O_g, as soon as its P is in
 #pragma unroll
         for (int g = 0; g < kGroups; ++g) {
-          if (!mbar_wait(&p_ready[s * kGroups + g], (i >> 1) & 1, a.status)) return false;
+          if (!mbar_wait(&p_ready[s * kGroups + g], static_cast<uint32_t>((gg >> 1) & 1),
+                         a.status))
+            return false;
           tc_fence_after();
 #pragma unroll
           for (int kk = 4 * g; kk < 4 * g + 4; ++kk) {
@@ -221,43 +265,63 @@ __global__ void __launch_bounds__(kThreads, 1)
             // groups 1024 B apart (SBO); 16 keys = 2048 B per step.
             const uint64_t bdesc = umma_desc_sw128(vb + kk * 2048, kBoxBytes, 1024);
             umma_ts(tmem + kColO + 128 * g, tmem + col_s(s) + kk * 8, bdesc, idesc_pv,
-                    (i > 0 || kk > 4 * g) ? 1u : 0u);
+                    (!first_of_item || kk > 4 * g) ? 1u : 0u);
           }
         }
         umma_commit(&v_empty[vs]);
         umma_commit(pv_done);
         return true;
       };
-      for (int j = 0; ok && j < n; ++j) {
-        const int s = j & 1;
-        const int ks = j % kKStages;
-        if (!mbar_wait(&k_full[ks], (j / kKStages) & 1, a.status)) {
+      int64_t g = 0;
+      int li = 0;
+      bool ok = true;
+      bool have_prev = false, prev_first = false;
+      int prev_li = 0;
+      for (int64_t it = blockIdx.x; ok && it < n_items; it += gridDim.x, ++li) {
+        int qt, b, head;
+        item_of(it, qt, b, head);
+        const int n = a.off[qt + 1] - a.off[qt];
+        const int qb = li % kQStages;
+        if (!mbar_wait(&q_full[qb], (li / kQStages) & 1, a.status)) {
           ok = false;
           break;
         }
-        // S buffer s held P_{j-2}: PV_{j-2} must have finished reading it
-        if (j >= 2 && !mbar_wait(pv_done, (j - 2) & 1, a.status)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t kb = k_addr + ks * kTileBytes;
+        const uint32_t q_addr = smem_u32(sQ + qb * kTileBytes);
+        for (int j = 0; j < n; ++j, ++g) {
+          const int s = static_cast<int>(g & 1);
+          const int ks = static_cast<int>(g % kKStages);
+          if (!mbar_wait(&k_full[ks], static_cast<uint32_t>((g / kKStages) & 1), a.status)) {
+            ok = false;
+            break;
+          }
+          // S buffer s held P of tile g-2: its PV must have finished reading it
+          if (g >= 2 && !mbar_wait(pv_done, static_cast<uint32_t>((g - 2) & 1), a.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t kb = k_addr + ks * kTileBytes;
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          // A = Q, B = K: K-major, 128-byte rows, 8-row groups 1024 B apart; 16 columns =
-          // 32 B per step inside a 64-column half.
-          const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
-          umma_ss(tmem + col_s(s), umma_desc_sw128(q_addr + off, 16, 1024),
-                  umma_desc_sw128(kb + off, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
-        }
-        umma_commit(&s_full[s]);
-        umma_commit(&k_empty[ks]);
-        if (j >= 1 && !issue_pv(j - 1)) {
-          ok = false;
-          break;
+          for (int kk = 0; kk < 8; ++kk) {
+            // A = Q, B = K: K-major, 128-byte rows, 8-row groups 1024 B apart; 16 columns =
+            // 32 B per step inside a 64-column half.
+            const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
+            umma_ss(tmem + col_s(s), umma_desc_sw128(q_addr + off, 16, 1024),
+                    umma_desc_sw128(kb + off, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
+          }
+          umma_commit(&s_full[s]);
+          umma_commit(&k_empty[ks]);
+          if (j == n - 1) umma_commit(&q_empty[qb]);
+          if (have_prev && !issue_pv(g - 1, prev_first, prev_li)) {
+            ok = false;
+            break;
+          }
+          have_prev = true;
+          prev_first = (j == 0);
+          prev_li = li;
         }
       }
-      if (ok && n > 0) issue_pv(n - 1);
+      if (ok && have_prev) issue_pv(g - 1, prev_first, prev_li);
       umma_commit(mma_done);
       mbar_wait(mma_done, 0, a.status);
     }
@@ -269,149 +333,172 @@ __global__ void __launch_bounds__(kThreads, 1)
     // wait for each other inside the loop; the epilogue combines the two halves once.
     const int wg = threadIdx.x >> 7;
     const int r = threadIdx.x & 127;  // row within the tile == TMEM lane
-    const int64_t row = (int64_t)qt * kBq + r;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
     const uint32_t cs0 = static_cast<uint32_t>(kCols * wg);  // S column offset
     const uint32_t og = kColO + 128u * wg;                    // this group's O_g
-    float* red = reinterpret_cast<float*>(tmem_slot + 4);     // [kGroups][2][128]
+    float* red = reinterpret_cast<float*>(tmem_slot + 4);     // [2 parity][kGroups][2][128]
     const float sl2 = a.scale_log2;
     const uint64_t sl2x2 = pack_f32x2(sl2, sl2);
-    float m = -INFINITY;  // running max of raw scores (softmax scale > 0 keeps the order)
-    float l = 0.f;
     bool ok = true;
-    for (int j = 0; j < n; ++j) {
-      const int s = j & 1;
-      const int kt = a.ent[2 * (e0 + j)];
-      const int flag = a.ent[2 * (e0 + j) + 1];
-      // warp-uniform outcome: the tcgen05.ld/st below are warp-collective
-      ok = ok && __all_sync(0xffffffffu, mbar_wait(&s_full[s], (j >> 1) & 1, a.status));
-      if (!ok) continue;  // keep iterating: every warp must reach the epilogue barrier
-      tc_fence_after();
-      float x[kCols];
+    int64_t g = 0;
+    int li = 0;
+    for (int64_t it = blockIdx.x; it < n_items; it += gridDim.x, ++li) {
+      int qt, b, head;
+      item_of(it, qt, b, head);
+      const int e0 = a.off[qt];
+      const int n = a.off[qt + 1] - e0;
+      const int64_t row = (int64_t)qt * kBq + r;
+      float m = -INFINITY;  // running max of raw scores (softmax scale > 0 keeps the order)
+      float l = 0.f;
+      for (int j = 0; j < n; ++j, ++g) {
+        const int s = static_cast<int>(g & 1);
+        const int kt = a.ent[2 * (e0 + j)];
+        const int flag = a.ent[2 * (e0 + j) + 1];
+        // warp-uniform outcome: the tcgen05.ld/st below are warp-collective
+        ok = ok && __all_sync(0xffffffffu, mbar_wait(&s_full[s],
+                                                      static_cast<uint32_t>((g >> 1) & 1),
+                                                      a.status));
+        if (!ok) continue;  // keep iterating: every warp must reach the epilogue barriers
+        tc_fence_after();
+        float x[kCols];
 #pragma unroll
-      for (int c = 0; c < kCols / 32; ++c) {
-        uint32_t raw[32];
-        tmem_ld32(lane_base + col_s(s) + cs0 + 32 * c, raw);
-        tmem_wait_ld();
+        for (int c = 0; c < kCols / 32; ++c) {
+          uint32_t raw[32];
+          tmem_ld32(lane_base + col_s(s) + cs0 + 32 * c, raw);
+          tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 32; ++i) x[32 * c + i] = __uint_as_float(raw[i]);
-      }
-      if (flag == PS_TILE_PARTIAL) {
-        // visible keys of this row inside the slice: two intervals, as a 64-bit mask
-        const uint64_t vis = visible_bits(row, (int64_t)kt * kBk + cs0, a.seq, a.lp, a.w);
-        const uint32_t vlo = static_cast<uint32_t>(vis), vhi = static_cast<uint32_t>(vis >> 32);
-#pragma unroll
-        for (int i = 0; i < kCols; ++i) {
-          const uint32_t word = i < 32 ? vlo : vhi;
-          if (!(word & (1u << (i & 31)))) x[i] = -INFINITY;
+          for (int i = 0; i < 32; ++i) x[32 * c + i] = __uint_as_float(raw[i]);
         }
-      }
-      float t8[kCols / 4];
+        if (flag == PS_TILE_PARTIAL) {
+          // visible keys of this row inside the slice: two intervals, as a 64-bit mask
+          const uint64_t vis = visible_bits(row, (int64_t)kt * kBk + cs0, a.seq, a.lp, a.w);
+          const uint32_t vlo = static_cast<uint32_t>(vis), vhi = static_cast<uint32_t>(vis >> 32);
 #pragma unroll
-      for (int i = 0; i < kCols / 4; ++i)
-        t8[i] = max3f(x[4 * i], x[4 * i + 1], fmaxf(x[4 * i + 2], x[4 * i + 3]));
-#pragma unroll
-      for (int n2 = kCols / 4; n2 > 1; n2 = (n2 + 1) / 2) {
-#pragma unroll
-        for (int i = 0; i < n2 / 2; ++i) t8[i] = fmaxf(t8[2 * i], t8[2 * i + 1]);
-        if (n2 & 1) t8[n2 / 2] = t8[n2 - 1];
-      }
-      const float m_new = fmaxf(m, t8[0]);
-      // Rescale O_g (and l) when the max of some row of this warp grew by more than 2^8.
-      if (__any_sync(0xffffffffu, (m_new - m) * sl2 > kRescaleThreshold)) {
-        float f = 1.f;
-        if (m_new != -INFINITY) f = (m == -INFINITY) ? 0.f : fast_exp2((m - m_new) * sl2);
-        if (j > 0) {
-          // O_g holds PV_0..PV_{j-1}: wait for the last one, then scale it in place
-          if (__all_sync(0xffffffffu, mbar_wait(pv_done, (j - 1) & 1, a.status))) {
-            tc_fence_after();
-            const uint64_t f2 = pack_f32x2(f, f);
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-              uint32_t o[32];
-              tmem_ld32(lane_base + og + 32 * c, o);
-              tmem_wait_ld();
-#pragma unroll
-              for (int i = 0; i < 16; ++i) {
-                const uint64_t v = fmul2(pack_f32x2(__uint_as_float(o[2 * i]),
-                                                    __uint_as_float(o[2 * i + 1])), f2);
-                const float2 w2 = unpack_f32x2(v);
-                o[2 * i] = __float_as_uint(w2.x);
-                o[2 * i + 1] = __float_as_uint(w2.y);
-              }
-              tmem_st32(lane_base + og + 32 * c, o);
-            }
-            tmem_wait_st();
-          } else {
-            ok = false;
-            continue;
+          for (int i = 0; i < kCols; ++i) {
+            const uint32_t word = i < 32 ? vlo : vhi;
+            if (!(word & (1u << (i & 31)))) x[i] = -INFINITY;
           }
         }
-        l *= f;
-        if (m_new != -INFINITY) m = m_new;
-      }
-      // p = 2^(x * scale*log2e - m * scale*log2e), two lanes per instruction
-      const float ms = (m == -INFINITY) ? 0.f : m * sl2;
-      const uint64_t nms2 = pack_f32x2(-ms, -ms);
-      uint64_t acc0 = pack_f32x2(0.f, 0.f), acc1 = acc0;
-      uint32_t pk[kCols / 2];
+        float t8[kCols / 4];
 #pragma unroll
-      for (int i = 0; i < kCols / 2; ++i) {
-        const float2 e = unpack_f32x2(ffma2(pack_f32x2(x[2 * i], x[2 * i + 1]), sl2x2, nms2));
-        const float p0 = fast_exp2(e.x), p1 = fast_exp2(e.y);
-        if (i & 1)
-          acc1 = fadd2(acc1, pack_f32x2(p0, p1));
-        else
-          acc0 = fadd2(acc0, pack_f32x2(p0, p1));
-        pk[i] = cvt_bf16x2(p0, p1);
-      }
-      tmem_st32(lane_base + col_s(s) + cs0 / 2, pk);
-      const float2 a0 = unpack_f32x2(acc0), a1 = unpack_f32x2(acc1);
-      l += (a0.x + a0.y) + (a1.x + a1.y);
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&p_ready[s * kGroups + wg]);
-    }
-    // ------------------------------------------------------------ epilogue
-    // O = (2^(m_0 - M) O_0 + 2^(m_1 - M) O_1) / (2^(m_0 - M) l_0 + 2^(m_1 - M) l_1)
-    const bool fin = ok && n > 0 && mbar_wait(pv_done, (n - 1) & 1, a.status);
-    red[(wg * 2 + 0) * 128 + r] = m;
-    red[(wg * 2 + 1) * 128 + r] = l;
-    const bool all_fin = named_bar_and(1, kSoftmaxThreads, fin);
-    if (all_fin) {
-      tc_fence_after();
-      const float m0 = red[0 * 128 + r], l0 = red[1 * 128 + r];
-      const float m1 = red[2 * 128 + r], l1 = red[3 * 128 + r];
-      const float M = fmaxf(m0, m1);
-      const float f0 = (m0 == -INFINITY) ? 0.f : fast_exp2((m0 - M) * sl2);
-      const float f1 = (m1 == -INFINITY) ? 0.f : fast_exp2((m1 - M) * sl2);
-      const float lt = f0 * l0 + f1 * l1;
-      const float inv_l = lt > 0.f ? 1.f / lt : 0.f;
-      const float g0 = f0 * inv_l, g1 = f1 * inv_l;
-      const bool store = row < a.seq;
-      __nv_bfloat16* orow = a.out + (((int64_t)b * a.seq + row) * a.hq + head) * kHeadDim + cs0;
+        for (int i = 0; i < kCols / 4; ++i)
+          t8[i] = max3f(x[4 * i], x[4 * i + 1], fmaxf(x[4 * i + 2], x[4 * i + 3]));
 #pragma unroll
-      for (int c = 0; c < kCols / 32; ++c) {
-        uint32_t oa[32], ob[32];
-        tmem_ld32(lane_base + kColO + cs0 + 32 * c, oa);
-        tmem_ld32(lane_base + kColO + 128 + cs0 + 32 * c, ob);
-        tmem_wait_ld();
-        uint32_t pk[16];
+        for (int n2 = kCols / 4; n2 > 1; n2 = (n2 + 1) / 2) {
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
-          pk[i] = cvt_bf16x2(g0 * __uint_as_float(oa[2 * i]) + g1 * __uint_as_float(ob[2 * i]),
-                             g0 * __uint_as_float(oa[2 * i + 1]) + g1 * __uint_as_float(ob[2 * i + 1]));
-        if (store) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
-#pragma unroll
-          for (int v = 0; v < 4; ++v)
-            dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+          for (int i = 0; i < n2 / 2; ++i) t8[i] = fmaxf(t8[2 * i], t8[2 * i + 1]);
+          if (n2 & 1) t8[n2 / 2] = t8[n2 - 1];
         }
+        const float m_new = fmaxf(m, t8[0]);
+        // Rescale O_g (and l) when the max of some row of this warp grew by more than 2^8.
+        if (__any_sync(0xffffffffu, (m_new - m) * sl2 > kRescaleThreshold)) {
+          float f = 1.f;
+          if (m_new != -INFINITY) f = (m == -INFINITY) ? 0.f : fast_exp2((m - m_new) * sl2);
+          if (j > 0) {
+            // O_g holds this item's PVs up to tile g-1: wait for it, then scale in place
+            if (__all_sync(0xffffffffu,
+                           mbar_wait(pv_done, static_cast<uint32_t>((g - 1) & 1), a.status))) {
+              tc_fence_after();
+              const uint64_t f2 = pack_f32x2(f, f);
+#pragma unroll
+              for (int c = 0; c < 4; ++c) {
+                uint32_t o[32];
+                tmem_ld32(lane_base + og + 32 * c, o);
+                tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                  const uint64_t v = fmul2(pack_f32x2(__uint_as_float(o[2 * i]),
+                                                      __uint_as_float(o[2 * i + 1])), f2);
+                  const float2 w2 = unpack_f32x2(v);
+                  o[2 * i] = __float_as_uint(w2.x);
+                  o[2 * i + 1] = __float_as_uint(w2.y);
+                }
+                tmem_st32(lane_base + og + 32 * c, o);
+              }
+              tmem_wait_st();
+            } else {
+              ok = false;
+              continue;
+            }
+          }
+          l *= f;
+          if (m_new != -INFINITY) m = m_new;
+        }
+        // p = 2^(x * scale*log2e - m * scale*log2e), two lanes per instruction
+        const float ms = (m == -INFINITY) ? 0.f : m * sl2;
+        const uint64_t nms2 = pack_f32x2(-ms, -ms);
+        uint64_t acc0 = pack_f32x2(0.f, 0.f), acc1 = acc0;
+        uint32_t pk[kCols / 2];
+#pragma unroll
+        for (int i = 0; i < kCols / 2; ++i) {
+          const float2 e = unpack_f32x2(ffma2(pack_f32x2(x[2 * i], x[2 * i + 1]), sl2x2, nms2));
+          const float p0 = fast_exp2(e.x), p1 = fast_exp2(e.y);
+          if (i & 1)
+            acc1 = fadd2(acc1, pack_f32x2(p0, p1));
+          else
+            acc0 = fadd2(acc0, pack_f32x2(p0, p1));
+          pk[i] = cvt_bf16x2(p0, p1);
+        }
+        tmem_st32(lane_base + col_s(s) + cs0 / 2, pk);
+        const float2 a0 = unpack_f32x2(acc0), a1 = unpack_f32x2(acc1);
+        l += (a0.x + a0.y) + (a1.x + a1.y);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&p_ready[s * kGroups + wg]);
       }
-      if (store && wg == 0 && a.lse)
-        a.lse[((int64_t)b * a.hq + head) * a.seq + row] =
-            lt > 0.f ? (M * sl2 + log2f(lt)) * kLn2 : -INFINITY;
+      // ---------------------------------------------------------- epilogue of the item
+      // O = (2^(m_0 - M) O_0 + 2^(m_1 - M) O_1) / (2^(m_0 - M) l_0 + 2^(m_1 - M) l_1)
+      const bool fin =
+          ok && n > 0 && mbar_wait(pv_done, static_cast<uint32_t>((g - 1) & 1), a.status);
+      float* rd = red + (li & 1) * (kGroups * 2 * 128);
+      rd[(wg * 2 + 0) * 128 + r] = m;
+      rd[(wg * 2 + 1) * 128 + r] = l;
+      const bool all_fin = named_bar_and(1, kSoftmaxThreads, fin);
+      ok = ok && all_fin;
+      if (all_fin) {
+        tc_fence_after();
+        const float m0 = rd[0 * 128 + r], l0 = rd[1 * 128 + r];
+        const float m1 = rd[2 * 128 + r], l1 = rd[3 * 128 + r];
+        const float M = fmaxf(m0, m1);
+        const float f0 = (m0 == -INFINITY) ? 0.f : fast_exp2((m0 - M) * sl2);
+        const float f1 = (m1 == -INFINITY) ? 0.f : fast_exp2((m1 - M) * sl2);
+        const float lt = f0 * l0 + f1 * l1;
+        const float inv_l = lt > 0.f ? 1.f / lt : 0.f;
+        const float g0 = f0 * inv_l, g1 = f1 * inv_l;
+        uint32_t oa[2][32], ob[2][32];
+#pragma unroll
+        for (int c = 0; c < kCols / 32; ++c) {
+          tmem_ld32(lane_base + kColO + cs0 + 32 * c, oa[c]);
+          tmem_ld32(lane_base + kColO + 128 + cs0 + 32 * c, ob[c]);
+        }
+        tmem_wait_ld();
+        // O is in registers: the next item's first PV may overwrite it
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(o_free);
+        const bool store = row < a.seq;
+        __nv_bfloat16* orow =
+            a.out + (((int64_t)b * a.seq + row) * a.hq + head) * kHeadDim + cs0;
+#pragma unroll
+        for (int c = 0; c < kCols / 32; ++c) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            pk[i] = cvt_bf16x2(
+                g0 * __uint_as_float(oa[c][2 * i]) + g1 * __uint_as_float(ob[c][2 * i]),
+                g0 * __uint_as_float(oa[c][2 * i + 1]) + g1 * __uint_as_float(ob[c][2 * i + 1]));
+          if (store) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
+#pragma unroll
+            for (int v = 0; v < 4; ++v)
+              dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+          }
+        }
+        if (store && wg == 0 && a.lse)
+          a.lse[((int64_t)b * a.hq + head) * a.seq + row] =
+              lt > 0.f ? (M * sl2 + log2f(lt)) * kLn2 : -INFINITY;
+      }
     }
   }
   tc_fence_before();
@@ -472,11 +559,14 @@ int launch_prefill(const PrefillLaunch& l, cudaStream_t stream) {
     if (rc != PS_OK) return rc;
     attr_set[dev] = true;
   }
-  const int64_t grid = l.batch * l.hq * nq;
-  if (grid <= 0) return PS_OK;
-  if (grid > 0x7fffffffLL) return fail(PS_ERR_UNSUPPORTED, "prefill grid too large");
-  prefill_kernel<<<static_cast<unsigned>(grid), kThreads, kSmemBytes, stream>>>(mq, mk, mv, a);
-  return check_cuda(cudaGetLastError(), "prefill_kernel launch");
+  const int64_t items = l.batch * l.hq * nq;
+  if (items <= 0) return PS_OK;
+  if (items > 0x7fffffffLL) return fail(PS_ERR_UNSUPPORTED, "prefill problem too large");
+  // persistent: one CTA per SM walks items blockIdx.x, blockIdx.x + grid, ...
+  const int64_t grid = items < sm_count() ? items : sm_count();
+  return check_cuda(launch_pdl(prefill_kernel, dim3(static_cast<unsigned>(grid)), dim3(kThreads),
+                               kSmemBytes, stream, mq, mk, mv, a),
+                    "prefill_kernel launch");
 }
 
 }  // namespace ps
