@@ -350,10 +350,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int64_t row = (int64_t)qt * kBq + r;
       float m = -INFINITY;  // running max of raw scores (softmax scale > 0 keeps the order)
       float l = 0.f;
+      int2 ent_next = n > 0 ? reinterpret_cast<const int2*>(a.ent)[e0] : make_int2(0, 0);
       for (int j = 0; j < n; ++j, ++g) {
         const int s = static_cast<int>(g & 1);
-        const int kt = a.ent[2 * (e0 + j)];
-        const int flag = a.ent[2 * (e0 + j) + 1];
+        const int kt = ent_next.x;
+        const int flag = ent_next.y;
+        if (j + 1 < n) ent_next = reinterpret_cast<const int2*>(a.ent)[e0 + j + 1];
         // warp-uniform outcome: the tcgen05.ld/st below are warp-collective
         ok = ok && __all_sync(0xffffffffu, mbar_wait(&s_full[s],
                                                       static_cast<uint32_t>((g >> 1) & 1),
@@ -361,13 +363,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) continue;  // keep iterating: every warp must reach the epilogue barriers
         tc_fence_after();
         float x[kCols];
+        {
+          // both 32-column loads in flight before one wait
+          uint32_t raw[kCols / 32][32];
 #pragma unroll
-        for (int c = 0; c < kCols / 32; ++c) {
-          uint32_t raw[32];
-          tmem_ld32(lane_base + col_s(s) + cs0 + 32 * c, raw);
+          for (int c = 0; c < kCols / 32; ++c)
+            tmem_ld32(lane_base + col_s(s) + cs0 + 32 * c, raw[c]);
           tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) x[32 * c + i] = __uint_as_float(raw[i]);
+          for (int c = 0; c < kCols / 32; ++c)
+#pragma unroll
+            for (int i = 0; i < 32; ++i) x[32 * c + i] = __uint_as_float(raw[c][i]);
         }
         if (flag == PS_TILE_PARTIAL) {
           // visible keys of this row inside the slice: two intervals, as a 64-bit mask
@@ -553,7 +559,8 @@ int launch_prefill(const PrefillLaunch& l, cudaStream_t stream) {
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    rc = check_cuda(cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    rc = check_cuda(cudaFuncSetAttribute(prefill_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)kSmemBytes),
                     "cudaFuncSetAttribute(prefill_kernel)");
     if (rc != PS_OK) return rc;
