@@ -12,17 +12,17 @@
 // Persistent: one CTA per SM walks the (batch, query head, 128-row query tile) items
 // blockIdx.x, blockIdx.x + gridDim.x, ... (heaviest query tiles first); TMEM, barriers and
 // the TMA rings live across items, so the next item's Q tile and first QK^T overlap the
-// previous item's tail.  11 warps:
+// previous item's tail.  12 warps:
 //   warps 8, 9 - TMA producers: warp 8 loads the query tiles (two buffers) and the K tiles
 //             of the plan into a 2-stage ring, warp 9 the V tiles into a 2-stage ring (4-D
 //             tensor maps, 128-byte swizzle).  A query buffer is released after its item's
 //             last QK^T, a K stage when its QK^T completes, a V stage when its PV completes.
-//   warp 10 - allocates 512 TMEM columns; one lane issues the MMAs:
-//               S[buf] = Q K^T             (tcgen05.mma kind::f16, A and B from smem)
-//               O_g   += P_g V_g, g = 0, 1 (A = P from TMEM, B = V from smem, MN-major;
-//                                           P_g, V_g: keys [64g, 64g+64) of the tile)
-//             and commits them to mbarriers.  S of tile j+1 is issued before PV of tile j,
-//             so the tensor pipe computes the next scores while softmax runs.
+//   warp 10 - allocates 512 TMEM columns; one lane issues S[buf] = Q K^T (tcgen05.mma
+//             kind::f16, A and B from smem) as soon as K is in and the buffer's previous P
+//             has been consumed, so the next scores are computed while softmax runs.
+//   warp 11 - one lane issues O_g += P_g V_g, g = 0, 1 (A = P from TMEM, B = V from smem,
+//             MN-major; P_g, V_g: keys [64g, 64g+64) of the tile) as soon as that group's P
+//             and the V tile are in.  Each issuer commits its own MMAs to mbarriers.
 //   warps 0-7 - softmax, two warpgroups: row r lives in TMEM lane r; group g handles the
 //             64 score columns [64g, 64g+64) of every row as an independent online softmax
 //             (its own max m_g, sum l_g and accumulator O_g), so the groups never wait for
@@ -58,8 +58,9 @@ constexpr int kSoftmaxWarps = 4 * kGroups;
 constexpr int kSoftmaxThreads = kSoftmaxWarps * 32;
 constexpr int kKProducerWarp = kSoftmaxWarps;
 constexpr int kVProducerWarp = kSoftmaxWarps + 1;
-constexpr int kMmaWarp = kSoftmaxWarps + 2;
-constexpr int kThreads = (kSoftmaxWarps + 3) * 32;
+constexpr int kMmaWarp = kSoftmaxWarps + 2;   // issues QK^T, owns TMEM
+constexpr int kPvWarp = kSoftmaxWarps + 3;    // issues PV
+constexpr int kThreads = (kSoftmaxWarps + 4) * 32;
 constexpr int kQStages = 2;
 constexpr int kKStages = 2;
 constexpr int kVStages = 2;
@@ -126,8 +127,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* v_empty = v_full + kVStages;             // [kVStages]
   uint64_t* s_full = v_empty + kVStages;             // [2]
   uint64_t* p_ready = s_full + 2;                    // [2 buffers][kGroups]
-  uint64_t* pv_done = p_ready + 2 * kGroups;
-  uint64_t* o_free = pv_done + 1;
+  uint64_t* pv_done = p_ready + 2 * kGroups;          // [2]: PV of tile g -> g & 1
+  uint64_t* o_free = pv_done + 2;
   uint64_t* mma_done = o_free + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
 
@@ -160,9 +161,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&s_full[s], 1);
       for (int g = 0; g < kGroups; ++g) mbar_init(&p_ready[s * kGroups + g], 4);
     }
-    mbar_init(pv_done, 1);
+    mbar_init(&pv_done[0], 1);
+    mbar_init(&pv_done[1], 1);
     mbar_init(o_free, kSoftmaxWarps);
-    mbar_init(mma_done, 1);
+    mbar_init(mma_done, 2);  // both MMA issuers
     fence_mbar_init();
   }
   if (warp == kMmaWarp) {
@@ -236,47 +238,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_wait(&q_full[j % kQStages], (j / kQStages) & 1, a.status);
     }
   } else if (warp == kMmaWarp) {
-    // ------------------------------------------------------------ MMA issuer
+    // ------------------------------------------------------------ QK^T issuer
     if (lane == 0) {
       constexpr uint32_t idesc_qk = umma_idesc_bf16(128, 128, false);
-      constexpr uint32_t idesc_pv = umma_idesc_bf16(128, 128, true);
       const uint32_t k_addr = smem_u32(sK);
-      const uint32_t v_addr = smem_u32(sV);
-      // PV of global tile gg; the first PV of an item zero-initialises O_0 / O_1, after the
-      // previous item's epilogue has read them (o_free)
-      auto issue_pv = [&](int64_t gg, bool first_of_item, int item_li) -> bool {
-        const int s = static_cast<int>(gg & 1);
-        const int vs = static_cast<int>(gg % kVStages);
-        if (!mbar_wait(&v_full[vs], static_cast<uint32_t>((gg / kVStages) & 1), a.status))
-          return false;
-        if (first_of_item && item_li > 0 && !mbar_wait(o_free, (item_li - 1) & 1, a.status))
-          return false;
-        const uint32_t vb = v_addr + vs * kTileBytes;
-        // group g's keys [64g, 64g+64) accumulate into its own O_g, as soon as its P is in
-#pragma unroll
-        for (int g = 0; g < kGroups; ++g) {
-          if (!mbar_wait(&p_ready[s * kGroups + g], static_cast<uint32_t>((gg >> 1) & 1),
-                         a.status))
-            return false;
-          tc_fence_after();
-#pragma unroll
-          for (int kk = 4 * g; kk < 4 * g + 4; ++kk) {
-            // B = V[16 keys][128 d]: MN-major, 64-column halves 16 KB apart (LBO), 8-key
-            // groups 1024 B apart (SBO); 16 keys = 2048 B per step.
-            const uint64_t bdesc = umma_desc_sw128(vb + kk * 2048, kBoxBytes, 1024);
-            umma_ts(tmem + kColO + 128 * g, tmem + col_s(s) + kk * 8, bdesc, idesc_pv,
-                    (!first_of_item || kk > 4 * g) ? 1u : 0u);
-          }
-        }
-        umma_commit(&v_empty[vs]);
-        umma_commit(pv_done);
-        return true;
-      };
       int64_t g = 0;
       int li = 0;
       bool ok = true;
-      bool have_prev = false, prev_first = false;
-      int prev_li = 0;
       for (int64_t it = blockIdx.x; ok && it < n_items; it += gridDim.x, ++li) {
         int qt, b, head;
         item_of(it, qt, b, head);
@@ -295,7 +263,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           // S buffer s held P of tile g-2: its PV must have finished reading it
-          if (g >= 2 && !mbar_wait(pv_done, static_cast<uint32_t>((g - 2) & 1), a.status)) {
+          if (g >= 2 &&
+              !mbar_wait(&pv_done[s], static_cast<uint32_t>(((g >> 1) - 1) & 1), a.status)) {
             ok = false;
             break;
           }
@@ -312,16 +281,63 @@ __global__ void __launch_bounds__(kThreads, 1)
           umma_commit(&s_full[s]);
           umma_commit(&k_empty[ks]);
           if (j == n - 1) umma_commit(&q_empty[qb]);
-          if (have_prev && !issue_pv(g - 1, prev_first, prev_li)) {
+        }
+      }
+      umma_commit(mma_done);  // arrives once this thread's MMAs have all completed
+      mbar_wait(mma_done, 0, a.status);
+    }
+  } else if (warp == kPvWarp) {
+    // ------------------------------------------------------------ PV issuer
+    // Separate from the QK^T issuer, so PV of a tile goes out as soon as its P and V are in,
+    // instead of queueing behind the next tile's QK^T (which waits for an older PV).
+    if (lane == 0) {
+      constexpr uint32_t idesc_pv = umma_idesc_bf16(128, 128, true);
+      const uint32_t v_addr = smem_u32(sV);
+      int64_t g = 0;
+      int li = 0;
+      bool ok = true;
+      for (int64_t it = blockIdx.x; ok && it < n_items; it += gridDim.x, ++li) {
+        int qt, b, head;
+        item_of(it, qt, b, head);
+        const int n = a.off[qt + 1] - a.off[qt];
+        for (int j = 0; j < n; ++j, ++g) {
+          const int s = static_cast<int>(g & 1);
+          const int vs = static_cast<int>(g % kVStages);
+          if (!mbar_wait(&v_full[vs], static_cast<uint32_t>((g / kVStages) & 1), a.status)) {
             ok = false;
             break;
           }
-          have_prev = true;
-          prev_first = (j == 0);
-          prev_li = li;
+          // the first PV of an item zero-initialises O_0 / O_1, after the previous item's
+          // epilogue has read them
+          if (j == 0 && li > 0 && !mbar_wait(o_free, (li - 1) & 1, a.status)) {
+            ok = false;
+            break;
+          }
+          const uint32_t vb = v_addr + vs * kTileBytes;
+          // group gr's keys [64gr, 64gr+64) accumulate into its own O_gr, as soon as its P is in
+#pragma unroll
+          for (int gr = 0; gr < kGroups; ++gr) {
+            if (!mbar_wait(&p_ready[s * kGroups + gr], static_cast<uint32_t>((g >> 1) & 1),
+                           a.status)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 4 * gr; kk < 4 * gr + 4; ++kk) {
+              // B = V[16 keys][128 d]: MN-major, 64-column halves 16 KB apart (LBO), 8-key
+              // groups 1024 B apart (SBO); 16 keys = 2048 B per step.
+              const uint64_t bdesc = umma_desc_sw128(vb + kk * 2048, kBoxBytes, 1024);
+              umma_ts(tmem + kColO + 128 * gr, tmem + col_s(s) + kk * 8, bdesc, idesc_pv,
+                      (j > 0 || kk > 4 * gr) ? 1u : 0u);
+            }
+          }
+          if (!ok) break;
+          umma_commit(&v_empty[vs]);
+          // one completion barrier per S buffer keeps every waiter within one phase of it
+          umma_commit(&pv_done[s]);
         }
       }
-      if (ok && have_prev) issue_pv(g - 1, prev_first, prev_li);
       umma_commit(mma_done);
       mbar_wait(mma_done, 0, a.status);
     }
@@ -402,8 +418,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (m_new != -INFINITY) f = (m == -INFINITY) ? 0.f : fast_exp2((m - m_new) * sl2);
           if (j > 0) {
             // O_g holds this item's PVs up to tile g-1: wait for it, then scale in place
-            if (__all_sync(0xffffffffu,
-                           mbar_wait(pv_done, static_cast<uint32_t>((g - 1) & 1), a.status))) {
+            const int64_t gp = g - 1;
+            if (__all_sync(0xffffffffu, mbar_wait(&pv_done[gp & 1],
+                                                  static_cast<uint32_t>((gp >> 1) & 1),
+                                                  a.status))) {
               tc_fence_after();
               const uint64_t f2 = pack_f32x2(f, f);
 #pragma unroll
@@ -455,8 +473,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // ---------------------------------------------------------- epilogue of the item
       // O = (2^(m_0 - M) O_0 + 2^(m_1 - M) O_1) / (2^(m_0 - M) l_0 + 2^(m_1 - M) l_1)
-      const bool fin =
-          ok && n > 0 && mbar_wait(pv_done, static_cast<uint32_t>((g - 1) & 1), a.status);
+      const bool fin = ok && n > 0 &&
+                       mbar_wait(&pv_done[(g - 1) & 1], static_cast<uint32_t>(((g - 1) >> 1) & 1),
+                                 a.status);
       float* rd = red + (li & 1) * (kGroups * 2 * 128);
       rd[(wg * 2 + 0) * 128 + r] = m;
       rd[(wg * 2 + 1) * 128 + r] = l;
