@@ -137,22 +137,30 @@ def _barrier(world):
         dist.barrier()
 
 
-def _max_over_ranks(x: float, world: int) -> float:
+def _max_over_ranks(x: float, world: int, device: str = "cuda") -> float:
+    """Step time of the job: the slowest rank's."""
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
 
-def _sum_over_ranks(x: float, world: int) -> float:
+def _sum_over_ranks(x: float, world: int, device: str = "cuda") -> float:
+    """Work of the whole job: every rank decodes its own batch (weak scaling)."""
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.SUM)
     return float(t.item())
+
+
+def rank_seed(index: int, rank: int, k: int) -> int:
+    """Seed of input stream k of workload `index` on `rank`: every rank draws its own
+    sequences (the batch is sharded, not replicated)."""
+    return synth.seed_for(index, 10 * rank + k)
 
 
 # ------------------------------------------------------------- decode setup
@@ -167,7 +175,7 @@ class DecodeWorkload:
         self.dev = dev
         Bn, hq, hkv, lp, w = wl.batch, wl.n_q_heads, wl.n_kv_heads, wl.l_prefix, wl.window
         self.params = B.make_params(hq, hkv, D, lp, w, wl.rope_theta)
-        s = lambda k: synth.seed_for(wl.index, 10 * rank + k)  # noqa: E731
+        s = lambda k: rank_seed(wl.index, rank, k)  # noqa: E731
         self.pos_start = synth.uniform_positions(Bn, wl.pos_lo, wl.pos_hi, s(0), dev)
         self.cache = PrefixSlidingCache(Bn, hkv, lp, w, D, dev, fill=None)
         st = torch.zeros(1, dtype=torch.int32, device=dev)
@@ -233,26 +241,46 @@ def run_decode(args, world, rank, dev):
     for i in range(W):
         step(i)
     torch.cuda.synchronize()
-    sampler = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
-    if sampler:
-        sampler.start()
-    # soak: a few more untimed steps so the clocks are sampled under this load
-    for _ in range(3):
-        for i in range(W):
-            step(i)
+    # per-launch duration of ps_decode_attn (decode + merge), CUDA events on the stream
+    work.q.copy_(work.q_raw)
     ev_dec = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(K)]
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    _barrier(world)
-    torch.cuda.synchronize()
-    t_host0 = time.perf_counter()
-    ev0.record(stream)
     for j in range(K):
         i = W + j
         work.append(i)
         ev_dec[j][0].record(stream)
         work.decode(i)
         ev_dec[j][1].record(stream)
+    torch.cuda.synchronize()
+    work.q.copy_(work.q_raw)
+    graph = None
+    if not args.no_graph:
+        # the K timed steps as one CUDA graph (kernel launches only; programmatic
+        # dependencies between append, decode and merge are kept as graph edges)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            for j in range(K):
+                step(W + j)
+        torch.cuda.synchronize()
+    sampler = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
+    if sampler:
+        sampler.start()
+    # soak: the same work once more, untimed, so the clocks are sampled under this load
+    if graph is not None:
+        graph.replay()
+    else:
+        for j in range(K):
+            step(W + j)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    _barrier(world)
+    torch.cuda.synchronize()
+    t_host0 = time.perf_counter()
+    ev0.record(stream)
+    if graph is not None:
+        graph.replay()
+    else:
+        for j in range(K):
+            step(W + j)
     ev1.record(stream)
     torch.cuda.synchronize()
     t_host1 = time.perf_counter()
@@ -288,6 +316,7 @@ def run_decode(args, world, rank, dev):
                    "l_prefix": wl.l_prefix, "window": wl.window,
                    "positions": f"U[{wl.pos_lo},{wl.pos_hi}]", "layers": 1,
                    "step": "ps_kv_append_rope + ps_decode_attn",
+                   "launch": "CUDA graph of the timed steps" if graph is not None else "eager",
                    "l2": "inputs larger than L2 (275 MB of K/V read per step vs 126 MB L2)",
                    "parallelism": f"dp{world} (independent sequences, no collective)"},
         "roofline": roof,
@@ -457,6 +486,51 @@ def run_full_attention(work: DecodeWorkload, steps: int = 16, warmup: int = 3):
             "ms_per_step": round(ms, 4), "tok_per_s": round(Bn / (ms / 1e3), 1),
             "kv_gb_per_step": round(kv_bytes / 1e9, 3),
             "gbs": round(kv_bytes / (ms / 1e3) / 1e9, 1)}
+
+
+# ------------------------------------------------------------- latency leg
+def run_latency(dev, steps: int = 256, warmup: int = 8):
+    """Single-sequence decode latency: batch 1, 16/2/128, L_prefix 100, W 512, positions past
+    the point where the window slides (612); one step = append + decode, replayed as a CUDA
+    graph and also launched eagerly."""
+    wl = synth.WORKLOADS["decode_b1_w512"]
+    import dataclasses
+    wl = dataclasses.replace(wl, pos_lo=2047 - steps - warmup, pos_hi=2047 - steps - warmup)
+    n = steps + warmup
+    work = DecodeWorkload(wl, dev, 0, n)
+    stream = torch.cuda.current_stream()
+
+    def step(i):
+        work.append(i)
+        work.decode(i)
+
+    for i in range(warmup):
+        step(i)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(warmup, n):
+        step(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    eager_us = e0.elapsed_time(e1) / steps * 1e3
+    work.q.copy_(work.q_raw)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for i in range(warmup, n):
+            step(i)
+    g.replay()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    g.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    assert work.status.item() == 0
+    graph_us = e0.elapsed_time(e1) / steps * 1e3
+    return {"leg": "latency", "workload": wl.name, "positions": f"{wl.pos_lo + warmup}.."
+            f"{wl.pos_lo + n - 1}", "visible_keys": wl.l_prefix + wl.window,
+            "step_us_graph": round(graph_us, 2), "step_us_eager": round(eager_us, 2),
+            "kernels_per_step": work.kernels_per_step()}
 
 
 # ------------------------------------------------------ long-trace sweep leg
@@ -698,7 +772,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=8)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--leg", default="main", choices=["main", "prefill", "sweep", "stack"],
+    ap.add_argument("--no-graph", action="store_true",
+                    help="launch the timed steps one by one instead of as a CUDA graph")
+    ap.add_argument("--leg", default="main", choices=["main", "prefill", "sweep", "stack", "latency"],
                     help="main: the driver's line; prefill/sweep/stack: one extra workload")
     ap.add_argument("--stack-batch", type=int, default=1024)
     ap.add_argument("--stack-distinct", type=int, default=6)
@@ -722,6 +798,8 @@ def main():
             res = {"leg": "prefill", **run_prefill(dev, steps=args.steps, warmup=args.warmup)}
         elif args.leg == "sweep":
             res = run_sweep(dev)
+        elif args.leg == "latency":
+            res = run_latency(dev)
         else:
             res = run_stack(dev, args.stack_batch, args.stack_distinct)
         if rank == 0:

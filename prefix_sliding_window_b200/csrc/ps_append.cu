@@ -65,22 +65,6 @@ __global__ void __launch_bounds__(kAppendThreads) append_rope_kernel(const Appen
     if (threadIdx.x == 0 && a.status) atomicOr(a.status, PS_DEV_POS_RANGE);
     return;
   }
-  if (threadIdx.x < kHalf) {
-    // angle = p * inv_f[i] in float64, reduced to [-pi, pi] by subtracting k * 2*pi with
-    // 2*pi split in two parts (Cody-Waite): the first has 24 significant bits, so k * part1
-    // is exact for |k| < 2^29; the second carries the rest of 2*pi in double precision.
-    // The remainder is small, so the fp32 sincosf of it is accurate to ~1e-7.
-    const double ang = double(p) * a.inv_freq[threadIdx.x];
-    const double k = rint(ang * 0.15915494309189535);
-    double red = fma(-k, 6.2831854820251465, ang);
-    red = fma(-k, -1.748455600074497e-07, red);
-    float sf, cf;
-    sincosf(static_cast<float>(red), &sf, &cf);
-    s_cos[threadIdx.x] = cf;
-    s_sin[threadIdx.x] = sf;
-  }
-  __syncthreads();
-
   // where this token's K/V row goes (or nowhere, if a later token of this call owns it)
   const __nv_bfloat16* k_src = static_cast<const __nv_bfloat16*>(a.k_new) + tok * a.hkv * kHeadDim;
   const __nv_bfloat16* v_src = static_cast<const __nv_bfloat16*>(a.v_new) + tok * a.hkv * kHeadDim;
@@ -98,43 +82,71 @@ __global__ void __launch_bounds__(kAppendThreads) append_rope_kernel(const Appen
     row_stride_rows = a.w;
     row = (p - a.lp) % a.w;
   }
+  __nv_bfloat16* qb = static_cast<__nv_bfloat16*>(a.q) + tok * a.hq * kHeadDim;
 
-  // K: rotate; V: copy.  Items: hkv heads x kChunks rotate items, hkv x 16 copy items.
-  const int n_k = a.hkv * kChunks;
-  const int n_v = a.hkv * (kHeadDim / 8);
-  if (k_dst_base != nullptr) {
-    for (int it = threadIdx.x; it < n_k + n_v; it += blockDim.x) {
-      if (it < n_k) {
-        const int h = it / kChunks, c = it % kChunks;
-        const __nv_bfloat16* src = k_src + h * kHeadDim;
-        const uint4 x1 = *reinterpret_cast<const uint4*>(src + 8 * c);
-        const uint4 x2 = *reinterpret_cast<const uint4*>(src + kHalf + 8 * c);
-        uint4 y1, y2;
-        rotate8(x1, x2, s_cos + 8 * c, s_sin + 8 * c, y1, y2);
-        __nv_bfloat16* dst = k_dst_base + ((b * a.hkv + h) * row_stride_rows + row) * kHeadDim;
-        *reinterpret_cast<uint4*>(dst + 8 * c) = y1;
-        *reinterpret_cast<uint4*>(dst + kHalf + 8 * c) = y2;
-      } else {
-        const int j = it - n_k;
-        const int h = j / (kHeadDim / 8), c = j % (kHeadDim / 8);
-        const uint4 x = *reinterpret_cast<const uint4*>(v_src + h * kHeadDim + 8 * c);
-        __nv_bfloat16* dst = v_dst_base + ((b * a.hkv + h) * row_stride_rows + row) * kHeadDim;
-        *reinterpret_cast<uint4*>(dst + 8 * c) = x;
-      }
+  // Work items: K rotate (hkv x kChunks), V copy (hkv x 16), q rotate (hq x kChunks).
+  const int n_k = k_dst_base ? a.hkv * kChunks : 0;
+  const int n_v = k_dst_base ? a.hkv * (kHeadDim / 8) : 0;
+  const int n_q = a.q ? a.hq * kChunks : 0;
+  const int n_items = n_k + n_v + n_q;
+  auto load = [&](int it, uint4& x1, uint4& x2) {
+    if (it < n_k) {
+      const __nv_bfloat16* src = k_src + (it / kChunks) * kHeadDim + 8 * (it % kChunks);
+      x1 = *reinterpret_cast<const uint4*>(src);
+      x2 = *reinterpret_cast<const uint4*>(src + kHalf);
+    } else if (it < n_k + n_v) {
+      const int j = it - n_k;
+      x1 = *reinterpret_cast<const uint4*>(v_src + (j / 16) * kHeadDim + 8 * (j % 16));
+    } else {
+      const int j = it - n_k - n_v;
+      const __nv_bfloat16* src = qb + (j / kChunks) * kHeadDim + 8 * (j % kChunks);
+      x1 = *reinterpret_cast<const uint4*>(src);
+      x2 = *reinterpret_cast<const uint4*>(src + kHalf);
     }
+  };
+  // the first item's inputs are fetched before the angles, so both latencies overlap
+  uint4 x1 = make_uint4(0, 0, 0, 0), x2 = x1;
+  if (threadIdx.x < n_items) load(threadIdx.x, x1, x2);
+
+  if (threadIdx.x < kHalf) {
+    // angle = p * inv_f[i] in float64, reduced to [-pi, pi] by subtracting k * 2*pi with
+    // 2*pi split in two parts (Cody-Waite): the first has 24 significant bits, so k * part1
+    // is exact for |k| < 2^29; the second carries the rest of 2*pi in double precision.
+    // The remainder is small, so the fp32 sincosf of it is accurate to ~1e-7.
+    const double ang = double(p) * a.inv_freq[threadIdx.x];
+    const double k = rint(ang * 0.15915494309189535);
+    double red = fma(-k, 6.2831854820251465, ang);
+    red = fma(-k, -1.748455600074497e-07, red);
+    float sf, cf;
+    sincosf(static_cast<float>(red), &sf, &cf);
+    s_cos[threadIdx.x] = cf;
+    s_sin[threadIdx.x] = sf;
   }
-  // q rotated in place at the token's own absolute position
-  if (a.q != nullptr) {
-    __nv_bfloat16* qb = static_cast<__nv_bfloat16*>(a.q) + tok * a.hq * kHeadDim;
-    for (int it = threadIdx.x; it < a.hq * kChunks; it += blockDim.x) {
+  __syncthreads();
+
+  for (int it = threadIdx.x; it < n_items; it += blockDim.x) {
+    if (it != threadIdx.x) load(it, x1, x2);
+    if (it < n_k) {
       const int h = it / kChunks, c = it % kChunks;
-      __nv_bfloat16* src = qb + h * kHeadDim;
-      const uint4 x1 = *reinterpret_cast<const uint4*>(src + 8 * c);
-      const uint4 x2 = *reinterpret_cast<const uint4*>(src + kHalf + 8 * c);
       uint4 y1, y2;
       rotate8(x1, x2, s_cos + 8 * c, s_sin + 8 * c, y1, y2);
-      *reinterpret_cast<uint4*>(src + 8 * c) = y1;
-      *reinterpret_cast<uint4*>(src + kHalf + 8 * c) = y2;
+      __nv_bfloat16* dst = k_dst_base + ((b * a.hkv + h) * row_stride_rows + row) * kHeadDim;
+      *reinterpret_cast<uint4*>(dst + 8 * c) = y1;
+      *reinterpret_cast<uint4*>(dst + kHalf + 8 * c) = y2;
+    } else if (it < n_k + n_v) {
+      const int j = it - n_k;
+      const int h = j / 16, c = j % 16;
+      __nv_bfloat16* dst = v_dst_base + ((b * a.hkv + h) * row_stride_rows + row) * kHeadDim;
+      *reinterpret_cast<uint4*>(dst + 8 * c) = x1;
+    } else {
+      // q rotated in place at the token's own absolute position
+      const int j = it - n_k - n_v;
+      const int h = j / kChunks, c = j % kChunks;
+      uint4 y1, y2;
+      rotate8(x1, x2, s_cos + 8 * c, s_sin + 8 * c, y1, y2);
+      __nv_bfloat16* dst = qb + h * kHeadDim;
+      *reinterpret_cast<uint4*>(dst + 8 * c) = y1;
+      *reinterpret_cast<uint4*>(dst + kHalf + 8 * c) = y2;
     }
   }
 }

@@ -534,22 +534,43 @@ __global__ void __launch_bounds__(128)
     auto empty_cta = [&](int c) {
       return maybe_empty && total * c / grid == total * (c + 1) / grid;
     };
-    float M = -INFINITY;
-    for (int c = c_lo; c <= c_hi; ++c)
-      if (!empty_cta(c)) M = fmaxf(M, ws_lse[(unit + c) * 8 + hh]);
-    if (M != -INFINITY) {
-      float wsum = 0.f;
-      for (int c = c_lo; c <= c_hi; ++c) {
-        if (empty_cta(c)) continue;
-        const int64_t slot = (unit + c) * 8 + hh;
-        const float f = fast_exp2(ws_lse[slot] - M);
-        const float4 v = reinterpret_cast<const float4*>(ws_o + slot * kHeadDim)[lane];
-        wsum += f;
-        acc.x += f * v.x;
-        acc.y += f * v.y;
-        acc.z += f * v.z;
-        acc.w += f * v.w;
+    // online combine, four pieces per round: their lse and o are loaded together
+    float M = -INFINITY, wsum = 0.f;
+    for (int c0 = c_lo; c0 <= c_hi; c0 += 4) {
+      float lv[4];
+      float4 ov[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int c = c0 + k;
+        lv[k] = -INFINITY;
+        ov[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (c <= c_hi && !empty_cta(c)) {
+          const int64_t slot = (unit + c) * 8 + hh;
+          lv[k] = ws_lse[slot];
+          ov[k] = reinterpret_cast<const float4*>(ws_o + slot * kHeadDim)[lane];
+        }
       }
+      const float mc = fmaxf(fmaxf(lv[0], lv[1]), fmaxf(lv[2], lv[3]));
+      const float Mn = fmaxf(M, mc);
+      if (Mn == -INFINITY) continue;
+      const float corr = (M == -INFINITY) ? 0.f : fast_exp2(M - Mn);
+      wsum *= corr;
+      acc.x *= corr;
+      acc.y *= corr;
+      acc.z *= corr;
+      acc.w *= corr;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float f = (lv[k] == -INFINITY) ? 0.f : fast_exp2(lv[k] - Mn);
+        wsum += f;
+        acc.x += f * ov[k].x;
+        acc.y += f * ov[k].y;
+        acc.z += f * ov[k].z;
+        acc.w += f * ov[k].w;
+      }
+      M = Mn;
+    }
+    if (M != -INFINITY) {
       const float inv = 1.f / wsum;
       acc.x *= inv;
       acc.y *= inv;
