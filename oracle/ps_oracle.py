@@ -65,6 +65,7 @@ __all__ = [
     "decode_reference",
     "full_attention_decode",
     "prefill_reference",
+    "prefill_backward_reference",
     "tile_plan",
     "tile_counts",
     "kv_bytes_per_token",
@@ -250,6 +251,78 @@ def prefill_reference(Q: np.ndarray, K: np.ndarray, V: np.ndarray, l_prefix: int
         outs.append(o)
         lses.append(l)
     return np.stack(outs), np.stack(lses)
+
+
+def prefill_backward_reference(Q: np.ndarray, K: np.ndarray, V: np.ndarray, dO: np.ndarray,
+                               l_prefix: int, window: int, scale: float,
+                               rows: Optional[Sequence[int]] = None,
+                               keys: Optional[Sequence[int]] = None):
+    """Gradients of the masked prefill with respect to Q, K and V.
+
+    The truncated-backprop trainer ("Prefix Sliding 完全拆解", §截断回传) back-propagates
+    through the same masked attention it ran forward; this is the chain rule of
+    O_i = sum_{j in V(i)} softmax_j(s_ij) V_j with s_ij = scale * <Q_i, K_j>, written out
+    per query head h (KV head h // g):
+
+        P_ij  = softmax over j in V(i) of s_ij              (0 for j not in V(i))
+        dV_j  = sum_i P_ij dO_i                             (summed over the heads of a group)
+        dP_ij = <dO_i, V_j>
+        D_i   = sum_j P_ij dP_ij  (= <dO_i, O_i>)
+        dS_ij = P_ij (dP_ij - D_i)
+        dQ_i  = scale * sum_j dS_ij K_j
+        dK_j  = scale * sum_i dS_ij Q_i                     (summed over the heads of a group)
+
+    Q, dO: [S, Hq, D]; K, V: [S, Hkv, D] (already rotated).  ``rows`` selects the query
+    rows of dQ and ``keys`` the key rows of dK/dV to return (default: all).  Each head's
+    masked score matrix is formed densely over the query rows that are needed (the
+    selected rows plus every row that sees a selected key) and the keys [0, last row].
+    Returns (dQ [R, Hq, D], dK [K, Hkv, D], dV [K, Hkv, D]) in float64.
+    """
+    Q = np.asarray(Q, np.float64)
+    K = np.asarray(K, np.float64)
+    V = np.asarray(V, np.float64)
+    dO = np.asarray(dO, np.float64)
+    S, hq, d = Q.shape
+    hkv = K.shape[1]
+    g = hq // hkv
+    rows = np.arange(S) if rows is None else np.asarray(rows, np.int64)
+    keys = np.arange(S) if keys is None else np.asarray(keys, np.int64)
+    # every query row that sees one of the selected keys: i >= j, and i < j + W unless
+    # j is a prefix key
+    need = np.zeros(S, bool)
+    need[rows] = True
+    for j in keys:
+        hi = S if j < l_prefix else min(S, j + window)
+        need[j:hi] = True
+    R = np.nonzero(need)[0]
+    if R.size == 0:
+        return (np.zeros((0, hq, d)), np.zeros((len(keys), hkv, d)),
+                np.zeros((len(keys), hkv, d)))
+    ncol = int(R.max()) + 1
+    j = np.arange(ncol)
+    vis = (j[None, :] <= R[:, None]) & ((j[None, :] < l_prefix) | (j[None, :] > R[:, None] - window))
+    where_row = {int(i): r for r, i in enumerate(R)}
+    sel_rows = np.array([where_row[int(i)] for i in rows], np.int64)
+    dQ = np.zeros((len(rows), hq, d))
+    dK = np.zeros((len(keys), hkv, d))
+    dV = np.zeros((len(keys), hkv, d))
+    for h in range(hq):
+        kv = h // g
+        Kh, Vh = K[:ncol, kv], V[:ncol, kv]
+        s = np.where(vis, (Q[R, h] @ Kh.T) * scale, -np.inf)
+        m = s.max(axis=1, keepdims=True)
+        e = np.exp(s - m)
+        P = e / e.sum(axis=1, keepdims=True)
+        O = P @ Vh
+        dP = dO[R, h] @ Vh.T
+        Dr = (dO[R, h] * O).sum(axis=1, keepdims=True)
+        dS = P * (dP - Dr)
+        dQ[:, h] = scale * (dS[sel_rows] @ Kh)
+        kin = keys < ncol
+        kk = keys[kin]
+        dK[kin, kv] += scale * (dS[:, kk].T @ Q[R, h])
+        dV[kin, kv] += P[:, kk].T @ dO[R, h]
+    return dQ, dK, dV
 
 
 # ------------------------------------------------------------------- tile plan

@@ -333,3 +333,82 @@ def test_tile_plan_flags_from_interval_counts(seq, lp, w, bq, bk):
     want = [(q, k, O.TILE_FULL if c == bq * bk else O.TILE_PARTIAL)
             for q in range(cnt.shape[0]) for k in range(cnt.shape[1]) for c in [cnt[q, k]] if c > 0]
     assert [tuple(r) for r in O.tile_plan(seq, lp, w, bq, bk).tolist()] == want
+
+
+# ------------------------------------------------------- masked prefill backward
+def _autograd_grads(Q, K, V, dO, lp, w, scale):
+    """Gradients from torch autograd through SDPA in float64 with an explicit boolean
+    mask built from the 0-indexed eq. A(i) and torch's own GQA expansion."""
+    S = Q.shape[0]
+    i = torch.arange(S)[:, None]
+    j = torch.arange(S)[None, :]
+    mask = (j <= i) & ((j < lp) | (j > i - w))
+    tq = torch.from_numpy(Q).permute(1, 0, 2)[None].requires_grad_(True)
+    tk = torch.from_numpy(K).permute(1, 0, 2)[None].requires_grad_(True)
+    tv = torch.from_numpy(V).permute(1, 0, 2)[None].requires_grad_(True)
+    out = torch.nn.functional.scaled_dot_product_attention(
+        tq, tk, tv, attn_mask=mask, scale=scale, enable_gqa=True)
+    out.backward(torch.from_numpy(dO).permute(1, 0, 2)[None])
+    return [t.grad[0].permute(1, 0, 2).numpy() for t in (tq, tk, tv)]
+
+
+@pytest.mark.parametrize("S,lp,w,hq,hkv", [(24, 3, 5, 4, 2), (30, 0, 7, 6, 2), (17, 17, 1, 2, 1),
+                                          (20, 4, 40, 8, 1), (33, 2, 1, 3, 3)])
+def test_prefill_backward_matches_autograd(S, lp, w, hq, hkv):
+    d, scale = 8, 0.37
+    Q, K, V = _rand((S, hq, d), 40), _rand((S, hkv, d), 41), _rand((S, hkv, d), 42)
+    dO = _rand((S, hq, d), 43)
+    dq, dk, dv = O.prefill_backward_reference(Q, K, V, dO, lp, w, scale)
+    wq, wk, wv = _autograd_grads(Q, K, V, dO, lp, w, scale)
+    for got, want in ((dq, wq), (dk, wk), (dv, wv)):
+        np.testing.assert_allclose(got, want, rtol=0, atol=1e-11)
+
+
+def test_prefill_backward_central_differences_of_forward():
+    """Brute force: d/dx of L = sum(dO * O) by central differences of the forward oracle,
+    for every element of a tiny Q, K and V."""
+    S, lp, w, hq, hkv, d, scale = 7, 2, 3, 2, 1, 3, 0.8
+    Q, K, V = _rand((S, hq, d), 44), _rand((S, hkv, d), 45), _rand((S, hkv, d), 46)
+    dO = _rand((S, hq, d), 47)
+    dq, dk, dv = O.prefill_backward_reference(Q, K, V, dO, lp, w, scale)
+
+    def loss(q, k, v):
+        return float((O.prefill_reference(q, k, v, lp, w, scale)[0] * dO).sum())
+
+    eps = 1e-6
+    for which, grad in ((0, dq), (1, dk), (2, dv)):
+        args = [Q, K, V]
+        num = np.zeros_like(grad)
+        for idx in np.ndindex(*grad.shape):
+            hi = [a.copy() for a in args]
+            lo = [a.copy() for a in args]
+            hi[which][idx] += eps
+            lo[which][idx] -= eps
+            num[idx] = (loss(*hi) - loss(*lo)) / (2 * eps)
+        np.testing.assert_allclose(grad, num, rtol=0, atol=1e-7)
+
+
+def test_prefill_backward_closed_form_sums():
+    """Each softmax row sums to one, so sum_j dV_j = sum_i dO_i over a KV head's group,
+    and each dS row sums to zero, so sum_j dK_j = 0."""
+    S, lp, w, hq, hkv, d = 50, 6, 11, 6, 2, 16
+    Q, K, V = _rand((S, hq, d), 48), _rand((S, hkv, d), 49), _rand((S, hkv, d), 50)
+    dO = _rand((S, hq, d), 51)
+    _, dk, dv = O.prefill_backward_reference(Q, K, V, dO, lp, w, 0.25)
+    np.testing.assert_allclose(dk.sum(axis=0), 0.0, rtol=0, atol=1e-12)
+    want = dO.reshape(S, hkv, hq // hkv, d).sum(axis=(0, 2))
+    np.testing.assert_allclose(dv.sum(axis=0), want, rtol=0, atol=1e-12)
+
+
+def test_prefill_backward_selected_rows_and_keys():
+    """Selecting rows/keys returns exactly those rows of the full gradients (prefix keys,
+    window keys, the last key; first, middle and last rows)."""
+    S, lp, w, hq, hkv, d = 40, 5, 8, 4, 2, 8
+    Q, K, V = _rand((S, hq, d), 52), _rand((S, hkv, d), 53), _rand((S, hkv, d), 54)
+    dO = _rand((S, hq, d), 55)
+    fq, fk, fv = O.prefill_backward_reference(Q, K, V, dO, lp, w, 0.5)
+    rows, keys = [0, 17, 39], [0, 4, 5, 20, 39]
+    sq, sk, sv = O.prefill_backward_reference(Q, K, V, dO, lp, w, 0.5, rows=rows, keys=keys)
+    np.testing.assert_allclose(sq, fq[rows], rtol=0, atol=1e-13)
+    np.testing.assert_allclose(sk, fk[keys], rtol=0, atol=1e-13)
+    np.testing.assert_allclose(sv, fv[keys], rtol=0, atol=1e-13)
