@@ -431,7 +431,46 @@ def run_prefill(dev, steps: int = 10, warmup: int = 3):
             "tflops_computed_tiles": round(computed / med / 1e12, 1),
             "unmasked_gflop": round(flops / 1e9, 1), "computed_gflop": round(computed / 1e9, 1),
             "tiles_per_head": {"full": n_full, "partial": n_part, "skip": nq * nq - n},
-            "launches_per_call": 2, "inputs": "Q 235 MB + K,V 67 MB per call (> L2)"}
+            "launches_per_call": 2, "inputs": "Q 235 MB + K,V 67 MB per call (> L2)",
+            "backward": run_prefill_bwd(dev, params, wl, q, k, v, out, lse, st, pairs, n,
+                                        steps, warmup, peaks)}
+
+
+def run_prefill_bwd(dev, params, wl, q, k, v, out, lse, st, pairs, n_tiles, steps, warmup, peaks):
+    """Backward of the same prefill (dQ, dK, dV from dO, the forward's output and lse).
+    Algorithmic FLOPs = 10 * D per visible pair per query head (the score recompute, dP,
+    dV, dK and dQ products: 2.5x the forward); the computed-tile figure counts the 7
+    products per planned tile the two-kernel design runs (S and dP are formed twice)."""
+    from prefix_sliding_window_b200 import binding as B
+    Bn, S, hq, hkv = wl.batch, wl.seq, wl.n_q_heads, wl.n_kv_heads
+    do = synth.normal_bf16((Bn, S, hq, D), synth.seed_for(3, 4), dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = torch.empty(B.ps_prefill_bwd_workspace_bytes(params, Bn, S), dtype=torch.uint8,
+                     device=dev)
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        B.ps_masked_prefill_attn_bwd(params, q, k, v, out, do, lse, Bn, S, dq, dk, dv, ws, st)
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(steps)]
+    for a, b in evs:
+        a.record(stream)
+        B.ps_masked_prefill_attn_bwd(params, q, k, v, out, do, lse, Bn, S, dq, dk, dv, ws, st)
+        b.record(stream)
+    torch.cuda.synchronize()
+    assert st.item() == 0, f"device status {st.item()}"
+    ms = [a.elapsed_time(b) for a, b in evs]
+    med = statistics.median(ms) / 1e3
+    flops = 10 * D * pairs * hq * Bn
+    computed = 14 * D * 128 * 128 * n_tiles * hq * Bn
+    tflops = flops / med / 1e12
+    return {"ms": round(med * 1e3, 4), "ms_p10": round(float(np.percentile(ms, 10)), 4),
+            "ms_p90": round(float(np.percentile(ms, 90)), 4),
+            "tflops_algorithmic": round(tflops, 1), "unit": "TFLOP/s",
+            "frac": round(tflops / peaks["bf16_tflops"], 4),
+            "tflops_computed": round(computed / med / 1e12, 1),
+            "algorithmic_gflop": round(flops / 1e9, 1), "computed_gflop": round(computed / 1e9, 1),
+            "launches_per_call": 4}
 
 
 # -------------------------------------------------------- full attention leg

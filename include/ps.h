@@ -190,6 +190,35 @@ int ps_masked_prefill_attn(const ps_params* params, const void* q, const void* k
                            int64_t tile_plan_cap, int64_t* n_tiles, void* workspace,
                            size_t ws_bytes, int32_t* dev_status, ps_stream_t stream);
 
+/* Bytes of device workspace ps_masked_prefill_attn_bwd needs: the tile plan, two fp32 row
+ * statistics per (batch, head, row) padded to whole 128-row tiles, and a work counter. */
+size_t ps_prefill_bwd_workspace_bytes(const ps_params* params, int64_t batch, int64_t seq);
+
+/* Backward of ps_masked_prefill_attn: gradients of the masked attention with respect to
+ * q, k and v.  Source: §截断回传 of "Prefix Sliding 完全拆解" (the trainer back-propagates
+ * through the masked attention over the last 4W tokens of a rollout), eq. A(i) for the
+ * mask, §Kernel 实现 for the tile skipping (the same plan as the forward).
+ * With P the masked softmax of the forward and D_i = <dout_i, out_i>:
+ *   dv_j = sum_i P_ij dout_i,  dS_ij = P_ij (<dout_i, v_j> - D_i),
+ *   dq_i = scale sum_j dS_ij k_j,  dk_j = scale sum_i dS_ij q_i,
+ * dk and dv summed over the query heads that share a KV head.
+ *   q, k, v  : the forward's inputs (layouts as ps_masked_prefill_attn).
+ *   out      : device bf16 [batch, seq, Hq, D], the forward's output.
+ *   dout     : device bf16 [batch, seq, Hq, D], gradient of the loss with respect to out.
+ *   lse      : device fp32 [batch, Hq, seq], the forward's log-sum-exp (required).
+ *   dq       : device bf16 [batch, seq, Hq, D] (written).
+ *   dk, dv   : device bf16 [batch, seq, Hkv, D] (written).
+ *   workspace, ws_bytes : device scratch of at least ps_prefill_bwd_workspace_bytes(),
+ *              256-byte aligned.
+ *   dev_status : device int32 or NULL (PS_DEV_TIMEOUT only).
+ * Requires seq >= 1, Hq / Hkv integral.  All of q, k, v, out, dout, dq, dk, dv 16-byte
+ * aligned.  Outputs are written in full (no accumulation into existing values). */
+int ps_masked_prefill_attn_bwd(const ps_params* params, const void* q, const void* k,
+                               const void* v, const void* out, const void* dout,
+                               const float* lse, int64_t batch, int64_t seq, void* dq, void* dk,
+                               void* dv, void* workspace, size_t ws_bytes, int32_t* dev_status,
+                               ps_stream_t stream);
+
 /* Introspection for bit-exact checks: the visible-range descriptor the decode kernel
  * uses, computed by the same device code.  ranges_out: device int32 [batch, 4] =
  * (pre_len, seg0_start, seg0_len, seg1_len): the prefix rows [0, pre_len) and the ring

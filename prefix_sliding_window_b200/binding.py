@@ -82,6 +82,11 @@ _SIGS = {
                                          c_int64, c_void_p, c_void_p, c_void_p, c_int64,
                                          POINTER(c_int64), c_void_p, c_size_t, c_void_p,
                                          c_void_p]),
+    "ps_prefill_bwd_workspace_bytes": (c_size_t, [POINTER(PsParams), c_int64, c_int64]),
+    "ps_masked_prefill_attn_bwd": (c_int32, [POINTER(PsParams), c_void_p, c_void_p, c_void_p,
+                                             c_void_p, c_void_p, c_void_p, c_int64, c_int64,
+                                             c_void_p, c_void_p, c_void_p, c_void_p, c_size_t,
+                                             c_void_p, c_void_p]),
     "ps_decode_visible_ranges": (c_int32, [POINTER(PsParams), c_void_p, c_int64, c_void_p,
                                            c_void_p]),
     "ps_last_error": (c_char_p, []),
@@ -220,6 +225,20 @@ def ps_masked_prefill_attn(params: PsParams, q, k, v, batch: int, seq: int, out,
                                        _ptr(dev_status), _stream(stream))
     _check(rc, "ps_masked_prefill_attn")
     return n_tiles.value
+
+
+def ps_prefill_bwd_workspace_bytes(params: PsParams, batch: int, seq: int) -> int:
+    return int(load().ps_prefill_bwd_workspace_bytes(ctypes.byref(params), int(batch), int(seq)))
+
+
+def ps_masked_prefill_attn_bwd(params: PsParams, q, k, v, out, dout, lse, batch: int, seq: int,
+                               dq, dk, dv, workspace=None, dev_status=None, stream=None) -> None:
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rc = load().ps_masked_prefill_attn_bwd(ctypes.byref(params), _ptr(q), _ptr(k), _ptr(v),
+                                           _ptr(out), _ptr(dout), _ptr(lse), int(batch), int(seq),
+                                           _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace), ws_bytes,
+                                           _ptr(dev_status), _stream(stream))
+    _check(rc, "ps_masked_prefill_attn_bwd")
 
 
 def ps_decode_visible_ranges(params: PsParams, pos, batch: int, ranges_out, stream=None) -> None:

@@ -449,4 +449,60 @@ int ps_masked_prefill_attn(const ps_params* params, const void* q, const void* k
   return launch_prefill(l, reinterpret_cast<cudaStream_t>(stream));
 }
 
+size_t ps_prefill_bwd_workspace_bytes(const ps_params* params, int64_t batch, int64_t seq) {
+  if (check_params(params, true) != PS_OK || batch < 0 || seq < 1 || seq > (1LL << 30)) return 0;
+  return prefill_bwd_workspace_bytes(batch, params->n_q_heads, seq, params->l_prefix,
+                                     params->window);
+}
+
+int ps_masked_prefill_attn_bwd(const ps_params* params, const void* q, const void* k,
+                               const void* v, const void* out, const void* dout,
+                               const float* lse, int64_t batch, int64_t seq, void* dq, void* dk,
+                               void* dv, void* workspace, size_t ws_bytes, int32_t* dev_status,
+                               ps_stream_t stream) {
+  g_last_error.clear();
+  PS_TRY(check_params(params, true));
+  if (batch < 0) return fail(PS_ERR_INVALID_ARG, "batch must be >= 0");
+  if (seq < 1 || seq > (1LL << 30)) return fail(PS_ERR_INVALID_ARG, "seq out of range");
+  if (batch == 0) return PS_OK;
+  if (batch > 0x7fffffffLL) return fail(PS_ERR_UNSUPPORTED, "batch too large");
+  PS_TRY(check_ptr(q, "q"));
+  PS_TRY(check_ptr(k, "k"));
+  PS_TRY(check_ptr(v, "v"));
+  PS_TRY(check_ptr(out, "out"));
+  PS_TRY(check_ptr(dout, "dout"));
+  PS_TRY(check_ptr(lse, "lse"));
+  PS_TRY(check_ptr(dq, "dq"));
+  PS_TRY(check_ptr(dk, "dk"));
+  PS_TRY(check_ptr(dv, "dv"));
+  if ((reinterpret_cast<uintptr_t>(dev_status) & 3u) != 0)
+    return fail(PS_ERR_INVALID_ARG, "dev_status is not 4-byte aligned");
+  const size_t need = prefill_bwd_workspace_bytes(batch, params->n_q_heads, seq,
+                                                  params->l_prefix, params->window);
+  if (!workspace || ws_bytes < need)
+    return fail(PS_ERR_WORKSPACE, "workspace smaller than ps_prefill_bwd_workspace_bytes()");
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return fail(PS_ERR_INVALID_ARG, "workspace is not 256-byte aligned");
+  PrefillBwdLaunch l{};
+  l.q = q;
+  l.k = k;
+  l.v = v;
+  l.out = out;
+  l.dout = dout;
+  l.lse = lse;
+  l.dq = dq;
+  l.dk = dk;
+  l.dv = dv;
+  l.workspace = workspace;
+  l.batch = batch;
+  l.seq = seq;
+  l.hq = params->n_q_heads;
+  l.hkv = params->n_kv_heads;
+  l.lp = params->l_prefix;
+  l.w = params->window;
+  l.scale = resolve_scale(params);
+  l.status = dev_status;
+  return launch_prefill_bwd(l, reinterpret_cast<cudaStream_t>(stream));
+}
+
 }  // extern "C"

@@ -119,4 +119,24 @@ cudaError_t launch_plan(int64_t seq, int32_t lp, int32_t w, int64_t n_tiles, voi
 int64_t prefill_plan_tiles(int64_t seq, int32_t lp, int32_t w);
 int launch_prefill(const PrefillLaunch& a, cudaStream_t stream);
 
+// ---------------------------------------------------------------- prefill backward
+struct PrefillBwdLaunch {
+  const void* q;
+  const void* k;
+  const void* v;
+  const void* out;
+  const void* dout;
+  const float* lse;
+  void* dq;
+  void* dk;
+  void* dv;
+  void* workspace;
+  int64_t batch, seq;
+  int32_t hq, hkv, lp, w;
+  float scale;
+  int32_t* status;
+};
+size_t prefill_bwd_workspace_bytes(int64_t batch, int32_t hq, int64_t seq, int32_t lp, int32_t w);
+int launch_prefill_bwd(const PrefillBwdLaunch& l, cudaStream_t stream);
+
 }  // namespace ps

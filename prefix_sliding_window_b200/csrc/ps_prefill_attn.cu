@@ -27,8 +27,8 @@
 //             64 score columns [64g, 64g+64) of every row as an independent online softmax
 //             (its own max m_g, sum l_g and accumulator O_g), so the groups never wait for
 //             each other inside the loop.  On PARTIAL tiles each thread masks its slice with
-//             a 64-bit interval mask built once per row; it then writes P as bf16 over its
-//             columns of the same S buffer (packed fp32x2 FMA/add, one ex2 per element) and
+//             a 64-bit interval mask built once per row; it then writes P as bf16 over the
+//             first half of its own columns of the same S buffer (packed fp32x2 FMA/add, one ex2 per element) and
 //             signals the MMA warp.  O_g is rescaled in TMEM only when the max of some row
 //             of the warp grows by more than 8 (log2 units); otherwise P stays below 2^8
 //             and the stale max keeps fp32 sums exact enough.  The decision is warp-uniform
@@ -327,9 +327,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int kk = 4 * gr; kk < 4 * gr + 4; ++kk) {
               // B = V[16 keys][128 d]: MN-major, 64-column halves 16 KB apart (LBO), 8-key
               // groups 1024 B apart (SBO); 16 keys = 2048 B per step.
+              // A = P_gr: group gr wrote its bf16 pairs over the first 32 of its own 64 S
+              // columns, [64 gr, 64 gr + 32), 8 columns per 16 keys
               const uint64_t bdesc = umma_desc_sw128(vb + kk * 2048, kBoxBytes, 1024);
-              umma_ts(tmem + kColO + 128 * gr, tmem + col_s(s) + kk * 8, bdesc, idesc_pv,
-                      (j > 0 || kk > 4 * gr) ? 1u : 0u);
+              umma_ts(tmem + kColO + 128 * gr, tmem + col_s(s) + 64 * gr + (kk - 4 * gr) * 8,
+                      bdesc, idesc_pv, (j > 0 || kk > 4 * gr) ? 1u : 0u);
             }
           }
           if (!ok) break;
@@ -463,7 +465,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             acc0 = fadd2(acc0, pack_f32x2(p0, p1));
           pk[i] = cvt_bf16x2(p0, p1);
         }
-        tmem_st32(lane_base + col_s(s) + cs0 / 2, pk);
+        // P over this group's own S columns: the other group may not have read its scores
+        tmem_st32(lane_base + col_s(s) + cs0, pk);
         const float2 a0 = unpack_f32x2(acc0), a1 = unpack_f32x2(acc1);
         l += (a0.x + a0.y) + (a1.x + a1.y);
         tmem_wait_st();

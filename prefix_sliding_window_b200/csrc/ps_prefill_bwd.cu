@@ -1,0 +1,958 @@
+// Masked prefill backward (dQ, dK, dV) on 5th-generation tensor cores, sm_100a.
+//
+// What it computes ("Prefix Sliding 完全拆解", §截断回传: the trainer back-propagates through
+// the masked attention it ran over the last 4W tokens): with P_ij the masked softmax of
+// s_ij = scale <q_i, k_j> over j in V(i) (eq. A(i), §核心机制), and D_i = <dO_i, O_i>,
+//   dV_j = sum_i P_ij dO_i,   dS_ij = P_ij (<dO_i, V_j> - D_i),
+//   dQ_i = scale sum_j dS_ij K_j,   dK_j = scale sum_i dS_ij Q_i,
+// dK and dV summed over the query heads of a KV head.  P is rebuilt from the forward's
+// log-sum-exp, so no running max is needed.  Only the tiles of the two-level plan
+// (§Kernel 实现) are visited; PARTIAL tiles are masked element-wise.
+//
+// Three kernels:
+//   bwd_prep_kernel - one warp per (batch, head, row): -D_i and -lse_i*log2(e) into
+//             workspace rows padded to whole 128-row tiles (padding: 0 and -inf, so padded
+//             rows contribute nothing); zeroes the key-tile work counter.
+//   bwd_dq_kernel - query-tile-major, persistent like the forward: per planned key tile,
+//             S = Q K^T and dP = dO V^T into TMEM, the softmax warps form
+//             dS = P (dP - D) as bf16 over S, and dQ += dS K accumulates in TMEM.
+//   bwd_dkdv_kernel - key-tile-major over (batch, KV head, key tile) items taken from an
+//             atomic counter (a prefix key tile is seen by every later query tile, a window
+//             key tile by about W/128 of them, so static striding would leave SMs idle): per
+//             (query head of the group, query tile), S^T = K Q^T and dP^T = V dO^T into
+//             TMEM, P^T and dS^T as bf16 over them, dV += P^T dO and dK += dS^T Q in TMEM
+//             across the whole group, so no atomics are needed.
+// Both big kernels use the forward's roles: warps 0-7 two softmax warpgroups (group g owns
+// columns [64g, 64g+64) of every TMEM lane), warps 8-9 TMA producers, warp 10 issues the
+// smem x smem products (and owns TMEM), warp 11 the TMEM x smem accumulations.
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <math.h>
+
+#include "ps_device.cuh"
+#include "ps_internal.h"
+#include "ps_ranges.cuh"
+
+namespace ps {
+namespace {
+
+constexpr int kT = 128;  // query and key tile rows
+static_assert(kPrefillBq == kT && kPrefillBk == kT, "backward assumes square 128-row tiles");
+constexpr int kBoxBytes = 128 * 128;       // [128 rows][64 bf16], 128-byte swizzle
+constexpr int kTileBytes = 2 * kBoxBytes;  // [128 rows][128 bf16]
+constexpr int kGroups = 2;
+constexpr int kCols = 64;  // columns per softmax group
+constexpr int kSoftmaxWarps = 8;
+constexpr int kProdA = 8;
+constexpr int kProdB = 9;
+constexpr int kIssA = 10;
+constexpr int kIssB = 11;
+constexpr int kThreads = 12 * 32;
+constexpr uint32_t kTmemCols = 512;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr int kPrepThreads = 256;
+constexpr int kItemRing = 4;
+
+struct BwdArgs {
+  int32_t* status;
+  int64_t seq, s_pad;
+  int32_t batch, hq, hkv, group, nq;
+  int32_t lp, w;
+  float scale, scale_log2;
+  const float* nl;  // [B][Hq][s_pad]: -lse * log2(e)
+  const float* nd;  // [B][Hq][s_pad]: -D
+  const int32_t* off;  // query-tile-major plan: [nq + 1] offsets
+  const int32_t* ent;  // [n][2] (k_tile, flag)
+  int32_t* counter;    // key-tile work counter
+  __nv_bfloat16* dq;   // [B, S, Hq, D]
+  __nv_bfloat16* dk;   // [B, S, Hkv, D]
+  __nv_bfloat16* dv;
+};
+
+// K-major 128x128 x 128x128 product: both operands [128 rows][128 cols] in two 64-column
+// 128-byte-swizzled halves; 16 columns = 32 B per step inside a half.
+__device__ __forceinline__ void mma_kmajor(uint32_t d_tmem, uint32_t a_addr, uint32_t b_addr) {
+  constexpr uint32_t idesc = umma_idesc_bf16(128, 128, false);
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk) {
+    const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
+    umma_ss(d_tmem, umma_desc_sw128(a_addr + off, 16, 1024),
+            umma_desc_sw128(b_addr + off, 16, 1024), idesc, kk > 0 ? 1u : 0u);
+  }
+}
+
+// D += A * B[rows 64 grp .. 64 grp + 63] for one softmax group: A = the group's bf16 pairs in
+// TMEM (written over the first 32 of its own 64 columns, buffer column 64 grp, 8 columns per
+// 16 rows of B), B = smem [128 rows][128 cols] MN-major.
+__device__ __forceinline__ void mma_tmem_a(uint32_t d_tmem, uint32_t a_buf, uint32_t b_addr,
+                                           int grp, bool first) {
+  constexpr uint32_t idesc = umma_idesc_bf16(128, 128, true);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int kk = 4 * grp + i;
+    // B rows 16kk..16kk+15: 2048 B per step; 64-column halves 16 KB apart (LBO), 8-row
+    // groups 1024 B apart (SBO)
+    const uint64_t bdesc = umma_desc_sw128(b_addr + kk * 2048, kBoxBytes, 1024);
+    umma_ts(d_tmem, a_buf + 64 * grp + 8 * i, bdesc, idesc, (first && i == 0) ? 0u : 1u);
+  }
+}
+
+__device__ __forceinline__ void load64(uint32_t taddr, float (&x)[kCols]) {
+  uint32_t raw[2][32];
+  tmem_ld32(taddr, raw[0]);
+  tmem_ld32(taddr + 32, raw[1]);
+  tmem_wait_ld();
+#pragma unroll
+  for (int c = 0; c < 2; ++c)
+#pragma unroll
+    for (int i = 0; i < 32; ++i) x[32 * c + i] = __uint_as_float(raw[c][i]);
+}
+
+// Bit c (c < 64) set iff c + base lies in [lo, hi).
+__device__ __forceinline__ uint64_t span_bits(int64_t lo, int64_t hi, int64_t base) {
+  lo -= base;
+  hi -= base;
+  if (lo < 0) lo = 0;
+  if (hi > 64) hi = 64;
+  if (hi <= lo) return 0ull;
+  const uint64_t len = static_cast<uint64_t>(hi - lo);
+  return (len >= 64 ? ~0ull : ((1ull << len) - 1ull)) << lo;
+}
+
+// ------------------------------------------------------------------ prep
+__global__ void __launch_bounds__(kPrepThreads)
+    bwd_prep_kernel(const __nv_bfloat16* __restrict__ out, const __nv_bfloat16* __restrict__ dout,
+                    const float* __restrict__ lse, int64_t seq, int32_t hq, int64_t s_pad,
+                    int64_t n_rows, float* __restrict__ nl, float* __restrict__ nd,
+                    int32_t* __restrict__ counter) {
+  pdl_trigger();
+  pdl_wait();
+  if (blockIdx.x == 0 && threadIdx.x == 0) *counter = 0;
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * (kPrepThreads / 32) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= n_rows) return;
+  const int64_t i = row % s_pad;
+  const int64_t bh = row / s_pad;
+  float dot = 0.f, l2 = -INFINITY;
+  if (i < seq) {
+    const int64_t h = bh % hq, b = bh / hq;
+    const int64_t base = ((b * seq + i) * hq + h) * kHeadDim + 4 * lane;
+    const uint2 o = *reinterpret_cast<const uint2*>(out + base);
+    const uint2 d = *reinterpret_cast<const uint2*>(dout + base);
+    const float2 o0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&o.x));
+    const float2 o1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&o.y));
+    const float2 d0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&d.x));
+    const float2 d1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&d.y));
+    dot = o0.x * d0.x + o0.y * d0.y + o1.x * d1.x + o1.y * d1.y;
+#pragma unroll
+    for (int sh = 16; sh > 0; sh >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, sh);
+    l2 = -lse[bh * seq + i] * kLog2e;
+  }
+  if (lane == 0) {
+    nl[row] = l2;
+    nd[row] = -dot;
+  }
+}
+
+// ------------------------------------------------------------------ dQ
+// TMEM: S0 [0,128), S1 [128,256), dP [256,384), dQ [384,512).
+constexpr uint32_t kQColDP = 256;
+constexpr uint32_t kQColDQ = 384;
+__device__ __forceinline__ uint32_t col_s(int s) { return s ? 128u : 0u; }
+constexpr size_t kDqSmem = 1024 + 6 * size_t(kTileBytes) + 256;
+
+__global__ void __launch_bounds__(kThreads, 1)
+    bwd_dq_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mdo,
+                  const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtensorMap mv,
+                  const BwdArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* sQ = smem;
+  uint8_t* sDO = sQ + kTileBytes;
+  uint8_t* sK = sDO + kTileBytes;  // [2]
+  uint8_t* sV = sK + 2 * kTileBytes;  // [2]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + 2 * kTileBytes);
+  uint64_t* qdo_full = bars;
+  uint64_t* qdo_empty = bars + 1;
+  uint64_t* k_full = bars + 2;     // [2]
+  uint64_t* k_empty = bars + 4;    // [2]
+  uint64_t* v_full = bars + 6;     // [2]
+  uint64_t* v_empty = bars + 8;    // [2]
+  uint64_t* s_full = bars + 10;    // [2]
+  uint64_t* s_free = bars + 12;    // [2]: dQ MMA of the buffer's tile done
+  uint64_t* ds_ready = bars + 14;  // [2 buffers][2 groups]
+  uint64_t* dp_full = bars + 18;
+  uint64_t* dp_free = bars + 19;
+  uint64_t* dq_full = bars + 20;
+  uint64_t* dq_free = bars + 21;
+  uint64_t* mma_done = bars + 22;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 23);
+
+  const int64_t bh = (int64_t)a.batch * a.hq;
+  const int64_t n_items = bh * a.nq;
+  auto item_of = [&](int64_t it, int& qt, int& b, int& head) {
+    qt = a.nq - 1 - static_cast<int>(it / bh);  // heaviest query tiles first
+    const int rem = static_cast<int>(it % bh);
+    head = rem % a.hq;
+    b = rem / a.hq;
+  };
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    mbar_init(qdo_full, 1);
+    mbar_init(qdo_empty, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&k_full[s], 1);
+      mbar_init(&k_empty[s], 1);
+      mbar_init(&v_full[s], 1);
+      mbar_init(&v_empty[s], 1);
+      mbar_init(&s_full[s], 1);
+      mbar_init(&s_free[s], 1);
+      for (int g = 0; g < kGroups; ++g) mbar_init(&ds_ready[s * kGroups + g], 4);
+    }
+    mbar_init(dp_full, 1);
+    mbar_init(dp_free, kSoftmaxWarps);
+    mbar_init(dq_full, 1);
+    mbar_init(dq_free, kSoftmaxWarps);
+    mbar_init(mma_done, 2);
+    fence_mbar_init();
+  }
+  if (warp == kIssA) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  if (warp == kProdA && lane == 0) {
+    prefetch_tensormap(&mq);
+    prefetch_tensormap(&mdo);
+    prefetch_tensormap(&mk);
+    prefetch_tensormap(&mv);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  pdl_wait();  // plan and row statistics come from the kernels launched before
+
+  if (warp == kProdA || warp == kProdB) {
+    // warp 8: Q and dO of each item, then the K tiles of its plan; warp 9: the V tiles
+    if (lane == 0) {
+      const bool is_k = (warp == kProdA);
+      const CUtensorMap* map = is_k ? &mk : &mv;
+      uint8_t* ring = is_k ? sK : sV;
+      uint64_t* full = is_k ? k_full : v_full;
+      uint64_t* empty = is_k ? k_empty : v_empty;
+      int64_t g = 0;
+      int li = 0;
+      bool alive = true;
+      for (int64_t it = blockIdx.x; alive && it < n_items; it += gridDim.x, ++li) {
+        int qt, b, head;
+        item_of(it, qt, b, head);
+        const int kvh = head / a.group;
+        const int e0 = a.off[qt];
+        const int n = a.off[qt + 1] - e0;
+        if (is_k) {
+          if (li > 0 && !mbar_wait(qdo_empty, (li - 1) & 1, a.status)) {
+            alive = false;
+            break;
+          }
+          mbar_arrive_expect_tx(qdo_full, 2 * kTileBytes);
+          tma_load_4d(sQ, &mq, 0, head, qt * kT, b, qdo_full);
+          tma_load_4d(sQ + kBoxBytes, &mq, 64, head, qt * kT, b, qdo_full);
+          tma_load_4d(sDO, &mdo, 0, head, qt * kT, b, qdo_full);
+          tma_load_4d(sDO + kBoxBytes, &mdo, 64, head, qt * kT, b, qdo_full);
+        }
+        for (int j = 0; j < n; ++j, ++g) {
+          const int s = static_cast<int>(g & 1);
+          if (g >= 2 && !mbar_wait(&empty[s], static_cast<uint32_t>(((g >> 1) - 1) & 1), a.status)) {
+            alive = false;
+            break;
+          }
+          const int kt = a.ent[2 * (e0 + j)];
+          uint8_t* dst = ring + s * kTileBytes;
+          mbar_arrive_expect_tx(&full[s], kTileBytes);
+          tma_load_4d(dst, map, 0, kvh, kt * kT, b, &full[s]);
+          tma_load_4d(dst + kBoxBytes, map, 64, kvh, kt * kT, b, &full[s]);
+        }
+      }
+      // every issued copy lands before the CTA may exit
+      for (int64_t j = (g > 2 ? g - 2 : 0); j < g; ++j)
+        mbar_wait(&full[j & 1], static_cast<uint32_t>((j >> 1) & 1), a.status);
+      if (is_k && li > 0) mbar_wait(qdo_full, (li - 1) & 1, a.status);
+    }
+  } else if (warp == kIssA) {
+    // S[buf] = Q K^T and dP = dO V^T
+    if (lane == 0) {
+      const uint32_t q_addr = smem_u32(sQ), do_addr = smem_u32(sDO);
+      const uint32_t k_addr = smem_u32(sK), v_addr = smem_u32(sV);
+      int64_t g = 0;
+      int li = 0;
+      bool ok = true;
+      for (int64_t it = blockIdx.x; ok && it < n_items; it += gridDim.x, ++li) {
+        int qt, b, head;
+        item_of(it, qt, b, head);
+        const int n = a.off[qt + 1] - a.off[qt];
+        if (!mbar_wait(qdo_full, li & 1, a.status)) {
+          ok = false;
+          break;
+        }
+        for (int j = 0; j < n; ++j, ++g) {
+          const int s = static_cast<int>(g & 1);
+          const uint32_t ph = static_cast<uint32_t>((g >> 1) & 1);
+          if (!mbar_wait(&k_full[s], ph, a.status) ||
+              (g >= 2 && !mbar_wait(&s_free[s], ph ^ 1, a.status))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          mma_kmajor(tmem + col_s(s), q_addr, k_addr + s * kTileBytes);
+          umma_commit(&s_full[s]);
+          if (!mbar_wait(&v_full[s], ph, a.status) ||
+              (g >= 1 && !mbar_wait(dp_free, static_cast<uint32_t>((g - 1) & 1), a.status))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          mma_kmajor(tmem + kQColDP, do_addr, v_addr + s * kTileBytes);
+          umma_commit(dp_full);
+          umma_commit(&v_empty[s]);
+          if (j == n - 1) umma_commit(qdo_empty);
+        }
+      }
+      umma_commit(mma_done);
+      mbar_wait(mma_done, 0, a.status);
+    }
+  } else if (warp == kIssB) {
+    // dQ += dS K, group by group as each softmax group's dS lands
+    if (lane == 0) {
+      const uint32_t k_addr = smem_u32(sK);
+      int64_t g = 0;
+      int li = 0;
+      bool ok = true;
+      for (int64_t it = blockIdx.x; ok && it < n_items; it += gridDim.x, ++li) {
+        int qt, b, head;
+        item_of(it, qt, b, head);
+        const int n = a.off[qt + 1] - a.off[qt];
+        for (int j = 0; j < n; ++j, ++g) {
+          const int s = static_cast<int>(g & 1);
+          if (j == 0 && li > 0 && !mbar_wait(dq_free, (li - 1) & 1, a.status)) {
+            ok = false;
+            break;
+          }
+#pragma unroll
+          for (int gr = 0; gr < kGroups; ++gr) {
+            if (!mbar_wait(&ds_ready[s * kGroups + gr], static_cast<uint32_t>((g >> 1) & 1),
+                           a.status)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            mma_tmem_a(tmem + kQColDQ, tmem + col_s(s), k_addr + s * kTileBytes, gr,
+                       j == 0 && gr == 0);
+          }
+          if (!ok) break;
+          umma_commit(&k_empty[s]);
+          umma_commit(&s_free[s]);
+        }
+        if (ok) umma_commit(dq_full);
+      }
+      umma_commit(mma_done);
+      mbar_wait(mma_done, 0, a.status);
+    }
+  } else {
+    // softmax warpgroups: dS = P (dP - D) with P = 2^(s*scale*log2e - lse*log2e)
+    const int wg = threadIdx.x >> 7;
+    const int r = threadIdx.x & 127;
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+    const uint32_t cs0 = static_cast<uint32_t>(kCols * wg);
+    const uint64_t sl2x2 = pack_f32x2(a.scale_log2, a.scale_log2);
+    bool ok = true;
+    int64_t g = 0;
+    int li = 0;
+    for (int64_t it = blockIdx.x; it < n_items; it += gridDim.x, ++li) {
+      int qt, b, head;
+      item_of(it, qt, b, head);
+      const int e0 = a.off[qt];
+      const int n = a.off[qt + 1] - e0;
+      const int64_t row = (int64_t)qt * kT + r;
+      const int64_t srow = ((int64_t)b * a.hq + head) * a.s_pad + row;
+      const float nl = a.nl[srow], nd = a.nd[srow];
+      const uint64_t nl2 = pack_f32x2(nl, nl), nd2 = pack_f32x2(nd, nd);
+      int2 ent_next = n > 0 ? reinterpret_cast<const int2*>(a.ent)[e0] : make_int2(0, 0);
+      for (int j = 0; j < n; ++j, ++g) {
+        const int s = static_cast<int>(g & 1);
+        const int kt = ent_next.x;
+        const int flag = ent_next.y;
+        if (j + 1 < n) ent_next = reinterpret_cast<const int2*>(a.ent)[e0 + j + 1];
+        ok = ok && __all_sync(0xffffffffu, mbar_wait(&s_full[s], static_cast<uint32_t>((g >> 1) & 1),
+                                                      a.status));
+        if (!ok) continue;
+        tc_fence_after();
+        float x[kCols];
+        load64(lane_base + col_s(s) + cs0, x);
+        if (flag == PS_TILE_PARTIAL) {
+          const int64_t end = row + 1 < a.seq ? row + 1 : a.seq;
+          int64_t win_lo = row - a.w + 1;
+          if (win_lo < a.lp) win_lo = a.lp;
+          const int64_t k0 = (int64_t)kt * kT + cs0;
+          const uint64_t vis = span_bits(0, a.lp < end ? a.lp : end, k0) | span_bits(win_lo, end, k0);
+#pragma unroll
+          for (int i = 0; i < kCols; ++i)
+            if (!((vis >> i) & 1ull)) x[i] = -INFINITY;
+        }
+#pragma unroll
+        for (int i = 0; i < kCols / 2; ++i) {
+          const float2 e = unpack_f32x2(ffma2(pack_f32x2(x[2 * i], x[2 * i + 1]), sl2x2, nl2));
+          x[2 * i] = fast_exp2(e.x);
+          x[2 * i + 1] = fast_exp2(e.y);
+        }
+        ok = ok && __all_sync(0xffffffffu, mbar_wait(dp_full, static_cast<uint32_t>(g & 1), a.status));
+        if (!ok) continue;
+        tc_fence_after();
+        float dp[kCols];
+        load64(lane_base + kQColDP + cs0, dp);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(dp_free);
+        uint32_t pk[kCols / 2];
+#pragma unroll
+        for (int i = 0; i < kCols / 2; ++i) {
+          const float2 d = unpack_f32x2(
+              fmul2(pack_f32x2(x[2 * i], x[2 * i + 1]), fadd2(pack_f32x2(dp[2 * i], dp[2 * i + 1]), nd2)));
+          pk[i] = cvt_bf16x2(d.x, d.y);
+        }
+        tmem_st32(lane_base + col_s(s) + cs0, pk);  // over this group's own columns
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ds_ready[s * kGroups + wg]);
+      }
+      // epilogue: dQ = scale * accumulated dS K
+      const bool fin = __all_sync(0xffffffffu, ok && mbar_wait(dq_full, li & 1, a.status));
+      ok = ok && fin;
+      if (!fin) continue;
+      tc_fence_after();
+      float acc[kCols];
+      load64(lane_base + kQColDQ + cs0, acc);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(dq_free);
+      if (row < a.seq) {
+        uint4* dst = reinterpret_cast<uint4*>(a.dq + (((int64_t)b * a.seq + row) * a.hq + head) *
+                                                         kHeadDim + cs0);
+#pragma unroll
+        for (int v = 0; v < kCols / 8; ++v) {
+          dst[v] = make_uint4(cvt_bf16x2(a.scale * acc[8 * v], a.scale * acc[8 * v + 1]),
+                              cvt_bf16x2(a.scale * acc[8 * v + 2], a.scale * acc[8 * v + 3]),
+                              cvt_bf16x2(a.scale * acc[8 * v + 4], a.scale * acc[8 * v + 5]),
+                              cvt_bf16x2(a.scale * acc[8 * v + 6], a.scale * acc[8 * v + 7]));
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kIssA) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// ------------------------------------------------------------------ dK, dV
+// TMEM: S^T [0,128), dP^T [128,256), dV [256,384), dK [384,512).
+constexpr uint32_t kKColS = 0;
+constexpr uint32_t kKColDP = 128;
+constexpr uint32_t kKColDV = 256;
+constexpr uint32_t kKColDK = 384;
+constexpr int kStatBytes = kT * 4;  // one tile of -lse*log2e (or -D)
+constexpr size_t kDkdvSmem = 1024 + 6 * size_t(kTileBytes) + 4 * kStatBytes + 512;
+
+struct KvItem {
+  int b, kvh, kt;
+  int qlo, nqt;
+};
+__device__ __forceinline__ KvItem kv_item(int64_t it, const BwdArgs& a) {
+  KvItem m;
+  const int64_t per = (int64_t)a.batch * a.hkv;
+  m.kt = static_cast<int>(it / per);  // ascending key tiles: prefix tiles (the heaviest) first
+  const int rem = static_cast<int>(it % per);
+  m.kvh = rem % a.hkv;
+  m.b = rem / a.hkv;
+  int64_t lo = 0, hi = -1;
+  ktile_qrange(m.kt, a.seq, a.lp, a.w, kT, &lo, &hi);
+  m.qlo = static_cast<int>(lo);
+  m.nqt = static_cast<int>(hi - lo + 1);
+  return m;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    bwd_dkdv_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mdo,
+                    const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtensorMap mv,
+                    const BwdArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* sK = smem;
+  uint8_t* sV = sK + kTileBytes;
+  uint8_t* sQ = sV + kTileBytes;      // [2 stages]
+  uint8_t* sDO = sQ + 2 * kTileBytes;  // [2 stages]
+  float* sNL = reinterpret_cast<float*>(sDO + 2 * kTileBytes);  // [2][128]
+  float* sND = sNL + 2 * kT;                                      // [2][128]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sND + 2 * kT);
+  uint64_t* item_full = bars;                  // [kItemRing]
+  uint64_t* item_empty = bars + kItemRing;     // [kItemRing]
+  uint64_t* kv_full = bars + 2 * kItemRing;
+  uint64_t* kv_empty = kv_full + 1;
+  uint64_t* st_full = kv_full + 2;   // [2]
+  uint64_t* st_empty = kv_full + 4;  // [2]
+  uint64_t* s_full = kv_full + 6;
+  uint64_t* dp_full = kv_full + 7;
+  uint64_t* p_ready = kv_full + 8;   // [2 groups]
+  uint64_t* ds_ready = kv_full + 10;  // [2 groups]
+  uint64_t* s_free = kv_full + 12;
+  uint64_t* dp_free = kv_full + 13;
+  uint64_t* acc_full = kv_full + 14;
+  uint64_t* acc_free = kv_full + 15;
+  uint64_t* mma_done = kv_full + 16;
+  int32_t* s_items = reinterpret_cast<int32_t*>(kv_full + 17);  // [kItemRing]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(s_items + kItemRing);
+
+  const int64_t n_items = (int64_t)a.batch * a.hkv * a.nq;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  constexpr int kItemReaders = 3 + kSoftmaxWarps;  // producer A, both issuers, softmax warps
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kItemRing; ++i) {
+      mbar_init(&item_full[i], 1);
+      mbar_init(&item_empty[i], kItemReaders);
+    }
+    mbar_init(kv_full, 1);
+    mbar_init(kv_empty, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&st_full[s], 1);
+      mbar_init(&st_empty[s], 1);
+      mbar_init(&p_ready[s], 4);
+      mbar_init(&ds_ready[s], 4);
+    }
+    mbar_init(s_full, 1);
+    mbar_init(dp_full, 1);
+    mbar_init(s_free, 1);
+    mbar_init(dp_free, 1);
+    mbar_init(acc_full, 1);
+    mbar_init(acc_free, kSoftmaxWarps);
+    mbar_init(mma_done, 2);
+    fence_mbar_init();
+  }
+  if (warp == kIssA) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  if (warp == kProdA && lane == 0) {
+    prefetch_tensormap(&mq);
+    prefetch_tensormap(&mdo);
+    prefetch_tensormap(&mk);
+    prefetch_tensormap(&mv);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  pdl_wait();  // row statistics and the zeroed counter come from earlier kernels
+
+  // Item i of this CTA from the ring (slot i % kItemRing); -1 on timeout.
+  auto next_item = [&](int li) -> int64_t {
+    const int slot = li % kItemRing;
+    if (!mbar_wait(&item_full[slot], static_cast<uint32_t>((li / kItemRing) & 1), a.status))
+      return -1;
+    return *reinterpret_cast<volatile int32_t*>(&s_items[slot]);
+  };
+
+  if (warp == kProdB) {
+    // ---------------------------------------------------- item fetcher + K/V producer
+    if (lane == 0) {
+      int li = 0;
+      for (;; ++li) {
+        const int slot = li % kItemRing;
+        if (li >= kItemRing &&
+            !mbar_wait(&item_empty[slot], static_cast<uint32_t>(((li / kItemRing) - 1) & 1),
+                       a.status))
+          break;
+        // take the next item only once this CTA's K/V buffer is free again
+        if (li > 0 && !mbar_wait(kv_empty, (li - 1) & 1, a.status)) break;
+        const int32_t it = atomicAdd(a.counter, 1);
+        s_items[slot] = it >= n_items ? static_cast<int32_t>(n_items) : it;
+        mbar_arrive(&item_full[slot]);
+        if (it >= n_items) break;
+        const KvItem m = kv_item(it, a);
+        mbar_arrive_expect_tx(kv_full, 2 * kTileBytes);
+        tma_load_4d(sK, &mk, 0, m.kvh, m.kt * kT, m.b, kv_full);
+        tma_load_4d(sK + kBoxBytes, &mk, 64, m.kvh, m.kt * kT, m.b, kv_full);
+        tma_load_4d(sV, &mv, 0, m.kvh, m.kt * kT, m.b, kv_full);
+        tma_load_4d(sV + kBoxBytes, &mv, 64, m.kvh, m.kt * kT, m.b, kv_full);
+      }
+      // li items were loaded (the last fetch returned the end marker or a wait failed)
+      if (li > 0) mbar_wait(kv_full, (li - 1) & 1, a.status);
+    }
+  } else if (warp == kProdA) {
+    // ---------------------------------------------------- Q, dO and row statistics
+    if (lane == 0) {
+      int64_t g = 0;
+      bool alive = true;
+      for (int li = 0; alive; ++li) {
+        const int64_t it = next_item(li);
+        if (it < 0) break;
+        mbar_arrive(&item_empty[li % kItemRing]);
+        if (it >= n_items) break;
+        const KvItem m = kv_item(it, a);
+        const int n = a.group * m.nqt;
+        for (int j = 0; j < n; ++j, ++g) {
+          const int st = static_cast<int>(g & 1);
+          if (g >= 2 &&
+              !mbar_wait(&st_empty[st], static_cast<uint32_t>(((g >> 1) - 1) & 1), a.status)) {
+            alive = false;
+            break;
+          }
+          const int h = m.kvh * a.group + j / m.nqt;
+          const int qt = m.qlo + j % m.nqt;
+          mbar_arrive_expect_tx(&st_full[st], 2 * kTileBytes + 2 * kStatBytes);
+          uint8_t* q = sQ + st * kTileBytes;
+          uint8_t* d = sDO + st * kTileBytes;
+          tma_load_4d(q, &mq, 0, h, qt * kT, m.b, &st_full[st]);
+          tma_load_4d(q + kBoxBytes, &mq, 64, h, qt * kT, m.b, &st_full[st]);
+          tma_load_4d(d, &mdo, 0, h, qt * kT, m.b, &st_full[st]);
+          tma_load_4d(d + kBoxBytes, &mdo, 64, h, qt * kT, m.b, &st_full[st]);
+          const int64_t srow = ((int64_t)m.b * a.hq + h) * a.s_pad + (int64_t)qt * kT;
+          bulk_load(sNL + st * kT, a.nl + srow, kStatBytes, &st_full[st]);
+          bulk_load(sND + st * kT, a.nd + srow, kStatBytes, &st_full[st]);
+        }
+      }
+      for (int64_t j = (g > 2 ? g - 2 : 0); j < g; ++j)
+        mbar_wait(&st_full[j & 1], static_cast<uint32_t>((j >> 1) & 1), a.status);
+    }
+  } else if (warp == kIssA) {
+    // ---------------------------------------------------- S^T = K Q^T, dP^T = V dO^T
+    if (lane == 0) {
+      const uint32_t k_addr = smem_u32(sK), v_addr = smem_u32(sV);
+      const uint32_t q_addr = smem_u32(sQ), do_addr = smem_u32(sDO);
+      int64_t g = 0;
+      bool ok = true;
+      for (int li = 0; ok; ++li) {
+        const int64_t it = next_item(li);
+        if (it < 0) break;
+        mbar_arrive(&item_empty[li % kItemRing]);
+        if (it >= n_items) break;
+        const KvItem m = kv_item(it, a);
+        const int n = a.group * m.nqt;
+        if (!mbar_wait(kv_full, li & 1, a.status)) break;
+        for (int j = 0; j < n; ++j, ++g) {
+          const int st = static_cast<int>(g & 1);
+          const uint32_t prev = static_cast<uint32_t>((g - 1) & 1);
+          if (!mbar_wait(&st_full[st], static_cast<uint32_t>((g >> 1) & 1), a.status) ||
+              (g >= 1 && !mbar_wait(s_free, prev, a.status))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          mma_kmajor(tmem + kKColS, k_addr, q_addr + st * kTileBytes);
+          umma_commit(s_full);
+          if (g >= 1 && !mbar_wait(dp_free, prev, a.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          mma_kmajor(tmem + kKColDP, v_addr, do_addr + st * kTileBytes);
+          umma_commit(dp_full);
+        }
+        if (!ok) break;
+        umma_commit(kv_empty);  // K and V of this item are no longer read
+      }
+      umma_commit(mma_done);
+      mbar_wait(mma_done, 0, a.status);
+    }
+  } else if (warp == kIssB) {
+    // ---------------------------------------------------- dV += P^T dO, dK += dS^T Q
+    if (lane == 0) {
+      const uint32_t q_addr = smem_u32(sQ), do_addr = smem_u32(sDO);
+      int64_t g = 0;
+      bool ok = true;
+      for (int li = 0; ok; ++li) {
+        const int64_t it = next_item(li);
+        if (it < 0) break;
+        mbar_arrive(&item_empty[li % kItemRing]);
+        if (it >= n_items) break;
+        const KvItem m = kv_item(it, a);
+        const int n = a.group * m.nqt;
+        for (int j = 0; j < n; ++j, ++g) {
+          const int st = static_cast<int>(g & 1);
+          const uint32_t ph = static_cast<uint32_t>(g & 1);
+          if (j == 0 && li > 0 && !mbar_wait(acc_free, (li - 1) & 1, a.status)) {
+            ok = false;
+            break;
+          }
+#pragma unroll
+          for (int gr = 0; gr < kGroups; ++gr) {
+            if (!mbar_wait(&p_ready[gr], ph, a.status)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            mma_tmem_a(tmem + kKColDV, tmem + kKColS, do_addr + st * kTileBytes, gr,
+                       j == 0 && gr == 0);
+          }
+          if (!ok) break;
+          umma_commit(s_free);
+#pragma unroll
+          for (int gr = 0; gr < kGroups; ++gr) {
+            if (!mbar_wait(&ds_ready[gr], ph, a.status)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            mma_tmem_a(tmem + kKColDK, tmem + kKColDP, q_addr + st * kTileBytes, gr,
+                       j == 0 && gr == 0);
+          }
+          if (!ok) break;
+          umma_commit(dp_free);
+          umma_commit(&st_empty[st]);
+        }
+        if (!ok) break;
+        umma_commit(acc_full);
+      }
+      umma_commit(mma_done);
+      mbar_wait(mma_done, 0, a.status);
+    }
+  } else {
+    // ---------------------------------------------------- softmax warpgroups
+    // TMEM lane r = key row kt*128 + r; group wg owns query columns [64 wg, 64 wg + 64).
+    const int wg = threadIdx.x >> 7;
+    const int r = threadIdx.x & 127;
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+    const uint32_t cs0 = static_cast<uint32_t>(kCols * wg);
+    const uint64_t sl2x2 = pack_f32x2(a.scale_log2, a.scale_log2);
+    bool ok = true;
+    int64_t g = 0;
+    for (int li = 0;; ++li) {
+      const int64_t it = next_item(li);
+      __syncwarp();
+      if (lane == 0 && it >= 0) mbar_arrive(&item_empty[li % kItemRing]);
+      if (it < 0 || it >= n_items) break;
+      const KvItem m = kv_item(it, a);
+      const int n = a.group * m.nqt;
+      const int64_t kr = (int64_t)m.kt * kT + r;  // this thread's key
+      // queries that see key kr: [kr, vis_end)
+      int64_t vis_end = kr;
+      if (kr < a.seq) vis_end = (kr < a.lp || kr + a.w > a.seq) ? a.seq : kr + a.w;
+      for (int j = 0; j < n; ++j, ++g) {
+        const int st = static_cast<int>(g & 1);
+        const uint32_t ph = static_cast<uint32_t>(g & 1);
+        const int qt = m.qlo + j % m.nqt;
+        const int flag = classify_tile(qt, m.kt, a.seq, a.lp, a.w, kT, kT);
+        ok = ok && __all_sync(0xffffffffu,
+                              mbar_wait(s_full, ph, a.status) &&
+                                  mbar_wait(&st_full[st], static_cast<uint32_t>((g >> 1) & 1),
+                                            a.status));
+        if (!ok) continue;
+        tc_fence_after();
+        float x[kCols];
+        load64(lane_base + kKColS + cs0, x);
+        if (flag == PS_TILE_PARTIAL) {
+          const uint64_t vis = span_bits(kr, vis_end, (int64_t)qt * kT + cs0);
+#pragma unroll
+          for (int i = 0; i < kCols; ++i)
+            if (!((vis >> i) & 1ull)) x[i] = -INFINITY;
+        }
+        const float2* nl = reinterpret_cast<const float2*>(sNL + st * kT + cs0);
+        const float2* nd = reinterpret_cast<const float2*>(sND + st * kT + cs0);
+        uint32_t pk[kCols / 2];
+#pragma unroll
+        for (int i = 0; i < kCols / 2; ++i) {
+          const float2 l = nl[i];
+          const float2 e =
+              unpack_f32x2(ffma2(pack_f32x2(x[2 * i], x[2 * i + 1]), sl2x2, pack_f32x2(l.x, l.y)));
+          x[2 * i] = fast_exp2(e.x);
+          x[2 * i + 1] = fast_exp2(e.y);
+          pk[i] = cvt_bf16x2(x[2 * i], x[2 * i + 1]);
+        }
+        tmem_st32(lane_base + kKColS + cs0, pk);  // over this group's own columns
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&p_ready[wg]);
+        ok = ok && __all_sync(0xffffffffu, mbar_wait(dp_full, ph, a.status));
+        if (!ok) continue;
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          uint32_t raw[32];
+          tmem_ld32(lane_base + kKColDP + cs0 + 32 * c, raw);
+          tmem_wait_ld();
+          uint32_t dk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int e = 32 * c + 2 * i;
+            const float2 d = nd[e / 2];
+            const float2 v = unpack_f32x2(
+                fmul2(pack_f32x2(x[e], x[e + 1]),
+                      fadd2(pack_f32x2(__uint_as_float(raw[2 * i]), __uint_as_float(raw[2 * i + 1])),
+                            pack_f32x2(d.x, d.y))));
+            dk[i] = cvt_bf16x2(v.x, v.y);
+          }
+          tmem_st16(lane_base + kKColDP + cs0 + 16 * c, dk);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ds_ready[wg]);
+      }
+      // epilogue: dV and dK (times the softmax scale) of this key tile
+      const bool fin = __all_sync(0xffffffffu, ok && mbar_wait(acc_full, li & 1, a.status));
+      ok = ok && fin;
+      if (!fin) continue;
+      tc_fence_after();
+      uint32_t pv[kCols / 2], pkk[kCols / 2];
+      {
+        float acc[kCols];
+        load64(lane_base + kKColDV + cs0, acc);
+#pragma unroll
+        for (int i = 0; i < kCols / 2; ++i) pv[i] = cvt_bf16x2(acc[2 * i], acc[2 * i + 1]);
+        load64(lane_base + kKColDK + cs0, acc);
+#pragma unroll
+        for (int i = 0; i < kCols / 2; ++i)
+          pkk[i] = cvt_bf16x2(a.scale * acc[2 * i], a.scale * acc[2 * i + 1]);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acc_free);
+      if (kr < a.seq) {
+        const int64_t o = (((int64_t)m.b * a.seq + kr) * a.hkv + m.kvh) * kHeadDim + cs0;
+        uint4* dv = reinterpret_cast<uint4*>(a.dv + o);
+        uint4* dk = reinterpret_cast<uint4*>(a.dk + o);
+#pragma unroll
+        for (int v = 0; v < kCols / 8; ++v) {
+          dv[v] = make_uint4(pv[4 * v], pv[4 * v + 1], pv[4 * v + 2], pv[4 * v + 3]);
+          dk[v] = make_uint4(pkk[4 * v], pkk[4 * v + 1], pkk[4 * v + 2], pkk[4 * v + 3]);
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kIssA) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct BwdLayout {
+  size_t plan, stats, counter, total;
+};
+BwdLayout bwd_layout(int64_t batch, int32_t hq, int64_t seq, int32_t lp, int32_t w) {
+  BwdLayout L;
+  L.plan = prefill_plan_bytes(seq, prefill_plan_tiles(seq, lp, w));
+  const int64_t s_pad = (seq + kT - 1) / kT * kT;
+  L.stats = align256(size_t(batch) * hq * s_pad * 4);
+  L.counter = 256;
+  L.total = align256(L.plan) + 2 * L.stats + L.counter;
+  return L;
+}
+
+bool set_smem(const void* fn, size_t bytes, bool* done, const char* what, int* rc) {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) dev = 0;
+  if (!done[dev]) {
+    *rc = check_cuda(cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          static_cast<int>(bytes)),
+                     what);
+    if (*rc != PS_OK) return false;
+    done[dev] = true;
+  }
+  return true;
+}
+
+}  // namespace
+
+size_t prefill_bwd_workspace_bytes(int64_t batch, int32_t hq, int64_t seq, int32_t lp, int32_t w) {
+  return bwd_layout(batch, hq, seq, lp, w).total;
+}
+
+int launch_prefill_bwd(const PrefillBwdLaunch& l, cudaStream_t stream) {
+  const int64_t nq = (l.seq + kT - 1) / kT;
+  const int64_t s_pad = nq * kT;
+  const BwdLayout L = bwd_layout(l.batch, l.hq, l.seq, l.lp, l.w);
+  char* ws = static_cast<char*>(l.workspace);
+  const int64_t n_tiles = prefill_plan_tiles(l.seq, l.lp, l.w);
+  int rc = check_cuda(launch_plan(l.seq, l.lp, l.w, n_tiles, ws, nullptr, stream),
+                      "plan_kernel launch");
+  if (rc != PS_OK) return rc;
+
+  BwdArgs a;
+  a.status = l.status;
+  a.seq = l.seq;
+  a.s_pad = s_pad;
+  a.batch = static_cast<int32_t>(l.batch);
+  a.hq = l.hq;
+  a.hkv = l.hkv;
+  a.group = l.hq / l.hkv;
+  a.nq = static_cast<int32_t>(nq);
+  a.lp = l.lp;
+  a.w = l.w;
+  a.scale = l.scale;
+  a.scale_log2 = l.scale * kLog2e;
+  a.off = reinterpret_cast<const int32_t*>(ws);
+  a.ent = reinterpret_cast<const int32_t*>(ws + align256(size_t(nq + 1) * 4));
+  float* nl = reinterpret_cast<float*>(ws + align256(L.plan));
+  float* nd = reinterpret_cast<float*>(ws + align256(L.plan) + L.stats);
+  a.nl = nl;
+  a.nd = nd;
+  a.counter = reinterpret_cast<int32_t*>(ws + align256(L.plan) + 2 * L.stats);
+  a.dq = static_cast<__nv_bfloat16*>(l.dq);
+  a.dk = static_cast<__nv_bfloat16*>(l.dk);
+  a.dv = static_cast<__nv_bfloat16*>(l.dv);
+
+  const int64_t n_rows = l.batch * l.hq * s_pad;
+  const int rows_per_block = kPrepThreads / 32;
+  const int64_t prep_blocks = (n_rows + rows_per_block - 1) / rows_per_block;
+  if (prep_blocks > 0x7fffffffLL) return fail(PS_ERR_UNSUPPORTED, "prefill backward too large");
+  rc = check_cuda(launch_pdl(bwd_prep_kernel, dim3(static_cast<unsigned>(prep_blocks)),
+                             dim3(kPrepThreads), 0, stream,
+                             static_cast<const __nv_bfloat16*>(l.out),
+                             static_cast<const __nv_bfloat16*>(l.dout), l.lse, l.seq, l.hq, s_pad,
+                             n_rows, nl, nd, a.counter),
+                  "bwd_prep_kernel launch");
+  if (rc != PS_OK) return rc;
+
+  CUtensorMap mq, mdo, mk, mv;
+  const uint64_t dq_dims[4] = {kHeadDim, (uint64_t)l.hq, (uint64_t)l.seq, (uint64_t)l.batch};
+  const uint64_t dk_dims[4] = {kHeadDim, (uint64_t)l.hkv, (uint64_t)l.seq, (uint64_t)l.batch};
+  const uint32_t box[4] = {64, 1, 128, 1};
+  if (!make_map_4d(&mq, l.q, dq_dims, box) || !make_map_4d(&mdo, l.dout, dq_dims, box) ||
+      !make_map_4d(&mk, l.k, dk_dims, box) || !make_map_4d(&mv, l.v, dk_dims, box))
+    return PS_ERR_CUDA;
+
+  static bool dq_attr[64] = {false}, kv_attr[64] = {false};
+  if (!set_smem(reinterpret_cast<const void*>(bwd_dq_kernel), kDqSmem, dq_attr,
+                "cudaFuncSetAttribute(bwd_dq_kernel)", &rc) ||
+      !set_smem(reinterpret_cast<const void*>(bwd_dkdv_kernel), kDkdvSmem, kv_attr,
+                "cudaFuncSetAttribute(bwd_dkdv_kernel)", &rc))
+    return rc;
+  const int64_t sms = sm_count();
+  const int64_t q_items = l.batch * l.hq * nq;
+  const int64_t kv_items = l.batch * l.hkv * nq;
+  if (q_items > 0x7fffffffLL) return fail(PS_ERR_UNSUPPORTED, "prefill backward too large");
+  rc = check_cuda(launch_pdl(bwd_dq_kernel, dim3(static_cast<unsigned>(q_items < sms ? q_items : sms)),
+                             dim3(kThreads), kDqSmem, stream, mq, mdo, mk, mv, a),
+                  "bwd_dq_kernel launch");
+  if (rc != PS_OK) return rc;
+  return check_cuda(
+      launch_pdl(bwd_dkdv_kernel, dim3(static_cast<unsigned>(kv_items < sms ? kv_items : sms)),
+                 dim3(kThreads), kDkdvSmem, stream, mq, mdo, mk, mv, a),
+      "bwd_dkdv_kernel launch");
+}
+
+}  // namespace ps

@@ -191,4 +191,23 @@ PS_HD int64_t qtile_count(int64_t qt, int64_t seq, int32_t lp, int32_t w, int32_
   return c;
 }
 
+// Query tiles that hold a visible pair with key tile kt (square tiles, b = Bq = Bk):
+// key k is seen by the queries [k, seq) when k < lp and [k, min(seq, k + w)) otherwise; over
+// the keys of the tile these intervals overlap, so their union [k0, last] is contiguous and
+// every query tile in [k0 / b, last / b] is non-SKIP.  Returns false if the tile is empty.
+PS_HD bool ktile_qrange(int64_t kt, int64_t seq, int32_t lp, int32_t w, int32_t b, int64_t* qlo,
+                        int64_t* qhi) {
+  const int64_t k0 = kt * b;
+  if (k0 >= seq) return false;
+  const int64_t k1 = (k0 + b < seq ? k0 + b : seq);  // one past the last in-range key
+  int64_t last = seq - 1;
+  if (k0 >= lp) {
+    const int64_t l = k1 - 1 + w - 1;  // last query that sees the tile's last key
+    if (l < last) last = l;
+  }
+  *qlo = k0 / b;
+  *qhi = last / b;
+  return true;
+}
+
 }  // namespace ps

@@ -133,3 +133,26 @@ def test_workspace_too_small_rejected(lib):
     rc = lib.ps_masked_prefill_attn(ctypes.byref(p), 16, 16, 16, 1, 8192, 16, None, None, 0, None,
                                     16, need - 1, None, None)
     assert rc == B.PS_ERR_WORKSPACE
+
+
+def test_prefill_bwd_host_validation(lib):
+    """The backward checks pointers, alignment and workspace on the host, before any launch."""
+    p = _params(n_q_heads=28, n_kv_heads=4, l_prefix=256, window=2048)
+    need = B.ps_prefill_bwd_workspace_bytes(p, 4, 8192)
+    # plan + two fp32 statistics per (batch, head, row) + the work counter
+    plan = B.ps_prefill_workspace_bytes(p, 4, 8192)
+    assert need >= plan + 2 * 4 * 28 * 8192 * 4 + 256
+    f = lib.ps_masked_prefill_attn_bwd
+    ok = [16] * 5
+    args = lambda ptrs, lse=16, grads=(16, 16, 16), ws=256, wsb=need: (  # noqa: E731
+        ctypes.byref(p), *ptrs, lse, 4, 8192, *grads, ws, wsb, None, None)
+    assert f(*args(ok, lse=None)) == B.PS_ERR_INVALID_ARG          # lse is required
+    assert f(*args([16, 16, 16, 16, None])) == B.PS_ERR_INVALID_ARG  # dout NULL
+    assert f(*args([16, 16, 8, 16, 16])) == B.PS_ERR_INVALID_ARG     # v misaligned
+    assert f(*args(ok, grads=(16, None, 16))) == B.PS_ERR_INVALID_ARG
+    assert f(*args(ok, wsb=need - 1)) == B.PS_ERR_WORKSPACE
+    assert f(*args(ok, ws=None)) == B.PS_ERR_WORKSPACE
+    assert f(*args(ok, ws=272)) == B.PS_ERR_INVALID_ARG              # workspace not 256-aligned
+    assert f(ctypes.byref(p), *ok, 16, 4, 0, 16, 16, 16, 256, need, None, None) == \
+        B.PS_ERR_INVALID_ARG                                          # seq < 1
+    assert f(ctypes.byref(p), *ok, 16, 0, 8192, 16, 16, 16, None, 0, None, None) == B.PS_OK
