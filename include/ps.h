@@ -79,7 +79,10 @@ typedef struct {
  *   k_prefix, v_prefix : [batch, Hkv, l_prefix, D]   (may be NULL when l_prefix == 0)
  *   k_ring,   v_ring   : [batch, Hkv, W, D]
  * A linear full-attention cache is the same struct with l_prefix = Lmax, window = 1 and
- * the ring pointers NULL; every position must then be < Lmax. */
+ * the ring pointers NULL; every position must then be < Lmax.
+ * A ring-only cache has both prefix pointers NULL (and the ring set): ps_kv_append_rope then
+ * writes only ring slots and skips tokens below l_prefix (PS_DEV_POS_RANGE); the prefix rows
+ * live elsewhere, e.g. shared by a group of sequences (ps_decode_attn_shared_prefix). */
 typedef struct {
   void* k_prefix;
   void* v_prefix;
@@ -142,6 +145,34 @@ int ps_decode_attn(const ps_params* params, const ps_kv_cache* cache, const void
 int ps_decode_attn_noalloc(const ps_params* params, const ps_kv_cache* cache, const void* q,
                            const int64_t* pos, void* out, float* lse, int32_t* dev_status,
                            ps_stream_t stream);
+
+/* Bytes of device workspace ps_decode_attn_shared_prefix needs (the split-K partials of
+ * the window pass plus one fp32 prefix partial per (sequence, query head)).  0 on invalid
+ * arguments. */
+size_t ps_decode_shared_prefix_workspace_bytes(const ps_params* params, int64_t batch);
+
+/* Decode step for groups of sequences that share one prompt prefix.  Source: eq. A(i)
+ * (§核心机制: every sequence pins its prompt as the prefix), §Kernel 实现 (the sampling code
+ * sends one prompt per request; the accuracy tables average many samples of one problem):
+ * the sequences of a group attend the same l_prefix rows, so those rows are read once per
+ * group instead of once per sequence.  Results equal ps_decode_attn on a cache whose
+ * prefix of every sequence is its group's prefix.
+ *   cache->k_prefix, v_prefix : device bf16 [batch / group_size, Hkv, l_prefix, D]: the
+ *                  prefix of group j is shared by sequences [j * group_size, (j+1) * group_size).
+ *                  Fill it with ps_kv_append_rope on a linear cache of batch / group_size
+ *                  sequences (ring NULL, positions 0 .. l_prefix - 1).
+ *   cache->k_ring, v_ring     : device bf16 [batch, Hkv, W, D], one ring per sequence; append
+ *                  decode tokens with a ring-only cache (prefix pointers NULL).
+ *   cache->batch  : number of sequences, a multiple of group_size.
+ *   group_size    : sequences per shared prefix, >= 1.
+ *   q, pos, out, lse, dev_status : as ps_decode_attn.
+ *   workspace, ws_bytes : device scratch of at least
+ *                  ps_decode_shared_prefix_workspace_bytes(), 256-byte aligned.
+ * Requires l_prefix >= 1 and 1 <= Hq / Hkv <= 8. */
+int ps_decode_attn_shared_prefix(const ps_params* params, const ps_kv_cache* cache,
+                                 int64_t group_size, const void* q, const int64_t* pos,
+                                 void* out, float* lse, void* workspace, size_t ws_bytes,
+                                 int32_t* dev_status, ps_stream_t stream);
 
 /* Bytes of device workspace ps_full_attn_ref needs (same split-K layout as decode). */
 size_t ps_full_attn_workspace_bytes(const ps_params* params, int64_t batch, int64_t lmax);

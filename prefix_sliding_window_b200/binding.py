@@ -82,6 +82,10 @@ _SIGS = {
                                          c_int64, c_void_p, c_void_p, c_void_p, c_int64,
                                          POINTER(c_int64), c_void_p, c_size_t, c_void_p,
                                          c_void_p]),
+    "ps_decode_shared_prefix_workspace_bytes": (c_size_t, [POINTER(PsParams), c_int64]),
+    "ps_decode_attn_shared_prefix": (c_int32, [POINTER(PsParams), POINTER(PsKVCache), c_int64,
+                                               c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                               c_size_t, c_void_p, c_void_p]),
     "ps_prefill_bwd_workspace_bytes": (c_size_t, [POINTER(PsParams), c_int64, c_int64]),
     "ps_masked_prefill_attn_bwd": (c_int32, [POINTER(PsParams), c_void_p, c_void_p, c_void_p,
                                              c_void_p, c_void_p, c_void_p, c_int64, c_int64,
@@ -180,6 +184,23 @@ def ps_decode_attn_noalloc(params: PsParams, cache: PsKVCache, q, pos, out, lse=
                                        _ptr(pos), _ptr(out), _ptr(lse), _ptr(dev_status),
                                        _stream(stream))
     _check(rc, "ps_decode_attn_noalloc")
+
+
+def ps_decode_shared_prefix_workspace_bytes(params: PsParams, batch: int) -> int:
+    return int(load().ps_decode_shared_prefix_workspace_bytes(ctypes.byref(params), int(batch)))
+
+
+def ps_decode_attn_shared_prefix(params: PsParams, cache: PsKVCache, group_size: int, q, pos,
+                                 out, lse=None, workspace=None, dev_status=None,
+                                 stream=None) -> None:
+    """Decode where sequences [j*group_size, (j+1)*group_size) share prefix j of
+    cache.k_prefix / v_prefix ([batch / group_size, Hkv, l_prefix, D])."""
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rc = load().ps_decode_attn_shared_prefix(ctypes.byref(params), ctypes.byref(cache),
+                                             int(group_size), _ptr(q), _ptr(pos), _ptr(out),
+                                             _ptr(lse), _ptr(workspace), ws_bytes,
+                                             _ptr(dev_status), _stream(stream))
+    _check(rc, "ps_decode_attn_shared_prefix")
 
 
 def ps_full_attn_workspace_bytes(params: PsParams, batch: int, lmax: int) -> int:

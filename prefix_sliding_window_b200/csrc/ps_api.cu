@@ -177,7 +177,10 @@ int ps_kv_append_rope(const ps_params* params, const ps_kv_cache* cache, const v
     PS_TRY(check_ptr(cache->k_ring, "cache->k_ring"));
     PS_TRY(check_ptr(cache->v_ring, "cache->v_ring"));
   }
-  if (params->l_prefix > 0 || linear) {
+  // a ring cache whose prefix pointers are both NULL is ring-only: tokens at positions
+  // below l_prefix are skipped (their prefix rows live elsewhere)
+  const bool ring_only = !linear && cache->k_prefix == nullptr && cache->v_prefix == nullptr;
+  if ((params->l_prefix > 0 && !ring_only) || linear) {
     PS_TRY(check_ptr(cache->k_prefix, "cache->k_prefix"));
     PS_TRY(check_ptr(cache->v_prefix, "cache->v_prefix"));
   }
@@ -503,6 +506,96 @@ int ps_masked_prefill_attn_bwd(const ps_params* params, const void* q, const voi
   l.scale = resolve_scale(params);
   l.status = dev_status;
   return launch_prefill_bwd(l, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t ps_decode_shared_prefix_workspace_bytes(const ps_params* params, int64_t batch) {
+  if (check_params(params, true) != PS_OK || batch < 0) return 0;
+  const size_t dec = decode_workspace_bytes(batch, params->n_kv_heads,
+                                            (int64_t)params->l_prefix + params->window);
+  const size_t o = (size_t(batch) * params->n_q_heads * kHeadDim * 4 + 255) & ~size_t(255);
+  const size_t l = (size_t(batch) * params->n_q_heads * 4 + 255) & ~size_t(255);
+  return ((dec + 255) & ~size_t(255)) + o + l;
+}
+
+int ps_decode_attn_shared_prefix(const ps_params* params, const ps_kv_cache* cache,
+                                 int64_t group_size, const void* q, const int64_t* pos,
+                                 void* out, float* lse, void* workspace, size_t ws_bytes,
+                                 int32_t* dev_status, ps_stream_t stream) {
+  g_last_error.clear();
+  PS_TRY(check_params(params, true));
+  if (params->n_q_heads / params->n_kv_heads > kMaxGroup)
+    return fail(PS_ERR_UNSUPPORTED, "decode supports at most 8 query heads per KV head");
+  if (params->l_prefix < 1)
+    return fail(PS_ERR_INVALID_ARG, "shared-prefix decode needs l_prefix >= 1");
+  if (!cache) return fail(PS_ERR_INVALID_ARG, "cache is NULL");
+  if (cache->batch < 0) return fail(PS_ERR_INVALID_ARG, "cache->batch must be >= 0");
+  if (group_size < 1) return fail(PS_ERR_INVALID_ARG, "group_size must be >= 1");
+  if (cache->batch % group_size != 0)
+    return fail(PS_ERR_INVALID_ARG, "batch must be a multiple of group_size");
+  if (cache->batch == 0) return PS_OK;
+  if (group_size * (params->n_q_heads / params->n_kv_heads) > 0x7fffffffLL)
+    return fail(PS_ERR_UNSUPPORTED, "group_size too large");
+  PS_TRY(check_ptr(cache->k_ring, "cache->k_ring"));
+  PS_TRY(check_ptr(cache->v_ring, "cache->v_ring"));
+  PS_TRY(check_ptr(cache->k_prefix, "cache->k_prefix"));
+  PS_TRY(check_ptr(cache->v_prefix, "cache->v_prefix"));
+  PS_TRY(check_ptr(q, "q"));
+  PS_TRY(check_ptr(out, "out"));
+  PS_TRY(check_ptr(lse, "lse", true));
+  if (!pos) return fail(PS_ERR_INVALID_ARG, "pos is NULL");
+  if ((reinterpret_cast<uintptr_t>(pos) & 7u) != 0)
+    return fail(PS_ERR_INVALID_ARG, "pos is not 8-byte aligned");
+  if ((reinterpret_cast<uintptr_t>(dev_status) & 3u) != 0)
+    return fail(PS_ERR_INVALID_ARG, "dev_status is not 4-byte aligned");
+  const size_t need = ps_decode_shared_prefix_workspace_bytes(params, cache->batch);
+  if (!workspace || ws_bytes < need)
+    return fail(PS_ERR_WORKSPACE, "workspace smaller than ps_decode_shared_prefix_workspace_bytes()");
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return fail(PS_ERR_INVALID_ARG, "workspace is not 256-byte aligned");
+  const size_t dec = decode_workspace_bytes(cache->batch, params->n_kv_heads,
+                                            (int64_t)params->l_prefix + params->window);
+  char* ws = static_cast<char*>(workspace);
+  float* o_pre = reinterpret_cast<float*>(ws + ((dec + 255) & ~size_t(255)));
+  float* lse2_pre = reinterpret_cast<float*>(
+      reinterpret_cast<char*>(o_pre) +
+      ((size_t(cache->batch) * params->n_q_heads * kHeadDim * 4 + 255) & ~size_t(255)));
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  SharedPrefixLaunch sp{};
+  sp.q = q;
+  sp.pos = pos;
+  sp.k_pre = cache->k_prefix;
+  sp.v_pre = cache->v_prefix;
+  sp.o_pre = o_pre;
+  sp.lse2_pre = lse2_pre;
+  sp.status = dev_status;
+  sp.batch = cache->batch;
+  sp.gsize = group_size;
+  sp.hq = params->n_q_heads;
+  sp.hkv = params->n_kv_heads;
+  sp.lp = params->l_prefix;
+  sp.scale = resolve_scale(params);
+  PS_TRY(launch_shared_prefix(sp, st));
+  DecodeLaunch l{};
+  l.q = q;
+  l.pos = pos;
+  l.out = out;
+  l.lse = lse;
+  l.workspace = dec > 0 ? workspace : nullptr;
+  l.status = dev_status;
+  l.batch = cache->batch;
+  l.hq = params->n_q_heads;
+  l.hkv = params->n_kv_heads;
+  l.lp = params->l_prefix;
+  l.w = params->window;
+  l.scale = resolve_scale(params);
+  l.k0 = cache->k_prefix;
+  l.v0 = cache->v_prefix;
+  l.k1 = cache->k_ring;
+  l.v1 = cache->v_ring;
+  l.skip_prefix = 1;
+  l.pre_o = o_pre;
+  l.pre_lse2 = lse2_pre;
+  return launch_decode(l, st);
 }
 
 }  // extern "C"

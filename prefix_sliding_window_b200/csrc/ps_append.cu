@@ -71,6 +71,11 @@ __global__ void __launch_bounds__(kAppendThreads) append_rope_kernel(const Appen
   __nv_bfloat16* k_dst_base = nullptr;
   __nv_bfloat16* v_dst_base = nullptr;
   int64_t row_stride_rows = 0, row = 0;
+  if (p < a.lp && a.k_pre == nullptr) {
+    // ring-only cache (the prefix lives elsewhere, e.g. shared by a group of sequences)
+    if (threadIdx.x == 0 && a.status) atomicOr(a.status, PS_DEV_POS_RANGE);
+    return;
+  }
   if (p < a.lp) {
     k_dst_base = static_cast<__nv_bfloat16*>(a.k_pre);
     v_dst_base = static_cast<__nv_bfloat16*>(a.v_pre);

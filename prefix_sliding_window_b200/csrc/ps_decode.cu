@@ -73,6 +73,9 @@ struct DecodeArgs {
   int32_t streamk, full_mode;
   int64_t lmax;
   float scale_log2;
+  int32_t skip_prefix;     // shared-prefix decode: window rows only
+  const float* pre_o;      // shared-prefix partials folded in at flush (per-unit schedule)
+  const float* pre_lse2;
 };
 
 // Offset of the 16-byte chunk `chunk` (0..7) of box row `row` under the 128-byte swizzle
@@ -92,6 +95,7 @@ __device__ __forceinline__ DecodeTiling tiling_of(const DecodeArgs& a, int64_t p
       r.pre_len = static_cast<int32_t>(p + 1);
     else
       r = visible_ranges(p, a.lp, a.w);
+    if (a.skip_prefix) r.pre_len = 0;  // the shared-prefix pass covers those rows
   }
   return make_tiling(r, a.dim0, a.w);
 }
@@ -353,6 +357,26 @@ __global__ void __launch_bounds__(kThreads)
       named_bar_sync(1, kConsumerThreads);
       if (warp == 0) {
         merge_state(m0, m1, l0, l1, o, flush + lane * 36);
+        if (a.pre_o && !a.streamk) {
+          // fold in the shared-prefix partial (normalised o, weight 2^lse2) of heads 2qq,
+          // 2qq + 1 at this lane's fragment positions; slots 32.. of the flush area are free
+          float* other = flush + (32 + lane) * 36;
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int hh = 2 * qq + e;
+            const bool valid = hh < a.group;
+            const int64_t row = (int64_t)b * a.hq + h * a.group + hh;
+            other[32 + e] = valid ? a.pre_lse2[row] : -INFINITY;
+            other[34 + e] = 1.f;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const int d0 = 16 * j + (lane >> 2);
+              other[4 * j + e] = valid ? a.pre_o[row * kHeadDim + d0] : 0.f;
+              other[4 * j + 2 + e] = valid ? a.pre_o[row * kHeadDim + d0 + 8] : 0.f;
+            }
+          }
+          merge_state(m0, m1, l0, l1, o, other);
+        }
         const int unit = b * a.hkv + h;
         const int64_t slot = (int64_t)unit + blockIdx.x;  // unique per (unit, CTA) piece
 #pragma unroll
@@ -515,7 +539,8 @@ __global__ void __launch_bounds__(128)
     merge_kernel(const float* __restrict__ ws_o, const float* __restrict__ ws_lse,
                  const int32_t* __restrict__ pref, const int32_t* __restrict__ span,
                  __nv_bfloat16* __restrict__ out, float* __restrict__ lse, int32_t batch,
-                 int32_t hq, int32_t hkv, int32_t group, int32_t grid) {
+                 int32_t hq, int32_t hkv, int32_t group, int32_t grid,
+                 const float* __restrict__ pre_o, const float* __restrict__ pre_lse2) {
   const int64_t bh = (int64_t)blockIdx.x * 4 + (threadIdx.x >> 5);
   if (bh >= (int64_t)batch * hq) return;
   const int lane = threadIdx.x & 31;
@@ -527,6 +552,16 @@ __global__ void __launch_bounds__(128)
   const int64_t total = (int64_t)hkv * pref[batch];
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   float lse2 = -INFINITY;
+  // online combine state; a shared-prefix partial (normalised, weight 2^lse2) starts it
+  float M = -INFINITY, wsum = 0.f;
+  if (pre_o) {
+    const float l2 = pre_lse2[bh];
+    if (l2 != -INFINITY) {
+      M = l2;
+      wsum = 1.f;
+      acc = reinterpret_cast<const float4*>(pre_o + bh * kHeadDim)[lane];
+    }
+  }
   if (sp.x <= sp.y) {
     const int c_lo = sp.x, c_hi = sp.y;
     // with fewer tiles than CTAs some CTAs own nothing and wrote no piece
@@ -535,7 +570,6 @@ __global__ void __launch_bounds__(128)
       return maybe_empty && total * c / grid == total * (c + 1) / grid;
     };
     // online combine, four pieces per round: their lse and o are loaded together
-    float M = -INFINITY, wsum = 0.f;
     for (int c0 = c_lo; c0 <= c_hi; c0 += 4) {
       float lv[4];
       float4 ov[4];
@@ -570,14 +604,14 @@ __global__ void __launch_bounds__(128)
       }
       M = Mn;
     }
-    if (M != -INFINITY) {
-      const float inv = 1.f / wsum;
-      acc.x *= inv;
-      acc.y *= inv;
-      acc.z *= inv;
-      acc.w *= inv;
-      lse2 = M + log2f(wsum);
-    }
+  }
+  if (M != -INFINITY) {
+    const float inv = 1.f / wsum;
+    acc.x *= inv;
+    acc.y *= inv;
+    acc.z *= inv;
+    acc.w *= inv;
+    lse2 = M + log2f(wsum);
   }
   uint2 pk;
   pk.x = pack_bf16x2(acc.x, acc.y);
@@ -651,7 +685,8 @@ int launch_decode(const DecodeLaunch& l, cudaStream_t stream) {
   const int64_t max_keys = l.full_mode ? l.lmax : (int64_t)l.lp + l.w;
   const int64_t g = streamk_grid(l.batch, l.hkv, max_keys);
   const int64_t units = l.batch * l.hkv;
-  const int32_t dim0 = l.full_mode ? static_cast<int32_t>(l.lmax) : l.lp;
+  // window-only decode reads no prefix rows: no prefix map (it may describe fewer units)
+  const int32_t dim0 = l.full_mode ? static_cast<int32_t>(l.lmax) : (l.skip_prefix ? 0 : l.lp);
 
   CUtensorMap mk0, mv0, mk1, mv1;
   // A zero-row tensor cannot be described; such a map is never used (no tiles), so it
@@ -702,6 +737,9 @@ int launch_decode(const DecodeLaunch& l, cudaStream_t stream) {
   a.full_mode = l.full_mode;
   a.lmax = l.lmax;
   a.scale_log2 = l.scale * kLog2e;
+  a.skip_prefix = l.skip_prefix;
+  a.pre_o = l.pre_o;
+  a.pre_lse2 = l.pre_lse2;
 
   const size_t sb = smem_bytes(kStages);
   occupancy_per_sm();  // sets the shared-memory attribute once per device
@@ -719,7 +757,7 @@ int launch_decode(const DecodeLaunch& l, cudaStream_t stream) {
                    0, stream, static_cast<const float*>(a.ws_o),
                    static_cast<const float*>(a.ws_lse), static_cast<const int32_t*>(a.ws_pref),
                    static_cast<const int32_t*>(a.ws_span), a.out, a.lse, a.batch, l.hq, l.hkv,
-                   group, static_cast<int32_t>(g)),
+                   group, static_cast<int32_t>(g), l.pre_o, l.pre_lse2),
         "merge_kernel launch");
   }
   return rc;

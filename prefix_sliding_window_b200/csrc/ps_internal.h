@@ -84,11 +84,32 @@ struct DecodeLaunch {
   float scale;
   const void *k0, *v0;  // prefix (or linear) cache
   const void *k1, *v1;  // ring (unused in full mode)
+  // Shared-prefix decode: read only the window (the prefix rows are skipped) and fold in a
+  // precomputed prefix partial per (sequence, query head): normalised fp32 o [batch, Hq, D]
+  // and its base-2 lse [batch, Hq] (scores scaled by scale * log2 e).
+  int32_t skip_prefix;
+  const float* pre_o;
+  const float* pre_lse2;
 };
 // Split count and workspace bytes for a decode of this shape on the current device.
 int decode_splits(int64_t batch, int32_t hkv, int64_t max_keys);
 size_t decode_workspace_bytes(int64_t batch, int32_t hkv, int64_t max_keys);
 int launch_decode(const DecodeLaunch& a, cudaStream_t stream);
+// Shared-prefix pass: attention of every (sequence, query head) of a group of `gsize`
+// sequences over the group's prefix rows [0, min(pos + 1, lp)); writes o_pre/lse2_pre.
+struct SharedPrefixLaunch {
+  const void* q;         // [batch, Hq, D]
+  const int64_t* pos;    // [batch]
+  const void* k_pre;     // [batch / gsize, Hkv, lp, D]
+  const void* v_pre;
+  float* o_pre;          // [batch, Hq, D]
+  float* lse2_pre;       // [batch, Hq]
+  int32_t* status;
+  int64_t batch, gsize;
+  int32_t hq, hkv, lp;
+  float scale;
+};
+int launch_shared_prefix(const SharedPrefixLaunch& l, cudaStream_t stream);
 // Decode whose split-K scratch is the library's file-scope device array (no allocation).
 constexpr size_t kDecodeScratchBytes = size_t(4) << 20;
 int launch_decode_static_scratch(const DecodeLaunch& a, cudaStream_t stream);
