@@ -660,6 +660,70 @@ def run_sweep(dev, steps: int = 20, warmup: int = 3):
             "peak_hbm_gbs": peaks["hbm_gbs"]}
 
 
+# ------------------------------------------------------- shared-prefix decode leg
+def run_shared(dev, steps: int = 20, warmup: int = 3):
+    """Shared-prefix decode: 256 sequences in 4 groups of 64 share their group's 2000-token
+    prompt prefix; W = 4096; positions U[8192, 131072] (full windows).  The same batch runs
+    through plain decode with the prefix copied into every sequence.  Attention calls only
+    (the append is the same for both); HBM GB/s on each path's algorithmic bytes."""
+    from prefix_sliding_window_b200 import binding as B
+    wl = synth.WORKLOADS["decode_shared_b256_g64_lp2000_w4096"]
+    Bn, hq, hkv, lp, w, gs = (wl.batch, wl.n_q_heads, wl.n_kv_heads, wl.l_prefix, wl.window,
+                              wl.group_size)
+    G = Bn // gs
+    peaks = _peaks()
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    seed = synth.seed_for(wl.index)
+    pos = synth.uniform_positions(Bn, wl.pos_lo, wl.pos_hi, seed, dev)
+    params = B.make_params(hq, hkv, D, lp, w, wl.rope_theta)
+    # cache contents do not change the work; N(0,1) values stand in for rotated keys
+    pre_k = synth.normal_bf16((G, hkv, lp, D), seed + 1, dev)
+    pre_v = synth.normal_bf16((G, hkv, lp, D), seed + 2, dev)
+    ring_k = synth.normal_bf16((Bn, hkv, w, D), seed + 3, dev)
+    ring_v = synth.normal_bf16((Bn, hkv, w, D), seed + 4, dev)
+    grp = torch.arange(Bn, device=dev) // gs
+    copy_k, copy_v = pre_k[grp].contiguous(), pre_v[grp].contiguous()
+    q = synth.normal_bf16((Bn, hq, D), seed + 5, dev)
+    out = torch.empty((Bn, hq, D), dtype=torch.bfloat16, device=dev)
+    shared = B.make_cache(pre_k, pre_v, ring_k, ring_v, Bn)
+    plain = B.make_cache(copy_k, copy_v, ring_k, ring_v, Bn)
+    ws_s = torch.empty(B.ps_decode_shared_prefix_workspace_bytes(params, Bn, gs),
+                       dtype=torch.uint8, device=dev)
+    ws_p = torch.empty(max(1, B.ps_decode_workspace_bytes(params, Bn)), dtype=torch.uint8,
+                       device=dev)
+    stream = torch.cuda.current_stream()
+    calls = {
+        "shared_prefix": lambda: B.ps_decode_attn_shared_prefix(params, shared, gs, q, pos, out,
+                                                                None, ws_s, st),
+        "plain": lambda: B.ps_decode_attn(params, plain, q, pos, out, None, ws_p, st),
+    }
+    kv_tok = 2 * hkv * D * 2
+    qo = 2 * Bn * hq * D * 2
+    bytes_ = {"shared_prefix": G * lp * kv_tok + Bn * w * kv_tok + qo,
+              "plain": Bn * (lp + w) * kv_tok + qo}
+    res = {}
+    for name, fn in calls.items():
+        for _ in range(warmup):
+            fn()
+        torch.cuda.synchronize()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(steps)]
+        for a, b in evs:
+            a.record(stream)
+            fn()
+            b.record(stream)
+        torch.cuda.synchronize()
+        assert st.item() == 0, st.item()
+        ms = statistics.median([a.elapsed_time(b) for a, b in evs])
+        gbs = bytes_[name] / (ms / 1e3) / 1e9
+        res[name] = {"attn_us": round(ms * 1e3, 1), "tok_per_s": round(Bn / (ms / 1e3), 1),
+                     "bytes_per_call": int(bytes_[name]), "gbs": round(gbs, 1),
+                     "frac": round(gbs / peaks["hbm_gbs"], 4)}
+    res["speedup"] = round(res["plain"]["attn_us"] / res["shared_prefix"]["attn_us"], 3)
+    return {"leg": "shared", "workload": wl.name, "groups": G, "group_size": gs, "steps": steps,
+            "peak_hbm_gbs": peaks["hbm_gbs"], **res}
+
+
 # ------------------------------------------------------- full-stack decode leg
 def run_stack(dev, batch: int, distinct: int, steps: int = 3, warmup: int = 1):
     """Full-stack decode step: 28 layers x (append + decode), 16/2/128, L_prefix 2000,
@@ -813,7 +877,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true",
                     help="launch the timed steps one by one instead of as a CUDA graph")
-    ap.add_argument("--leg", default="main", choices=["main", "prefill", "sweep", "stack", "latency"],
+    ap.add_argument("--leg", default="main", choices=["main", "prefill", "sweep", "stack", "latency",
+                                                      "shared"],
                     help="main: the driver's line; prefill/sweep/stack: one extra workload")
     ap.add_argument("--stack-batch", type=int, default=1024)
     ap.add_argument("--stack-distinct", type=int, default=6)
@@ -839,6 +904,8 @@ def main():
             res = run_sweep(dev)
         elif args.leg == "latency":
             res = run_latency(dev)
+        elif args.leg == "shared":
+            res = run_shared(dev)
         else:
             res = run_stack(dev, args.stack_batch, args.stack_distinct)
         if rank == 0:

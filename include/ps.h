@@ -146,10 +146,11 @@ int ps_decode_attn_noalloc(const ps_params* params, const ps_kv_cache* cache, co
                            const int64_t* pos, void* out, float* lse, int32_t* dev_status,
                            ps_stream_t stream);
 
-/* Bytes of device workspace ps_decode_attn_shared_prefix needs (the split-K partials of
- * the window pass plus one fp32 prefix partial per (sequence, query head)).  0 on invalid
- * arguments. */
-size_t ps_decode_shared_prefix_workspace_bytes(const ps_params* params, int64_t batch);
+/* Bytes of device workspace ps_decode_attn_shared_prefix needs for this batch and group
+ * size (the split-K partials of the window pass plus fp32 prefix partials per (sequence,
+ * query head) and prefix key range).  0 on invalid arguments. */
+size_t ps_decode_shared_prefix_workspace_bytes(const ps_params* params, int64_t batch,
+                                               int64_t group_size);
 
 /* Decode step for groups of sequences that share one prompt prefix.  Source: eq. A(i)
  * (§核心机制: every sequence pins its prompt as the prefix), §Kernel 实现 (the sampling code
@@ -168,7 +169,11 @@ size_t ps_decode_shared_prefix_workspace_bytes(const ps_params* params, int64_t 
  *   q, pos, out, lse, dev_status : as ps_decode_attn.
  *   workspace, ws_bytes : device scratch of at least
  *                  ps_decode_shared_prefix_workspace_bytes(), 256-byte aligned.
- * Requires l_prefix >= 1 and 1 <= Hq / Hkv <= 8. */
+ * The prefix pass runs on an internal side stream of the library (one per device, created
+ * on first use), forked from `stream` before the window decode and joined before the final
+ * merge, so it overlaps the window decode; the call stays asynchronous and ordered on
+ * `stream`.
+ * Requires l_prefix >= 1, 1 <= Hq / Hkv <= 8 and batch <= 1024 (PS_ERR_UNSUPPORTED). */
 int ps_decode_attn_shared_prefix(const ps_params* params, const ps_kv_cache* cache,
                                  int64_t group_size, const void* q, const int64_t* pos,
                                  void* out, float* lse, void* workspace, size_t ws_bytes,

@@ -82,7 +82,8 @@ _SIGS = {
                                          c_int64, c_void_p, c_void_p, c_void_p, c_int64,
                                          POINTER(c_int64), c_void_p, c_size_t, c_void_p,
                                          c_void_p]),
-    "ps_decode_shared_prefix_workspace_bytes": (c_size_t, [POINTER(PsParams), c_int64]),
+    "ps_decode_shared_prefix_workspace_bytes": (c_size_t, [POINTER(PsParams), c_int64,
+                                                           c_int64]),
     "ps_decode_attn_shared_prefix": (c_int32, [POINTER(PsParams), POINTER(PsKVCache), c_int64,
                                                c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                                c_size_t, c_void_p, c_void_p]),
@@ -186,8 +187,9 @@ def ps_decode_attn_noalloc(params: PsParams, cache: PsKVCache, q, pos, out, lse=
     _check(rc, "ps_decode_attn_noalloc")
 
 
-def ps_decode_shared_prefix_workspace_bytes(params: PsParams, batch: int) -> int:
-    return int(load().ps_decode_shared_prefix_workspace_bytes(ctypes.byref(params), int(batch)))
+def ps_decode_shared_prefix_workspace_bytes(params: PsParams, batch: int, group_size: int) -> int:
+    return int(load().ps_decode_shared_prefix_workspace_bytes(ctypes.byref(params), int(batch),
+                                                              int(group_size)))
 
 
 def ps_decode_attn_shared_prefix(params: PsParams, cache: PsKVCache, group_size: int, q, pos,

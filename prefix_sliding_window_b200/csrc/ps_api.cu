@@ -155,6 +155,67 @@ int sm_count() {
 
 }  // namespace ps
 
+namespace ps {
+namespace {
+// Shared-prefix decode workspace: [window-pass split-K partials][prefix partials o]
+// [prefix partials lse2], each part 256-byte aligned.
+struct SharedPrefixLayout {
+  size_t dec, o, lse, total;
+  int splits;
+};
+SharedPrefixLayout shared_prefix_layout(const ps_params* p, int64_t batch, int64_t gsize) {
+  SharedPrefixLayout L;
+  L.splits = shared_prefix_splits(batch, gsize, p->n_q_heads, p->n_kv_heads, p->l_prefix);
+  L.dec = (decode_workspace_bytes(batch, p->n_kv_heads, (int64_t)p->l_prefix + p->window, true) +
+           255) & ~size_t(255);
+  L.o = (size_t(L.splits) * batch * p->n_q_heads * kHeadDim * 4 + 255) & ~size_t(255);
+  L.lse = (size_t(L.splits) * batch * p->n_q_heads * 4 + 255) & ~size_t(255);
+  L.total = L.dec + L.o + L.lse;
+  return L;
+}
+// Side stream (one per device, created on first use) on which the shared-prefix pass runs
+// concurrently with the window decode.
+cudaStream_t side_stream(int* rc) {
+  static std::mutex mu;
+  static cudaStream_t streams[64] = {nullptr};
+  int dev = 0;
+  *rc = check_cuda(cudaGetDevice(&dev), "cudaGetDevice");
+  if (*rc != PS_OK) return nullptr;
+  if (dev < 0 || dev >= 64) {
+    *rc = fail(PS_ERR_UNSUPPORTED, "device index above 63");
+    return nullptr;
+  }
+  std::lock_guard<std::mutex> lock(mu);
+  if (!streams[dev]) {
+    *rc = check_cuda(cudaStreamCreateWithFlags(&streams[dev], cudaStreamNonBlocking),
+                     "cudaStreamCreateWithFlags");
+    if (*rc != PS_OK) return nullptr;
+  }
+  return streams[dev];
+}
+
+// Runs between the window decode and the merge: fork the caller's stream (at the point
+// recorded before the decode) onto the side stream, launch the prefix pass there, join.
+struct PrefixFork {
+  SharedPrefixLaunch sp;
+  cudaEvent_t fork;
+  cudaStream_t side;
+};
+int launch_prefix_forked(void* ctx, cudaStream_t stream) {
+  PrefixFork* f = static_cast<PrefixFork*>(ctx);
+  cudaEvent_t join = nullptr;
+  int rc = check_cuda(cudaEventCreateWithFlags(&join, cudaEventDisableTiming), "cudaEventCreate");
+  if (rc != PS_OK) return rc;
+  rc = check_cuda(cudaStreamWaitEvent(f->side, f->fork, 0), "cudaStreamWaitEvent");
+  if (rc == PS_OK) rc = launch_shared_prefix(f->sp, f->side);
+  if (rc == PS_OK) rc = check_cuda(cudaEventRecord(join, f->side), "cudaEventRecord");
+  if (rc == PS_OK) rc = check_cuda(cudaStreamWaitEvent(stream, join, 0), "cudaStreamWaitEvent");
+  cudaEventDestroy(join);  // released once the recorded work completes
+  return rc;
+}
+}  // namespace
+}  // namespace ps
+
 using namespace ps;
 
 extern "C" {
@@ -508,13 +569,12 @@ int ps_masked_prefill_attn_bwd(const ps_params* params, const void* q, const voi
   return launch_prefill_bwd(l, reinterpret_cast<cudaStream_t>(stream));
 }
 
-size_t ps_decode_shared_prefix_workspace_bytes(const ps_params* params, int64_t batch) {
-  if (check_params(params, true) != PS_OK || batch < 0) return 0;
-  const size_t dec = decode_workspace_bytes(batch, params->n_kv_heads,
-                                            (int64_t)params->l_prefix + params->window);
-  const size_t o = (size_t(batch) * params->n_q_heads * kHeadDim * 4 + 255) & ~size_t(255);
-  const size_t l = (size_t(batch) * params->n_q_heads * 4 + 255) & ~size_t(255);
-  return ((dec + 255) & ~size_t(255)) + o + l;
+size_t ps_decode_shared_prefix_workspace_bytes(const ps_params* params, int64_t batch,
+                                               int64_t group_size) {
+  if (check_params(params, true) != PS_OK || batch < 0 || group_size < 1 ||
+      batch % group_size != 0 || params->l_prefix < 1)
+    return 0;
+  return shared_prefix_layout(params, batch, group_size).total;
 }
 
 int ps_decode_attn_shared_prefix(const ps_params* params, const ps_kv_cache* cache,
@@ -547,18 +607,14 @@ int ps_decode_attn_shared_prefix(const ps_params* params, const ps_kv_cache* cac
     return fail(PS_ERR_INVALID_ARG, "pos is not 8-byte aligned");
   if ((reinterpret_cast<uintptr_t>(dev_status) & 3u) != 0)
     return fail(PS_ERR_INVALID_ARG, "dev_status is not 4-byte aligned");
-  const size_t need = ps_decode_shared_prefix_workspace_bytes(params, cache->batch);
-  if (!workspace || ws_bytes < need)
+  const SharedPrefixLayout L = shared_prefix_layout(params, cache->batch, group_size);
+  if (!workspace || ws_bytes < L.total)
     return fail(PS_ERR_WORKSPACE, "workspace smaller than ps_decode_shared_prefix_workspace_bytes()");
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
     return fail(PS_ERR_INVALID_ARG, "workspace is not 256-byte aligned");
-  const size_t dec = decode_workspace_bytes(cache->batch, params->n_kv_heads,
-                                            (int64_t)params->l_prefix + params->window);
   char* ws = static_cast<char*>(workspace);
-  float* o_pre = reinterpret_cast<float*>(ws + ((dec + 255) & ~size_t(255)));
-  float* lse2_pre = reinterpret_cast<float*>(
-      reinterpret_cast<char*>(o_pre) +
-      ((size_t(cache->batch) * params->n_q_heads * kHeadDim * 4 + 255) & ~size_t(255)));
+  float* o_pre = reinterpret_cast<float*>(ws + L.dec);
+  float* lse2_pre = reinterpret_cast<float*>(ws + L.dec + L.o);
   const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   SharedPrefixLaunch sp{};
   sp.q = q;
@@ -574,13 +630,26 @@ int ps_decode_attn_shared_prefix(const ps_params* params, const ps_kv_cache* cac
   sp.hkv = params->n_kv_heads;
   sp.lp = params->l_prefix;
   sp.scale = resolve_scale(params);
-  PS_TRY(launch_shared_prefix(sp, st));
+  int rc = PS_OK;
+  PrefixFork fk;
+  fk.sp = sp;
+  fk.side = side_stream(&rc);
+  if (rc != PS_OK) return rc;
+  rc = check_cuda(cudaEventCreateWithFlags(&fk.fork, cudaEventDisableTiming), "cudaEventCreate");
+  if (rc != PS_OK) return rc;
+  // the prefix pass may start as soon as the work queued so far on `stream` is done; it is
+  // launched after the window decode, so that decode is first in line for the SMs
+  rc = check_cuda(cudaEventRecord(fk.fork, st), "cudaEventRecord");
+  if (rc != PS_OK) {
+    cudaEventDestroy(fk.fork);
+    return rc;
+  }
   DecodeLaunch l{};
   l.q = q;
   l.pos = pos;
   l.out = out;
   l.lse = lse;
-  l.workspace = dec > 0 ? workspace : nullptr;
+  l.workspace = workspace;  // the window pass's split-K partials come first (L.dec bytes)
   l.status = dev_status;
   l.batch = cache->batch;
   l.hq = params->n_q_heads;
@@ -595,7 +664,12 @@ int ps_decode_attn_shared_prefix(const ps_params* params, const ps_kv_cache* cac
   l.skip_prefix = 1;
   l.pre_o = o_pre;
   l.pre_lse2 = lse2_pre;
-  return launch_decode(l, st);
+  l.pre_splits = L.splits;
+  l.before_merge = launch_prefix_forked;
+  l.before_merge_ctx = &fk;
+  rc = launch_decode(l, st);
+  cudaEventDestroy(fk.fork);
+  return rc;
 }
 
 }  // extern "C"

@@ -74,8 +74,6 @@ struct DecodeArgs {
   int64_t lmax;
   float scale_log2;
   int32_t skip_prefix;     // shared-prefix decode: window rows only
-  const float* pre_o;      // shared-prefix partials folded in at flush (per-unit schedule)
-  const float* pre_lse2;
 };
 
 // Offset of the 16-byte chunk `chunk` (0..7) of box row `row` under the 128-byte swizzle
@@ -357,26 +355,6 @@ __global__ void __launch_bounds__(kThreads)
       named_bar_sync(1, kConsumerThreads);
       if (warp == 0) {
         merge_state(m0, m1, l0, l1, o, flush + lane * 36);
-        if (a.pre_o && !a.streamk) {
-          // fold in the shared-prefix partial (normalised o, weight 2^lse2) of heads 2qq,
-          // 2qq + 1 at this lane's fragment positions; slots 32.. of the flush area are free
-          float* other = flush + (32 + lane) * 36;
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int hh = 2 * qq + e;
-            const bool valid = hh < a.group;
-            const int64_t row = (int64_t)b * a.hq + h * a.group + hh;
-            other[32 + e] = valid ? a.pre_lse2[row] : -INFINITY;
-            other[34 + e] = 1.f;
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              const int d0 = 16 * j + (lane >> 2);
-              other[4 * j + e] = valid ? a.pre_o[row * kHeadDim + d0] : 0.f;
-              other[4 * j + 2 + e] = valid ? a.pre_o[row * kHeadDim + d0 + 8] : 0.f;
-            }
-          }
-          merge_state(m0, m1, l0, l1, o, other);
-        }
         const int unit = b * a.hkv + h;
         const int64_t slot = (int64_t)unit + blockIdx.x;  // unique per (unit, CTA) piece
 #pragma unroll
@@ -540,7 +518,8 @@ __global__ void __launch_bounds__(128)
                  const int32_t* __restrict__ pref, const int32_t* __restrict__ span,
                  __nv_bfloat16* __restrict__ out, float* __restrict__ lse, int32_t batch,
                  int32_t hq, int32_t hkv, int32_t group, int32_t grid,
-                 const float* __restrict__ pre_o, const float* __restrict__ pre_lse2) {
+                 const float* __restrict__ pre_o, const float* __restrict__ pre_lse2,
+                 int32_t pre_splits) {
   const int64_t bh = (int64_t)blockIdx.x * 4 + (threadIdx.x >> 5);
   if (bh >= (int64_t)batch * hq) return;
   const int lane = threadIdx.x & 31;
@@ -552,15 +531,22 @@ __global__ void __launch_bounds__(128)
   const int64_t total = (int64_t)hkv * pref[batch];
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   float lse2 = -INFINITY;
-  // online combine state; a shared-prefix partial (normalised, weight 2^lse2) starts it
+  // online combine state; shared-prefix partials (normalised, weight 2^lse2) start it
   float M = -INFINITY, wsum = 0.f;
-  if (pre_o) {
-    const float l2 = pre_lse2[bh];
-    if (l2 != -INFINITY) {
-      M = l2;
-      wsum = 1.f;
-      acc = reinterpret_cast<const float4*>(pre_o + bh * kHeadDim)[lane];
-    }
+  for (int sp = 0; pre_o && sp < pre_splits; ++sp) {
+    const int64_t row = (int64_t)sp * batch * hq + bh;
+    const float l2 = pre_lse2[row];
+    if (l2 == -INFINITY) continue;
+    const float4 ov = reinterpret_cast<const float4*>(pre_o + row * kHeadDim)[lane];
+    const float Mn = fmaxf(M, l2);
+    const float fa = (M == -INFINITY) ? 0.f : fast_exp2(M - Mn);
+    const float fb = fast_exp2(l2 - Mn);
+    wsum = wsum * fa + fb;
+    acc.x = acc.x * fa + fb * ov.x;
+    acc.y = acc.y * fa + fb * ov.y;
+    acc.z = acc.z * fa + fb * ov.z;
+    acc.w = acc.w * fa + fb * ov.w;
+    M = Mn;
   }
   if (sp.x <= sp.y) {
     const int c_lo = sp.x, c_hi = sp.y;
@@ -651,11 +637,13 @@ int occupancy_per_sm() {
   return cached[dev];
 }
 
-// Stream-K grid size for this shape, or 0 for the per-unit schedule.
-int64_t streamk_grid(int64_t batch, int32_t hkv, int64_t max_keys) {
+// Stream-K grid size for this shape, or 0 for the per-unit schedule.  `force` selects
+// stream-K whenever the batch fits its prefix table (the caller then always gets partials
+// to merge, e.g. with a shared-prefix pass).
+int64_t streamk_grid(int64_t batch, int32_t hkv, int64_t max_keys, bool force = false) {
   const int64_t units = batch * hkv;
   const int64_t slots = (int64_t)sm_count() * occupancy_per_sm();
-  if (units >= slots || batch > kMaxStreamKSeqs) return 0;
+  if (batch > kMaxStreamKSeqs || (units >= slots && !force)) return 0;
   const int64_t max_tiles = units * ((max_keys + kDecodeTile - 1) / kDecodeTile + 2);
   int64_t g = max_tiles / kMinTilesPerCta;
   if (g > slots) g = slots;
@@ -670,8 +658,8 @@ int decode_splits(int64_t batch, int32_t hkv, int64_t max_keys) {
   return g > 0 ? static_cast<int>(g) : 1;
 }
 
-size_t decode_workspace_bytes(int64_t batch, int32_t hkv, int64_t max_keys) {
-  const int64_t g = streamk_grid(batch, hkv, max_keys);
+size_t decode_workspace_bytes(int64_t batch, int32_t hkv, int64_t max_keys, bool force_streamk) {
+  const int64_t g = streamk_grid(batch, hkv, max_keys, force_streamk);
   if (g == 0) return 0;
   const size_t slots = size_t(batch * hkv + g) * 8;
   const size_t o_bytes = slots * kHeadDim * sizeof(float);
@@ -683,7 +671,11 @@ size_t decode_workspace_bytes(int64_t batch, int32_t hkv, int64_t max_keys) {
 int launch_decode(const DecodeLaunch& l, cudaStream_t stream) {
   const int group = l.hq / l.hkv;
   const int64_t max_keys = l.full_mode ? l.lmax : (int64_t)l.lp + l.w;
-  const int64_t g = streamk_grid(l.batch, l.hkv, max_keys);
+  const bool force = l.pre_o != nullptr;  // prefix partials are combined by the merge
+  const int64_t g = streamk_grid(l.batch, l.hkv, max_keys, force);
+  if (force && g == 0) return fail(PS_ERR_UNSUPPORTED, "shared-prefix decode needs batch <= 1024");
+  if (g > 0 && l.workspace == nullptr)
+    return fail(PS_ERR_WORKSPACE, "split-K decode launched without a workspace");
   const int64_t units = l.batch * l.hkv;
   // window-only decode reads no prefix rows: no prefix map (it may describe fewer units)
   const int32_t dim0 = l.full_mode ? static_cast<int32_t>(l.lmax) : (l.skip_prefix ? 0 : l.lp);
@@ -738,8 +730,7 @@ int launch_decode(const DecodeLaunch& l, cudaStream_t stream) {
   a.lmax = l.lmax;
   a.scale_log2 = l.scale * kLog2e;
   a.skip_prefix = l.skip_prefix;
-  a.pre_o = l.pre_o;
-  a.pre_lse2 = l.pre_lse2;
+  const int32_t pre_splits = l.pre_o ? (l.pre_splits > 0 ? l.pre_splits : 1) : 0;
 
   const size_t sb = smem_bytes(kStages);
   occupancy_per_sm();  // sets the shared-memory attribute once per device
@@ -751,13 +742,17 @@ int launch_decode(const DecodeLaunch& l, cudaStream_t stream) {
                                  dim3(kThreads), sb, stream, mk0, mv0, mk1, mv1, a),
                       "decode_kernel launch");
   if (rc != PS_OK) return rc;
+  if (l.before_merge) {
+    rc = l.before_merge(l.before_merge_ctx, stream);
+    if (rc != PS_OK) return rc;
+  }
   if (g > 0) {
     rc = check_cuda(
         launch_pdl(merge_kernel, dim3(static_cast<unsigned>((l.batch * l.hq + 3) / 4)), dim3(128),
                    0, stream, static_cast<const float*>(a.ws_o),
                    static_cast<const float*>(a.ws_lse), static_cast<const int32_t*>(a.ws_pref),
                    static_cast<const int32_t*>(a.ws_span), a.out, a.lse, a.batch, l.hq, l.hkv,
-                   group, static_cast<int32_t>(g), l.pre_o, l.pre_lse2),
+                   group, static_cast<int32_t>(g), l.pre_o, l.pre_lse2, pre_splits),
         "merge_kernel launch");
   }
   return rc;

@@ -84,16 +84,22 @@ struct DecodeLaunch {
   float scale;
   const void *k0, *v0;  // prefix (or linear) cache
   const void *k1, *v1;  // ring (unused in full mode)
-  // Shared-prefix decode: read only the window (the prefix rows are skipped) and fold in a
-  // precomputed prefix partial per (sequence, query head): normalised fp32 o [batch, Hq, D]
-  // and its base-2 lse [batch, Hq] (scores scaled by scale * log2 e).
+  // Shared-prefix decode: read only the window (the prefix rows are skipped); the split-K
+  // merge folds in precomputed prefix partials per (sequence, query head): normalised fp32
+  // o and its base-2 lse (scores scaled by scale * log2 e).  Forces the stream-K schedule.
   int32_t skip_prefix;
-  const float* pre_o;
-  const float* pre_lse2;
+  const float* pre_o;     // [pre_splits][batch, Hq, D]
+  const float* pre_lse2;  // [pre_splits][batch, Hq]
+  int32_t pre_splits;     // partials per (sequence, query head), each over a key range
+  // called after the decode kernel is launched and before the merge (e.g. to launch the
+  // prefix pass on another stream and make `stream` wait for it); PS_OK to continue
+  int (*before_merge)(void* ctx, cudaStream_t stream);
+  void* before_merge_ctx;
 };
 // Split count and workspace bytes for a decode of this shape on the current device.
 int decode_splits(int64_t batch, int32_t hkv, int64_t max_keys);
-size_t decode_workspace_bytes(int64_t batch, int32_t hkv, int64_t max_keys);
+size_t decode_workspace_bytes(int64_t batch, int32_t hkv, int64_t max_keys,
+                              bool force_streamk = false);
 int launch_decode(const DecodeLaunch& a, cudaStream_t stream);
 // Shared-prefix pass: attention of every (sequence, query head) of a group of `gsize`
 // sequences over the group's prefix rows [0, min(pos + 1, lp)); writes o_pre/lse2_pre.
@@ -102,13 +108,15 @@ struct SharedPrefixLaunch {
   const int64_t* pos;    // [batch]
   const void* k_pre;     // [batch / gsize, Hkv, lp, D]
   const void* v_pre;
-  float* o_pre;          // [batch, Hq, D]
-  float* lse2_pre;       // [batch, Hq]
+  float* o_pre;          // [splits][batch, Hq, D]
+  float* lse2_pre;       // [splits][batch, Hq]
   int32_t* status;
   int64_t batch, gsize;
   int32_t hq, hkv, lp;
   float scale;
 };
+// Key-range splits of the shared-prefix pass (enough CTAs to cover the SMs).
+int shared_prefix_splits(int64_t batch, int64_t gsize, int32_t hq, int32_t hkv, int32_t lp);
 int launch_shared_prefix(const SharedPrefixLaunch& l, cudaStream_t stream);
 // Decode whose split-K scratch is the library's file-scope device array (no allocation).
 constexpr size_t kDecodeScratchBytes = size_t(4) << 20;

@@ -11,8 +11,10 @@
 // log-sum-exp; the window-only decode folds it in (log-sum-exp weighted), which gives exactly
 // the attention over the prefix and the window together.
 //
-// One CTA per (group, KV head, 128-row block of that group's query rows); row r is sequence
-// r / g of the group, query head h * g + r % g.  6 warps:
+// One CTA per (group, KV head, 128-row block of that group's query rows, key-range split):
+// row r is sequence r / g of the group, query head h * g + r % g; each split covers a run
+// of 128-key prefix tiles and writes its own partial, so few groups still fill the GPU.
+// 6 warps:
 //   all     - stage the query block into shared memory (128-byte swizzled, K-major);
 //   warp 4  - TMA producer: K and V prefix tiles (128 rows, two 64-column halves) into a
 //             2-stage ring;
@@ -53,6 +55,8 @@ struct SpArgs {
   int32_t* status;
   int32_t hq, hkv, group, gsize;
   int32_t lp, nkt, row_tiles;
+  int32_t splits, per;  // key-range splits of the prefix and tiles per split
+  int64_t split_rows;   // batch * Hq: stride between the splits' partials
   float scale_log2;
 };
 
@@ -79,8 +83,14 @@ __global__ void __launch_bounds__(kSpThreads, 1)
   uint64_t* mma_done = bars + 11;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 12);
 
-  const int t = blockIdx.x % a.row_tiles;
-  const int rest = blockIdx.x / a.row_tiles;
+  // block = (group, KV head, row block, key split); the split owns prefix tiles
+  // [kt0, kt0 + n), tile indices below are relative to kt0
+  const int split = blockIdx.x % a.splits;
+  const int item = blockIdx.x / a.splits;
+  const int kt0 = split * a.per;
+  const int n = (a.nkt - kt0 < a.per) ? a.nkt - kt0 : a.per;
+  const int t = item % a.row_tiles;
+  const int rest = item / a.row_tiles;
   const int h = rest % a.hkv;
   const int grp = rest / a.hkv;
   const int warp = threadIdx.x >> 5;
@@ -133,7 +143,7 @@ __global__ void __launch_bounds__(kSpThreads, 1)
     if (lane == 0) {
       const int unit = grp * a.hkv + h;
       int issued = 0;
-      for (int kt = 0; kt < a.nkt; ++kt) {
+      for (int kt = 0; kt < n; ++kt) {
         const int s = kt & 1;
         if (kt >= 2 && !mbar_wait(&kv_empty[s], static_cast<uint32_t>(((kt >> 1) - 1) & 1),
                                   a.status))
@@ -141,10 +151,11 @@ __global__ void __launch_bounds__(kSpThreads, 1)
         mbar_arrive_expect_tx(&kv_full[s], 2 * kTileBytes);
         uint8_t* k = sK + s * kTileBytes;
         uint8_t* v = sV + s * kTileBytes;
-        tma_load_3d(k, &mk, 0, kt * 128, unit, &kv_full[s]);
-        tma_load_3d(k + kBoxBytes, &mk, 64, kt * 128, unit, &kv_full[s]);
-        tma_load_3d(v, &mv, 0, kt * 128, unit, &kv_full[s]);
-        tma_load_3d(v + kBoxBytes, &mv, 64, kt * 128, unit, &kv_full[s]);
+        const int row0 = (kt0 + kt) * 128;
+        tma_load_3d(k, &mk, 0, row0, unit, &kv_full[s]);
+        tma_load_3d(k + kBoxBytes, &mk, 64, row0, unit, &kv_full[s]);
+        tma_load_3d(v, &mv, 0, row0, unit, &kv_full[s]);
+        tma_load_3d(v + kBoxBytes, &mv, 64, row0, unit, &kv_full[s]);
         issued = kt + 1;
       }
       for (int kt = (issued > 2 ? issued - 2 : 0); kt < issued; ++kt)
@@ -174,9 +185,9 @@ __global__ void __launch_bounds__(kSpThreads, 1)
         }
         umma_commit(&s_full[s]);
       };
-      if (a.nkt > 0) issue_s(0);
-      for (int kt = 0; ok && kt < a.nkt; ++kt) {
-        if (kt + 1 < a.nkt) issue_s(kt + 1);  // next scores while this tile's softmax runs
+      if (n > 0) issue_s(0);
+      for (int kt = 0; ok && kt < n; ++kt) {
+        if (kt + 1 < n) issue_s(kt + 1);  // next scores while this tile's softmax runs
         if (!ok) break;
         const int s = kt & 1;
         if (!mbar_wait(&p_ready[s], static_cast<uint32_t>((kt >> 1) & 1), a.status)) {
@@ -217,7 +228,7 @@ __global__ void __launch_bounds__(kSpThreads, 1)
     const float sl2 = a.scale_log2;
     float m = -INFINITY, l = 0.f;
     bool ok = true;
-    for (int kt = 0; kt < a.nkt; ++kt) {
+    for (int kt = 0; kt < n; ++kt) {
       const int s = kt & 1;
       ok = ok && __all_sync(0xffffffffu,
                             mbar_wait(&s_full[s], static_cast<uint32_t>((kt >> 1) & 1), a.status));
@@ -229,7 +240,7 @@ __global__ void __launch_bounds__(kSpThreads, 1)
 #pragma unroll
         for (int c = 0; c < 4; ++c) tmem_ld32(lane_base + 128u * s + 32 * c, raw[c]);
         tmem_wait_ld();
-        const int64_t lim = kvis - (int64_t)kt * 128;  // visible columns [0, lim)
+        const int64_t lim = kvis - (int64_t)(kt0 + kt) * 128;  // visible columns [0, lim)
 #pragma unroll
         for (int c = 0; c < 4; ++c)
 #pragma unroll
@@ -288,11 +299,12 @@ __global__ void __launch_bounds__(kSpThreads, 1)
     // epilogue: normalised prefix attention and its base-2 lse.  The TMEM loads are
     // warp-collective, so every lane runs them; only rows of the group are stored.
     const bool fin = __all_sync(0xffffffffu,
-                                ok && (a.nkt == 0 || mbar_wait(o_full, 0, a.status)));
+                                ok && (n == 0 || mbar_wait(o_full, 0, a.status)));
     if (fin) {
-      float* dst = a.o + (b * a.hq + head) * kHeadDim;
+      const int64_t orow = split * a.split_rows + b * a.hq + head;
+      float* dst = a.o + orow * kHeadDim;
       const float inv = l > 0.f ? 1.f / l : 0.f;
-      if (a.nkt > 0) {
+      if (n > 0) {
         tc_fence_after();
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
@@ -311,7 +323,7 @@ __global__ void __launch_bounds__(kSpThreads, 1)
         for (int v = 0; v < 32; ++v)
           reinterpret_cast<float4*>(dst)[v] = make_float4(0.f, 0.f, 0.f, 0.f);
       }
-      if (valid) a.lse2[b * a.hq + head] = l > 0.f ? m + log2f(l) : -INFINITY;
+      if (valid) a.lse2[orow] = l > 0.f ? m + log2f(l) : -INFINITY;
     }
   }
   tc_fence_before();
@@ -324,12 +336,28 @@ __global__ void __launch_bounds__(kSpThreads, 1)
 
 }  // namespace
 
+// Enough key-range splits that the blocks cover every SM once (each split keeps at least
+// one 128-key tile); the window pass and the merge fold the splits' partials together.
+int shared_prefix_splits(int64_t batch, int64_t gsize, int32_t hq, int32_t hkv, int32_t lp) {
+  const int64_t rows = gsize * (hq / hkv);
+  const int64_t items = (batch / gsize) * hkv * ((rows + 127) / 128);
+  const int64_t nkt = (lp + 127) / 128;
+  if (items <= 0 || nkt <= 0) return 1;
+  int64_t want = (sm_count() + items - 1) / items;
+  if (want > nkt) want = nkt;
+  if (want < 1) want = 1;
+  const int64_t per = (nkt + want - 1) / want;
+  return static_cast<int>((nkt + per - 1) / per);
+}
+
 int launch_shared_prefix(const SharedPrefixLaunch& l, cudaStream_t stream) {
   const int group = l.hq / l.hkv;
   const int64_t groups = l.batch / l.gsize;
   const int64_t rows = l.gsize * group;
   const int64_t row_tiles = (rows + 127) / 128;
-  const int64_t items = groups * l.hkv * row_tiles;
+  const int splits = shared_prefix_splits(l.batch, l.gsize, l.hq, l.hkv, l.lp);
+  const int64_t nkt = (l.lp + 127) / 128;
+  const int64_t items = groups * l.hkv * row_tiles * splits;
   if (items <= 0) return PS_OK;
   if (items > 0x7fffffffLL || rows > 0x7fffffffLL)
     return fail(PS_ERR_UNSUPPORTED, "shared-prefix problem too large");
@@ -350,6 +378,9 @@ int launch_shared_prefix(const SharedPrefixLaunch& l, cudaStream_t stream) {
   a.lp = l.lp;
   a.nkt = (l.lp + 127) / 128;
   a.row_tiles = static_cast<int32_t>(row_tiles);
+  a.splits = splits;
+  a.per = static_cast<int32_t>((nkt + splits - 1) / splits);
+  a.split_rows = l.batch * l.hq;
   a.scale_log2 = l.scale * kLog2e;
   static bool attr[64] = {false};
   int dev = 0;

@@ -43,6 +43,7 @@ class Workload:
     # prefill workloads: sequence length
     seq: Optional[int] = None
     n_layers: int = 1
+    group_size: int = 1  # sequences sharing one prompt prefix
     index: int = 0  # 1-based workload index used for the seed
 
 
@@ -66,6 +67,12 @@ WORKLOADS = {
         name="decode_stack_l28_b1024_w16384", batch=1024, n_q_heads=16, n_kv_heads=2,
         head_dim=128, l_prefix=2000, window=16384, pos_lo=32768, pos_hi=262144,
         n_layers=28, index=5),
+    # many samples of one prompt (the pages' accuracy tables average 64 samples per
+    # problem): 4 prompts x 64 samples, a 2000-token prompt kept as the prefix
+    "decode_shared_b256_g64_lp2000_w4096": Workload(
+        name="decode_shared_b256_g64_lp2000_w4096", batch=256, n_q_heads=16, n_kv_heads=2,
+        head_dim=128, l_prefix=2000, window=4096, pos_lo=8192, pos_hi=131072, group_size=64,
+        index=6),
 }
 
 

@@ -75,8 +75,8 @@ def _shared_prefix_case(dev, hq, hkv, lp, w, gsize, positions, seed, scale=0.0):
 
     out = torch.full((Bn, hq, D), float("nan"), dtype=torch.bfloat16, device=dev)
     lse = torch.full((Bn, hq), float("nan"), dtype=torch.float32, device=dev)
-    ws = torch.empty(B.ps_decode_shared_prefix_workspace_bytes(params, Bn), dtype=torch.uint8,
-                     device=dev)
+    ws = torch.empty(B.ps_decode_shared_prefix_workspace_bytes(params, Bn, gsize),
+                     dtype=torch.uint8, device=dev)
     B.ps_decode_attn_shared_prefix(params, shared, gsize, q, pos, out, lse, ws, st)
     out_p = torch.empty_like(out)
     lse_p = torch.empty_like(lse)
