@@ -64,6 +64,8 @@ __all__ = [
     "attend_gqa",
     "decode_reference",
     "full_attention_decode",
+    "reset_pe_positions",
+    "reset_pe_decode_reference",
     "prefill_reference",
     "prefill_backward_reference",
     "tile_plan",
@@ -234,6 +236,37 @@ def full_attention_decode(q: np.ndarray, k_rot: np.ndarray, v: np.ndarray, p: in
                           scale: float):
     """Full causal attention of the query at position p over keys [0, p]."""
     return attend_gqa(q, k_rot[: p + 1], v[: p + 1], scale)
+
+
+def reset_pe_positions(p: int, l_prefix: int, window: int):
+    """Reset PE ("Prefix Sliding 完全拆解", §位置编码): the visible keys of the query at
+    absolute position p, and the position ids Reset PE gives them and the query.
+
+    The prefix keeps its ids; the window tokens are renumbered to follow the prefix
+    directly (the first window token gets id L_prefix, the next L_prefix + 1, ...), and the
+    query, the newest window token, gets the last of those ids.
+    Returns (visible absolute positions, their Reset-PE ids, the query's Reset-PE id).
+    """
+    vis = visible_positions(p, l_prefix, window)
+    ids = vis.copy()
+    win = vis >= l_prefix
+    ids[win] = l_prefix + np.arange(int(win.sum()), dtype=np.int64)
+    q_id = int(ids[-1])  # the query is the last visible position (itself)
+    return vis, ids, q_id
+
+
+def reset_pe_decode_reference(q_raw: np.ndarray, k_raw: np.ndarray, v: np.ndarray, p: int,
+                              l_prefix: int, window: int, theta: float, scale: float):
+    """Decode output under Reset PE: every visible key and the query rotated at its Reset-PE
+    id (reset_pe_positions), then softmax attention (eq. A(i) for the visible set).
+
+    q_raw: [Hq, D] un-rotated query; k_raw, v: [>= p+1, Hkv, D] un-rotated keys and values
+    indexed by absolute position.  Returns (out [Hq, D], lse [Hq]).
+    """
+    vis, ids, q_id = reset_pe_positions(p, l_prefix, window)
+    q = rope_rotate(np.asarray(q_raw, np.float64), q_id, theta)
+    k = rope_rotate(np.asarray(k_raw, np.float64)[vis], ids[:, None], theta)
+    return attend_gqa(q, k, np.asarray(v, np.float64)[vis], scale)
 
 
 def prefill_reference(Q: np.ndarray, K: np.ndarray, V: np.ndarray, l_prefix: int,

@@ -412,3 +412,82 @@ def test_prefill_backward_selected_rows_and_keys():
     np.testing.assert_allclose(sq, fq[rows], rtol=0, atol=1e-13)
     np.testing.assert_allclose(sk, fk[keys], rtol=0, atol=1e-13)
     np.testing.assert_allclose(sv, fv[keys], rtol=0, atol=1e-13)
+
+
+# ------------------------------------------------------------------- Reset PE
+def test_reset_pe_positions_by_hand():
+    """L_prefix 3, W 4, query at 10: keys 0,1,2 keep their ids, window 7..10 -> 3..6."""
+    vis, ids, q_id = O.reset_pe_positions(10, 3, 4)
+    assert vis.tolist() == [0, 1, 2, 7, 8, 9, 10]
+    assert ids.tolist() == [0, 1, 2, 3, 4, 5, 6]
+    assert q_id == 6
+
+
+def _continue_pe(q_raw, k_raw, v, p, lp, w, theta, scale):
+    vis = O.visible_positions(p, lp, w)
+    q = O.rope_rotate(q_raw, p, theta)
+    k = O.rope_rotate(k_raw[vis], vis[:, None], theta)
+    return O.attend_gqa(q, k, v[vis], scale)
+
+
+@pytest.mark.parametrize("lp,w,p", [(5, 20, 10), (5, 20, 24), (0, 8, 30), (0, 1, 9)])
+def test_reset_pe_equals_continue_pe_without_renumbering_gap(lp, w, p):
+    """Warm-up (nothing evicted: ids are the absolute positions) and L_prefix = 0 (only
+    relative offsets inside the window matter) give Continue PE exactly."""
+    hq, hkv, d = 4, 2, 16
+    q, k, v = _rand((hq, d), 60), _rand((p + 1, hkv, d), 61), _rand((p + 1, hkv, d), 62)
+    got, gl = O.reset_pe_decode_reference(q, k, v, p, lp, w, 1e4, 0.3)
+    want, wl = _continue_pe(q, k, v, p, lp, w, 1e4, 0.3)
+    np.testing.assert_allclose(got, want, rtol=0, atol=1e-10)
+    np.testing.assert_allclose(gl, wl, rtol=0, atol=1e-10)
+
+
+def test_reset_pe_differs_from_continue_pe_after_eviction():
+    """After eviction with a prefix, the prefix-to-query offsets change: results differ."""
+    hq, hkv, d, lp, w, p = 4, 2, 16, 4, 6, 40
+    q, k, v = _rand((hq, d), 63), _rand((p + 1, hkv, d), 64), _rand((p + 1, hkv, d), 65)
+    got, _ = O.reset_pe_decode_reference(q, k, v, p, lp, w, 100.0, 0.5)
+    want, _ = _continue_pe(q, k, v, p, lp, w, 100.0, 0.5)
+    assert np.abs(got - want).max() > 1e-3
+
+
+def test_reset_pe_bruteforce_rotation_matrices():
+    """Tiny case with explicit 2x2 rotation blocks and a nested-loop softmax."""
+    hq, hkv, d, lp, w, p, theta, scale = 2, 1, 4, 2, 3, 9, 50.0, 0.7
+    q, k, v = _rand((hq, d), 66), _rand((p + 1, hkv, d), 67), _rand((p + 1, hkv, d), 68)
+    keys = [0, 1, 7, 8, 9]                # prefix 0,1; window 7,8,9
+    ids = {0: 0, 1: 1, 7: 2, 8: 3, 9: 4}  # window renumbered after the prefix
+    qid = 4
+
+    def rot(x, pos):
+        y = np.empty(d)
+        for i in range(d // 2):
+            a = pos * theta ** (-2.0 * i / d)
+            c, s_ = math.cos(a), math.sin(a)
+            y[i] = x[i] * c - x[i + d // 2] * s_
+            y[i + d // 2] = x[i + d // 2] * c + x[i] * s_
+        return y
+
+    got, _ = O.reset_pe_decode_reference(q, k, v, p, lp, w, theta, scale)
+    for h in range(hq):
+        qr = rot(q[h], qid)
+        sc = [scale * float(qr @ rot(k[j, 0], ids[j])) for j in keys]
+        m = max(sc)
+        e = [math.exp(x - m) for x in sc]
+        want = sum(ei * v[j, 0] for ei, j in zip(e, keys)) / sum(e)
+        np.testing.assert_allclose(got[h], want, rtol=0, atol=1e-12)
+
+
+def test_reset_pe_equals_shifted_query_for_prefix_keys():
+    """Relative form of RoPE: Reset PE scores against window keys equal Continue PE's, and
+    against prefix keys equal Continue PE's with the query moved to L_prefix + |win| - 1."""
+    hq, hkv, d, lp, w, p, theta = 2, 1, 8, 3, 5, 30, 1e3
+    q, k = _rand((hq, d), 69), _rand((p + 1, hkv, d), 70)
+    vis, ids, qid = O.reset_pe_positions(p, lp, w)
+    kr = O.rope_rotate(k[vis], vis[:, None], theta)[:, 0]   # Continue-PE cached keys
+    reset = O.rope_rotate(q, qid, theta) @ O.rope_rotate(k[vis], ids[:, None], theta)[:, 0].T
+    cont = O.rope_rotate(q, p, theta) @ kr.T
+    moved = O.rope_rotate(q, lp + w - 1, theta) @ kr.T
+    pre = vis < lp
+    np.testing.assert_allclose(reset[:, ~pre], cont[:, ~pre], rtol=0, atol=1e-10)
+    np.testing.assert_allclose(reset[:, pre], moved[:, pre], rtol=0, atol=1e-10)
