@@ -128,6 +128,22 @@ int ps_decode_attn(const ps_params* params, const ps_kv_cache* cache, const void
                    const int64_t* pos, void* out, float* lse, void* workspace, size_t ws_bytes,
                    int32_t* dev_status, ps_stream_t stream);
 
+/* One decode step under Reset PE, from the same Continue-PE cache ps_kv_append_rope fills.
+ * Source: §位置编码 of "Prefix Sliding 完全拆解": Reset PE renumbers the window so that it
+ * directly follows the prefix (the first window token gets id L_prefix, the next
+ * L_prefix + 1, ...; the query, the newest window token, the last id); prefix ids are kept.
+ * RoPE scores depend only on id differences, so against window keys these scores equal the
+ * Continue-PE ones, and against prefix keys they equal Continue PE with the query rotated at
+ * L_prefix + |window| - 1 instead of pos.  The kernel derives that second query from q (a
+ * further rotation by L_prefix + |window| - 1 - pos, angles reduced in float64) and uses it
+ * for the prefix rows; nothing in the cache is rotated again.  During warm-up (nothing
+ * evicted) and with l_prefix = 0 the result equals ps_decode_attn.
+ * Arguments, workspace (ps_decode_workspace_bytes), results and errors as ps_decode_attn;
+ * q is rotated at pos (ps_kv_append_rope), as for ps_decode_attn. */
+int ps_decode_attn_reset_pe(const ps_params* params, const ps_kv_cache* cache, const void* q,
+                            const int64_t* pos, void* out, float* lse, void* workspace,
+                            size_t ws_bytes, int32_t* dev_status, ps_stream_t stream);
+
 /* ps_decode_attn without a workspace argument, for callers that cannot allocate device
  * memory: for example a plugin that its host framework hands only the input and output
  * buffers, or a fixed-memory serving loop where a cudaMalloc (or a caching allocator

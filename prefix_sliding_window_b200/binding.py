@@ -82,6 +82,9 @@ _SIGS = {
                                          c_int64, c_void_p, c_void_p, c_void_p, c_int64,
                                          POINTER(c_int64), c_void_p, c_size_t, c_void_p,
                                          c_void_p]),
+    "ps_decode_attn_reset_pe": (c_int32, [POINTER(PsParams), POINTER(PsKVCache), c_void_p,
+                                          c_void_p, c_void_p, c_void_p, c_void_p, c_size_t,
+                                          c_void_p, c_void_p]),
     "ps_decode_shared_prefix_workspace_bytes": (c_size_t, [POINTER(PsParams), c_int64,
                                                            c_int64]),
     "ps_decode_attn_shared_prefix": (c_int32, [POINTER(PsParams), POINTER(PsKVCache), c_int64,
@@ -176,6 +179,17 @@ def ps_decode_attn(params: PsParams, cache: PsKVCache, q, pos, out, lse=None, wo
                                _ptr(out), _ptr(lse), _ptr(workspace), ws_bytes, _ptr(dev_status),
                                _stream(stream))
     _check(rc, "ps_decode_attn")
+
+
+def ps_decode_attn_reset_pe(params: PsParams, cache: PsKVCache, q, pos, out, lse=None,
+                            workspace=None, dev_status=None, stream=None) -> None:
+    """Decode under Reset PE from a Continue-PE cache (prefix rows see the query at its
+    Reset-PE id)."""
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rc = load().ps_decode_attn_reset_pe(ctypes.byref(params), ctypes.byref(cache), _ptr(q),
+                                        _ptr(pos), _ptr(out), _ptr(lse), _ptr(workspace),
+                                        ws_bytes, _ptr(dev_status), _stream(stream))
+    _check(rc, "ps_decode_attn_reset_pe")
 
 
 def ps_decode_attn_noalloc(params: PsParams, cache: PsKVCache, q, pos, out, lse=None,

@@ -283,9 +283,10 @@ size_t ps_decode_workspace_bytes(const ps_params* params, int64_t batch) {
                                 (int64_t)params->l_prefix + params->window);
 }
 
-int ps_decode_attn(const ps_params* params, const ps_kv_cache* cache, const void* q,
-                   const int64_t* pos, void* out, float* lse, void* workspace, size_t ws_bytes,
-                   int32_t* dev_status, ps_stream_t stream) {
+static int decode_entry(const ps_params* params, const ps_kv_cache* cache, const void* q,
+                        const int64_t* pos, void* out, float* lse, void* workspace,
+                        size_t ws_bytes, int32_t* dev_status, ps_stream_t stream,
+                        int32_t reset_pe) {
   g_last_error.clear();
   PS_TRY(check_params(params, true));
   if (params->n_q_heads / params->n_kv_heads > kMaxGroup)
@@ -333,7 +334,23 @@ int ps_decode_attn(const ps_params* params, const ps_kv_cache* cache, const void
   l.v0 = cache->v_prefix;
   l.k1 = cache->k_ring;
   l.v1 = cache->v_ring;
+  l.reset_pe = reset_pe;
+  l.rope_theta = params->rope_theta;
   return launch_decode(l, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int ps_decode_attn(const ps_params* params, const ps_kv_cache* cache, const void* q,
+                   const int64_t* pos, void* out, float* lse, void* workspace, size_t ws_bytes,
+                   int32_t* dev_status, ps_stream_t stream) {
+  return decode_entry(params, cache, q, pos, out, lse, workspace, ws_bytes, dev_status, stream,
+                      0);
+}
+
+int ps_decode_attn_reset_pe(const ps_params* params, const ps_kv_cache* cache, const void* q,
+                            const int64_t* pos, void* out, float* lse, void* workspace,
+                            size_t ws_bytes, int32_t* dev_status, ps_stream_t stream) {
+  return decode_entry(params, cache, q, pos, out, lse, workspace, ws_bytes, dev_status, stream,
+                      1);
 }
 
 int ps_decode_attn_noalloc(const ps_params* params, const ps_kv_cache* cache, const void* q,

@@ -74,6 +74,10 @@ struct DecodeArgs {
   int64_t lmax;
   float scale_log2;
   int32_t skip_prefix;     // shared-prefix decode: window rows only
+  // Reset PE: prefix tiles use the query rotated by delta = L_prefix + |window| - 1 - p
+  // more (its Reset-PE id); inv_freq = theta^(-2i/D) in float64
+  int32_t reset_pe;
+  double inv_freq[kHeadDim / 2];
 };
 
 // Offset of the 16-byte chunk `chunk` (0..7) of box row `row` under the 128-byte swizzle
@@ -319,6 +323,37 @@ __global__ void __launch_bounds__(kThreads)
     float o[8][4];
     float m0, m1, l0, l1;
     uint32_t qf[8][2];
+    uint32_t qp[8][2];  // Reset PE: the query at its Reset-PE id, for prefix tiles
+    // qp = R_delta qf (rotate-half RoPE composes: R_a R_b = R_(a+b)).  This lane's pairs are
+    // (d, d + 64) for d = 16 ks + 2 qq + {0, 1, 8, 9}, ks < 4: fragments ks and ks + 4.
+    // delta * inv_freq is formed and reduced modulo 2 pi in float64, as in the append.
+    auto rotate_prefix_q = [&](int64_t p) {
+      const int64_t n = p + 1;
+      int64_t ws = n - a.w;
+      if (ws < a.lp) ws = a.lp;
+      const int64_t delta = (int64_t)a.lp - ws;  // <= 0; 0 while nothing is evicted
+#pragma unroll
+      for (int ks = 0; ks < 4; ++ks) {
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+          const uint32_t lo = qf[ks][r], hi = qf[ks + 4][r];
+          const float2 x1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&lo));
+          const float2 x2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&hi));
+          float c[2], sn[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int d = 16 * ks + 8 * r + 2 * qq + e;
+            const double ang = double(delta) * a.inv_freq[d];
+            const double k = rint(ang * 0.15915494309189535);
+            double red = fma(-k, 6.2831854820251465, ang);
+            red = fma(-k, -1.748455600074497e-07, red);
+            sincosf(static_cast<float>(red), &sn[e], &c[e]);
+          }
+          qp[ks][r] = pack_bf16x2(x1.x * c[0] - x2.x * sn[0], x1.y * c[1] - x2.y * sn[1]);
+          qp[ks + 4][r] = pack_bf16x2(x2.x * c[0] + x1.x * sn[0], x2.y * c[1] + x1.y * sn[1]);
+        }
+      }
+    };
     auto reset = [&]() {
       m0 = m1 = -INFINITY;
       l0 = l1 = 0.f;
@@ -423,6 +458,7 @@ __global__ void __launch_bounds__(kThreads)
     };
     if (ntiles > 0) {
       load_q(cw.b, cw.h);
+      if (a.reset_pe) rotate_prefix_q(a.pos[cw.b]);
       note_span(cw, cw.t, (cw.pu1 < wk.t_end ? cw.pu1 : wk.t_end) - 1);
       prefetch_next_q(cw);
     }
@@ -437,6 +473,7 @@ __global__ void __launch_bounds__(kThreads)
           qf[ks][0] = qn[ks][0];
           qf[ks][1] = qn[ks][1];
         }
+        if (a.reset_pe) rotate_prefix_q(a.pos[cw.b]);
         note_span(cw, cw.t, (cw.pu1 < wk.t_end ? cw.pu1 : wk.t_end) - 1);
         prefetch_next_q(cw);
       }
@@ -456,7 +493,10 @@ __global__ void __launch_bounds__(kThreads)
         const uint32_t addr =
             kbase + (ks >> 2) * kBoxBytes + swz(arow, ((ks & 3) << 1) + achunk);
         ldmatrix_x4(addr, a0, a1, a2, a3);
-        mma_bf16_16816(sc, a0, a1, a2, a3, qf[ks][0], qf[ks][1]);
+        // Reset PE: prefix tiles (map 0) see the query at its Reset-PE id
+        const bool pre_q = a.reset_pe && d.map_id == 0;
+        mma_bf16_16816(sc, a0, a1, a2, a3, pre_q ? qp[ks][0] : qf[ks][0],
+                       pre_q ? qp[ks][1] : qf[ks][1]);
       }
       const bool v0 = (r0 >= d.lo) && (r0 < d.hi);
       const bool v1 = (r1 >= d.lo) && (r1 < d.hi);
@@ -730,6 +770,9 @@ int launch_decode(const DecodeLaunch& l, cudaStream_t stream) {
   a.lmax = l.lmax;
   a.scale_log2 = l.scale * kLog2e;
   a.skip_prefix = l.skip_prefix;
+  a.reset_pe = l.reset_pe;
+  for (int i = 0; i < kHeadDim / 2; ++i)
+    a.inv_freq[i] = l.reset_pe ? pow(l.rope_theta, -2.0 * i / double(kHeadDim)) : 0.0;
   const int32_t pre_splits = l.pre_o ? (l.pre_splits > 0 ? l.pre_splits : 1) : 0;
 
   const size_t sb = smem_bytes(kStages);

@@ -95,6 +95,10 @@ struct DecodeLaunch {
   // prefix pass on another stream and make `stream` wait for it); PS_OK to continue
   int (*before_merge)(void* ctx, cudaStream_t stream);
   void* before_merge_ctx;
+  // Reset PE (window renumbered after the prefix): prefix tiles use the query rotated at its
+  // Reset-PE id L_prefix + |window| - 1 instead of its absolute position
+  int32_t reset_pe;
+  double rope_theta;
 };
 // Split count and workspace bytes for a decode of this shape on the current device.
 int decode_splits(int64_t batch, int32_t hkv, int64_t max_keys);
