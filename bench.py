@@ -724,6 +724,87 @@ def run_shared(dev, steps: int = 20, warmup: int = 3):
             "peak_hbm_gbs": peaks["hbm_gbs"], **res}
 
 
+# ------------------------------------------------------------- Reset PE leg
+def run_reset(dev, steps: int = 16, warmup: int = 3):
+    """Reset PE vs Continue PE on the batch-64 decode workload (16/2/128, L_prefix 100,
+    W 4096, positions U[8192, 131072]).  Per step: Continue PE = append (T = 1) + decode;
+    Reset PE here = append + Reset-PE decode (the same cache; only the query is rotated
+    again for the prefix rows); Reset PE done literally = the visible tokens re-appended at
+    their renumbered ids (T = L_prefix + W from un-rotated keys) + the query + decode."""
+    from prefix_sliding_window_b200 import binding as B
+    from prefix_sliding_window_b200.cache import PrefixSlidingCache
+    wl = synth.WORKLOADS[WORKLOAD]
+    Bn, hq, hkv, lp, w = wl.batch, wl.n_q_heads, wl.n_kv_heads, wl.l_prefix, wl.window
+    peaks = _peaks()
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    seed = synth.seed_for(wl.index, 9)
+    params = B.make_params(hq, hkv, D, lp, w, wl.rope_theta)
+    pos0 = synth.uniform_positions(Bn, wl.pos_lo, wl.pos_hi, seed, dev)
+    cache = PrefixSlidingCache(Bn, hkv, lp, w, D, dev, fill=None)
+    ring_k = synth.normal_bf16((Bn, hkv, w, D), seed + 1, dev)
+    cache.k_ring.copy_(ring_k)
+    cache.v_ring.copy_(ring_k)
+    cache.k_prefix.normal_()
+    cache.v_prefix.normal_()
+    del ring_k
+    T = lp + w  # visible tokens once the window is full
+    raw_k = synth.normal_bf16((Bn, T, hkv, D), seed + 2, dev)  # un-rotated, in id order
+    raw_v = synth.normal_bf16((Bn, T, hkv, D), seed + 3, dev)
+    scratch = PrefixSlidingCache(Bn, hkv, lp, w, D, dev, fill=None)
+    n = warmup + steps
+    k_new = synth.normal_bf16((n, Bn, 1, hkv, D), seed + 4, dev)
+    v_new = synth.normal_bf16((n, Bn, 1, hkv, D), seed + 5, dev)
+    q_raw = synth.normal_bf16((n, Bn, hq, D), seed + 6, dev)
+    out = torch.empty((Bn, hq, D), dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(max(1, B.ps_decode_workspace_bytes(params, Bn)), dtype=torch.uint8,
+                     device=dev)
+    zeros = torch.zeros(Bn, dtype=torch.int64, device=dev)
+    qid = torch.full((Bn,), T - 1, dtype=torch.int64, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def continue_pe(i, q):
+        p = pos0 + i
+        B.ps_kv_append_rope(params, cache.struct, k_new[i], v_new[i], q, p, 1, st)
+        B.ps_decode_attn(params, cache.struct, q, p, out, None, ws, st)
+
+    def reset_here(i, q):
+        p = pos0 + i
+        B.ps_kv_append_rope(params, cache.struct, k_new[i], v_new[i], q, p, 1, st)
+        B.ps_decode_attn_reset_pe(params, cache.struct, q, p, out, None, ws, st)
+
+    def reset_literal(i, q):
+        B.ps_kv_append_rope(params, scratch.struct, raw_k, raw_v, None, zeros, T, st)
+        B.ps_kv_append_rope(params, scratch.struct, k_new[i], v_new[i], q, qid, 1, st)
+        B.ps_decode_attn(params, scratch.struct, q, qid, out, None, ws, st)
+
+    res = {}
+    kv_tok = 2 * hkv * D * 2
+    for name, fn in (("continue_pe", continue_pe), ("reset_pe", reset_here),
+                     ("reset_pe_literal", reset_literal)):
+        qs = q_raw.clone()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(n)]
+        for i in range(n):
+            evs[i][0].record(stream)
+            fn(i, qs[i])
+            evs[i][1].record(stream)
+        torch.cuda.synchronize()
+        assert st.item() == 0, st.item()
+        ms = statistics.median([a.elapsed_time(b) for a, b in evs[warmup:]])
+        res[name] = {"step_us": round(ms * 1e3, 1), "tok_per_s": round(Bn / (ms / 1e3), 1)}
+    # bytes per step: decode reads the visible K/V; the literal path also reads the
+    # un-rotated keys/values and writes them rotated
+    res["continue_pe"]["kv_bytes"] = Bn * T * kv_tok
+    res["reset_pe"]["kv_bytes"] = Bn * T * kv_tok
+    res["reset_pe_literal"]["kv_bytes"] = 3 * Bn * T * kv_tok
+    res["literal_over_here"] = round(res["reset_pe_literal"]["step_us"] /
+                                     res["reset_pe"]["step_us"], 2)
+    res["here_over_continue"] = round(res["reset_pe"]["step_us"] /
+                                      res["continue_pe"]["step_us"], 3)
+    return {"leg": "reset", "workload": wl.name, "steps": steps,
+            "peak_hbm_gbs": peaks["hbm_gbs"], **res}
+
+
 # ------------------------------------------------------- full-stack decode leg
 def run_stack(dev, batch: int, distinct: int, steps: int = 3, warmup: int = 1):
     """Full-stack decode step: 28 layers x (append + decode), 16/2/128, L_prefix 2000,
@@ -878,7 +959,7 @@ def main():
     ap.add_argument("--no-graph", action="store_true",
                     help="launch the timed steps one by one instead of as a CUDA graph")
     ap.add_argument("--leg", default="main", choices=["main", "prefill", "sweep", "stack", "latency",
-                                                      "shared"],
+                                                      "shared", "reset"],
                     help="main: the driver's line; prefill/sweep/stack: one extra workload")
     ap.add_argument("--stack-batch", type=int, default=1024)
     ap.add_argument("--stack-distinct", type=int, default=6)
@@ -906,6 +987,8 @@ def main():
             res = run_latency(dev)
         elif args.leg == "shared":
             res = run_shared(dev)
+        elif args.leg == "reset":
+            res = run_reset(dev)
         else:
             res = run_stack(dev, args.stack_batch, args.stack_distinct)
         if rank == 0:
