@@ -65,6 +65,8 @@ __all__ = [
     "decode_reference",
     "full_attention_decode",
     "reset_pe_positions",
+    "pinned_visible_positions",
+    "pinned_decode_reference",
     "reset_pe_decode_reference",
     "prefill_reference",
     "prefill_backward_reference",
@@ -236,6 +238,28 @@ def full_attention_decode(q: np.ndarray, k_rot: np.ndarray, v: np.ndarray, p: in
                           scale: float):
     """Full causal attention of the query at position p over keys [0, p]."""
     return attend_gqa(q, k_rot[: p + 1], v[: p + 1], scale)
+
+
+def pinned_visible_positions(p: int, l_prefix: int, window: int, pinned) -> np.ndarray:
+    """Visible keys when tokens are appended to the pinned prefix at run time
+    ("Prefix Sliding 完全拆解", §局限: a mechanism for the model to append important tokens to
+    the prefix; multi-turn: pinning later user messages into the prefix).
+
+    The pinned set becomes the prompt rows [0, L_prefix) plus the promoted positions; a
+    pinned token is never evicted.  V(p) = eq. A(i)'s set united with the promoted
+    positions <= p (a promoted token still inside the window is counted once).
+    """
+    base = visible_positions(p, l_prefix, window)
+    extra = np.asarray([t for t in pinned if t <= p], dtype=np.int64)
+    return np.union1d(base, extra).astype(np.int64)
+
+
+def pinned_decode_reference(q: np.ndarray, k_rot: np.ndarray, v: np.ndarray, p: int,
+                            l_prefix: int, window: int, pinned, scale: float):
+    """Decode output of the query at p over pinned_visible_positions (Continue PE: keys
+    already rotated at their absolute positions).  Returns (out [Hq, D], lse [Hq])."""
+    vis = pinned_visible_positions(p, l_prefix, window, pinned)
+    return attend_gqa(q, k_rot[vis], v[vis], scale)
 
 
 def reset_pe_positions(p: int, l_prefix: int, window: int):

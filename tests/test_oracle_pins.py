@@ -491,3 +491,35 @@ def test_reset_pe_equals_shifted_query_for_prefix_keys():
     pre = vis < lp
     np.testing.assert_allclose(reset[:, ~pre], cont[:, ~pre], rtol=0, atol=1e-10)
     np.testing.assert_allclose(reset[:, pre], moved[:, pre], rtol=0, atol=1e-10)
+
+
+# ------------------------------------------------------------ appended prefix
+def test_pinned_visible_by_hand():
+    """L_prefix 2, W 3, promoted {5, 6}: at p = 12 the visible keys are 0, 1, 5, 6, 10..12;
+    at p = 7 the promoted tokens are still in the window (no double count)."""
+    assert O.pinned_visible_positions(12, 2, 3, [5, 6]).tolist() == [0, 1, 5, 6, 10, 11, 12]
+    assert O.pinned_visible_positions(7, 2, 3, [5, 6]).tolist() == [0, 1, 5, 6, 7]
+    assert O.pinned_visible_positions(4, 2, 3, [5, 6]).tolist() == [0, 1, 2, 3, 4]
+
+
+@given(st.integers(0, 20), st.integers(1, 30), st.integers(0, 120),
+       st.lists(st.integers(0, 150), max_size=12))
+@settings(max_examples=150, deadline=None)
+def test_pinned_visible_closed_form(lp, w, p, pinned):
+    """Count = |V(p)| + #{promoted t <= p outside V(p)}; no pins = eq. A(i)'s set."""
+    got = O.pinned_visible_positions(p, lp, w, pinned)
+    base = set(O.visible_positions(p, lp, w).tolist())
+    extra = {t for t in pinned if t <= p} - base
+    assert len(got) == min(p + 1, lp + w) + len(extra)
+    assert O.pinned_visible_positions(p, lp, w, []).tolist() == sorted(base)
+    assert np.all(np.diff(got) > 0)
+
+
+def test_pinned_decode_equals_sdpa_over_the_union():
+    hq, hkv, d, lp, w, p = 4, 2, 16, 3, 5, 40
+    q, k, v = _rand((hq, d), 71), _rand((p + 1, hkv, d), 72), _rand((p + 1, hkv, d), 73)
+    pinned = [10, 11, 12, 30, 38]
+    got, _ = O.pinned_decode_reference(q, k, v, p, lp, w, pinned, 0.25)
+    keys = sorted(set(range(lp)) | {10, 11, 12, 30} | set(range(p - w + 1, p + 1)))
+    want = _sdpa(q[None], k[keys], v[keys], 0.25)[0]
+    np.testing.assert_allclose(got, want, rtol=0, atol=1e-12)
