@@ -195,6 +195,43 @@ int ps_decode_attn_shared_prefix(const ps_params* params, const ps_kv_cache* cac
                                  void* out, float* lse, void* workspace, size_t ws_bytes,
                                  int32_t* dev_status, ps_stream_t stream);
 
+/* Append tokens to the pinned prefix at run time.  Source: §局限 of "Prefix Sliding 完全拆解"
+ * (a mechanism for the model to append important tokens to the prefix; whether later user
+ * messages of a conversation should be pinned into the prefix).  A promoted token is
+ * never evicted: from then on every query sees it, together with eq. A(i)'s set.
+ * The prefix store has room for appended tokens: cache->k_prefix / v_prefix are
+ * [batch, Hkv, prefix_capacity, D]; rows [0, l_prefix) hold the prompt (fill them with
+ * ps_kv_append_rope on a linear view of the store, ring NULL, params with
+ * l_prefix = prefix_capacity), rows [l_prefix, l_prefix + pin_count[b]) the promoted
+ * tokens in ascending position order.  Decode-phase appends go through a ring-only view
+ * (prefix pointers NULL).
+ *   pin_count : device int32 [batch], promoted tokens so far (start at 0); updated.
+ *   pin_pos   : device int64 [batch, prefix_capacity - l_prefix], their positions; updated.
+ *   t0, t1    : device int64 [batch]; tokens [t0[b], t1[b]) of sequence b are promoted
+ *               (t1 <= t0: nothing).  They must still be in the window of pos[b] (the latest
+ *               appended position): l_prefix <= t0, t0 > pos - W, t1 - 1 <= pos; follow the
+ *               previous promoted position; and fit the capacity.  Otherwise the sequence
+ *               is left unchanged and PS_DEV_POS_RANGE is set.
+ * Their K/V rows are copied from the ring unchanged (Continue PE: already rotated). */
+int ps_kv_pin(const ps_params* params, const ps_kv_cache* cache, int32_t prefix_capacity,
+              int32_t* pin_count, int64_t* pin_pos, const int64_t* t0, const int64_t* t1,
+              const int64_t* pos, int32_t* dev_status, ps_stream_t stream);
+
+/* Bytes of device workspace ps_decode_attn_pinned needs.  0 on invalid arguments. */
+size_t ps_decode_pinned_workspace_bytes(const ps_params* params, int64_t batch,
+                                        int32_t prefix_capacity);
+
+/* Decode step with promoted tokens (ps_kv_pin): the query at pos[b] attends the prompt
+ * rows, every promoted token at a position <= pos[b], and the window, each key once (a
+ * promoted token still inside the window is read from the ring).  Promoted rows whose
+ * positions precede the window start are read with the prefix (a binary search over
+ * pin_pos per sequence).  Other arguments and results as ps_decode_attn. */
+int ps_decode_attn_pinned(const ps_params* params, const ps_kv_cache* cache,
+                          int32_t prefix_capacity, const int32_t* pin_count,
+                          const int64_t* pin_pos, const void* q, const int64_t* pos, void* out,
+                          float* lse, void* workspace, size_t ws_bytes, int32_t* dev_status,
+                          ps_stream_t stream);
+
 /* Bytes of device workspace ps_full_attn_ref needs (same split-K layout as decode). */
 size_t ps_full_attn_workspace_bytes(const ps_params* params, int64_t batch, int64_t lmax);
 

@@ -85,6 +85,12 @@ _SIGS = {
     "ps_decode_attn_reset_pe": (c_int32, [POINTER(PsParams), POINTER(PsKVCache), c_void_p,
                                           c_void_p, c_void_p, c_void_p, c_void_p, c_size_t,
                                           c_void_p, c_void_p]),
+    "ps_kv_pin": (c_int32, [POINTER(PsParams), POINTER(PsKVCache), c_int32, c_void_p, c_void_p,
+                            c_void_p, c_void_p, c_void_p, c_void_p, c_void_p]),
+    "ps_decode_pinned_workspace_bytes": (c_size_t, [POINTER(PsParams), c_int64, c_int32]),
+    "ps_decode_attn_pinned": (c_int32, [POINTER(PsParams), POINTER(PsKVCache), c_int32,
+                                        c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                        c_void_p, c_void_p, c_size_t, c_void_p, c_void_p]),
     "ps_decode_shared_prefix_workspace_bytes": (c_size_t, [POINTER(PsParams), c_int64,
                                                            c_int64]),
     "ps_decode_attn_shared_prefix": (c_int32, [POINTER(PsParams), POINTER(PsKVCache), c_int64,
@@ -190,6 +196,31 @@ def ps_decode_attn_reset_pe(params: PsParams, cache: PsKVCache, q, pos, out, lse
                                         _ptr(pos), _ptr(out), _ptr(lse), _ptr(workspace),
                                         ws_bytes, _ptr(dev_status), _stream(stream))
     _check(rc, "ps_decode_attn_reset_pe")
+
+
+def ps_kv_pin(params: PsParams, cache: PsKVCache, prefix_capacity: int, pin_count, pin_pos, t0,
+              t1, pos, dev_status=None, stream=None) -> None:
+    """Promote tokens [t0[b], t1[b]) (still in the window) into the pinned prefix."""
+    rc = load().ps_kv_pin(ctypes.byref(params), ctypes.byref(cache), int(prefix_capacity),
+                          _ptr(pin_count), _ptr(pin_pos), _ptr(t0), _ptr(t1), _ptr(pos),
+                          _ptr(dev_status), _stream(stream))
+    _check(rc, "ps_kv_pin")
+
+
+def ps_decode_pinned_workspace_bytes(params: PsParams, batch: int, prefix_capacity: int) -> int:
+    return int(load().ps_decode_pinned_workspace_bytes(ctypes.byref(params), int(batch),
+                                                       int(prefix_capacity)))
+
+
+def ps_decode_attn_pinned(params: PsParams, cache: PsKVCache, prefix_capacity: int, pin_count,
+                          pin_pos, q, pos, out, lse=None, workspace=None, dev_status=None,
+                          stream=None) -> None:
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rc = load().ps_decode_attn_pinned(ctypes.byref(params), ctypes.byref(cache),
+                                      int(prefix_capacity), _ptr(pin_count), _ptr(pin_pos),
+                                      _ptr(q), _ptr(pos), _ptr(out), _ptr(lse), _ptr(workspace),
+                                      ws_bytes, _ptr(dev_status), _stream(stream))
+    _check(rc, "ps_decode_attn_pinned")
 
 
 def ps_decode_attn_noalloc(params: PsParams, cache: PsKVCache, q, pos, out, lse=None,

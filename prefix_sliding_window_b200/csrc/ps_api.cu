@@ -286,7 +286,8 @@ size_t ps_decode_workspace_bytes(const ps_params* params, int64_t batch) {
 static int decode_entry(const ps_params* params, const ps_kv_cache* cache, const void* q,
                         const int64_t* pos, void* out, float* lse, void* workspace,
                         size_t ws_bytes, int32_t* dev_status, ps_stream_t stream,
-                        int32_t reset_pe) {
+                        int32_t reset_pe, int32_t lcap = 0, const int32_t* pin_count = nullptr,
+                        const int64_t* pin_pos = nullptr) {
   g_last_error.clear();
   PS_TRY(check_params(params, true));
   if (params->n_q_heads / params->n_kv_heads > kMaxGroup)
@@ -308,11 +309,12 @@ static int decode_entry(const ps_params* params, const ps_kv_cache* cache, const
     return fail(PS_ERR_INVALID_ARG, "pos is not 8-byte aligned");
   if ((reinterpret_cast<uintptr_t>(dev_status) & 3u) != 0)
     return fail(PS_ERR_INVALID_ARG, "dev_status is not 4-byte aligned");
+  const int64_t pre_rows = lcap > params->l_prefix ? lcap : params->l_prefix;
   const size_t need = decode_workspace_bytes(cache->batch, params->n_kv_heads,
-                                             (int64_t)params->l_prefix + params->window);
+                                             pre_rows + params->window);
   if (need > 0) {
     if (!workspace || ws_bytes < need)
-      return fail(PS_ERR_WORKSPACE, "workspace smaller than ps_decode_workspace_bytes()");
+      return fail(PS_ERR_WORKSPACE, "workspace smaller than the decode workspace size");
     PS_TRY(check_ptr(workspace, "workspace"));
   }
   DecodeLaunch l{};
@@ -336,6 +338,9 @@ static int decode_entry(const ps_params* params, const ps_kv_cache* cache, const
   l.v1 = cache->v_ring;
   l.reset_pe = reset_pe;
   l.rope_theta = params->rope_theta;
+  l.lcap = lcap;
+  l.pin_count = pin_count;
+  l.pin_pos = pin_pos;
   return launch_decode(l, reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -687,6 +692,72 @@ int ps_decode_attn_shared_prefix(const ps_params* params, const ps_kv_cache* cac
   rc = launch_decode(l, st);
   cudaEventDestroy(fk.fork);
   return rc;
+}
+
+int ps_kv_pin(const ps_params* params, const ps_kv_cache* cache, int32_t prefix_capacity,
+              int32_t* pin_count, int64_t* pin_pos, const int64_t* t0, const int64_t* t1,
+              const int64_t* pos, int32_t* dev_status, ps_stream_t stream) {
+  g_last_error.clear();
+  PS_TRY(check_params(params, true));
+  if (!cache) return fail(PS_ERR_INVALID_ARG, "cache is NULL");
+  if (cache->batch < 0) return fail(PS_ERR_INVALID_ARG, "cache->batch must be >= 0");
+  if (prefix_capacity <= params->l_prefix)
+    return fail(PS_ERR_INVALID_ARG, "prefix_capacity must exceed l_prefix");
+  if (cache->batch == 0) return PS_OK;
+  PS_TRY(check_ptr(cache->k_prefix, "cache->k_prefix"));
+  PS_TRY(check_ptr(cache->v_prefix, "cache->v_prefix"));
+  PS_TRY(check_ptr(cache->k_ring, "cache->k_ring"));
+  PS_TRY(check_ptr(cache->v_ring, "cache->v_ring"));
+  if (!pin_count || !pin_pos || !t0 || !t1 || !pos)
+    return fail(PS_ERR_INVALID_ARG, "pin_count, pin_pos, t0, t1 and pos are required");
+  if (((reinterpret_cast<uintptr_t>(pin_pos) | reinterpret_cast<uintptr_t>(t0) |
+        reinterpret_cast<uintptr_t>(t1) | reinterpret_cast<uintptr_t>(pos)) & 7u) != 0 ||
+      (reinterpret_cast<uintptr_t>(pin_count) & 3u) != 0)
+    return fail(PS_ERR_INVALID_ARG, "misaligned pin metadata or positions");
+  if ((reinterpret_cast<uintptr_t>(dev_status) & 3u) != 0)
+    return fail(PS_ERR_INVALID_ARG, "dev_status is not 4-byte aligned");
+  PinArgs a;
+  a.k_ring = cache->k_ring;
+  a.v_ring = cache->v_ring;
+  a.k_pre = cache->k_prefix;
+  a.v_pre = cache->v_prefix;
+  a.pin_count = pin_count;
+  a.pin_pos = pin_pos;
+  a.t0 = t0;
+  a.t1 = t1;
+  a.pos = pos;
+  a.status = dev_status;
+  a.batch = cache->batch;
+  a.hkv = params->n_kv_heads;
+  a.lp = params->l_prefix;
+  a.w = params->window;
+  a.lcap = prefix_capacity;
+  return check_cuda(launch_pin(a, reinterpret_cast<cudaStream_t>(stream)), "pin_kernel launch");
+}
+
+size_t ps_decode_pinned_workspace_bytes(const ps_params* params, int64_t batch,
+                                        int32_t prefix_capacity) {
+  if (check_params(params, true) != PS_OK || batch < 0 || prefix_capacity < params->l_prefix)
+    return 0;
+  return decode_workspace_bytes(batch, params->n_kv_heads,
+                                (int64_t)prefix_capacity + params->window);
+}
+
+int ps_decode_attn_pinned(const ps_params* params, const ps_kv_cache* cache,
+                          int32_t prefix_capacity, const int32_t* pin_count,
+                          const int64_t* pin_pos, const void* q, const int64_t* pos, void* out,
+                          float* lse, void* workspace, size_t ws_bytes, int32_t* dev_status,
+                          ps_stream_t stream) {
+  g_last_error.clear();
+  if (!params) return fail(PS_ERR_INVALID_ARG, "params is NULL");
+  if (prefix_capacity <= params->l_prefix)
+    return fail(PS_ERR_INVALID_ARG, "prefix_capacity must exceed l_prefix");
+  if (!pin_count || !pin_pos) return fail(PS_ERR_INVALID_ARG, "pin_count and pin_pos required");
+  if ((reinterpret_cast<uintptr_t>(pin_pos) & 7u) != 0 ||
+      (reinterpret_cast<uintptr_t>(pin_count) & 3u) != 0)
+    return fail(PS_ERR_INVALID_ARG, "misaligned pin metadata");
+  return decode_entry(params, cache, q, pos, out, lse, workspace, ws_bytes, dev_status, stream,
+                      0, prefix_capacity, pin_count, pin_pos);
 }
 
 }  // extern "C"

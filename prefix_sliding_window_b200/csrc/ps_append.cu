@@ -156,7 +156,53 @@ __global__ void __launch_bounds__(kAppendThreads) append_rope_kernel(const Appen
   }
 }
 
+// One CTA per sequence: validate the range (inside the window of the latest position, in
+// ascending order after the last promoted token, within capacity), then copy 16-byte chunks
+// of K and V rows from ring slots (t - lp) mod w to prefix rows lp + pin_count + (t - t0).
+// Keys stay as cached: Continue PE rotated them at their absolute positions already.
+__global__ void __launch_bounds__(256) pin_kernel(const PinArgs a) {
+  const int64_t b = blockIdx.x;
+  const int64_t t0 = a.t0[b], t1 = a.t1[b], p = a.pos[b];
+  const int32_t cnt = a.pin_count[b];
+  const int64_t m = t1 - t0;
+  if (m <= 0) return;
+  const int32_t cap = a.lcap - a.lp;
+  const int64_t* pp = a.pin_pos + b * cap;
+  const bool ok = t0 >= a.lp && t1 - 1 <= p && t0 > p - a.w && cnt + m <= cap &&
+                  (cnt == 0 || t0 > pp[cnt - 1]);
+  if (!ok) {
+    if (threadIdx.x == 0 && a.status) atomicOr(a.status, PS_DEV_POS_RANGE);
+    return;
+  }
+  constexpr int kChunks = kHeadDim / 8;  // 16-byte chunks per row
+  const int64_t items = m * a.hkv * 2 * kChunks;
+  for (int64_t it = threadIdx.x; it < items; it += blockDim.x) {
+    const int c = static_cast<int>(it % kChunks);
+    const int kv = static_cast<int>((it / kChunks) % 2);
+    const int h = static_cast<int>((it / (2 * kChunks)) % a.hkv);
+    const int64_t i = it / (2 * kChunks * a.hkv);
+    const int64_t slot = (t0 + i - a.lp) % a.w;
+    const int64_t row = a.lp + cnt + i;
+    const uint4* src = static_cast<const uint4*>(kv ? a.v_ring : a.k_ring) +
+                       ((b * a.hkv + h) * a.w + slot) * kChunks + c;
+    uint4* dst = static_cast<uint4*>(kv ? a.v_pre : a.k_pre) +
+                 ((b * a.hkv + h) * a.lcap + row) * kChunks + c;
+    *dst = *src;
+  }
+  int64_t* wp = a.pin_pos + b * cap;
+  for (int64_t i = threadIdx.x; i < m; i += blockDim.x) wp[cnt + i] = t0 + i;
+  __syncthreads();  // every thread has read cnt before it changes
+  if (threadIdx.x == 0) a.pin_count[b] = cnt + static_cast<int32_t>(m);
+}
+
 }  // namespace
+
+cudaError_t launch_pin(const PinArgs& a, cudaStream_t stream) {
+  if (a.batch <= 0) return cudaSuccess;
+  if (a.batch > 0x7fffffff) return cudaErrorInvalidConfiguration;
+  pin_kernel<<<static_cast<unsigned>(a.batch), 256, 0, stream>>>(a);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_append(const AppendArgs& a, cudaStream_t stream) {
   const int64_t tokens = a.batch * a.T;

@@ -78,6 +78,11 @@ struct DecodeArgs {
   // more (its Reset-PE id); inv_freq = theta^(-2i/D) in float64
   int32_t reset_pe;
   double inv_freq[kHeadDim / 2];
+  // tokens appended to the pinned prefix: rows [L_prefix, L_prefix + pin_count[b]) of the
+  // prefix store hold the promoted positions pin_pos[b][0..) (ascending)
+  const int32_t* pin_count;
+  const int64_t* pin_pos;
+  int32_t pin_cap;
 };
 
 // Offset of the 16-byte chunk `chunk` (0..7) of box row `row` under the 128-byte swizzle
@@ -90,7 +95,7 @@ __device__ __forceinline__ bool bad_position(const DecodeArgs& a, int64_t p) {
   return (p < 0) || (a.full_mode && p >= a.lmax);
 }
 
-__device__ __forceinline__ DecodeTiling tiling_of(const DecodeArgs& a, int64_t p) {
+__device__ __forceinline__ DecodeTiling tiling_of(const DecodeArgs& a, int64_t b, int64_t p) {
   VisibleRanges r{0, 0, 0, 0};
   if (!bad_position(a, p)) {
     if (a.full_mode)
@@ -98,6 +103,19 @@ __device__ __forceinline__ DecodeTiling tiling_of(const DecodeArgs& a, int64_t p
     else
       r = visible_ranges(p, a.lp, a.w);
     if (a.skip_prefix) r.pre_len = 0;  // the shared-prefix pass covers those rows
+    if (a.pin_count && p >= a.lp) {
+      // promoted rows whose positions precede the window start are read with the prefix;
+      // the rest are still in the window (ascending positions: a binary search)
+      int64_t ws = p + 1 - a.w;
+      if (ws < a.lp) ws = a.lp;
+      const int64_t* pp = a.pin_pos + b * a.pin_cap;
+      int lo = 0, hi = a.pin_count[b];
+      while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if (pp[mid] < ws) lo = mid + 1; else hi = mid;
+      }
+      r.pre_len += lo;
+    }
   }
   return make_tiling(r, a.dim0, a.w);
 }
@@ -114,7 +132,7 @@ struct TileWalker {
     const int64_t cnt = pref[b + 1] - pref[b];
     pu = (int64_t)a.hkv * pref[b] + h * cnt;
     pu1 = pu + cnt;
-    tiling = tiling_of(a, a.pos[b]);
+    tiling = tiling_of(a, b, a.pos[b]);
   }
   // position the walker on global tile t0 (t0 < total)
   __device__ void seek(const DecodeArgs& a, const int32_t* pref, int64_t t0) {
@@ -226,7 +244,7 @@ __global__ void __launch_bounds__(kThreads)
     // tiles per sequence, then an inclusive scan (batch <= kMaxStreamKSeqs)
     for (int b = threadIdx.x; b < a.batch; b += kThreads) {
       const int64_t p = a.pos[b];
-      const int32_t cnt = tiling_of(a, p).total;
+      const int32_t cnt = tiling_of(a, b, p).total;
       pref[b + 1] = cnt;
       if (blockIdx.x == 0 && cnt == 0) {
         if (bad_position(a, p) && a.status)
@@ -273,7 +291,7 @@ __global__ void __launch_bounds__(kThreads)
     const int64_t p = a.pos[wk.b];
     if (bad_position(a, p) && threadIdx.x == 0 && wk.h == 0 && a.status)
       atomicOr(a.status, p < 0 ? PS_DEV_BAD_POS : PS_DEV_POS_RANGE);
-    wk.tiling = tiling_of(a, p);
+    wk.tiling = tiling_of(a, wk.b, p);
     wk.t = 0;
     wk.t_end = wk.tiling.total;
     wk.pu = 0;
@@ -710,15 +728,19 @@ size_t decode_workspace_bytes(int64_t batch, int32_t hkv, int64_t max_keys, bool
 
 int launch_decode(const DecodeLaunch& l, cudaStream_t stream) {
   const int group = l.hq / l.hkv;
-  const int64_t max_keys = l.full_mode ? l.lmax : (int64_t)l.lp + l.w;
+  const int64_t max_keys =
+      l.full_mode ? l.lmax : (int64_t)(l.lcap > l.lp ? l.lcap : l.lp) + l.w;
   const bool force = l.pre_o != nullptr;  // prefix partials are combined by the merge
   const int64_t g = streamk_grid(l.batch, l.hkv, max_keys, force);
   if (force && g == 0) return fail(PS_ERR_UNSUPPORTED, "shared-prefix decode needs batch <= 1024");
   if (g > 0 && l.workspace == nullptr)
     return fail(PS_ERR_WORKSPACE, "split-K decode launched without a workspace");
   const int64_t units = l.batch * l.hkv;
-  // window-only decode reads no prefix rows: no prefix map (it may describe fewer units)
-  const int32_t dim0 = l.full_mode ? static_cast<int32_t>(l.lmax) : (l.skip_prefix ? 0 : l.lp);
+  // window-only decode reads no prefix rows: no prefix map (it may describe fewer units);
+  // a prefix store with room for appended tokens has lcap rows per (sequence, KV head)
+  const int32_t pre_rows = l.lcap > l.lp ? l.lcap : l.lp;
+  const int32_t dim0 =
+      l.full_mode ? static_cast<int32_t>(l.lmax) : (l.skip_prefix ? 0 : pre_rows);
 
   CUtensorMap mk0, mv0, mk1, mv1;
   // A zero-row tensor cannot be described; such a map is never used (no tiles), so it
@@ -771,6 +793,9 @@ int launch_decode(const DecodeLaunch& l, cudaStream_t stream) {
   a.scale_log2 = l.scale * kLog2e;
   a.skip_prefix = l.skip_prefix;
   a.reset_pe = l.reset_pe;
+  a.pin_count = l.pin_count;
+  a.pin_pos = l.pin_pos;
+  a.pin_cap = (l.lcap > l.lp) ? l.lcap - l.lp : 0;
   for (int i = 0; i < kHeadDim / 2; ++i)
     a.inv_freq[i] = l.reset_pe ? pow(l.rope_theta, -2.0 * i / double(kHeadDim)) : 0.0;
   const int32_t pre_splits = l.pre_o ? (l.pre_splits > 0 ? l.pre_splits : 1) : 0;

@@ -68,6 +68,25 @@ struct AppendArgs {
 };
 cudaError_t launch_append(const AppendArgs& a, cudaStream_t stream);
 
+// Appends tokens [t0[b], t1[b]) of each sequence, still in its window, to its pinned
+// prefix: copies their (already rotated) K/V rows from the ring into prefix rows
+// [lp + pin_count[b], ...) of a store with lcap rows and records their positions.
+struct PinArgs {
+  const void* k_ring;
+  const void* v_ring;
+  void* k_pre;
+  void* v_pre;
+  int32_t* pin_count;
+  int64_t* pin_pos;
+  const int64_t* t0;
+  const int64_t* t1;
+  const int64_t* pos;
+  int32_t* status;
+  int64_t batch;
+  int32_t hkv, lp, w, lcap;
+};
+cudaError_t launch_pin(const PinArgs& a, cudaStream_t stream);
+
 // ---------------------------------------------------------------- decode
 struct DecodeLaunch {
   const void* q;
@@ -99,6 +118,11 @@ struct DecodeLaunch {
   // Reset-PE id L_prefix + |window| - 1 instead of its absolute position
   int32_t reset_pe;
   double rope_theta;
+  // prefix store with room for tokens appended at run time: lcap rows per (sequence, KV
+  // head); rows [lp, lp + pin_count[b]) hold promoted positions pin_pos[b][..] (ascending)
+  int32_t lcap;
+  const int32_t* pin_count;
+  const int64_t* pin_pos;
 };
 // Split count and workspace bytes for a decode of this shape on the current device.
 int decode_splits(int64_t batch, int32_t hkv, int64_t max_keys);
