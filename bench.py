@@ -805,6 +805,79 @@ def run_reset(dev, steps: int = 16, warmup: int = 3):
             "peak_hbm_gbs": peaks["hbm_gbs"], **res}
 
 
+# ------------------------------------------------------- appended-prefix leg
+def run_pin(dev, steps: int = 20, warmup: int = 3, n_pin: int = 1024):
+    """Tokens appended to the pinned prefix: the batch-64 decode workload (16/2/128,
+    L_prefix 100, W 4096, positions U[8192, 131072]) where every sequence has promoted
+    n_pin earlier tokens (now outside its window).  Decode reads L_prefix + n_pin + W keys
+    per sequence; compared with the same batch without promotions, and the promotion of
+    256 window tokens per sequence (ps_kv_pin) is timed on its own."""
+    from prefix_sliding_window_b200 import binding as B
+    wl = synth.WORKLOADS[WORKLOAD]
+    Bn, hq, hkv, lp, w = wl.batch, wl.n_q_heads, wl.n_kv_heads, wl.l_prefix, wl.window
+    lcap = lp + n_pin + 256
+    peaks = _peaks()
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    seed = synth.seed_for(wl.index, 11)
+    pos = synth.uniform_positions(Bn, wl.pos_lo, wl.pos_hi, seed, dev)
+    params = B.make_params(hq, hkv, D, lp, w, wl.rope_theta)
+    k_pre = synth.normal_bf16((Bn, hkv, lcap, D), seed + 1, dev)
+    v_pre = synth.normal_bf16((Bn, hkv, lcap, D), seed + 2, dev)
+    k_ring = synth.normal_bf16((Bn, hkv, w, D), seed + 3, dev)
+    v_ring = synth.normal_bf16((Bn, hkv, w, D), seed + 4, dev)
+    cache = B.make_cache(k_pre, v_pre, k_ring, v_ring, Bn)
+    # n_pin promoted tokens per sequence, all before the window start
+    start = (pos - w - n_pin).clamp(min=lp).view(Bn, 1)
+    pin_pos = torch.full((Bn, lcap - lp), -1, dtype=torch.int64, device=dev)
+    pin_pos[:, :n_pin] = start + torch.arange(n_pin, device=dev).view(1, n_pin)
+    pin_count = torch.full((Bn,), n_pin, dtype=torch.int32, device=dev)
+    no_pins = torch.zeros(Bn, dtype=torch.int32, device=dev)
+    q = synth.normal_bf16((Bn, hq, D), seed + 5, dev)
+    out = torch.empty((Bn, hq, D), dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(max(1, B.ps_decode_pinned_workspace_bytes(params, Bn, lcap)),
+                     dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def timed(fn, n=steps):
+        for _ in range(warmup):
+            fn()
+        torch.cuda.synchronize()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(n)]
+        for a, b in evs:
+            a.record(stream)
+            fn()
+            b.record(stream)
+        torch.cuda.synchronize()
+        assert st.item() == 0, st.item()
+        return statistics.median([a.elapsed_time(b) for a, b in evs])
+
+    kv_tok = 2 * hkv * D * 2
+    res = {}
+    for name, cnt, keys in (("with_pins", pin_count, lp + n_pin + w), ("no_pins", no_pins,
+                                                                        lp + w)):
+        ms = timed(lambda cnt=cnt: B.ps_decode_attn_pinned(params, cache, lcap, cnt, pin_pos, q,
+                                                           pos, out, None, ws, st))
+        gbs = Bn * keys * kv_tok / (ms / 1e3) / 1e9
+        res[name] = {"attn_us": round(ms * 1e3, 1), "keys_per_seq": keys,
+                     "tok_per_s": round(Bn / (ms / 1e3), 1), "gbs": round(gbs, 1),
+                     "frac": round(gbs / peaks["hbm_gbs"], 4)}
+    # promotion of the newest 256 window tokens of every sequence (a copy of 256 KB each)
+    t0 = pos - 255
+    t1 = pos + 1
+    base = pin_count.clone()
+    pp = pin_pos.clone()
+
+    def promote():
+        pin_count.copy_(base)
+        B.ps_kv_pin(params, cache, lcap, pin_count, pp, t0, t1, pos, st)
+    ms = timed(promote)
+    res["pin_256_tokens_us"] = round(ms * 1e3, 1)
+    res["pin_bytes"] = 2 * Bn * 256 * kv_tok
+    return {"leg": "pin", "workload": wl.name, "n_pin": n_pin, "peak_hbm_gbs": peaks["hbm_gbs"],
+            **res}
+
+
 # ------------------------------------------------------- full-stack decode leg
 def run_stack(dev, batch: int, distinct: int, steps: int = 3, warmup: int = 1):
     """Full-stack decode step: 28 layers x (append + decode), 16/2/128, L_prefix 2000,
@@ -959,7 +1032,7 @@ def main():
     ap.add_argument("--no-graph", action="store_true",
                     help="launch the timed steps one by one instead of as a CUDA graph")
     ap.add_argument("--leg", default="main", choices=["main", "prefill", "sweep", "stack", "latency",
-                                                      "shared", "reset"],
+                                                      "shared", "reset", "pin"],
                     help="main: the driver's line; prefill/sweep/stack: one extra workload")
     ap.add_argument("--stack-batch", type=int, default=1024)
     ap.add_argument("--stack-distinct", type=int, default=6)
@@ -989,6 +1062,8 @@ def main():
             res = run_shared(dev)
         elif args.leg == "reset":
             res = run_reset(dev)
+        elif args.leg == "pin":
+            res = run_pin(dev)
         else:
             res = run_stack(dev, args.stack_batch, args.stack_distinct)
         if rank == 0:
