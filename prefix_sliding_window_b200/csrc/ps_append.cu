@@ -156,43 +156,69 @@ __global__ void __launch_bounds__(kAppendThreads) append_rope_kernel(const Appen
   }
 }
 
-// One CTA per sequence: validate the range (inside the window of the latest position, in
-// ascending order after the last promoted token, within capacity), then copy 16-byte chunks
-// of K and V rows from ring slots (t - lp) mod w to prefix rows lp + pin_count + (t - t0).
-// Keys stay as cached: Continue PE rotated them at their absolute positions already.
-__global__ void __launch_bounds__(256) pin_kernel(const PinArgs a) {
-  const int64_t b = blockIdx.x;
+// Whether sequence b's promotion request is valid: inside the window of the latest position,
+// after the last promoted token (ascending order), within capacity.  Both pin kernels
+// evaluate it on the same inputs (pin_count changes only in the second).
+__device__ __forceinline__ bool pin_valid(const PinArgs& a, int64_t b, int64_t* m_out,
+                                          int32_t* cnt_out) {
   const int64_t t0 = a.t0[b], t1 = a.t1[b], p = a.pos[b];
   const int32_t cnt = a.pin_count[b];
   const int64_t m = t1 - t0;
-  if (m <= 0) return;
   const int32_t cap = a.lcap - a.lp;
+  *m_out = m;
+  *cnt_out = cnt;
+  if (m <= 0) return false;
   const int64_t* pp = a.pin_pos + b * cap;
-  const bool ok = t0 >= a.lp && t1 - 1 <= p && t0 > p - a.w && cnt + m <= cap &&
-                  (cnt == 0 || t0 > pp[cnt - 1]);
-  if (!ok) {
-    if (threadIdx.x == 0 && a.status) atomicOr(a.status, PS_DEV_POS_RANGE);
-    return;
-  }
+  return t0 >= a.lp && t1 - 1 <= p && t0 > p - a.w && cnt + m <= cap &&
+         (cnt == 0 || t0 > pp[cnt - 1]);
+}
+
+constexpr int kPinTokens = 32;  // tokens per copy block (one warp per token, 8 warps)
+
+// Block (b, chunk) copies tokens [32 chunk, 32 chunk + 32) of sequence b's range: K and V
+// rows from ring slots (t - lp) mod w to prefix rows lp + pin_count + (t - t0), 16 bytes per
+// lane, and records their positions.  Keys stay as cached (Continue PE rotated them at their
+// absolute positions already).
+__global__ void __launch_bounds__(256) pin_copy_kernel(const PinArgs a) {
+  const int64_t b = blockIdx.x;
+  int64_t m;
+  int32_t cnt;
+  if (!pin_valid(a, b, &m, &cnt)) return;
+  const int64_t first = (int64_t)blockIdx.y * kPinTokens;
+  if (first >= m) return;
+  const int n = static_cast<int>(m - first < kPinTokens ? m - first : kPinTokens);
+  const int64_t t0 = a.t0[b] + first;
   constexpr int kChunks = kHeadDim / 8;  // 16-byte chunks per row
-  const int64_t items = m * a.hkv * 2 * kChunks;
-  for (int64_t it = threadIdx.x; it < items; it += blockDim.x) {
-    const int c = static_cast<int>(it % kChunks);
-    const int kv = static_cast<int>((it / kChunks) % 2);
-    const int h = static_cast<int>((it / (2 * kChunks)) % a.hkv);
-    const int64_t i = it / (2 * kChunks * a.hkv);
+  const int per_token = a.hkv * 2 * kChunks;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int i = warp; i < n; i += 8) {
     const int64_t slot = (t0 + i - a.lp) % a.w;
-    const int64_t row = a.lp + cnt + i;
-    const uint4* src = static_cast<const uint4*>(kv ? a.v_ring : a.k_ring) +
-                       ((b * a.hkv + h) * a.w + slot) * kChunks + c;
-    uint4* dst = static_cast<uint4*>(kv ? a.v_pre : a.k_pre) +
-                 ((b * a.hkv + h) * a.lcap + row) * kChunks + c;
-    *dst = *src;
+    const int64_t row = a.lp + cnt + first + i;
+    for (int j = lane; j < per_token; j += 32) {
+      const int c = j % kChunks;
+      const int kv = (j / kChunks) & 1;
+      const int h = j / (2 * kChunks);
+      const int64_t bh = b * a.hkv + h;
+      const uint4* src = static_cast<const uint4*>(kv ? a.v_ring : a.k_ring) +
+                         (bh * a.w + slot) * kChunks + c;
+      uint4* dst = static_cast<uint4*>(kv ? a.v_pre : a.k_pre) + (bh * a.lcap + row) * kChunks + c;
+      *dst = *src;
+    }
   }
-  int64_t* wp = a.pin_pos + b * cap;
-  for (int64_t i = threadIdx.x; i < m; i += blockDim.x) wp[cnt + i] = t0 + i;
-  __syncthreads();  // every thread has read cnt before it changes
-  if (threadIdx.x == 0) a.pin_count[b] = cnt + static_cast<int32_t>(m);
+  if (threadIdx.x < n) a.pin_pos[b * (a.lcap - a.lp) + cnt + first + threadIdx.x] = t0 + threadIdx.x;
+}
+
+// One thread per sequence: advance pin_count (or flag an invalid request).
+__global__ void pin_commit_kernel(const PinArgs a) {
+  const int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (b >= a.batch) return;
+  int64_t m;
+  int32_t cnt;
+  if (pin_valid(a, b, &m, &cnt)) {
+    a.pin_count[b] = cnt + static_cast<int32_t>(m);
+  } else if (m > 0 && a.status) {
+    atomicOr(a.status, PS_DEV_POS_RANGE);
+  }
 }
 
 }  // namespace
@@ -200,7 +226,13 @@ __global__ void __launch_bounds__(256) pin_kernel(const PinArgs a) {
 cudaError_t launch_pin(const PinArgs& a, cudaStream_t stream) {
   if (a.batch <= 0) return cudaSuccess;
   if (a.batch > 0x7fffffff) return cudaErrorInvalidConfiguration;
-  pin_kernel<<<static_cast<unsigned>(a.batch), 256, 0, stream>>>(a);
+  const int64_t chunks = (a.lcap - a.lp + kPinTokens - 1) / kPinTokens;
+  if (chunks > 65535) return cudaErrorInvalidConfiguration;
+  pin_copy_kernel<<<dim3(static_cast<unsigned>(a.batch), static_cast<unsigned>(chunks)), 256, 0,
+                    stream>>>(a);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  pin_commit_kernel<<<static_cast<unsigned>((a.batch + 255) / 256), 256, 0, stream>>>(a);
   return cudaGetLastError();
 }
 
