@@ -459,8 +459,8 @@ def run_prefill(dev, steps: int = 10, warmup: int = 3):
 def run_prefill_bwd(dev, params, wl, q, k, v, out, lse, st, pairs, n_tiles, steps, warmup, peaks):
     """Backward of the same prefill (dQ, dK, dV from dO, the forward's output and lse).
     Algorithmic FLOPs = 10 * D per visible pair per query head (the score recompute, dP,
-    dV, dK and dQ products: 2.5x the forward); the computed-tile figure counts the 7
-    products per planned tile the two-kernel design runs (S and dP are formed twice)."""
+    dV, dK and dQ products: 2.5x the forward); the computed-tile figure counts the same 5
+    products over every planned 128 x 128 tile (masked elements included)."""
     from prefix_sliding_window_b200 import binding as B
     Bn, S, hq, hkv = wl.batch, wl.seq, wl.n_q_heads, wl.n_kv_heads
     do = synth.normal_bf16((Bn, S, hq, D), synth.seed_for(3, 4), dev)
@@ -482,7 +482,7 @@ def run_prefill_bwd(dev, params, wl, q, k, v, out, lse, st, pairs, n_tiles, step
     ms = [a.elapsed_time(b) for a, b in evs]
     med = statistics.median(ms) / 1e3
     flops = 10 * D * pairs * hq * Bn
-    computed = 14 * D * 128 * 128 * n_tiles * hq * Bn
+    computed = 10 * D * 128 * 128 * n_tiles * hq * Bn
     tflops = flops / med / 1e12
     return {"ms": round(med * 1e3, 4), "ms_p10": round(float(np.percentile(ms, 10)), 4),
             "ms_p90": round(float(np.percentile(ms, 90)), 4),

@@ -10,18 +10,18 @@
 // (§Kernel 实现) are visited; PARTIAL tiles are masked element-wise.
 //
 // Three kernels:
-//   bwd_prep_kernel - one warp per (batch, head, row): -D_i and -lse_i*log2(e) into
-//             workspace rows padded to whole 128-row tiles (padding: 0 and -inf, so padded
-//             rows contribute nothing); zeroes the key-tile work counter.
-//   bwd_dq_kernel - query-tile-major, persistent like the forward: per planned key tile,
-//             S = Q K^T and dP = dO V^T into TMEM, the softmax warps form
-//             dS = P (dP - D) as bf16 over S, and dQ += dS K accumulates in TMEM.
+//   bwd_prep_kernel - -D_i and -lse_i*log2(e) per (batch, head, row) into workspace rows
+//             padded to whole 128-row tiles (padding: 0 and -inf, so padded rows contribute
+//             nothing); zeroes the key-tile work counter.
 //   bwd_dkdv_kernel - key-tile-major over (batch, KV head, key tile) items taken from an
 //             atomic counter (a prefix key tile is seen by every later query tile, a window
 //             key tile by about W/128 of them, so static striding would leave SMs idle): per
 //             (query head of the group, query tile), S^T = K Q^T and dP^T = V dO^T into
 //             TMEM, P^T and dS^T as bf16 over them, dV += P^T dO and dK += dS^T Q in TMEM
-//             across the whole group, so no atomics are needed.
+//             across the whole group, so no atomics are needed.  It also stores each dS^T
+//             tile (bf16) for the dQ pass.
+//   bwd_dq_kernel - dQ = scale * dS K over the plan: a GEMM reading the stored dS^T tiles as
+//             the MN-major A operand, so S and dP are formed only once.
 // Both big kernels use the forward's roles: warps 0-7 two softmax warpgroups (group g owns
 // columns [64g, 64g+64) of every TMEM lane), warps 8-9 TMA producers, warp 10 issues the
 // smem x smem products (and owns TMEM), warp 11 the TMEM x smem accumulations.
@@ -65,6 +65,8 @@ struct BwdArgs {
   const int32_t* off;  // query-tile-major plan: [nq + 1] offsets
   const int32_t* ent;  // [n][2] (k_tile, flag)
   int32_t* counter;    // key-tile work counter
+  __nv_bfloat16* ds;   // dS^T tiles [B * Hq * n_plan][16 query chunks][128 key rows][8]
+  int64_t n_plan;      // plan entries per (batch, head)
   __nv_bfloat16* dq;   // [B, S, Hq, D]
   __nv_bfloat16* dk;   // [B, S, Hkv, D]
   __nv_bfloat16* dv;
@@ -121,74 +123,76 @@ __device__ __forceinline__ uint64_t span_bits(int64_t lo, int64_t hi, int64_t ba
 }
 
 // ------------------------------------------------------------------ prep
+// Rows are taken in memory order (batch, row, head): 16 lanes read one 256-byte row of O
+// and of dO with 16-byte loads, so a warp covers two rows per step.  Padded rows (past seq)
+// get -D = 0 and -lse*log2(e) = -inf.
 __global__ void __launch_bounds__(kPrepThreads)
     bwd_prep_kernel(const __nv_bfloat16* __restrict__ out, const __nv_bfloat16* __restrict__ dout,
                     const float* __restrict__ lse, int64_t seq, int32_t hq, int64_t s_pad,
-                    int64_t n_rows, float* __restrict__ nl, float* __restrict__ nd,
+                    int64_t batch, float* __restrict__ nl, float* __restrict__ nd,
                     int32_t* __restrict__ counter) {
   pdl_trigger();
   pdl_wait();
-  if (blockIdx.x == 0 && threadIdx.x == 0) *counter = 0;
-  const int64_t row = static_cast<int64_t>(blockIdx.x) * (kPrepThreads / 32) + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (row >= n_rows) return;
-  const int64_t i = row % s_pad;
-  const int64_t bh = row / s_pad;
-  float dot = 0.f, l2 = -INFINITY;
-  if (i < seq) {
-    const int64_t h = bh % hq, b = bh / hq;
-    const int64_t base = ((b * seq + i) * hq + h) * kHeadDim + 4 * lane;
-    const uint2 o = *reinterpret_cast<const uint2*>(out + base);
-    const uint2 d = *reinterpret_cast<const uint2*>(dout + base);
-    const float2 o0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&o.x));
-    const float2 o1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&o.y));
-    const float2 d0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&d.x));
-    const float2 d1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&d.y));
-    dot = o0.x * d0.x + o0.y * d0.y + o1.x * d1.x + o1.y * d1.y;
+  const int64_t tid = (int64_t)blockIdx.x * kPrepThreads + threadIdx.x;
+  if (tid == 0) *counter = 0;
+  const int64_t real = batch * seq * hq;   // rows with data, (b, i, h) order
+  const int64_t half_warps = (int64_t)gridDim.x * kPrepThreads / 16;
+  const int sub = threadIdx.x & 15;
+  for (int64_t row = tid >> 4; row < real; row += half_warps) {
+    const uint4 o = reinterpret_cast<const uint4*>(out + row * kHeadDim)[sub];
+    const uint4 d = reinterpret_cast<const uint4*>(dout + row * kHeadDim)[sub];
+    const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(&o);
+    const __nv_bfloat162* d2 = reinterpret_cast<const __nv_bfloat162*>(&d);
+    float dot = 0.f;
 #pragma unroll
-    for (int sh = 16; sh > 0; sh >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, sh);
-    l2 = -lse[bh * seq + i] * kLog2e;
+    for (int e = 0; e < 4; ++e) {
+      const float2 x = __bfloat1622float2(o2[e]), y = __bfloat1622float2(d2[e]);
+      dot = fmaf(x.x, y.x, fmaf(x.y, y.y, dot));
+    }
+#pragma unroll
+    for (int sh = 8; sh > 0; sh >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, sh);
+    if (sub == 0) {
+      const int64_t h = row % hq, bi = row / hq;
+      const int64_t i = bi % seq, b = bi / seq;
+      const int64_t srow = (b * hq + h) * s_pad + i;
+      nd[srow] = -dot;
+      nl[srow] = -lse[(b * hq + h) * seq + i] * kLog2e;
+    }
   }
-  if (lane == 0) {
-    nl[row] = l2;
-    nd[row] = -dot;
+  // padding rows [seq, s_pad) of every (batch, head)
+  const int64_t pad = s_pad - seq;
+  for (int64_t k = tid; k < batch * hq * pad; k += (int64_t)gridDim.x * kPrepThreads) {
+    const int64_t bh = k / pad, i = seq + k % pad;
+    nd[bh * s_pad + i] = 0.f;
+    nl[bh * s_pad + i] = -INFINITY;
   }
 }
 
 // ------------------------------------------------------------------ dQ
-// TMEM: S0 [0,128), S1 [128,256), dP [256,384), dQ [384,512).
-constexpr uint32_t kQColDP = 256;
-constexpr uint32_t kQColDQ = 384;
-__device__ __forceinline__ uint32_t col_s(int s) { return s ? 128u : 0u; }
-constexpr size_t kDqSmem = 1024 + 6 * size_t(kTileBytes) + 256;
+// dQ_i = scale * sum over the planned key tiles of dS K, with dS stored by the key-tile kernel
+// (bf16 dS^T tiles, [key row][query col]): a plain GEMM over the plan, read as the MN-major A
+// operand.  Persistent over (batch, head, query tile) items, heaviest first; warp 4 streams
+// (dS tile, K tile) pairs through a 3-stage ring, warp 5 issues dQ[buf] += dS K into one of two
+// TMEM accumulators, warps 0-3 drain the finished accumulator (scale, bf16, one row each) while
+// the next item accumulates in the other.
+constexpr int kDqThreads = 192;
+constexpr int kDqStages = 3;
+constexpr size_t kDqSmem = 1024 + size_t(kDqStages) * 2 * kTileBytes + 256;
 
-__global__ void __launch_bounds__(kThreads, 1)
-    bwd_dq_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mdo,
-                  const __grid_constant__ CUtensorMap mk, const __grid_constant__ CUtensorMap mv,
-                  const BwdArgs a) {
+__global__ void __launch_bounds__(kDqThreads, 1)
+    bwd_dq_kernel(const __grid_constant__ CUtensorMap mk, const BwdArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  uint8_t* sQ = smem;
-  uint8_t* sDO = sQ + kTileBytes;
-  uint8_t* sK = sDO + kTileBytes;  // [2]
-  uint8_t* sV = sK + 2 * kTileBytes;  // [2]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + 2 * kTileBytes);
-  uint64_t* qdo_full = bars;
-  uint64_t* qdo_empty = bars + 1;
-  uint64_t* k_full = bars + 2;     // [2]
-  uint64_t* k_empty = bars + 4;    // [2]
-  uint64_t* v_full = bars + 6;     // [2]
-  uint64_t* v_empty = bars + 8;    // [2]
-  uint64_t* s_full = bars + 10;    // [2]
-  uint64_t* s_free = bars + 12;    // [2]: dQ MMA of the buffer's tile done
-  uint64_t* ds_ready = bars + 14;  // [2 buffers][2 groups]
-  uint64_t* dp_full = bars + 18;
-  uint64_t* dp_free = bars + 19;
-  uint64_t* dq_full = bars + 20;
-  uint64_t* dq_free = bars + 21;
-  uint64_t* mma_done = bars + 22;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 23);
+  uint8_t* sDS = smem;                              // [kDqStages] dS tiles (no swizzle)
+  uint8_t* sK = sDS + kDqStages * kTileBytes;       // [kDqStages] K tiles
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sK + kDqStages * kTileBytes);
+  uint64_t* full = bars;                        // [kDqStages]
+  uint64_t* empty = bars + kDqStages;           // [kDqStages]
+  uint64_t* acc_full = bars + 2 * kDqStages;    // [2]
+  uint64_t* acc_free = acc_full + 2;            // [2]
+  uint64_t* mma_done = acc_free + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
 
   const int64_t bh = (int64_t)a.batch * a.hq;
   const int64_t n_items = bh * a.nq;
@@ -202,91 +206,67 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    mbar_init(qdo_full, 1);
-    mbar_init(qdo_empty, 1);
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&k_full[s], 1);
-      mbar_init(&k_empty[s], 1);
-      mbar_init(&v_full[s], 1);
-      mbar_init(&v_empty[s], 1);
-      mbar_init(&s_full[s], 1);
-      mbar_init(&s_free[s], 1);
-      for (int g = 0; g < kGroups; ++g) mbar_init(&ds_ready[s * kGroups + g], 4);
+    for (int s = 0; s < kDqStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
     }
-    mbar_init(dp_full, 1);
-    mbar_init(dp_free, kSoftmaxWarps);
-    mbar_init(dq_full, 1);
-    mbar_init(dq_free, kSoftmaxWarps);
-    mbar_init(mma_done, 2);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&acc_full[s], 1);
+      mbar_init(&acc_free[s], 4);
+    }
+    mbar_init(mma_done, 1);
     fence_mbar_init();
   }
-  if (warp == kIssA) {
-    tmem_alloc(tmem_slot, kTmemCols);
+  if (warp == 5) {
+    tmem_alloc(tmem_slot, 256);
     tmem_relinquish();
   }
-  if (warp == kProdA && lane == 0) {
-    prefetch_tensormap(&mq);
-    prefetch_tensormap(&mdo);
-    prefetch_tensormap(&mk);
-    prefetch_tensormap(&mv);
-  }
+  if (warp == 4 && lane == 0) prefetch_tensormap(&mk);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  pdl_wait();  // plan and row statistics come from the kernels launched before
+  pdl_wait();  // the dS tiles come from the key-tile kernel launched just before
 
-  if (warp == kProdA || warp == kProdB) {
-    // warp 8: Q and dO of each item, then the K tiles of its plan; warp 9: the V tiles
+  if (warp == 4) {
     if (lane == 0) {
-      const bool is_k = (warp == kProdA);
-      const CUtensorMap* map = is_k ? &mk : &mv;
-      uint8_t* ring = is_k ? sK : sV;
-      uint64_t* full = is_k ? k_full : v_full;
-      uint64_t* empty = is_k ? k_empty : v_empty;
       int64_t g = 0;
-      int li = 0;
       bool alive = true;
-      for (int64_t it = blockIdx.x; alive && it < n_items; it += gridDim.x, ++li) {
+      for (int64_t it = blockIdx.x; alive && it < n_items; it += gridDim.x) {
         int qt, b, head;
         item_of(it, qt, b, head);
         const int kvh = head / a.group;
         const int e0 = a.off[qt];
         const int n = a.off[qt + 1] - e0;
-        if (is_k) {
-          if (li > 0 && !mbar_wait(qdo_empty, (li - 1) & 1, a.status)) {
-            alive = false;
-            break;
-          }
-          mbar_arrive_expect_tx(qdo_full, 2 * kTileBytes);
-          tma_load_4d(sQ, &mq, 0, head, qt * kT, b, qdo_full);
-          tma_load_4d(sQ + kBoxBytes, &mq, 64, head, qt * kT, b, qdo_full);
-          tma_load_4d(sDO, &mdo, 0, head, qt * kT, b, qdo_full);
-          tma_load_4d(sDO + kBoxBytes, &mdo, 64, head, qt * kT, b, qdo_full);
-        }
+        const int64_t tile0 = ((int64_t)b * a.hq + head) * a.n_plan + e0;
         for (int j = 0; j < n; ++j, ++g) {
-          const int s = static_cast<int>(g & 1);
-          if (g >= 2 && !mbar_wait(&empty[s], static_cast<uint32_t>(((g >> 1) - 1) & 1), a.status)) {
+          const int s = static_cast<int>(g % kDqStages);
+          if (g >= kDqStages &&
+              !mbar_wait(&empty[s], static_cast<uint32_t>(((g / kDqStages) - 1) & 1), a.status)) {
             alive = false;
             break;
           }
           const int kt = a.ent[2 * (e0 + j)];
-          uint8_t* dst = ring + s * kTileBytes;
-          mbar_arrive_expect_tx(&full[s], kTileBytes);
-          tma_load_4d(dst, map, 0, kvh, kt * kT, b, &full[s]);
-          tma_load_4d(dst + kBoxBytes, map, 64, kvh, kt * kT, b, &full[s]);
+          mbar_arrive_expect_tx(&full[s], 2 * kTileBytes);
+          uint8_t* ds = sDS + s * kTileBytes;
+          uint8_t* k = sK + s * kTileBytes;
+          bulk_load(ds, a.ds + (tile0 + j) * kT * kT, kTileBytes, &full[s]);
+          tma_load_4d(k, &mk, 0, kvh, kt * kT, b, &full[s]);
+          tma_load_4d(k + kBoxBytes, &mk, 64, kvh, kt * kT, b, &full[s]);
         }
       }
-      // every issued copy lands before the CTA may exit
-      for (int64_t j = (g > 2 ? g - 2 : 0); j < g; ++j)
-        mbar_wait(&full[j & 1], static_cast<uint32_t>((j >> 1) & 1), a.status);
-      if (is_k && li > 0) mbar_wait(qdo_full, (li - 1) & 1, a.status);
+      for (int64_t j = (g > kDqStages ? g - kDqStages : 0); j < g; ++j)
+        mbar_wait(&full[j % kDqStages], static_cast<uint32_t>((j / kDqStages) & 1), a.status);
     }
-  } else if (warp == kIssA) {
-    // S[buf] = Q K^T and dP = dO V^T
+  } else if (warp == 5) {
     if (lane == 0) {
-      const uint32_t q_addr = smem_u32(sQ), do_addr = smem_u32(sDO);
-      const uint32_t k_addr = smem_u32(sK), v_addr = smem_u32(sV);
+      // A = dS [128 query rows][128 keys], MN-major without swizzle: the stored tile is
+      // [query chunk][key row][8 bf16], i.e. core matrices of 8 queries x 8 keys (128 B),
+      // 2048 B apart along the queries (SBO) and 128 B apart along the keys (LBO); a 16-key
+      // step advances 256 B.  B = K [128 keys][128 dims], MN-major, 128-byte swizzle: 2048 B
+      // per 16-key step, 64-column halves 16 KB apart (LBO), 8-row groups 1024 B (SBO).
+      constexpr uint32_t idesc = umma_idesc_bf16(128, 128, true, true);
+      const uint32_t ds_addr = smem_u32(sDS), k_addr = smem_u32(sK);
       int64_t g = 0;
       int li = 0;
       bool ok = true;
@@ -294,169 +274,80 @@ __global__ void __launch_bounds__(kThreads, 1)
         int qt, b, head;
         item_of(it, qt, b, head);
         const int n = a.off[qt + 1] - a.off[qt];
-        if (!mbar_wait(qdo_full, li & 1, a.status)) {
+        const int ab = li & 1;
+        if (li >= 2 &&
+            !mbar_wait(&acc_free[ab], static_cast<uint32_t>(((li >> 1) - 1) & 1), a.status)) {
           ok = false;
           break;
         }
         for (int j = 0; j < n; ++j, ++g) {
-          const int s = static_cast<int>(g & 1);
-          const uint32_t ph = static_cast<uint32_t>((g >> 1) & 1);
-          if (!mbar_wait(&k_full[s], ph, a.status) ||
-              (g >= 2 && !mbar_wait(&s_free[s], ph ^ 1, a.status))) {
+          const int s = static_cast<int>(g % kDqStages);
+          if (!mbar_wait(&full[s], static_cast<uint32_t>((g / kDqStages) & 1), a.status)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          mma_kmajor(tmem + col_s(s), q_addr, k_addr + s * kTileBytes);
-          umma_commit(&s_full[s]);
-          if (!mbar_wait(&v_full[s], ph, a.status) ||
-              (g >= 1 && !mbar_wait(dp_free, static_cast<uint32_t>((g - 1) & 1), a.status))) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          mma_kmajor(tmem + kQColDP, do_addr, v_addr + s * kTileBytes);
-          umma_commit(dp_full);
-          umma_commit(&v_empty[s]);
-          if (j == n - 1) umma_commit(qdo_empty);
-        }
-      }
-      umma_commit(mma_done);
-      mbar_wait(mma_done, 0, a.status);
-    }
-  } else if (warp == kIssB) {
-    // dQ += dS K, group by group as each softmax group's dS lands
-    if (lane == 0) {
-      const uint32_t k_addr = smem_u32(sK);
-      int64_t g = 0;
-      int li = 0;
-      bool ok = true;
-      for (int64_t it = blockIdx.x; ok && it < n_items; it += gridDim.x, ++li) {
-        int qt, b, head;
-        item_of(it, qt, b, head);
-        const int n = a.off[qt + 1] - a.off[qt];
-        for (int j = 0; j < n; ++j, ++g) {
-          const int s = static_cast<int>(g & 1);
-          if (j == 0 && li > 0 && !mbar_wait(dq_free, (li - 1) & 1, a.status)) {
-            ok = false;
-            break;
-          }
+          const uint32_t da = ds_addr + s * kTileBytes, kb = k_addr + s * kTileBytes;
 #pragma unroll
-          for (int gr = 0; gr < kGroups; ++gr) {
-            if (!mbar_wait(&ds_ready[s * kGroups + gr], static_cast<uint32_t>((g >> 1) & 1),
-                           a.status)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            mma_tmem_a(tmem + kQColDQ, tmem + col_s(s), k_addr + s * kTileBytes, gr,
-                       j == 0 && gr == 0);
+          for (int kk = 0; kk < 8; ++kk) {
+            umma_ss(tmem + 128u * ab, umma_desc_noswz(da + kk * 256, 128, 2048),
+                    umma_desc_sw128(kb + kk * 2048, kBoxBytes, 1024), idesc,
+                    (j > 0 || kk > 0) ? 1u : 0u);
           }
-          if (!ok) break;
-          umma_commit(&k_empty[s]);
-          umma_commit(&s_free[s]);
+          umma_commit(&empty[s]);
         }
-        if (ok) umma_commit(dq_full);
+        if (!ok) break;
+        umma_commit(&acc_full[ab]);
       }
       umma_commit(mma_done);
       mbar_wait(mma_done, 0, a.status);
     }
   } else {
-    // softmax warpgroups: dS = P (dP - D) with P = 2^(s*scale*log2e - lse*log2e)
-    const int wg = threadIdx.x >> 7;
-    const int r = threadIdx.x & 127;
-    const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
-    const uint32_t cs0 = static_cast<uint32_t>(kCols * wg);
-    const uint64_t sl2x2 = pack_f32x2(a.scale_log2, a.scale_log2);
-    bool ok = true;
-    int64_t g = 0;
+    // epilogue warps: row r of the finished accumulator -> dQ (times the softmax scale)
+    const int r = threadIdx.x;
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
     int li = 0;
+    bool ok = true;
     for (int64_t it = blockIdx.x; it < n_items; it += gridDim.x, ++li) {
       int qt, b, head;
       item_of(it, qt, b, head);
-      const int e0 = a.off[qt];
-      const int n = a.off[qt + 1] - e0;
-      const int64_t row = (int64_t)qt * kT + r;
-      const int64_t srow = ((int64_t)b * a.hq + head) * a.s_pad + row;
-      const float nl = a.nl[srow], nd = a.nd[srow];
-      const uint64_t nl2 = pack_f32x2(nl, nl), nd2 = pack_f32x2(nd, nd);
-      int2 ent_next = n > 0 ? reinterpret_cast<const int2*>(a.ent)[e0] : make_int2(0, 0);
-      for (int j = 0; j < n; ++j, ++g) {
-        const int s = static_cast<int>(g & 1);
-        const int kt = ent_next.x;
-        const int flag = ent_next.y;
-        if (j + 1 < n) ent_next = reinterpret_cast<const int2*>(a.ent)[e0 + j + 1];
-        ok = ok && __all_sync(0xffffffffu, mbar_wait(&s_full[s], static_cast<uint32_t>((g >> 1) & 1),
-                                                      a.status));
-        if (!ok) continue;
-        tc_fence_after();
-        float x[kCols];
-        load64(lane_base + col_s(s) + cs0, x);
-        if (flag == PS_TILE_PARTIAL) {
-          const int64_t end = row + 1 < a.seq ? row + 1 : a.seq;
-          int64_t win_lo = row - a.w + 1;
-          if (win_lo < a.lp) win_lo = a.lp;
-          const int64_t k0 = (int64_t)kt * kT + cs0;
-          const uint64_t vis = span_bits(0, a.lp < end ? a.lp : end, k0) | span_bits(win_lo, end, k0);
-#pragma unroll
-          for (int i = 0; i < kCols; ++i)
-            if (!((vis >> i) & 1ull)) x[i] = -INFINITY;
-        }
-#pragma unroll
-        for (int i = 0; i < kCols / 2; ++i) {
-          const float2 e = unpack_f32x2(ffma2(pack_f32x2(x[2 * i], x[2 * i + 1]), sl2x2, nl2));
-          x[2 * i] = fast_exp2(e.x);
-          x[2 * i + 1] = fast_exp2(e.y);
-        }
-        ok = ok && __all_sync(0xffffffffu, mbar_wait(dp_full, static_cast<uint32_t>(g & 1), a.status));
-        if (!ok) continue;
-        tc_fence_after();
-        float dp[kCols];
-        load64(lane_base + kQColDP + cs0, dp);
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(dp_free);
-        uint32_t pk[kCols / 2];
-#pragma unroll
-        for (int i = 0; i < kCols / 2; ++i) {
-          const float2 d = unpack_f32x2(
-              fmul2(pack_f32x2(x[2 * i], x[2 * i + 1]), fadd2(pack_f32x2(dp[2 * i], dp[2 * i + 1]), nd2)));
-          pk[i] = cvt_bf16x2(d.x, d.y);
-        }
-        tmem_st32(lane_base + col_s(s) + cs0, pk);  // over this group's own columns
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&ds_ready[s * kGroups + wg]);
-      }
-      // epilogue: dQ = scale * accumulated dS K
-      const bool fin = __all_sync(0xffffffffu, ok && mbar_wait(dq_full, li & 1, a.status));
-      ok = ok && fin;
-      if (!fin) continue;
+      const int ab = li & 1;
+      ok = ok && __all_sync(0xffffffffu, mbar_wait(&acc_full[ab],
+                                                   static_cast<uint32_t>((li >> 1) & 1),
+                                                   a.status));
+      if (!ok) break;
       tc_fence_after();
-      float acc[kCols];
-      load64(lane_base + kQColDQ + cs0, acc);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(dq_free);
-      if (row < a.seq) {
-        uint4* dst = reinterpret_cast<uint4*>(a.dq + (((int64_t)b * a.seq + row) * a.hq + head) *
-                                                         kHeadDim + cs0);
+      const int64_t row = (int64_t)qt * kT + r;
+      __nv_bfloat16* dst = a.dq + (((int64_t)b * a.seq + row) * a.hq + head) * kHeadDim;
 #pragma unroll
-        for (int v = 0; v < kCols / 8; ++v) {
-          dst[v] = make_uint4(cvt_bf16x2(a.scale * acc[8 * v], a.scale * acc[8 * v + 1]),
-                              cvt_bf16x2(a.scale * acc[8 * v + 2], a.scale * acc[8 * v + 3]),
-                              cvt_bf16x2(a.scale * acc[8 * v + 4], a.scale * acc[8 * v + 5]),
-                              cvt_bf16x2(a.scale * acc[8 * v + 6], a.scale * acc[8 * v + 7]));
+      for (int c = 0; c < 4; ++c) {
+        uint32_t raw[32];
+        tmem_ld32(lane_base + 128u * ab + 32 * c, raw);
+        tmem_wait_ld();
+        if (c == 3) {
+          // the accumulator is in registers: the item after next may overwrite it
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&acc_free[ab]);
+        }
+        if (row < a.seq) {
+          uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * c);
+#pragma unroll
+          for (int v = 0; v < 4; ++v)
+            d4[v] = make_uint4(
+                cvt_bf16x2(a.scale * __uint_as_float(raw[8 * v]), a.scale * __uint_as_float(raw[8 * v + 1])),
+                cvt_bf16x2(a.scale * __uint_as_float(raw[8 * v + 2]), a.scale * __uint_as_float(raw[8 * v + 3])),
+                cvt_bf16x2(a.scale * __uint_as_float(raw[8 * v + 4]), a.scale * __uint_as_float(raw[8 * v + 5])),
+                cvt_bf16x2(a.scale * __uint_as_float(raw[8 * v + 6]), a.scale * __uint_as_float(raw[8 * v + 7])));
         }
       }
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == kIssA) {
+  if (warp == 5) {
     tc_fence_after();
-    tmem_dealloc(tmem, kTmemCols);
+    tmem_dealloc(tmem, 256);
   }
 }
 
@@ -784,6 +675,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = ok && __all_sync(0xffffffffu, mbar_wait(dp_full, ph, a.status));
         if (!ok) continue;
         tc_fence_after();
+        // this (query tile, key tile)'s dS^T tile in the store: its index in query tile qt's
+        // plan (ascending key tiles)
+        __nv_bfloat16* ds_row;
+        {
+          const int e0 = a.off[qt];
+          int lo = 0, hi = a.off[qt + 1] - e0 - 1;
+          while (lo < hi) {
+            const int mid = (lo + hi) >> 1;
+            if (a.ent[2 * (e0 + mid)] < m.kt) lo = mid + 1; else hi = mid;
+          }
+          const int h = m.kvh * a.group + j / m.nqt;
+          // tile layout: [16 column chunks of 8 query cols][128 key rows][8 bf16], so the
+          // 32 rows of a warp store 512 contiguous bytes per chunk
+          ds_row = a.ds + (((int64_t)m.b * a.hq + h) * a.n_plan + e0 + lo) * kT * kT + r * 8;
+        }
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
           uint32_t raw[32];
@@ -801,6 +707,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             dk[i] = cvt_bf16x2(v.x, v.y);
           }
           tmem_st16(lane_base + kKColDP + cs0 + 16 * c, dk);
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            const int chunk = (cs0 >> 3) + 4 * c + v;  // query cols [8 chunk, 8 chunk + 8)
+            *reinterpret_cast<uint4*>(ds_row + chunk * kT * 8) =
+                make_uint4(dk[4 * v], dk[4 * v + 1], dk[4 * v + 2], dk[4 * v + 3]);
+          }
         }
         tmem_wait_st();
         tc_fence_before();
@@ -848,16 +760,21 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// Workspace: [plan][-lse*log2e rows][-D rows][counter][dS^T tiles of every planned tile,
+// 32 KB each]
 struct BwdLayout {
-  size_t plan, stats, counter, total;
+  size_t plan, stats, counter, ds, total;
+  int64_t n_plan;
 };
 BwdLayout bwd_layout(int64_t batch, int32_t hq, int64_t seq, int32_t lp, int32_t w) {
   BwdLayout L;
-  L.plan = prefill_plan_bytes(seq, prefill_plan_tiles(seq, lp, w));
+  L.n_plan = prefill_plan_tiles(seq, lp, w);
+  L.plan = prefill_plan_bytes(seq, L.n_plan);
   const int64_t s_pad = (seq + kT - 1) / kT * kT;
   L.stats = align256(size_t(batch) * hq * s_pad * 4);
   L.counter = 256;
-  L.total = align256(L.plan) + 2 * L.stats + L.counter;
+  L.ds = size_t(batch) * hq * L.n_plan * kT * kT * 2;
+  L.total = align256(L.plan) + 2 * L.stats + L.counter + L.ds;
   return L;
 }
 
@@ -911,19 +828,23 @@ int launch_prefill_bwd(const PrefillBwdLaunch& l, cudaStream_t stream) {
   a.nl = nl;
   a.nd = nd;
   a.counter = reinterpret_cast<int32_t*>(ws + align256(L.plan) + 2 * L.stats);
+  a.ds = reinterpret_cast<__nv_bfloat16*>(ws + align256(L.plan) + 2 * L.stats + L.counter);
+  a.n_plan = L.n_plan;
   a.dq = static_cast<__nv_bfloat16*>(l.dq);
   a.dk = static_cast<__nv_bfloat16*>(l.dk);
   a.dv = static_cast<__nv_bfloat16*>(l.dv);
 
-  const int64_t n_rows = l.batch * l.hq * s_pad;
-  const int rows_per_block = kPrepThreads / 32;
-  const int64_t prep_blocks = (n_rows + rows_per_block - 1) / rows_per_block;
-  if (prep_blocks > 0x7fffffffLL) return fail(PS_ERR_UNSUPPORTED, "prefill backward too large");
+  // row statistics: a grid of a few waves of the SMs, each half-warp striding over rows
+  const int64_t sms = sm_count();
+  const int64_t real_rows = l.batch * l.seq * l.hq;
+  int64_t prep_blocks = (real_rows * 16 + kPrepThreads - 1) / kPrepThreads;
+  if (prep_blocks > sms * 16) prep_blocks = sms * 16;
+  if (prep_blocks < 1) prep_blocks = 1;
   rc = check_cuda(launch_pdl(bwd_prep_kernel, dim3(static_cast<unsigned>(prep_blocks)),
                              dim3(kPrepThreads), 0, stream,
                              static_cast<const __nv_bfloat16*>(l.out),
                              static_cast<const __nv_bfloat16*>(l.dout), l.lse, l.seq, l.hq, s_pad,
-                             n_rows, nl, nd, a.counter),
+                             l.batch, nl, nd, a.counter),
                   "bwd_prep_kernel launch");
   if (rc != PS_OK) return rc;
 
@@ -935,24 +856,26 @@ int launch_prefill_bwd(const PrefillBwdLaunch& l, cudaStream_t stream) {
       !make_map_4d(&mk, l.k, dk_dims, box) || !make_map_4d(&mv, l.v, dk_dims, box))
     return PS_ERR_CUDA;
 
+
   static bool dq_attr[64] = {false}, kv_attr[64] = {false};
   if (!set_smem(reinterpret_cast<const void*>(bwd_dq_kernel), kDqSmem, dq_attr,
                 "cudaFuncSetAttribute(bwd_dq_kernel)", &rc) ||
       !set_smem(reinterpret_cast<const void*>(bwd_dkdv_kernel), kDkdvSmem, kv_attr,
                 "cudaFuncSetAttribute(bwd_dkdv_kernel)", &rc))
     return rc;
-  const int64_t sms = sm_count();
   const int64_t q_items = l.batch * l.hq * nq;
   const int64_t kv_items = l.batch * l.hkv * nq;
   if (q_items > 0x7fffffffLL) return fail(PS_ERR_UNSUPPORTED, "prefill backward too large");
-  rc = check_cuda(launch_pdl(bwd_dq_kernel, dim3(static_cast<unsigned>(q_items < sms ? q_items : sms)),
-                             dim3(kThreads), kDqSmem, stream, mq, mdo, mk, mv, a),
-                  "bwd_dq_kernel launch");
-  if (rc != PS_OK) return rc;
-  return check_cuda(
+  // dK, dV (and the dS^T tiles) first, then dQ from the stored tiles
+  rc = check_cuda(
       launch_pdl(bwd_dkdv_kernel, dim3(static_cast<unsigned>(kv_items < sms ? kv_items : sms)),
                  dim3(kThreads), kDkdvSmem, stream, mq, mdo, mk, mv, a),
       "bwd_dkdv_kernel launch");
+  if (rc != PS_OK) return rc;
+  return check_cuda(
+      launch_pdl(bwd_dq_kernel, dim3(static_cast<unsigned>(q_items < sms ? q_items : sms)),
+                 dim3(kDqThreads), kDqSmem, stream, mk, a),
+      "bwd_dq_kernel launch");
 }
 
 }  // namespace ps
