@@ -641,6 +641,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t ph = static_cast<uint32_t>(g & 1);
         const int qt = m.qlo + j % m.nqt;
         const int flag = classify_tile(qt, m.kt, a.seq, a.lp, a.w, kT, kT);
+        // this (query tile, key tile)'s dS^T tile in the store: its index in query tile qt's
+        // plan (ascending key tiles), looked up before the scores are waited for
+        __nv_bfloat16* ds_row;
+        {
+          const int e0 = a.off[qt];
+          int lo = 0, hi = a.off[qt + 1] - e0 - 1;
+          while (lo < hi) {
+            const int mid = (lo + hi) >> 1;
+            if (a.ent[2 * (e0 + mid)] < m.kt) lo = mid + 1; else hi = mid;
+          }
+          const int h = m.kvh * a.group + j / m.nqt;
+          // tile layout: [16 column chunks of 8 query cols][128 key rows][8 bf16], so the
+          // 32 rows of a warp store 512 contiguous bytes per chunk
+          ds_row = a.ds + (((int64_t)m.b * a.hq + h) * a.n_plan + e0 + lo) * kT * kT + r * 8;
+        }
         ok = ok && __all_sync(0xffffffffu,
                               mbar_wait(s_full, ph, a.status) &&
                                   mbar_wait(&st_full[st], static_cast<uint32_t>((g >> 1) & 1),
@@ -655,17 +670,22 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int i = 0; i < kCols; ++i)
             if (!((vis >> i) & 1ull)) x[i] = -INFINITY;
         }
-        const float2* nl = reinterpret_cast<const float2*>(sNL + st * kT + cs0);
-        const float2* nd = reinterpret_cast<const float2*>(sND + st * kT + cs0);
+        const float4* nl = reinterpret_cast<const float4*>(sNL + st * kT + cs0);
+        const float4* nd4 = reinterpret_cast<const float4*>(sND + st * kT + cs0);
         uint32_t pk[kCols / 2];
 #pragma unroll
-        for (int i = 0; i < kCols / 2; ++i) {
-          const float2 l = nl[i];
-          const float2 e =
-              unpack_f32x2(ffma2(pack_f32x2(x[2 * i], x[2 * i + 1]), sl2x2, pack_f32x2(l.x, l.y)));
-          x[2 * i] = fast_exp2(e.x);
-          x[2 * i + 1] = fast_exp2(e.y);
-          pk[i] = cvt_bf16x2(x[2 * i], x[2 * i + 1]);
+        for (int i = 0; i < kCols / 4; ++i) {
+          const float4 l = nl[i];
+          const float2 e0 = unpack_f32x2(
+              ffma2(pack_f32x2(x[4 * i], x[4 * i + 1]), sl2x2, pack_f32x2(l.x, l.y)));
+          const float2 e1 = unpack_f32x2(
+              ffma2(pack_f32x2(x[4 * i + 2], x[4 * i + 3]), sl2x2, pack_f32x2(l.z, l.w)));
+          x[4 * i] = fast_exp2(e0.x);
+          x[4 * i + 1] = fast_exp2(e0.y);
+          x[4 * i + 2] = fast_exp2(e1.x);
+          x[4 * i + 3] = fast_exp2(e1.y);
+          pk[2 * i] = cvt_bf16x2(x[4 * i], x[4 * i + 1]);
+          pk[2 * i + 1] = cvt_bf16x2(x[4 * i + 2], x[4 * i + 3]);
         }
         tmem_st32(lane_base + kKColS + cs0, pk);  // over this group's own columns
         tmem_wait_st();
@@ -675,21 +695,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = ok && __all_sync(0xffffffffu, mbar_wait(dp_full, ph, a.status));
         if (!ok) continue;
         tc_fence_after();
-        // this (query tile, key tile)'s dS^T tile in the store: its index in query tile qt's
-        // plan (ascending key tiles)
-        __nv_bfloat16* ds_row;
-        {
-          const int e0 = a.off[qt];
-          int lo = 0, hi = a.off[qt + 1] - e0 - 1;
-          while (lo < hi) {
-            const int mid = (lo + hi) >> 1;
-            if (a.ent[2 * (e0 + mid)] < m.kt) lo = mid + 1; else hi = mid;
-          }
-          const int h = m.kvh * a.group + j / m.nqt;
-          // tile layout: [16 column chunks of 8 query cols][128 key rows][8 bf16], so the
-          // 32 rows of a warp store 512 contiguous bytes per chunk
-          ds_row = a.ds + (((int64_t)m.b * a.hq + h) * a.n_plan + e0 + lo) * kT * kT + r * 8;
-        }
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
           uint32_t raw[32];
@@ -697,14 +702,20 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_wait_ld();
           uint32_t dk[16];
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const int e = 32 * c + 2 * i;
-            const float2 d = nd[e / 2];
-            const float2 v = unpack_f32x2(
+          for (int i = 0; i < 8; ++i) {
+            const int e = 32 * c + 4 * i;
+            const float4 d = nd4[e / 4];
+            const float2 v0 = unpack_f32x2(
                 fmul2(pack_f32x2(x[e], x[e + 1]),
-                      fadd2(pack_f32x2(__uint_as_float(raw[2 * i]), __uint_as_float(raw[2 * i + 1])),
+                      fadd2(pack_f32x2(__uint_as_float(raw[4 * i]), __uint_as_float(raw[4 * i + 1])),
                             pack_f32x2(d.x, d.y))));
-            dk[i] = cvt_bf16x2(v.x, v.y);
+            const float2 v1 = unpack_f32x2(
+                fmul2(pack_f32x2(x[e + 2], x[e + 3]),
+                      fadd2(pack_f32x2(__uint_as_float(raw[4 * i + 2]),
+                                       __uint_as_float(raw[4 * i + 3])),
+                            pack_f32x2(d.z, d.w))));
+            dk[2 * i] = cvt_bf16x2(v0.x, v0.y);
+            dk[2 * i + 1] = cvt_bf16x2(v1.x, v1.y);
           }
           tmem_st16(lane_base + kKColDP + cs0 + 16 * c, dk);
 #pragma unroll
