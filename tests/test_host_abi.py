@@ -156,3 +156,57 @@ def test_prefill_bwd_host_validation(lib):
     assert f(ctypes.byref(p), *ok, 16, 4, 0, 16, 16, 16, 256, need, None, None) == \
         B.PS_ERR_INVALID_ARG                                          # seq < 1
     assert f(ctypes.byref(p), *ok, 16, 0, 8192, 16, 16, 16, None, 0, None, None) == B.PS_OK
+
+
+def test_shared_prefix_host_validation(lib):
+    p = _params(l_prefix=2000, window=4096)
+    need = B.ps_decode_shared_prefix_workspace_bytes(p, 256, 64)
+    # prefix partials alone: >= one fp32 o + lse per (sequence, head)
+    assert need >= 256 * 16 * (128 + 1) * 4
+    assert B.ps_decode_shared_prefix_workspace_bytes(p, 256, 60) == 0   # not a multiple
+    assert B.ps_decode_shared_prefix_workspace_bytes(p, 256, 0) == 0
+    assert B.ps_decode_shared_prefix_workspace_bytes(_params(l_prefix=0), 256, 64) == 0
+    f = lib.ps_decode_attn_shared_prefix
+    cache = B.PsKVCache(16, 16, 16, 16, 256)
+    args = lambda gs, ws=256, wsb=need, prm=p: (ctypes.byref(prm), ctypes.byref(cache), gs,  # noqa: E731
+                                                 16, 16, 16, None, ws, wsb, None, None)
+    assert f(*args(60)) == B.PS_ERR_INVALID_ARG          # batch not a multiple of the group
+    assert f(*args(0)) == B.PS_ERR_INVALID_ARG
+    assert f(*args(64, prm=_params(l_prefix=0, window=4096))) == B.PS_ERR_INVALID_ARG
+    assert f(*args(64, wsb=need - 1)) == B.PS_ERR_WORKSPACE
+    assert f(*args(64, ws=272)) == B.PS_ERR_INVALID_ARG  # workspace not 256-aligned
+    assert f(*args(64, prm=_params(n_q_heads=32, n_kv_heads=2))) == B.PS_ERR_UNSUPPORTED
+
+
+def test_reset_pe_host_validation(lib):
+    p = _params()
+    f = lib.ps_decode_attn_reset_pe
+    cache = B.PsKVCache(16, 16, 16, 16, 4)
+    assert f(ctypes.byref(p), ctypes.byref(cache), 16, None, 16, None, None, 0, None,
+             None) == B.PS_ERR_INVALID_ARG                      # pos NULL
+    assert f(ctypes.byref(p), ctypes.byref(cache), 16, 12, 16, None, None, 0, None,
+             None) == B.PS_ERR_INVALID_ARG                      # pos not 8-byte aligned
+    empty = B.PsKVCache(None, None, None, None, 0)
+    assert f(ctypes.byref(p), ctypes.byref(empty), 16, 16, 16, None, None, 0, None,
+             None) == B.PS_OK                                   # batch 0: nothing to do
+
+
+def test_pin_host_validation(lib):
+    p = _params(l_prefix=100, window=512)
+    cache = B.PsKVCache(16, 16, 16, 16, 4)
+    f = lib.ps_kv_pin
+    ok = dict(cnt=16, pp=16, t0=16, t1=16, pos=16)
+    call = lambda cap, **kw: f(ctypes.byref(p), ctypes.byref(cache), cap,  # noqa: E731
+                               *[kw.get(k, v) for k, v in ok.items()], None, None)
+    assert call(100) == B.PS_ERR_INVALID_ARG     # capacity must exceed l_prefix
+    assert call(200, cnt=None) == B.PS_ERR_INVALID_ARG
+    assert call(200, pp=12) == B.PS_ERR_INVALID_ARG   # pin positions not 8-byte aligned
+    assert call(200, cnt=18) == B.PS_ERR_INVALID_ARG  # counts not 4-byte aligned
+    assert B.ps_decode_pinned_workspace_bytes(p, 64, 99) == 0
+    assert B.ps_decode_pinned_workspace_bytes(p, 64, 1124) >= \
+        B.ps_decode_pinned_workspace_bytes(p, 64, 100)
+    g = lib.ps_decode_attn_pinned
+    assert g(ctypes.byref(p), ctypes.byref(cache), 100, 16, 16, 16, 16, 16, None, None, 0,
+             None, None) == B.PS_ERR_INVALID_ARG    # capacity must exceed l_prefix
+    assert g(ctypes.byref(p), ctypes.byref(cache), 200, None, 16, 16, 16, 16, None, None, 0,
+             None, None) == B.PS_ERR_INVALID_ARG
