@@ -237,6 +237,11 @@ class DecodeWorkload:
         self.B.ps_decode_attn(self.params, self.cache.struct, self.q[i], self.pos[i], self.out[i],
                               None, self.ws, self.status)
 
+    def step(self, i):
+        """One decode step through the single-call API (append at pos, then decode)."""
+        self.B.ps_decode_step(self.params, self.cache.struct, self.k_new[i], self.v_new[i],
+                              self.q[i], self.pos[i], self.out[i], None, self.ws, self.status)
+
     def algorithmic_bytes_per_decode(self) -> int:
         """K+V of every visible key plus q and out: 1024 B per visible token per sequence
         (2 KV heads x 128 x 2 B x 2) + 2 x Hq x D x 2 B."""
@@ -254,8 +259,7 @@ def run_decode(args, world, rank, dev):
     stream = torch.cuda.current_stream()
 
     def step(i):
-        work.append(i)
-        work.decode(i)
+        work.step(i)
 
     for i in range(W):
         step(i)
@@ -335,7 +339,7 @@ def run_decode(args, world, rank, dev):
                    "n_q_heads": wl.n_q_heads, "n_kv_heads": wl.n_kv_heads, "head_dim": D,
                    "l_prefix": wl.l_prefix, "window": wl.window,
                    "positions": f"U[{wl.pos_lo},{wl.pos_hi}]", "layers": 1,
-                   "step": "ps_kv_append_rope + ps_decode_attn",
+                   "step": "ps_decode_step (append with Continue-PE RoPE + decode)",
                    "launch": "CUDA graph of the timed steps" if graph is not None else "eager",
                    "l2": "inputs larger than L2 (275 MB of K/V read per step vs 126 MB L2)",
                    "parallelism": f"dp{world} (independent sequences, no collective)"},
@@ -350,30 +354,38 @@ def run_decode(args, world, rank, dev):
 
 def run_decode_e2e(work: DecodeWorkload, K: int, W: int, world: int):
     """Same metric through the C ABI with host buffers: every step copies its inputs
-    (q, k_new, v_new, pos) host->device from pinned memory and reads out device->host."""
+    (q, k_new, v_new, pos: packed in one pinned host buffer, so one DMA) host->device and
+    reads out device->host, in stream order: step i+1's inputs are copied after step i's
+    output has been read back, as a decode loop whose next inputs depend on it would."""
     B = work.B
     dev = work.dev
-    stream = torch.cuda.current_stream()
     n = K + W
-    h_k = work.k_new.cpu().pin_memory()
-    h_v = work.v_new.cpu().pin_memory()
-    h_q = work.q_raw.cpu().pin_memory()
-    h_pos = work.pos.cpu().pin_memory()
+    parts = [("k", work.k_new[0]), ("v", work.v_new[0]), ("q", work.q[0]), ("pos", work.pos[0])]
+    offs, size = {}, 0
+    for name, t in parts:
+        offs[name] = size
+        size += (t.numel() * t.element_size() + 255) // 256 * 256
+    h_in = torch.empty((n, size), dtype=torch.uint8).pin_memory()
+    for i in range(n):
+        for name, src in (("k", work.k_new[i]), ("v", work.v_new[i]), ("q", work.q_raw[i]),
+                          ("pos", work.pos[i])):
+            nb = src.numel() * src.element_size()
+            h_in[i, offs[name]:offs[name] + nb].copy_(src.cpu().contiguous().view(-1).view(torch.uint8))
+    d_in = torch.empty((size,), dtype=torch.uint8, device=dev)
+
+    def view(name, like):
+        nb = like.numel() * like.element_size()
+        return d_in[offs[name]:offs[name] + nb].view(like.dtype).view(like.shape)
+    d_k, d_v = view("k", work.k_new[0]), view("v", work.v_new[0])
+    d_q, d_pos = view("q", work.q[0]), view("pos", work.pos[0])
     h_out = torch.empty((n,) + tuple(work.out.shape[1:]), dtype=torch.bfloat16).pin_memory()
-    d_k = torch.empty_like(work.k_new[0])
-    d_v = torch.empty_like(work.v_new[0])
-    d_q = torch.empty_like(work.q[0])
-    d_pos = torch.empty_like(work.pos[0])
     d_out = torch.empty_like(work.out[0])
+    stream = torch.cuda.current_stream()
 
     def step(i):
-        d_k.copy_(h_k[i], non_blocking=True)
-        d_v.copy_(h_v[i], non_blocking=True)
-        d_q.copy_(h_q[i], non_blocking=True)
-        d_pos.copy_(h_pos[i], non_blocking=True)
-        B.ps_kv_append_rope(work.params, work.cache.struct, d_k, d_v, d_q, d_pos, 1, work.status)
-        B.ps_decode_attn(work.params, work.cache.struct, d_q, d_pos, d_out, None, work.ws,
-                         work.status)
+        d_in.copy_(h_in[i], non_blocking=True)
+        B.ps_decode_step(work.params, work.cache.struct, d_k, d_v, d_q, d_pos, d_out, None,
+                         work.ws, work.status)
         h_out[i].copy_(d_out, non_blocking=True)
 
     for i in range(W):
@@ -391,7 +403,7 @@ def run_decode_e2e(work: DecodeWorkload, K: int, W: int, world: int):
     bi = (d_k.numel() + d_v.numel() + d_q.numel()) * 2 + d_pos.numel() * 8
     bo = d_out.numel() * 2
     return {"value": round(tokens / (ms / 1e3), 1), "unit": UNIT, "h2d_bytes_per_step": bi,
-            "d2h_bytes_per_step": bo}
+            "d2h_bytes_per_step": bo, "h2d_copies_per_step": 1, "d2h_copies_per_step": 1}
 
 
 # ------------------------------------------------------------- prefill leg

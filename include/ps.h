@@ -128,6 +128,20 @@ int ps_decode_attn(const ps_params* params, const ps_kv_cache* cache, const void
                    const int64_t* pos, void* out, float* lse, void* workspace, size_t ws_bytes,
                    int32_t* dev_status, ps_stream_t stream);
 
+/* One whole decode step: ps_kv_append_rope of one token per sequence at pos[b] (q rotated
+ * in place), then ps_decode_attn at the same pos.  Source: §核心机制 and §位置编码 (append
+ * with Continue PE, then attend the visible keys).  Results equal the two calls made one
+ * after the other; because the library knows the append wrote exactly the newest row of
+ * every sequence, the decode streams every other key tile while the append is still
+ * running and waits for it only before that row and q.
+ *   k_new, v_new : device bf16 [batch, Hkv, D], raw keys and values of the new token.
+ *   q_inout      : device bf16 [batch, Hq, D], raw query; rotated at pos in place.
+ * Other arguments, errors and the workspace (ps_decode_workspace_bytes) as ps_decode_attn;
+ * a linear cache (ring NULL) is not accepted. */
+int ps_decode_step(const ps_params* params, const ps_kv_cache* cache, const void* k_new,
+                   const void* v_new, void* q_inout, const int64_t* pos, void* out, float* lse,
+                   void* workspace, size_t ws_bytes, int32_t* dev_status, ps_stream_t stream);
+
 /* One decode step under Reset PE, from the same Continue-PE cache ps_kv_append_rope fills.
  * Source: §位置编码 of "Prefix Sliding 完全拆解": Reset PE renumbers the window so that it
  * directly follows the prefix (the first window token gets id L_prefix, the next

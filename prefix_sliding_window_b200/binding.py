@@ -82,6 +82,9 @@ _SIGS = {
                                          c_int64, c_void_p, c_void_p, c_void_p, c_int64,
                                          POINTER(c_int64), c_void_p, c_size_t, c_void_p,
                                          c_void_p]),
+    "ps_decode_step": (c_int32, [POINTER(PsParams), POINTER(PsKVCache), c_void_p, c_void_p,
+                                 c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_size_t,
+                                 c_void_p, c_void_p]),
     "ps_decode_attn_reset_pe": (c_int32, [POINTER(PsParams), POINTER(PsKVCache), c_void_p,
                                           c_void_p, c_void_p, c_void_p, c_void_p, c_size_t,
                                           c_void_p, c_void_p]),
@@ -185,6 +188,16 @@ def ps_decode_attn(params: PsParams, cache: PsKVCache, q, pos, out, lse=None, wo
                                _ptr(out), _ptr(lse), _ptr(workspace), ws_bytes, _ptr(dev_status),
                                _stream(stream))
     _check(rc, "ps_decode_attn")
+
+
+def ps_decode_step(params: PsParams, cache: PsKVCache, k_new, v_new, q_inout, pos, out,
+                   lse=None, workspace=None, dev_status=None, stream=None) -> None:
+    """Append one token per sequence at pos (q rotated in place), then decode at pos."""
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rc = load().ps_decode_step(ctypes.byref(params), ctypes.byref(cache), _ptr(k_new),
+                               _ptr(v_new), _ptr(q_inout), _ptr(pos), _ptr(out), _ptr(lse),
+                               _ptr(workspace), ws_bytes, _ptr(dev_status), _stream(stream))
+    _check(rc, "ps_decode_step")
 
 
 def ps_decode_attn_reset_pe(params: PsParams, cache: PsKVCache, q, pos, out, lse=None,

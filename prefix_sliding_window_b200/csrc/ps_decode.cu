@@ -77,6 +77,10 @@ struct DecodeArgs {
   // Reset PE: prefix tiles use the query rotated by delta = L_prefix + |window| - 1 - p
   // more (its Reset-PE id); inv_freq = theta^(-2i/D) in float64
   int32_t reset_pe;
+  // launched right after a one-token append at pos (ps_decode_step): only the tile holding
+  // each sequence's newest row and the rotated q depend on that kernel, so everything else
+  // may stream before the programmatic wait
+  int32_t after_append;
   double inv_freq[kHeadDim / 2];
   // tokens appended to the pinned prefix: rows [L_prefix, L_prefix + pin_count[b]) of the
   // prefix store hold the promoted positions pin_pos[b][0..) (ascending)
@@ -235,7 +239,7 @@ __global__ void __launch_bounds__(kThreads)
   }
   // launched with programmatic serialization: everything above overlapped the previous
   // kernel (usually the append); positions, q and the cache are read only after this
-  pdl_wait();
+  if (!a.after_append) pdl_wait();
   pdl_trigger();  // the merge may be scheduled now; it waits for this grid to finish
 
   // ---------------------------------------------------------------- work range
@@ -304,6 +308,7 @@ __global__ void __launch_bounds__(kThreads)
     if (lane == 0 && ntiles > 0) {
       const uint64_t pol = l2_policy_evict_first();
       int issued = 0;
+      bool waited = !a.after_append;
       TileWalker pw = wk;
       for (int i = 0; i < ntiles; ++i, ++pw.t) {
         if (pw.t >= pw.pu1) pw.next_unit(a, pref);
@@ -311,6 +316,16 @@ __global__ void __launch_bounds__(kThreads)
         const uint32_t ph = (i / STAGES) & 1;
         if (i >= STAGES && !mbar_wait(&empty[s], ph ^ 1, a.status)) break;
         const DecodeTile d = tiling_tile(pw.tiling, static_cast<int32_t>(pw.t - pw.pu));
+        if (!waited) {
+          // the newest row of sequence b: prefix row p, or ring slot (p - Lp) mod W
+          const int64_t p = a.pos[pw.b];
+          const bool pre = a.full_mode || p < a.lp;
+          const int64_t row = pre ? p : (p - a.lp) % a.w;
+          if (d.map_id == (pre ? 0 : 1) && row >= d.row0 + d.lo && row < d.row0 + d.hi) {
+            pdl_wait();
+            waited = true;
+          }
+        }
         const CUtensorMap* mk = d.map_id ? &mk1 : &mk0;
         const CUtensorMap* mv = d.map_id ? &mv1 : &mv0;
         const int unit = pw.b * a.hkv + pw.h;
@@ -474,6 +489,7 @@ __global__ void __launch_bounds__(kThreads)
         }
       }
     };
+    if (a.after_append) pdl_wait();  // q is rotated by the append just before
     if (ntiles > 0) {
       load_q(cw.b, cw.h);
       if (a.reset_pe) rotate_prefix_q(a.pos[cw.b]);
@@ -793,6 +809,7 @@ int launch_decode(const DecodeLaunch& l, cudaStream_t stream) {
   a.scale_log2 = l.scale * kLog2e;
   a.skip_prefix = l.skip_prefix;
   a.reset_pe = l.reset_pe;
+  a.after_append = l.after_append;
   a.pin_count = l.pin_count;
   a.pin_pos = l.pin_pos;
   a.pin_cap = (l.lcap > l.lp) ? l.lcap - l.lp : 0;

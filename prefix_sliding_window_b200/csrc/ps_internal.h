@@ -123,6 +123,8 @@ struct DecodeLaunch {
   int32_t lcap;
   const int32_t* pin_count;
   const int64_t* pin_pos;
+  // the previous kernel on the stream is the one-token append at pos (ps_decode_step)
+  int32_t after_append;
 };
 // Split count and workspace bytes for a decode of this shape on the current device.
 int decode_splits(int64_t batch, int32_t hkv, int64_t max_keys);

@@ -409,3 +409,47 @@ def test_prefix_sliding_equals_full_attention_in_warmup(cuda_device):
                        ws)
     torch.cuda.synchronize()
     assert_close(f64(o1), f64(o2), "warm-up PS vs full")
+
+
+@pytest.mark.parametrize("Bn,lp,w,lo,hi", [(64, 100, 4096, 8192, 131072),   # stream-K
+                                         (160, 100, 256, 0, 4000),         # one CTA per unit
+                                         (5, 300, 64, 0, 400)])            # prompt / warm-up
+def test_decode_step_equals_append_then_decode(cuda_device, Bn, lp, w, lo, hi):
+    """ps_decode_step (the decode streams before the append finishes, except the newest row)
+    is bit-identical to ps_kv_append_rope followed by ps_decode_attn."""
+    dev = cuda_device
+    hq, hkv = 16, 2
+    params = B.make_params(hq, hkv, D, lp, w, THETA)
+    pos = synth.uniform_positions(Bn, lo, hi, seed=77, device=dev)
+    if Bn == 5:
+        pos[0] = -3  # a bad position: both paths flag it and write zeros
+    caches = []
+    for _ in range(2):
+        c = PrefixSlidingCache(Bn, hkv, lp, w, D, dev, fill=None)
+        if lp:
+            c.k_prefix.copy_(synth.normal_bf16(c.k_prefix.shape, 78, dev))
+            c.v_prefix.copy_(synth.normal_bf16(c.v_prefix.shape, 79, dev))
+        c.k_ring.copy_(synth.normal_bf16(c.k_ring.shape, 80, dev))
+        c.v_ring.copy_(synth.normal_bf16(c.v_ring.shape, 81, dev))
+        caches.append(c)
+    k_new = synth.normal_bf16((Bn, 1, hkv, D), 82, dev)
+    v_new = synth.normal_bf16((Bn, 1, hkv, D), 83, dev)
+    q_raw = synth.normal_bf16((Bn, hq, D), 84, dev)
+    ws = torch.empty(max(1, B.ps_decode_workspace_bytes(params, Bn)), dtype=torch.uint8, device=dev)
+    outs = []
+    for i, c in enumerate(caches):
+        q = q_raw.clone()
+        out = torch.full((Bn, hq, D), float("nan"), dtype=torch.bfloat16, device=dev)
+        lse = torch.full((Bn, hq), float("nan"), dtype=torch.float32, device=dev)
+        st = torch.zeros(1, dtype=torch.int32, device=dev)
+        if i == 0:
+            B.ps_kv_append_rope(params, c.struct, k_new, v_new, q.view(Bn, 1, hq, D), pos, 1, st)
+            B.ps_decode_attn(params, c.struct, q, pos, out, lse, ws, st)
+        else:
+            B.ps_decode_step(params, c.struct, k_new, v_new, q, pos, out, lse, ws, st)
+        torch.cuda.synchronize()
+        outs.append((q, out, lse, st.item()))
+    (qa, oa, la, sa), (qb, ob, lb, sb) = outs
+    assert sa == sb
+    assert torch.equal(qa, qb) and torch.equal(oa, ob) and torch.equal(la, lb)
+    assert torch.equal(caches[0].k_ring, caches[1].k_ring)
