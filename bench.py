@@ -562,8 +562,8 @@ def run_full_attention(work: DecodeWorkload, steps: int = 16, warmup: int = 3):
 # ------------------------------------------------------------- latency leg
 def run_latency(dev, steps: int = 256, warmup: int = 8):
     """Single-sequence decode latency: batch 1, 16/2/128, L_prefix 100, W 512, positions past
-    the point where the window slides (612); one step = append + decode, replayed as a CUDA
-    graph and also launched eagerly."""
+    the point where the window slides (612); one step = ps_decode_step (append + decode),
+    replayed as a CUDA graph and also launched eagerly."""
     wl = synth.WORKLOADS["decode_b1_w512"]
     import dataclasses
     wl = dataclasses.replace(wl, pos_lo=2047 - steps - warmup, pos_hi=2047 - steps - warmup)
@@ -572,8 +572,7 @@ def run_latency(dev, steps: int = 256, warmup: int = 8):
     stream = torch.cuda.current_stream()
 
     def step(i):
-        work.append(i)
-        work.decode(i)
+        work.step(i)
 
     for i in range(warmup):
         step(i)
