@@ -909,6 +909,80 @@ def run_pin(dev, steps: int = 20, warmup: int = 3, n_pin: int = 1024):
             **res}
 
 
+def run_paged(dev, steps: int = 20, warmup: int = 3):
+    """Paged store: the batch-64 decode workload (16/2/128, L_prefix 100, W 4096, positions
+    U[8192, 131072]) held in a pool of 64-row blocks scattered in a seeded random order,
+    each sequence's block table listing its prefix blocks then its W/64 ring blocks.  Paged
+    decode is timed beside the contiguous store's decode of the same batch, and one step
+    (append of the new token into its block + decode) on its own."""
+    from prefix_sliding_window_b200 import binding as B
+    from prefix_sliding_window_b200.cache import PrefixSlidingCache
+    wl = synth.WORKLOADS[WORKLOAD]
+    Bn, hq, hkv, lp, w = wl.batch, wl.n_q_heads, wl.n_kv_heads, wl.l_prefix, wl.window
+    peaks = _peaks()
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    seed = synth.seed_for(wl.index, 13)
+    pos = synth.uniform_positions(Bn, wl.pos_lo, wl.pos_hi, seed, dev)
+    params = B.make_params(hq, hkv, D, lp, w, wl.rope_theta)
+    pre_blocks = -(-lp // 64)
+    per_seq = pre_blocks + w // 64
+    n_blocks = Bn * per_seq
+    g = torch.Generator(device="cpu").manual_seed(seed)
+    table = torch.randperm(n_blocks, generator=g).to(torch.int32).view(Bn, per_seq).to(dev)
+    k_pool = synth.normal_bf16((n_blocks, hkv, 64, D), seed + 1, dev)
+    v_pool = synth.normal_bf16((n_blocks, hkv, 64, D), seed + 2, dev)
+    cache = PrefixSlidingCache(Bn, hkv, lp, w, D, dev, fill=None)
+    for i, t in enumerate((cache.k_prefix, cache.v_prefix, cache.k_ring, cache.v_ring)):
+        t.copy_(synth.normal_bf16(tuple(t.shape), seed + 10 + i, dev))
+    q = synth.normal_bf16((Bn, hq, D), seed + 5, dev)
+    k_new = synth.normal_bf16((Bn, 1, hkv, D), seed + 6, dev)
+    v_new = synth.normal_bf16((Bn, 1, hkv, D), seed + 7, dev)
+    q_new = synth.normal_bf16((Bn, 1, hq, D), seed + 8, dev)
+    out = torch.empty((Bn, hq, D), dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(max(1, B.ps_decode_workspace_bytes(params, Bn)), dtype=torch.uint8,
+                     device=dev)
+    stream = torch.cuda.current_stream()
+
+    def timed(fn, n=steps):
+        for _ in range(warmup):
+            fn()
+        torch.cuda.synchronize()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(n)]
+        for a, b in evs:
+            a.record(stream)
+            fn()
+            b.record(stream)
+        torch.cuda.synchronize()
+        assert st.item() == 0, st.item()
+        return statistics.median([a.elapsed_time(b) for a, b in evs])
+
+    kv_tok = 2 * hkv * D * 2
+    alg = Bn * (lp + w) * kv_tok            # rows visible at a wrapped position
+    loaded = Bn * per_seq * 64 * kv_tok     # whole blocks: the last prefix block is partial
+    res = {}
+    for name, fn in (
+            ("paged", lambda: B.ps_decode_attn_paged(params, k_pool, v_pool, table, Bn, q, pos,
+                                                     out, None, ws, st)),
+            ("contiguous", lambda: B.ps_decode_attn(params, cache.struct, q, pos, out, None, ws,
+                                                    st))):
+        ms = timed(fn)
+        gbs = alg / (ms / 1e3) / 1e9
+        res[name] = {"attn_us": round(ms * 1e3, 1), "tok_per_s": round(Bn / (ms / 1e3), 1),
+                     "gbs": round(gbs, 1), "frac": round(gbs / peaks["hbm_gbs"], 4)}
+    res["paged"]["gbs_loaded"] = round(loaded / (res["paged"]["attn_us"] / 1e6) / 1e9, 1)
+
+    def step():
+        B.ps_kv_append_rope_paged(params, k_pool, v_pool, table, Bn, k_new, v_new, q_new, pos, 1,
+                                  st)
+        B.ps_decode_attn_paged(params, k_pool, v_pool, table, Bn, q_new.view(Bn, hq, D), pos,
+                               out, None, ws, st)
+    res["paged_step_us"] = round(timed(step) * 1e3, 1)
+    return {"leg": "paged", "workload": wl.name, "n_blocks": n_blocks,
+            "blocks_per_seq": per_seq, "alg_bytes": alg, "loaded_bytes": loaded,
+            "peak_hbm_gbs": peaks["hbm_gbs"], **res}
+
+
 # ------------------------------------------------------- full-stack decode leg
 def run_stack(dev, batch: int, distinct: int, steps: int = 3, warmup: int = 1):
     """Full-stack decode step: 28 layers x (append + decode), 16/2/128, L_prefix 2000,
@@ -1063,7 +1137,7 @@ def main():
     ap.add_argument("--no-graph", action="store_true",
                     help="launch the timed steps one by one instead of as a CUDA graph")
     ap.add_argument("--leg", default="main", choices=["main", "prefill", "sweep", "stack", "latency",
-                                                      "shared", "reset", "pin"],
+                                                      "shared", "reset", "pin", "paged"],
                     help="main: the driver's line; prefill/sweep/stack: one extra workload")
     ap.add_argument("--stack-batch", type=int, default=1024)
     ap.add_argument("--stack-distinct", type=int, default=6)
@@ -1095,6 +1169,8 @@ def main():
             res = run_reset(dev)
         elif args.leg == "pin":
             res = run_pin(dev)
+        elif args.leg == "paged":
+            res = run_paged(dev)
         else:
             res = run_stack(dev, args.stack_batch, args.stack_distinct)
         if rank == 0:

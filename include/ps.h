@@ -246,6 +246,36 @@ int ps_decode_attn_pinned(const ps_params* params, const ps_kv_cache* cache,
                           float* lse, void* workspace, size_t ws_bytes, int32_t* dev_status,
                           ps_stream_t stream);
 
+/* Paged store ("Prefix Sliding 完全拆解", §核心机制: with paged block management every
+ * sequence can pre-allocate a fixed number of blocks, since it never holds more than
+ * L_prefix + W tokens).  K and V of all sequences live in one pool of 64-token blocks:
+ *   k_pool, v_pool : device bf16 [n_blocks, Hkv, 64, D].
+ *   block_table    : device int32 [batch, table_stride]; for sequence b, entries
+ *                    0 .. ceil(L_prefix / 64) - 1 are its prefix blocks (position p < L_prefix
+ *                    is row p % 64 of entry p / 64) and the next W / 64 entries its ring blocks
+ *                    (ring slot s = (p - L_prefix) mod W is row s % 64 of entry
+ *                    ceil(L_prefix / 64) + s / 64).  Sequences may share blocks, e.g. the
+ *                    prefix blocks of one prompt.
+ * Rows of a block that no visible position maps to (the tail of the last prefix block, ring
+ * rows not yet written) may hold anything, NaN included: they never reach the result.
+ * Requires W a multiple of 64 and table_stride >= ceil(L_prefix / 64) + W / 64.  A table
+ * entry outside [0, n_blocks) sets PS_DEV_POS_RANGE: the append writes nothing for that
+ * token and the decode reads zeros for that block. */
+int ps_kv_append_rope_paged(const ps_params* params, void* k_pool, void* v_pool,
+                            int64_t n_blocks, const int32_t* block_table, int32_t table_stride,
+                            int64_t batch, const void* k_new, const void* v_new, void* q_inout,
+                            const int64_t* pos0, int32_t T, int32_t* dev_status,
+                            ps_stream_t stream);
+
+/* Decode step over a paged store: results equal ps_decode_attn on the same keys; every
+ * 64-row tile is one block, loaded where the table points.  Other arguments, the workspace
+ * (ps_decode_workspace_bytes) and errors as ps_decode_attn. */
+int ps_decode_attn_paged(const ps_params* params, void* k_pool, void* v_pool, int64_t n_blocks,
+                         const int32_t* block_table, int32_t table_stride, int64_t batch,
+                         const void* q, const int64_t* pos, void* out, float* lse,
+                         void* workspace, size_t ws_bytes, int32_t* dev_status,
+                         ps_stream_t stream);
+
 /* Bytes of device workspace ps_full_attn_ref needs (same split-K layout as decode). */
 size_t ps_full_attn_workspace_bytes(const ps_params* params, int64_t batch, int64_t lmax);
 

@@ -82,6 +82,12 @@ _SIGS = {
                                          c_int64, c_void_p, c_void_p, c_void_p, c_int64,
                                          POINTER(c_int64), c_void_p, c_size_t, c_void_p,
                                          c_void_p]),
+    "ps_kv_append_rope_paged": (c_int32, [POINTER(PsParams), c_void_p, c_void_p, c_int64,
+                                          c_void_p, c_int32, c_int64, c_void_p, c_void_p,
+                                          c_void_p, c_void_p, c_int32, c_void_p, c_void_p]),
+    "ps_decode_attn_paged": (c_int32, [POINTER(PsParams), c_void_p, c_void_p, c_int64, c_void_p,
+                                       c_int32, c_int64, c_void_p, c_void_p, c_void_p, c_void_p,
+                                       c_void_p, c_size_t, c_void_p, c_void_p]),
     "ps_decode_step": (c_int32, [POINTER(PsParams), POINTER(PsKVCache), c_void_p, c_void_p,
                                  c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_size_t,
                                  c_void_p, c_void_p]),
@@ -188,6 +194,28 @@ def ps_decode_attn(params: PsParams, cache: PsKVCache, q, pos, out, lse=None, wo
                                _ptr(out), _ptr(lse), _ptr(workspace), ws_bytes, _ptr(dev_status),
                                _stream(stream))
     _check(rc, "ps_decode_attn")
+
+
+def ps_kv_append_rope_paged(params: PsParams, k_pool, v_pool, block_table, batch: int, k_new,
+                            v_new, q_inout, pos0, T: int, dev_status=None, stream=None) -> None:
+    """Append into a paged store: pools [n_blocks, Hkv, 64, D], block_table [batch, stride]."""
+    rc = load().ps_kv_append_rope_paged(ctypes.byref(params), _ptr(k_pool), _ptr(v_pool),
+                                        int(k_pool.shape[0]), _ptr(block_table),
+                                        int(block_table.shape[1]), int(batch), _ptr(k_new),
+                                        _ptr(v_new), _ptr(q_inout), _ptr(pos0), int(T),
+                                        _ptr(dev_status), _stream(stream))
+    _check(rc, "ps_kv_append_rope_paged")
+
+
+def ps_decode_attn_paged(params: PsParams, k_pool, v_pool, block_table, batch: int, q, pos, out,
+                         lse=None, workspace=None, dev_status=None, stream=None) -> None:
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rc = load().ps_decode_attn_paged(ctypes.byref(params), _ptr(k_pool), _ptr(v_pool),
+                                     int(k_pool.shape[0]), _ptr(block_table),
+                                     int(block_table.shape[1]), int(batch), _ptr(q), _ptr(pos),
+                                     _ptr(out), _ptr(lse), _ptr(workspace), ws_bytes,
+                                     _ptr(dev_status), _stream(stream))
+    _check(rc, "ps_decode_attn_paged")
 
 
 def ps_decode_step(params: PsParams, cache: PsKVCache, k_new, v_new, q_inout, pos, out,

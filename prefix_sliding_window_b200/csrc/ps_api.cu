@@ -255,7 +255,7 @@ int ps_kv_append_rope(const ps_params* params, const ps_kv_cache* cache, const v
     return fail(PS_ERR_INVALID_ARG, "pos0 is not 8-byte aligned");
   if ((reinterpret_cast<uintptr_t>(dev_status) & 3u) != 0)
     return fail(PS_ERR_INVALID_ARG, "dev_status is not 4-byte aligned");
-  AppendArgs a;
+  AppendArgs a{};
   a.k_new = k_new;
   a.v_new = v_new;
   a.q = q_inout;
@@ -781,6 +781,116 @@ int ps_decode_step(const ps_params* params, const ps_kv_cache* cache, const void
   PS_TRY(ps_kv_append_rope(params, cache, k_new, v_new, q_inout, pos, 1, dev_status, stream));
   return decode_entry(params, cache, q_inout, pos, out, lse, workspace, ws_bytes, dev_status,
                       stream, 0, 0, nullptr, nullptr, 1);
+}
+
+// ---------------------------------------------------------------- paged store
+static int check_paged(const ps_params* params, const void* k_pool, const void* v_pool,
+                       int64_t n_blocks, const int32_t* block_table, int32_t table_stride,
+                       int64_t batch) {
+  PS_TRY(check_params(params, true));
+  if (params->window % kDecodeTile != 0)
+    return fail(PS_ERR_UNSUPPORTED, "a paged store needs a window that is a multiple of 64");
+  if (batch < 0) return fail(PS_ERR_INVALID_ARG, "batch must be >= 0");
+  if (n_blocks < 1 || n_blocks > 0x7fffffffLL)
+    return fail(PS_ERR_INVALID_ARG, "n_blocks out of range");
+  const int32_t need = (params->l_prefix + kDecodeTile - 1) / kDecodeTile +
+                       params->window / kDecodeTile;
+  if (table_stride < need)
+    return fail(PS_ERR_INVALID_ARG, "table_stride smaller than the blocks a sequence needs");
+  PS_TRY(check_ptr(k_pool, "k_pool"));
+  PS_TRY(check_ptr(v_pool, "v_pool"));
+  if (!block_table || (reinterpret_cast<uintptr_t>(block_table) & 3u) != 0)
+    return fail(PS_ERR_INVALID_ARG, "block_table is NULL or not 4-byte aligned");
+  return PS_OK;
+}
+
+int ps_kv_append_rope_paged(const ps_params* params, void* k_pool, void* v_pool,
+                            int64_t n_blocks, const int32_t* block_table, int32_t table_stride,
+                            int64_t batch, const void* k_new, const void* v_new, void* q_inout,
+                            const int64_t* pos0, int32_t T, int32_t* dev_status,
+                            ps_stream_t stream) {
+  g_last_error.clear();
+  PS_TRY(check_paged(params, k_pool, v_pool, n_blocks, block_table, table_stride, batch));
+  if (T < 1) return fail(PS_ERR_INVALID_ARG, "T must be >= 1");
+  if (batch == 0) return PS_OK;
+  PS_TRY(check_ptr(k_new, "k_new"));
+  PS_TRY(check_ptr(v_new, "v_new"));
+  PS_TRY(check_ptr(q_inout, "q_inout", true));
+  if (!pos0 || (reinterpret_cast<uintptr_t>(pos0) & 7u) != 0)
+    return fail(PS_ERR_INVALID_ARG, "pos0 is NULL or not 8-byte aligned");
+  if ((reinterpret_cast<uintptr_t>(dev_status) & 3u) != 0)
+    return fail(PS_ERR_INVALID_ARG, "dev_status is not 4-byte aligned");
+  AppendArgs a{};
+  a.k_new = k_new;
+  a.v_new = v_new;
+  a.q = q_inout;
+  a.pos0 = pos0;
+  a.k_pre = k_pool;
+  a.v_pre = v_pool;
+  a.k_ring = k_pool;
+  a.v_ring = v_pool;
+  a.status = dev_status;
+  a.batch = batch;
+  a.T = T;
+  a.hq = params->n_q_heads;
+  a.hkv = params->n_kv_heads;
+  a.lp = params->l_prefix;
+  a.w = params->window;
+  a.paged = 1;
+  a.table = block_table;
+  a.table_stride = table_stride;
+  a.pre_blocks = (params->l_prefix + kDecodeTile - 1) / kDecodeTile;
+  a.n_blocks = n_blocks;
+  for (int i = 0; i < kHeadDim / 2; ++i)
+    a.inv_freq[i] = pow(params->rope_theta, -2.0 * i / double(kHeadDim));
+  return check_cuda(launch_append(a, reinterpret_cast<cudaStream_t>(stream)),
+                    "append_rope_kernel launch");
+}
+
+int ps_decode_attn_paged(const ps_params* params, void* k_pool, void* v_pool, int64_t n_blocks,
+                         const int32_t* block_table, int32_t table_stride, int64_t batch,
+                         const void* q, const int64_t* pos, void* out, float* lse,
+                         void* workspace, size_t ws_bytes, int32_t* dev_status,
+                         ps_stream_t stream) {
+  g_last_error.clear();
+  PS_TRY(check_paged(params, k_pool, v_pool, n_blocks, block_table, table_stride, batch));
+  if (params->n_q_heads / params->n_kv_heads > kMaxGroup)
+    return fail(PS_ERR_UNSUPPORTED, "decode supports at most 8 query heads per KV head");
+  if (batch == 0) return PS_OK;
+  PS_TRY(check_ptr(q, "q"));
+  PS_TRY(check_ptr(out, "out"));
+  PS_TRY(check_ptr(lse, "lse", true));
+  if (!pos || (reinterpret_cast<uintptr_t>(pos) & 7u) != 0)
+    return fail(PS_ERR_INVALID_ARG, "pos is NULL or not 8-byte aligned");
+  if ((reinterpret_cast<uintptr_t>(dev_status) & 3u) != 0)
+    return fail(PS_ERR_INVALID_ARG, "dev_status is not 4-byte aligned");
+  const size_t need = decode_workspace_bytes(batch, params->n_kv_heads,
+                                             (int64_t)params->l_prefix + params->window);
+  if (need > 0 && (!workspace || ws_bytes < need))
+    return fail(PS_ERR_WORKSPACE, "workspace smaller than ps_decode_workspace_bytes()");
+  DecodeLaunch l{};
+  l.q = q;
+  l.pos = pos;
+  l.out = out;
+  l.lse = lse;
+  l.workspace = workspace;
+  l.status = dev_status;
+  l.batch = batch;
+  l.hq = params->n_q_heads;
+  l.hkv = params->n_kv_heads;
+  l.lp = params->l_prefix;
+  l.w = params->window;
+  l.scale = resolve_scale(params);
+  l.k0 = k_pool;
+  l.v0 = v_pool;
+  l.k1 = k_pool;
+  l.v1 = v_pool;
+  l.rope_theta = params->rope_theta;
+  l.paged = 1;
+  l.table = block_table;
+  l.table_stride = table_stride;
+  l.n_blocks = n_blocks;
+  return launch_decode(l, reinterpret_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

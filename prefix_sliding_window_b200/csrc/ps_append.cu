@@ -87,6 +87,18 @@ __global__ void __launch_bounds__(kAppendThreads) append_rope_kernel(const Appen
     row_stride_rows = a.w;
     row = (p - a.lp) % a.w;
   }
+  int64_t blk = b;  // the store's (sequence or pool block) index in its outermost dimension
+  if (a.paged && k_dst_base) {
+    // 64-row blocks of the pool: logical block row / 64 (prefix) or pre_blocks + slot / 64
+    const int64_t lb = (p < a.lp ? 0 : a.pre_blocks) + row / 64;
+    blk = a.table[b * a.table_stride + lb];
+    row_stride_rows = 64;
+    row %= 64;
+    if (blk < 0 || blk >= a.n_blocks) {  // a bad table entry: flag it, write nothing
+      if (threadIdx.x == 0 && a.status) atomicOr(a.status, PS_DEV_POS_RANGE);
+      k_dst_base = v_dst_base = nullptr;
+    }
+  }
   __nv_bfloat16* qb = static_cast<__nv_bfloat16*>(a.q) + tok * a.hq * kHeadDim;
 
   // Work items: K rotate (hkv x kChunks), V copy (hkv x 16), q rotate (hq x kChunks).
@@ -135,13 +147,13 @@ __global__ void __launch_bounds__(kAppendThreads) append_rope_kernel(const Appen
       const int h = it / kChunks, c = it % kChunks;
       uint4 y1, y2;
       rotate8(x1, x2, s_cos + 8 * c, s_sin + 8 * c, y1, y2);
-      __nv_bfloat16* dst = k_dst_base + ((b * a.hkv + h) * row_stride_rows + row) * kHeadDim;
+      __nv_bfloat16* dst = k_dst_base + ((blk * a.hkv + h) * row_stride_rows + row) * kHeadDim;
       *reinterpret_cast<uint4*>(dst + 8 * c) = y1;
       *reinterpret_cast<uint4*>(dst + kHalf + 8 * c) = y2;
     } else if (it < n_k + n_v) {
       const int j = it - n_k;
       const int h = j / 16, c = j % 16;
-      __nv_bfloat16* dst = v_dst_base + ((b * a.hkv + h) * row_stride_rows + row) * kHeadDim;
+      __nv_bfloat16* dst = v_dst_base + ((blk * a.hkv + h) * row_stride_rows + row) * kHeadDim;
       *reinterpret_cast<uint4*>(dst + 8 * c) = x1;
     } else {
       // q rotated in place at the token's own absolute position

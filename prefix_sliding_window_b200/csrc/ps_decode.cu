@@ -81,6 +81,13 @@ struct DecodeArgs {
   // each sequence's newest row and the rotated q depend on that kernel, so everything else
   // may stream before the programmatic wait
   int32_t after_append;
+  // paged store: K/V of every (sequence, KV head) in 64-row blocks of one pool
+  // [n_blocks][Hkv][64][D]; logical block i of sequence b is table[b * table_stride + i]
+  // (prefix blocks first, then W / 64 ring blocks)
+  int32_t paged;
+  const int32_t* table;
+  int32_t table_stride, pre_blocks;
+  int64_t n_blocks;
   double inv_freq[kHeadDim / 2];
   // tokens appended to the pinned prefix: rows [L_prefix, L_prefix + pin_count[b]) of the
   // prefix store hold the promoted positions pin_pos[b][0..) (ascending)
@@ -121,7 +128,7 @@ __device__ __forceinline__ DecodeTiling tiling_of(const DecodeArgs& a, int64_t b
       r.pre_len += lo;
     }
   }
-  return make_tiling(r, a.dim0, a.w);
+  return a.paged ? make_tiling_paged(r) : make_tiling(r, a.dim0, a.w);
 }
 
 // Walks a contiguous range of the global tile sequence: unit u = b * hkv + h owns tiles
@@ -331,10 +338,23 @@ __global__ void __launch_bounds__(kThreads)
         const int unit = pw.b * a.hkv + pw.h;
         uint8_t* st = smem + s * kStageBytes;
         mbar_arrive_expect_tx(&full[s], kStageBytes);
-        tma_load_3d_hint(st, mk, 0, d.row0, unit, &full[s], pol);
-        tma_load_3d_hint(st + kBoxBytes, mk, 64, d.row0, unit, &full[s], pol);
-        tma_load_3d_hint(st + kTileBytes, mv, 0, d.row0, unit, &full[s], pol);
-        tma_load_3d_hint(st + kTileBytes + kBoxBytes, mv, 64, d.row0, unit, &full[s], pol);
+        if (a.paged) {
+          // one tile = one block of the pool (a block id out of range reads zeros: TMA
+          // clips coordinates to the pool; it is flagged)
+          const int32_t blk =
+              a.table[(int64_t)pw.b * a.table_stride + (d.map_id ? a.pre_blocks : 0) +
+                      d.row0 / kDecodeTile];
+          if ((blk < 0 || blk >= a.n_blocks) && a.status) atomicOr(a.status, PS_DEV_POS_RANGE);
+          tma_load_4d(st, &mk0, 0, 0, pw.h, blk, &full[s]);
+          tma_load_4d(st + kBoxBytes, &mk0, 64, 0, pw.h, blk, &full[s]);
+          tma_load_4d(st + kTileBytes, &mv0, 0, 0, pw.h, blk, &full[s]);
+          tma_load_4d(st + kTileBytes + kBoxBytes, &mv0, 64, 0, pw.h, blk, &full[s]);
+        } else {
+          tma_load_3d_hint(st, mk, 0, d.row0, unit, &full[s], pol);
+          tma_load_3d_hint(st + kBoxBytes, mk, 64, d.row0, unit, &full[s], pol);
+          tma_load_3d_hint(st + kTileBytes, mv, 0, d.row0, unit, &full[s], pol);
+          tma_load_3d_hint(st + kTileBytes + kBoxBytes, mv, 64, d.row0, unit, &full[s], pol);
+        }
         issued = i + 1;
       }
       // every issued copy must land before the CTA may exit or reuse shared memory
@@ -563,13 +583,23 @@ __global__ void __launch_bounds__(kThreads)
       }
       const uint32_t b0 = movmatrix_trans(pack_bf16x2(p0, p1));
       const uint32_t b1 = movmatrix_trans(pack_bf16x2(p2, p3));
+      // V rows outside [lo, hi) get P = 0, but 0 x NaN is NaN: a paged block's rows past
+      // its segment may never have been written.  This lane's V elements are keys
+      // kv, kv+1 (a0, a1) and kv+8, kv+9 (a2, a3); drop those outside the segment.
+      uint32_t vm01 = 0xffffffffu, vm23 = 0xffffffffu;
+      if (d.lo > 0 || d.hi < kDecodeTile) {
+        const int kv = 16 * warp + 2 * qq;
+        auto in = [&](int k) { return k >= d.lo && k < d.hi; };
+        vm01 = (in(kv) ? 0x0000ffffu : 0u) | (in(kv + 1) ? 0xffff0000u : 0u);
+        vm23 = (in(kv + 8) ? 0x0000ffffu : 0u) | (in(kv + 9) ? 0xffff0000u : 0u);
+      }
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
         const int dd = 16 * j + vdoff;
         uint32_t a0, a1, a2, a3;
         ldmatrix_x4_trans(vbase + (dd >> 6) * kBoxBytes + swz(vkey, (dd & 63) >> 3), a0, a1, a2,
                           a3);
-        mma_bf16_16816(o[j], a0, a1, a2, a3, b0, b1);
+        mma_bf16_16816(o[j], a0 & vm01, a1 & vm01, a2 & vm23, a3 & vm23, b0, b1);
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[s]);
@@ -759,19 +789,26 @@ int launch_decode(const DecodeLaunch& l, cudaStream_t stream) {
       l.full_mode ? static_cast<int32_t>(l.lmax) : (l.skip_prefix ? 0 : pre_rows);
 
   CUtensorMap mk0, mv0, mk1, mv1;
-  // A zero-row tensor cannot be described; such a map is never used (no tiles), so it
-  // borrows the other map.
-  if (dim0 > 0) {
+  if (l.paged) {
+    // the pool [n_blocks][Hkv][64][D]: a 4-D map whose box is one half-row block
+    const uint64_t dims[4] = {kHeadDim, (uint64_t)kDecodeTile, (uint64_t)l.hkv,
+                              (uint64_t)l.n_blocks};
+    const uint32_t box[4] = {64, (uint32_t)kDecodeTile, 1, 1};
+    if (!make_map_4d(&mk0, l.k0, dims, box) || !make_map_4d(&mv0, l.v0, dims, box))
+      return PS_ERR_CUDA;
+    mk1 = mk0;
+    mv1 = mv0;
+  } else if (dim0 > 0) {
     if (!make_map_3d(&mk0, l.k0, kHeadDim, dim0, units, 64, kDecodeTile) ||
         !make_map_3d(&mv0, l.v0, kHeadDim, dim0, units, 64, kDecodeTile))
       return PS_ERR_CUDA;
   }
-  if (!l.full_mode) {
+  if (!l.full_mode && !l.paged) {
     if (!make_map_3d(&mk1, l.k1, kHeadDim, l.w, units, 64, kDecodeTile) ||
         !make_map_3d(&mv1, l.v1, kHeadDim, l.w, units, 64, kDecodeTile))
       return PS_ERR_CUDA;
   }
-  if (dim0 == 0) {
+  if (dim0 == 0 && !l.paged) {
     mk0 = mk1;
     mv0 = mv1;
   }
@@ -810,6 +847,11 @@ int launch_decode(const DecodeLaunch& l, cudaStream_t stream) {
   a.skip_prefix = l.skip_prefix;
   a.reset_pe = l.reset_pe;
   a.after_append = l.after_append;
+  a.paged = l.paged;
+  a.table = l.table;
+  a.table_stride = l.table_stride;
+  a.pre_blocks = (l.lp + kDecodeTile - 1) / kDecodeTile;
+  a.n_blocks = l.n_blocks;
   a.pin_count = l.pin_count;
   a.pin_pos = l.pin_pos;
   a.pin_cap = (l.lcap > l.lp) ? l.lcap - l.lp : 0;

@@ -64,6 +64,13 @@ struct AppendArgs {
   int32_t* status;
   int64_t batch;
   int32_t T, hq, hkv, lp, w;
+  // paged store: k_pre/v_pre and k_ring/v_ring all point to the pool [n_blocks][Hkv][64][D];
+  // position p lives in logical block p / 64 (prefix) or pre_blocks + slot / 64 (ring) of
+  // table[b * table_stride + ...]
+  int32_t paged;
+  const int32_t* table;
+  int32_t table_stride, pre_blocks;
+  int64_t n_blocks;
   double inv_freq[kHeadDim / 2];  // theta^(-2i/D), float64, filled by the host
 };
 cudaError_t launch_append(const AppendArgs& a, cudaStream_t stream);
@@ -125,6 +132,11 @@ struct DecodeLaunch {
   const int64_t* pin_pos;
   // the previous kernel on the stream is the one-token append at pos (ps_decode_step)
   int32_t after_append;
+  // paged store (k0/v0 = the pool [n_blocks][Hkv][64][D], table [batch][table_stride])
+  int32_t paged;
+  const int32_t* table;
+  int32_t table_stride;
+  int64_t n_blocks;
 };
 // Split count and workspace bytes for a decode of this shape on the current device.
 int decode_splits(int64_t batch, int32_t hkv, int64_t max_keys);

@@ -73,7 +73,8 @@ struct DecodeTiling {
   int32_t nt[3];       // tiles per segment
   int32_t begin[3];    // first row of the segment
   int32_t end[3];      // one past the last row
-  int32_t forward[3];  // 1: tiled forward from begin; 0: backward from end
+  int32_t forward[3];  // 1: tiled forward from begin; 0: backward from end; 2: tiles on
+                       // 64-row block boundaries (paged stores), rows outside masked
   int32_t map_id[3];
   int32_t total;
 };
@@ -104,6 +105,30 @@ PS_HD DecodeTiling make_tiling(const VisibleRanges& r, int32_t dim_prefix, int32
   return t;
 }
 
+// Tiling of a paged store: every segment cut on 64-row block boundaries (a tile is one block;
+// rows outside the segment are masked by the tile's [lo, hi)).
+PS_HD DecodeTiling make_tiling_paged(const VisibleRanges& r) {
+  DecodeTiling t;
+  t.begin[0] = 0;
+  t.end[0] = r.pre_len;
+  t.map_id[0] = 0;
+  t.begin[1] = r.seg0_start;
+  t.end[1] = r.seg0_start + r.seg0_len;
+  t.map_id[1] = 1;
+  t.begin[2] = 0;
+  t.end[2] = r.seg1_len;
+  t.map_id[2] = 1;
+  t.total = 0;
+  for (int s = 0; s < 3; ++s) {
+    t.forward[s] = 2;
+    t.nt[s] = t.end[s] > t.begin[s]
+                  ? ceil_div_i32(t.end[s], kDecodeTile) - t.begin[s] / kDecodeTile
+                  : 0;
+    t.total += t.nt[s];
+  }
+  return t;
+}
+
 PS_HD DecodeTile tiling_tile(const DecodeTiling& t, int32_t idx) {
   // segment selection with constant indices only (keeps the tiling in registers)
   int32_t begin, end, fwd, map_id, nt;
@@ -118,7 +143,12 @@ PS_HD DecodeTile tiling_tile(const DecodeTiling& t, int32_t idx) {
   }
   DecodeTile d;
   d.map_id = map_id;
-  if (fwd) {
+  if (fwd == 2) {
+    d.row0 = (begin / kDecodeTile + idx) * kDecodeTile;
+    d.lo = begin > d.row0 ? begin - d.row0 : 0;
+    const int32_t left = end - d.row0;
+    d.hi = left < kDecodeTile ? left : kDecodeTile;
+  } else if (fwd) {
     d.row0 = begin + idx * kDecodeTile;
     d.lo = 0;
     const int32_t left = end - d.row0;
