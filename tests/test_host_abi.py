@@ -210,3 +210,29 @@ def test_pin_host_validation(lib):
              None, None) == B.PS_ERR_INVALID_ARG    # capacity must exceed l_prefix
     assert g(ctypes.byref(p), ctypes.byref(cache), 200, None, 16, 16, 16, 16, None, None, 0,
              None, None) == B.PS_ERR_INVALID_ARG
+
+
+def test_paged_host_validation(lib):
+    """Window not a multiple of 64, a table too narrow for L_prefix + W, no blocks, and NULL
+    or misaligned pointers are refused before any launch."""
+    f, g = lib.ps_kv_append_rope_paged, lib.ps_decode_attn_paged
+    p = _params(l_prefix=100, window=512)          # 2 prefix + 8 ring blocks per sequence
+
+    def app(par=p, n_blocks=64, table=16, stride=10, k_pool=16, pos0=16, T=1):
+        return f(ctypes.byref(par), k_pool, 16, n_blocks, table, stride, 4, 16, 16, None, pos0,
+                 T, None, None)
+
+    def dec(par=p, n_blocks=64, table=16, stride=10, k_pool=16):
+        return g(ctypes.byref(par), k_pool, 16, n_blocks, table, stride, 4, 16, 16, 16, None,
+                 None, 0, None, None)
+
+    for call in (app, dec):
+        assert call(par=_params(l_prefix=100, window=500)) == B.PS_ERR_UNSUPPORTED
+        assert call(stride=9) == B.PS_ERR_INVALID_ARG
+        assert call(n_blocks=0) == B.PS_ERR_INVALID_ARG
+        assert call(table=None) == B.PS_ERR_INVALID_ARG
+        assert call(table=18) == B.PS_ERR_INVALID_ARG   # not 4-byte aligned
+        assert call(k_pool=None) == B.PS_ERR_INVALID_ARG
+    assert app(T=0) == B.PS_ERR_INVALID_ARG
+    assert app(pos0=None) == B.PS_ERR_INVALID_ARG
+    assert app(pos0=12) == B.PS_ERR_INVALID_ARG         # not 8-byte aligned
