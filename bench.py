@@ -330,7 +330,7 @@ def run_decode(args, world, rank, dev):
             "decode_us_p10": round(float(np.percentile(dec_ms, 10)) * 1e3, 2),
             "decode_us_p90": round(float(np.percentile(dec_ms, 90)) * 1e3, 2),
             "frac_of_8tbs_spec": round(achieved / 8000.0, 4)}
-    e2e = run_decode_e2e(work, K, W, world)
+    e2e = run_decode_e2e(work, K, W, world, use_graph=not args.no_graph)
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": K,
         "warmup": W, "ms_per_step": round(ms / K, 5), "higher_is_better": True,
@@ -352,7 +352,7 @@ def run_decode(args, world, rank, dev):
     return line, work
 
 
-def run_decode_e2e(work: DecodeWorkload, K: int, W: int, world: int):
+def run_decode_e2e(work: DecodeWorkload, K: int, W: int, world: int, use_graph: bool = True):
     """Same metric through the C ABI with host buffers: every step copies its inputs
     (q, k_new, v_new, pos: packed in one pinned host buffer, so one DMA) host->device and
     reads out device->host, in stream order: step i+1's inputs are copied after step i's
@@ -391,19 +391,35 @@ def run_decode_e2e(work: DecodeWorkload, K: int, W: int, world: int):
     for i in range(W):
         step(i)
     torch.cuda.synchronize()
+    graph = None
+    if use_graph:
+        # the same K steps (copy in, step, copy out, in stream order) as one CUDA graph
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            for j in range(K):
+                step(W + j)
+        torch.cuda.synchronize()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     _barrier(world)
     ev0.record(stream)
-    for j in range(K):
-        step(W + j)
+    if graph is not None:
+        graph.replay()
+    else:
+        for j in range(K):
+            step(W + j)
     ev1.record(stream)
     torch.cuda.synchronize()
     ms = _max_over_ranks(ev0.elapsed_time(ev1), world)
+    assert work.status.item() == 0, f"device status {work.status.item()}"
+    # the timed steps really moved the data: the last output read back equals the device's
+    assert torch.equal(h_out[W + K - 1], d_out.cpu())
+    del graph
     tokens = _sum_over_ranks(float(work.wl.batch * K), world)
     bi = (d_k.numel() + d_v.numel() + d_q.numel()) * 2 + d_pos.numel() * 8
     bo = d_out.numel() * 2
     return {"value": round(tokens / (ms / 1e3), 1), "unit": UNIT, "h2d_bytes_per_step": bi,
-            "d2h_bytes_per_step": bo, "h2d_copies_per_step": 1, "d2h_copies_per_step": 1}
+            "d2h_bytes_per_step": bo, "h2d_copies_per_step": 1, "d2h_copies_per_step": 1,
+            "launch": "CUDA graph of the timed steps" if use_graph else "eager"}
 
 
 # ------------------------------------------------------------- prefill leg

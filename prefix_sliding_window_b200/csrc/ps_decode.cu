@@ -216,7 +216,9 @@ __device__ __forceinline__ void store_state(float* dst, float m0, float m1, floa
   dst[35] = l1;
 }
 
-template <int STAGES>
+// RESET: Reset-PE mode (prefix tiles see the query at its renumbered id).  A template
+// flag, not a run-time one, so the plain decode carries none of its registers.
+template <int STAGES, bool RESET>
 __global__ void __launch_bounds__(kThreads)
     decode_kernel(const __grid_constant__ CUtensorMap mk0, const __grid_constant__ CUtensorMap mv0,
                   const __grid_constant__ CUtensorMap mk1, const __grid_constant__ CUtensorMap mv1,
@@ -512,7 +514,7 @@ __global__ void __launch_bounds__(kThreads)
     if (a.after_append) pdl_wait();  // q is rotated by the append just before
     if (ntiles > 0) {
       load_q(cw.b, cw.h);
-      if (a.reset_pe) rotate_prefix_q(a.pos[cw.b]);
+      if (RESET) rotate_prefix_q(a.pos[cw.b]);
       note_span(cw, cw.t, (cw.pu1 < wk.t_end ? cw.pu1 : wk.t_end) - 1);
       prefetch_next_q(cw);
     }
@@ -527,7 +529,7 @@ __global__ void __launch_bounds__(kThreads)
           qf[ks][0] = qn[ks][0];
           qf[ks][1] = qn[ks][1];
         }
-        if (a.reset_pe) rotate_prefix_q(a.pos[cw.b]);
+        if (RESET) rotate_prefix_q(a.pos[cw.b]);
         note_span(cw, cw.t, (cw.pu1 < wk.t_end ? cw.pu1 : wk.t_end) - 1);
         prefetch_next_q(cw);
       }
@@ -548,7 +550,7 @@ __global__ void __launch_bounds__(kThreads)
             kbase + (ks >> 2) * kBoxBytes + swz(arow, ((ks & 3) << 1) + achunk);
         ldmatrix_x4(addr, a0, a1, a2, a3);
         // Reset PE: prefix tiles (map 0) see the query at its Reset-PE id
-        const bool pre_q = a.reset_pe && d.map_id == 0;
+        const bool pre_q = RESET && d.map_id == 0;
         mma_bf16_16816(sc, a0, a1, a2, a3, pre_q ? qp[ks][0] : qf[ks][0],
                        pre_q ? qp[ks][1] : qf[ks][1]);
       }
@@ -586,20 +588,24 @@ __global__ void __launch_bounds__(kThreads)
       // V rows outside [lo, hi) get P = 0, but 0 x NaN is NaN: a paged block's rows past
       // its segment may never have been written.  This lane's V elements are keys
       // kv, kv+1 (a0, a1) and kv+8, kv+9 (a2, a3); drop those outside the segment.
-      uint32_t vm01 = 0xffffffffu, vm23 = 0xffffffffu;
+      // Full tiles take the unmasked copy of the loop (the masks fold away).
+      auto pv = [&](uint32_t vm01, uint32_t vm23) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int dd = 16 * j + vdoff;
+          uint32_t a0, a1, a2, a3;
+          ldmatrix_x4_trans(vbase + (dd >> 6) * kBoxBytes + swz(vkey, (dd & 63) >> 3), a0, a1,
+                            a2, a3);
+          mma_bf16_16816(o[j], a0 & vm01, a1 & vm01, a2 & vm23, a3 & vm23, b0, b1);
+        }
+      };
       if (d.lo > 0 || d.hi < kDecodeTile) {
         const int kv = 16 * warp + 2 * qq;
         auto in = [&](int k) { return k >= d.lo && k < d.hi; };
-        vm01 = (in(kv) ? 0x0000ffffu : 0u) | (in(kv + 1) ? 0xffff0000u : 0u);
-        vm23 = (in(kv + 8) ? 0x0000ffffu : 0u) | (in(kv + 9) ? 0xffff0000u : 0u);
-      }
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int dd = 16 * j + vdoff;
-        uint32_t a0, a1, a2, a3;
-        ldmatrix_x4_trans(vbase + (dd >> 6) * kBoxBytes + swz(vkey, (dd & 63) >> 3), a0, a1, a2,
-                          a3);
-        mma_bf16_16816(o[j], a0 & vm01, a1 & vm01, a2 & vm23, a3 & vm23, b0, b1);
+        pv((in(kv) ? 0x0000ffffu : 0u) | (in(kv + 1) ? 0xffff0000u : 0u),
+           (in(kv + 8) ? 0x0000ffffu : 0u) | (in(kv + 9) ? 0xffff0000u : 0u));
+      } else {
+        pv(0xffffffffu, 0xffffffffu);
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[s]);
@@ -730,10 +736,12 @@ int occupancy_per_sm() {
   if (cached[dev] == 0) {
     int occ = 0;
     const size_t sb = smem_bytes(kStages);
-    cudaFuncSetAttribute(decode_kernel<kStages>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)sb);
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, decode_kernel<kStages>, kThreads, sb) !=
-            cudaSuccess ||
+    cudaFuncSetAttribute(decode_kernel<kStages, false>,
+                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sb);
+    cudaFuncSetAttribute(decode_kernel<kStages, true>,
+                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sb);
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, decode_kernel<kStages, false>,
+                                                      kThreads, sb) != cudaSuccess ||
         occ < 1)
       occ = 1;
     cached[dev] = occ < kCtasPerSm ? occ : kCtasPerSm;
@@ -865,8 +873,10 @@ int launch_decode(const DecodeLaunch& l, cudaStream_t stream) {
   if (grid <= 0) return PS_OK;
   if (grid > 0x7fffffff || l.batch > 0x7fffffff)
     return fail(PS_ERR_UNSUPPORTED, "decode grid too large");
-  int rc = check_cuda(launch_pdl(decode_kernel<kStages>, dim3(static_cast<unsigned>(grid)),
-                                 dim3(kThreads), sb, stream, mk0, mv0, mk1, mv1, a),
+  int rc = check_cuda(launch_pdl(a.reset_pe ? decode_kernel<kStages, true>
+                                            : decode_kernel<kStages, false>,
+                                 dim3(static_cast<unsigned>(grid)), dim3(kThreads), sb, stream,
+                                 mk0, mv0, mk1, mv1, a),
                       "decode_kernel launch");
   if (rc != PS_OK) return rc;
   if (l.before_merge) {
