@@ -4,8 +4,8 @@
 Default workload: steady-state batched decode on one layer (batch 64, 16 query / 2 KV
 heads, head_dim 128, bf16, L_prefix = 100, W = 4096, positions drawn in [8192, 131072],
 KV prefilled with RoPE at every absolute position).  One step = one decode step of the
-whole batch: ps_kv_append_rope (new token, Continue-PE RoPE, ring write) + ps_decode_attn
-(split-K decode + merge).  Prints ONE JSON line on rank 0.
+whole batch through ps_decode_step: the new token's append (Continue-PE RoPE of k and q,
+ring write), then split-K decode + merge.  Prints ONE JSON line on rank 0.
 
   python bench.py [--gpus N --steps K --warmup W] [--impl reference]
 

@@ -453,3 +453,34 @@ def test_decode_step_equals_append_then_decode(cuda_device, Bn, lp, w, lo, hi):
     assert sa == sb
     assert torch.equal(qa, qb) and torch.equal(oa, ob) and torch.equal(la, lb)
     assert torch.equal(caches[0].k_ring, caches[1].k_ring)
+
+
+def test_graph_launched_steps_equal_eager_steps(cuda_device):
+    """The launch configuration bench.py times: ps_decode_step on the batch-64, W=4096
+    workload replayed as one CUDA graph of 8 steps is bit-identical (q, out, cache) to the
+    same 8 steps launched one by one."""
+    import bench
+    dev = cuda_device
+    wl = synth.WORKLOADS["decode_b64_w4096"]
+    K = 8
+    runs = []
+    for graph in (False, True):
+        work = bench.DecodeWorkload(wl, dev, 0, K)
+        if graph:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                for i in range(K):
+                    work.step(i)
+            g.replay()
+        else:
+            for i in range(K):
+                work.step(i)
+        torch.cuda.synchronize()
+        assert work.status.item() == 0
+        runs.append((work.q.clone(), work.out.clone(), work.cache.k_ring.clone(),
+                     work.cache.v_ring.clone()))
+        del work
+        torch.cuda.empty_cache()
+    for a, b in zip(*runs):
+        assert torch.equal(a, b)
+    assert torch.isfinite(runs[1][1].float()).all()

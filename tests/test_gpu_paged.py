@@ -136,3 +136,58 @@ def test_paged_bad_table_entry_is_flagged(cuda_device):
     B.ps_decode_attn_paged(params, k_pool, v_pool, bad, 2, q, pos, out, None, ws, st)
     torch.cuda.synchronize()
     assert st.item() == B.PS_DEV_POS_RANGE
+
+
+def test_paged_pure_window_step_flow(cuda_device):
+    """L_prefix = 0 (no prefix blocks), W = 64 (one ring block): each sequence appends its
+    history, then its newest token together with q (rotated in place, bit-identical to the
+    contiguous append's rotation), then decodes; held to the oracle."""
+    dev = cuda_device
+    lp, w, hq, hkv = 0, 64, 16, 2
+    positions = [0, 1, 63, 64, 65, 200, 1000]
+    Bn = len(positions)
+    params = B.make_params(hq, hkv, D, lp, w, THETA)
+    n_blocks = Bn + 2
+    table = torch.tensor(np.random.default_rng(3).permutation(n_blocks)[:Bn].reshape(Bn, 1),
+                         dtype=torch.int32, device=dev)
+    nan = float("nan")
+    k_pool = torch.full((n_blocks, hkv, 64, D), nan, dtype=torch.bfloat16, device=dev)
+    v_pool = torch.full_like(k_pool, nan)
+    Smax = max(positions) + 1
+    k_raw = synth.normal_bf16((Bn, Smax, hkv, D), 831, dev)
+    v_raw = synth.normal_bf16((Bn, Smax, hkv, D), 832, dev)
+    q_raw = synth.normal_bf16((Bn, hq, D), 833, dev)
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    zero = torch.zeros(1, dtype=torch.int64, device=dev)
+    for b, p in enumerate(positions):
+        if p > 0:
+            B.ps_kv_append_rope_paged(params, k_pool, v_pool, table[b:b + 1], 1,
+                                      k_raw[b:b + 1, :p].contiguous(),
+                                      v_raw[b:b + 1, :p].contiguous(), None, zero, p, st)
+    pos = torch.tensor(positions, dtype=torch.int64, device=dev)
+    k_last = torch.stack([k_raw[b, p] for b, p in enumerate(positions)]).view(Bn, 1, hkv, D)
+    v_last = torch.stack([v_raw[b, p] for b, p in enumerate(positions)]).view(Bn, 1, hkv, D)
+    q = q_raw.clone()
+    B.ps_kv_append_rope_paged(params, k_pool, v_pool, table, Bn, k_last.contiguous(),
+                              v_last.contiguous(), q.view(Bn, 1, hq, D), pos, 1, st)
+    q_ref = q_raw.clone()
+    scratch = PrefixSlidingCache(Bn, hkv, lp, w, D, dev)
+    B.ps_kv_append_rope(params, scratch.struct, k_last.contiguous(), v_last.contiguous(),
+                        q_ref.view(Bn, 1, hq, D), pos, 1, st)
+    torch.cuda.synchronize()
+    assert st.item() == 0, st.item()
+    assert torch.equal(q, q_ref)
+    out = torch.full((Bn, hq, D), nan, dtype=torch.bfloat16, device=dev)
+    lse = torch.full((Bn, hq), nan, dtype=torch.float32, device=dev)
+    ws = torch.empty(max(1, B.ps_decode_workspace_bytes(params, Bn)), dtype=torch.uint8,
+                     device=dev)
+    B.ps_decode_attn_paged(params, k_pool, v_pool, table, Bn, q, pos, out, lse, ws, st)
+    torch.cuda.synchronize()
+    assert st.item() == 0, st.item()
+    qr, kr, vr = f64(q_raw), f64(k_raw), f64(v_raw)
+    got, gl = f64(out), f64(lse)
+    for b, p in enumerate(positions):
+        o, l = _oracle_decode_from_history(B_rope(qr[b], p), kr[b, :p + 1], vr[b, :p + 1], p,
+                                           lp, w, 1 / math.sqrt(D))
+        assert_close(got[b], o, f"paged lp=0 b={b} p={p}")
+        assert np.abs(gl[b] - l).max() < 2e-2, (b, p)
