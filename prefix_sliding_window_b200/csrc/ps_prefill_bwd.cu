@@ -641,20 +641,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t ph = static_cast<uint32_t>(g & 1);
         const int qt = m.qlo + j % m.nqt;
         const int flag = classify_tile(qt, m.kt, a.seq, a.lp, a.w, kT, kT);
-        // this (query tile, key tile)'s dS^T tile in the store: its index in query tile qt's
-        // plan (ascending key tiles), looked up before the scores are waited for
+        // this (query tile, key tile)'s dS^T tile in the store: query tile qt's plan offset
+        // plus the key tile's closed-form position in it, formed before the scores are
+        // waited for
         __nv_bfloat16* ds_row;
         {
-          const int e0 = a.off[qt];
-          int lo = 0, hi = a.off[qt + 1] - e0 - 1;
-          while (lo < hi) {
-            const int mid = (lo + hi) >> 1;
-            if (a.ent[2 * (e0 + mid)] < m.kt) lo = mid + 1; else hi = mid;
-          }
+          const int64_t e = a.off[qt] + plan_index(qt, m.kt, a.lp, a.w, kT);
           const int h = m.kvh * a.group + j / m.nqt;
           // tile layout: [16 column chunks of 8 query cols][128 key rows][8 bf16], so the
           // 32 rows of a warp store 512 contiguous bytes per chunk
-          ds_row = a.ds + (((int64_t)m.b * a.hq + h) * a.n_plan + e0 + lo) * kT * kT + r * 8;
+          ds_row = a.ds + (((int64_t)m.b * a.hq + h) * a.n_plan + e) * kT * kT + r * 8;
         }
         ok = ok && __all_sync(0xffffffffu,
                               mbar_wait(s_full, ph, a.status) &&

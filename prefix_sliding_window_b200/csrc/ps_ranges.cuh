@@ -207,6 +207,21 @@ PS_HD void qtile_candidates(int64_t qt, int64_t seq, int32_t lp, int32_t w, int3
   if (*ws < *pe) *ws = *pe;  // union: do not list a tile twice
 }
 
+// Position of key tile kt in query tile qt's plan, for a (qt, kt) pair that is in it (square
+// tiles, b = Bq = Bk).  A prefix tile (kt < pe) is visible to qt iff kt <= qt, and every
+// window candidate in [ws, we] is non-SKIP (its first key is within W - 1 of the tile's
+// first row, its last key is at most the tile's last row), so the plan is [0, min(pe,
+// qt + 1)) followed by [ws, we].
+PS_HD int64_t plan_index(int64_t qt, int64_t kt, int32_t lp, int32_t w, int32_t b) {
+  const int64_t pe = (lp + b - 1) / b;
+  if (kt < pe) return kt;
+  int64_t first_win_col = qt * b - w + 1;
+  if (first_win_col < lp) first_win_col = lp;
+  int64_t ws = first_win_col / b;
+  if (ws < pe) ws = pe;
+  return (pe < qt + 1 ? pe : qt + 1) + (kt - ws);
+}
+
 // Number of non-SKIP tiles of query tile qt.
 PS_HD int64_t qtile_count(int64_t qt, int64_t seq, int32_t lp, int32_t w, int32_t bq,
                           int32_t bk) {
