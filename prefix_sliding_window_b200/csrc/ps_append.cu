@@ -44,8 +44,10 @@ __device__ __forceinline__ void rotate8(const uint4& x1, const uint4& x2, const 
 }
 
 __global__ void __launch_bounds__(kAppendThreads) append_rope_kernel(const AppendArgs a) {
-  // the decode that usually follows may start its prologue now (it waits for this grid
-  // to complete before reading anything)
+  // Launched with programmatic serialization: wait for the previous kernel in the stream
+  // (inputs may come from it) before reading anything, then let the decode that usually
+  // follows start its prologue (it reads q and the newest row only after this grid ends).
+  pdl_wait();
   pdl_trigger();
   __shared__ float s_cos[kHalf];
   __shared__ float s_sin[kHalf];
@@ -252,8 +254,8 @@ cudaError_t launch_append(const AppendArgs& a, cudaStream_t stream) {
   const int64_t tokens = a.batch * a.T;
   if (tokens <= 0) return cudaSuccess;
   if (tokens > 0x7fffffff) return cudaErrorInvalidConfiguration;
-  append_rope_kernel<<<static_cast<unsigned>(tokens), kAppendThreads, 0, stream>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(append_rope_kernel, dim3(static_cast<unsigned>(tokens)),
+                    dim3(kAppendThreads), 0, stream, a);
 }
 
 }  // namespace ps

@@ -637,6 +637,7 @@ __global__ void __launch_bounds__(128)
   const int h = head / group, hh = head % group;
   const int64_t unit = (int64_t)b * hkv + h;
   pdl_wait();  // the decode kernel's pieces and spans must be complete
+  pdl_trigger();  // a programmatically serialized successor waits for this grid itself
   const int2 sp = reinterpret_cast<const int2*>(span)[unit];
   const int64_t total = (int64_t)hkv * pref[batch];
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
