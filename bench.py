@@ -449,17 +449,17 @@ def prefill_visible_pairs(S: int, lp: int, w: int) -> int:
     return n1 * (n1 + 1) // 2 + (S - n1) * cap
 
 
-def run_prefill(dev, steps: int = 10, warmup: int = 3):
-    """Masked prefill / truncated-backprop context forward: batch 4, 8192 tokens,
-    28/4/128, L_prefix 256, W 2048.  TFLOP/s counts unmasked FLOPs only
+def run_prefill(dev, steps: int = 10, warmup: int = 3, workload: str = "prefill_b4_s8192_w2048"):
+    """Masked prefill / truncated-backprop context forward (default: batch 4, 8192 tokens,
+    28/4/128, L_prefix 256, W 2048) and its backward.  TFLOP/s counts unmasked FLOPs only
     (4 * D per visible pair per query head)."""
     from prefix_sliding_window_b200 import binding as B
-    wl = synth.WORKLOADS["prefill_b4_s8192_w2048"]
+    wl = synth.WORKLOADS[workload]
     Bn, S, hq, hkv, lp, w = wl.batch, wl.seq, wl.n_q_heads, wl.n_kv_heads, wl.l_prefix, wl.window
     params = B.make_params(hq, hkv, D, lp, w, wl.rope_theta)
-    q = synth.normal_bf16((Bn, S, hq, D), synth.seed_for(3, 1), dev)
-    k = synth.normal_bf16((Bn, S, hkv, D), synth.seed_for(3, 2), dev)
-    v = synth.normal_bf16((Bn, S, hkv, D), synth.seed_for(3, 3), dev)
+    q = synth.normal_bf16((Bn, S, hq, D), synth.seed_for(wl.index, 1), dev)
+    k = synth.normal_bf16((Bn, S, hkv, D), synth.seed_for(wl.index, 2), dev)
+    v = synth.normal_bf16((Bn, S, hkv, D), synth.seed_for(wl.index, 3), dev)
     out = torch.empty_like(q)
     lse = torch.empty((Bn, hq, S), dtype=torch.float32, device=dev)
     n = B.ps_prefill_plan_tiles(params, S)
@@ -498,7 +498,8 @@ def run_prefill(dev, steps: int = 10, warmup: int = 3):
             "tflops_computed_tiles": round(computed / med / 1e12, 1),
             "unmasked_gflop": round(flops / 1e9, 1), "computed_gflop": round(computed / 1e9, 1),
             "tiles_per_head": {"full": n_full, "partial": n_part, "skip": nq * nq - n},
-            "launches_per_call": 2, "inputs": "Q 235 MB + K,V 67 MB per call (> L2)",
+            "launches_per_call": 2,
+            "inputs": f"Q {q.numel() * 2 / 1e6:.0f} MB + K,V {2 * k.numel() * 2 / 1e6:.0f} MB per call",
             "backward": run_prefill_bwd(dev, params, wl, q, k, v, out, lse, st, pairs, n,
                                         steps, warmup, peaks)}
 
@@ -510,7 +511,7 @@ def run_prefill_bwd(dev, params, wl, q, k, v, out, lse, st, pairs, n_tiles, step
     products over every planned 128 x 128 tile (masked elements included)."""
     from prefix_sliding_window_b200 import binding as B
     Bn, S, hq, hkv = wl.batch, wl.seq, wl.n_q_heads, wl.n_kv_heads
-    do = synth.normal_bf16((Bn, S, hq, D), synth.seed_for(3, 4), dev)
+    do = synth.normal_bf16((Bn, S, hq, D), synth.seed_for(wl.index, 4), dev)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     ws = torch.empty(B.ps_prefill_bwd_workspace_bytes(params, Bn, S), dtype=torch.uint8,
                      device=dev)
@@ -1174,6 +1175,9 @@ def main():
     ap.add_argument("--leg", default="main", choices=["main", "prefill", "sweep", "stack", "latency",
                                                       "shared", "reset", "pin", "paged"],
                     help="main: the driver's line; prefill/sweep/stack: one extra workload")
+    ap.add_argument("--prefill-workload", default="prefill_b4_s8192_w2048",
+                    choices=[k for k in synth.WORKLOADS if k.startswith("prefill")],
+                    help="workload of the prefill leg")
     ap.add_argument("--stack-batch", type=int, default=1024)
     ap.add_argument("--stack-distinct", type=int, default=6)
     ap.add_argument("--no-extras", action="store_true",
@@ -1193,7 +1197,8 @@ def main():
     dev = torch.device("cuda", local)
     if args.leg != "main":
         if args.leg == "prefill":
-            res = {"leg": "prefill", **run_prefill(dev, steps=args.steps, warmup=args.warmup)}
+            res = {"leg": "prefill", **run_prefill(dev, steps=args.steps, warmup=args.warmup,
+                                                   workload=args.prefill_workload)}
         elif args.leg == "sweep":
             res = run_sweep(dev)
         elif args.leg == "latency":

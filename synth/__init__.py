@@ -73,6 +73,11 @@ WORKLOADS = {
         name="decode_shared_b256_g64_lp2000_w4096", batch=256, n_q_heads=16, n_kv_heads=2,
         head_dim=128, l_prefix=2000, window=4096, pos_lo=8192, pos_hi=131072, group_size=64,
         index=6),
+    # a quarter of the truncated-backprop prefill (one sequence of 4096 tokens): small
+    # enough for a full profiler capture, still larger than L2
+    "prefill_b1_s4096_w2048": Workload(
+        name="prefill_b1_s4096_w2048", batch=1, n_q_heads=28, n_kv_heads=4, head_dim=128,
+        l_prefix=256, window=2048, seq=4096, index=7),
 }
 
 
