@@ -72,6 +72,24 @@ struct BwdArgs {
   __nv_bfloat16* dv;
 };
 
+// Bulk copy global -> shared with an L2 cache-policy hint.
+__device__ __forceinline__ void bulk_load_hint(void* smem_dst, const void* gsrc, uint32_t bytes,
+                                               uint64_t* bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1], %2, [%3], %4;" ::"r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(gsrc)), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
+}
+
+// 16-byte global store with the streaming (evict-first) cache operator: data written once
+// and read back much later by another kernel.
+__device__ __forceinline__ void st_global_cs(void* gdst, uint4 v) {
+  asm volatile("st.global.cs.v4.b32 [%0], {%1, %2, %3, %4};" ::"l"(gdst), "r"(v.x), "r"(v.y),
+               "r"(v.z), "r"(v.w)
+               : "memory");
+}
+
 // K-major 128x128 x 128x128 product: both operands [128 rows][128 cols] in two 64-column
 // 128-byte-swizzled halves; 16 columns = 32 B per step inside a half.
 __device__ __forceinline__ void mma_kmajor(uint32_t d_tmem, uint32_t a_addr, uint32_t b_addr) {
@@ -250,7 +268,9 @@ __global__ void __launch_bounds__(kDqThreads, 1)
           mbar_arrive_expect_tx(&full[s], 2 * kTileBytes);
           uint8_t* ds = sDS + s * kTileBytes;
           uint8_t* k = sK + s * kTileBytes;
-          bulk_load(ds, a.ds + (tile0 + j) * kT * kT, kTileBytes, &full[s]);
+          // each stored tile is read once: keep it from displacing the K tiles in L2
+          bulk_load_hint(ds, a.ds + (tile0 + j) * kT * kT, kTileBytes, &full[s],
+                         l2_policy_evict_first());
           tma_load_4d(k, &mk, 0, kvh, kt * kT, b, &full[s]);
           tma_load_4d(k + kBoxBytes, &mk, 64, kvh, kt * kT, b, &full[s]);
         }
@@ -717,8 +737,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int v = 0; v < 4; ++v) {
             const int chunk = (cs0 >> 3) + 4 * c + v;  // query cols [8 chunk, 8 chunk + 8)
-            *reinterpret_cast<uint4*>(ds_row + chunk * kT * 8) =
-                make_uint4(dk[4 * v], dk[4 * v + 1], dk[4 * v + 2], dk[4 * v + 3]);
+            st_global_cs(ds_row + chunk * kT * 8,
+                         make_uint4(dk[4 * v], dk[4 * v + 1], dk[4 * v + 2], dk[4 * v + 3]));
           }
         }
         tmem_wait_st();
