@@ -387,6 +387,17 @@ __global__ void __launch_bounds__(kThreads)
       int64_t ws = n - a.w;
       if (ws < a.lp) ws = a.lp;
       const int64_t delta = (int64_t)a.lp - ws;  // <= 0; 0 while nothing is evicted
+      // This lane forms the angles of frequencies d = lane and lane + 32; every lane then
+      // reads the 16 it needs (each is needed by the 8 lanes of one qq) with shuffles.
+      float cw[2], sw[2];
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) {
+        const double ang = double(delta) * a.inv_freq[lane + 32 * hf];
+        const double k = rint(ang * 0.15915494309189535);
+        double red = fma(-k, 6.2831854820251465, ang);
+        red = fma(-k, -1.748455600074497e-07, red);
+        sincosf(static_cast<float>(red), &sw[hf], &cw[hf]);
+      }
 #pragma unroll
       for (int ks = 0; ks < 4; ++ks) {
 #pragma unroll
@@ -397,12 +408,9 @@ __global__ void __launch_bounds__(kThreads)
           float c[2], sn[2];
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
-            const int d = 16 * ks + 8 * r + 2 * qq + e;
-            const double ang = double(delta) * a.inv_freq[d];
-            const double k = rint(ang * 0.15915494309189535);
-            double red = fma(-k, 6.2831854820251465, ang);
-            red = fma(-k, -1.748455600074497e-07, red);
-            sincosf(static_cast<float>(red), &sn[e], &c[e]);
+            const int d = 16 * ks + 8 * r + 2 * qq + e;  // d >> 5 == ks >> 1
+            c[e] = __shfl_sync(0xffffffffu, cw[ks >> 1], d & 31);
+            sn[e] = __shfl_sync(0xffffffffu, sw[ks >> 1], d & 31);
           }
           qp[ks][r] = pack_bf16x2(x1.x * c[0] - x2.x * sn[0], x1.y * c[1] - x2.y * sn[1]);
           qp[ks + 4][r] = pack_bf16x2(x2.x * c[0] + x1.x * sn[0], x2.y * c[1] + x1.y * sn[1]);

@@ -13,6 +13,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle as O
 import synth
 from prefix_sliding_window_b200 import binding as B
 from prefix_sliding_window_b200.cache import PrefixSlidingCache
@@ -191,3 +192,69 @@ def test_paged_pure_window_step_flow(cuda_device):
                                            lp, w, 1 / math.sqrt(D))
         assert_close(got[b], o, f"paged lp=0 b={b} p={p}")
         assert np.abs(gl[b] - l).max() < 2e-2, (b, p)
+
+
+def test_paged_full_size_b64_w4096(cuda_device):
+    """The bench's paged leg at full size: batch 64, 16/2/128, L_prefix 100, W 4096,
+    positions drawn in [8192, 131072]; the contiguous store's rows copied into 66 scattered
+    blocks per sequence.  Sampled sequences against the oracle, every sequence against the
+    contiguous decode."""
+    dev = cuda_device
+    wl = synth.WORKLOADS["decode_b64_w4096"]
+    hq, hkv, lp, w, Bn = wl.n_q_heads, wl.n_kv_heads, wl.l_prefix, wl.window, wl.batch
+    pos = synth.uniform_positions(Bn, wl.pos_lo, wl.pos_hi, synth.seed_for(2, 10), dev)
+    k_pre = synth.normal_bf16((Bn, lp, hkv, D), synth.seed_for(2, 11), dev)
+    v_pre = synth.normal_bf16((Bn, lp, hkv, D), synth.seed_for(2, 12), dev)
+    k_win = synth.normal_bf16((Bn, w, hkv, D), synth.seed_for(2, 13), dev)
+    v_win = synth.normal_bf16((Bn, w, hkv, D), synth.seed_for(2, 14), dev)
+    q_raw = synth.normal_bf16((Bn, hq, D), synth.seed_for(2, 15), dev)
+    params = B.make_params(hq, hkv, D, lp, w, wl.rope_theta)
+    cache = PrefixSlidingCache(Bn, hkv, lp, w, D, dev, fill=float("nan"))
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    B.ps_kv_append_rope(params, cache.struct, k_pre, v_pre, None,
+                        torch.zeros(Bn, dtype=torch.int64, device=dev), lp, st)
+    q = q_raw.clone()
+    # window positions p - W + 1 .. p; q rotated with the newest token
+    B.ps_kv_append_rope(params, cache.struct, k_win[:, :w - 1].contiguous(),
+                        v_win[:, :w - 1].contiguous(), None, pos - (w - 1), w - 1, st)
+    B.ps_kv_append_rope(params, cache.struct, k_win[:, w - 1:].contiguous(),
+                        v_win[:, w - 1:].contiguous(), q.view(Bn, 1, hq, D), pos, 1, st)
+    pre_blocks, ring_blocks = -(-lp // 64), w // 64
+    per_seq = pre_blocks + ring_blocks
+    n_blocks = Bn * per_seq
+    perm = torch.from_numpy(np.random.default_rng(21).permutation(n_blocks)).to(dev)
+    table = perm.view(Bn, per_seq).to(torch.int32)
+    nan = float("nan")
+    k_pool = torch.full((n_blocks, hkv, 64, D), nan, dtype=torch.bfloat16, device=dev)
+    v_pool = torch.full_like(k_pool, nan)
+    for src_pre, src_ring, pool in ((cache.k_prefix, cache.k_ring, k_pool),
+                                    (cache.v_prefix, cache.v_ring, v_pool)):
+        pre = torch.full((Bn, hkv, pre_blocks * 64, D), nan, dtype=torch.bfloat16, device=dev)
+        pre[:, :, :lp] = src_pre
+        blocks = torch.cat([pre.view(Bn, hkv, pre_blocks, 64, D),
+                            src_ring.view(Bn, hkv, ring_blocks, 64, D)], dim=2)
+        pool[table.long().view(-1)] = blocks.permute(0, 2, 1, 3, 4).reshape(n_blocks, hkv, 64, D)
+    ws = torch.empty(max(1, B.ps_decode_workspace_bytes(params, Bn)), dtype=torch.uint8,
+                     device=dev)
+    out = torch.full((Bn, hq, D), nan, dtype=torch.bfloat16, device=dev)
+    lse = torch.full((Bn, hq), nan, dtype=torch.float32, device=dev)
+    B.ps_decode_attn_paged(params, k_pool, v_pool, table, Bn, q, pos, out, lse, ws, st)
+    out_c = torch.empty_like(out)
+    B.ps_decode_attn(params, cache.struct, q, pos, out_c, None, ws, st)
+    torch.cuda.synchronize()
+    assert st.item() == 0, st.item()
+    assert torch.isfinite(out.float()).all()
+    assert (out.float() - out_c.float()).abs().max().item() < 1e-2
+    P = pos.cpu().numpy()
+    kp, vp, kw, vw, qr = f64(k_pre), f64(v_pre), f64(k_win), f64(v_win), f64(q_raw)
+    got, gl = f64(out), f64(lse)
+    for b in (0, 21, 42, 63):
+        p = int(P[b])
+        vis = O.visible_positions(p, lp, w)
+        base = p - (w - 1)
+        kr = np.stack([kp[b, x] if x < lp else kw[b, x - base] for x in vis])
+        vr = np.stack([vp[b, x] if x < lp else vw[b, x - base] for x in vis])
+        o, l = O.attend_gqa(O.rope_rotate(qr[b], p, THETA), O.rope_rotate(kr, vis[:, None], THETA),
+                            vr, 1 / math.sqrt(D))
+        assert_close(got[b], o, f"paged full size b={b}")
+        assert np.abs(gl[b] - l).max() < 2e-2
