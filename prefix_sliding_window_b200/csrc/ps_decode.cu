@@ -767,7 +767,9 @@ int64_t streamk_grid(int64_t batch, int32_t hkv, int64_t max_keys, bool force = 
   if (batch > kMaxStreamKSeqs || (units >= slots && !force)) return 0;
   const int64_t max_tiles = units * ((max_keys + kDecodeTile - 1) / kDecodeTile + 2);
   int64_t g = max_tiles / kMinTilesPerCta;
-  if (g > slots) g = slots;
+  // forced (prefix partials to fold in) with more units than CTA slots: about one unit per
+  // CTA over several waves streams faster than one wave of long shares
+  if (g > slots) g = (force && units > slots) ? units : slots;
   if (g < 1) g = 1;
   return g;
 }
