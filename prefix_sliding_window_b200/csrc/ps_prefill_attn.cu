@@ -360,15 +360,28 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     int64_t g = 0;
     int li = 0;
+    // plan offsets and first entry of this CTA's next item, loaded ahead (during the previous
+    // item's epilogue) so that a new item does not start with two dependent global loads
+    int nx_e0 = 0, nx_n = 0;
+    int2 nx_ent = make_int2(0, 0);
+    auto fetch_item = [&](int64_t itn) {
+      if (itn >= n_items) return;
+      int qt, b, head;
+      item_of(itn, qt, b, head);
+      nx_e0 = a.off[qt];
+      nx_n = a.off[qt + 1] - nx_e0;
+      nx_ent = nx_n > 0 ? reinterpret_cast<const int2*>(a.ent)[nx_e0] : make_int2(0, 0);
+    };
+    fetch_item(blockIdx.x);
     for (int64_t it = blockIdx.x; it < n_items; it += gridDim.x, ++li) {
       int qt, b, head;
       item_of(it, qt, b, head);
-      const int e0 = a.off[qt];
-      const int n = a.off[qt + 1] - e0;
+      const int e0 = nx_e0;
+      const int n = nx_n;
       const int64_t row = (int64_t)qt * kBq + r;
       float m = -INFINITY;  // running max of raw scores (softmax scale > 0 keeps the order)
       float l = 0.f;
-      int2 ent_next = n > 0 ? reinterpret_cast<const int2*>(a.ent)[e0] : make_int2(0, 0);
+      int2 ent_next = nx_ent;
       for (int j = 0; j < n; ++j, ++g) {
         const int s = static_cast<int>(g & 1);
         const int kt = ent_next.x;
@@ -475,6 +488,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) mbar_arrive(&p_ready[s * kGroups + wg]);
       }
       // ---------------------------------------------------------- epilogue of the item
+      fetch_item(it + gridDim.x);
       // O = (2^(m_0 - M) O_0 + 2^(m_1 - M) O_1) / (2^(m_0 - M) l_0 + 2^(m_1 - M) l_1)
       const bool fin = ok && n > 0 &&
                        mbar_wait(&pv_done[(g - 1) & 1], static_cast<uint32_t>(((g - 1) >> 1) & 1),
@@ -506,8 +520,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(o_free);
         const bool store = row < a.seq;
-        __nv_bfloat16* orow =
-            a.out + (((int64_t)b * a.seq + row) * a.hq + head) * kHeadDim + cs0;
+        // this row's 64 outputs as 8 chunks of 8 bf16
+        uint4 ch[8];
 #pragma unroll
         for (int c = 0; c < kCols / 32; ++c) {
           uint32_t pk[16];
@@ -516,12 +530,40 @@ __global__ void __launch_bounds__(kThreads, 1)
             pk[i] = cvt_bf16x2(
                 g0 * __uint_as_float(oa[c][2 * i]) + g1 * __uint_as_float(ob[c][2 * i]),
                 g0 * __uint_as_float(oa[c][2 * i + 1]) + g1 * __uint_as_float(ob[c][2 * i + 1]));
-          if (store) {
-            uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
 #pragma unroll
-            for (int v = 0; v < 4; ++v)
-              dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+          for (int v = 0; v < 4; ++v)
+            ch[4 * c + v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+        }
+        // Rows are a head stride apart in `out`, so one row per lane would make every store
+        // instruction touch 32 lines.  Transpose 8 x 8 chunk blocks across each 8-lane group
+        // (lane 8q + i then holds chunk i of rows 8q .. 8q + 7) so that each instruction
+        // writes 4 whole 128-byte row slices.
+        const int i8 = lane & 7;
+#pragma unroll
+        for (int d = 4; d > 0; d >>= 1) {
+          const bool hi = (i8 & d) != 0;
+#pragma unroll
+          for (int j0 = 0; j0 < 8; ++j0) {
+            if (j0 & d) continue;
+            const uint4 snd = hi ? ch[j0] : ch[j0 | d];
+            uint4 rcv;
+            rcv.x = __shfl_xor_sync(0xffffffffu, snd.x, d);
+            rcv.y = __shfl_xor_sync(0xffffffffu, snd.y, d);
+            rcv.z = __shfl_xor_sync(0xffffffffu, snd.z, d);
+            rcv.w = __shfl_xor_sync(0xffffffffu, snd.w, d);
+            if (hi)
+              ch[j0] = rcv;
+            else
+              ch[j0 | d] = rcv;
           }
+        }
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const int64_t rk = (int64_t)qt * kBq + 32 * (warp & 3) + (lane & ~7) + k;
+          if (rk < a.seq)
+            *reinterpret_cast<uint4*>(
+                a.out + (((int64_t)b * a.seq + rk) * a.hq + head) * kHeadDim + cs0 + 8 * i8) =
+                ch[k];
         }
         if (store && wg == 0 && a.lse)
           a.lse[((int64_t)b * a.hq + head) * a.seq + row] =
