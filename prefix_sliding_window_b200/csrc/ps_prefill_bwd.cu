@@ -118,6 +118,19 @@ __device__ __forceinline__ void mma_tmem_a(uint32_t d_tmem, uint32_t a_buf, uint
   }
 }
 
+// The half `hf` (B rows 64 grp + 32 hf .. + 31, A columns 64 grp + 16 hf .. + 15) of
+// mma_tmem_a.
+__device__ __forceinline__ void mma_tmem_a_half(uint32_t d_tmem, uint32_t a_buf, uint32_t b_addr,
+                                                int grp, int hf, bool first) {
+  constexpr uint32_t idesc = umma_idesc_bf16(128, 128, true);
+#pragma unroll
+  for (int i = 2 * hf; i < 2 * hf + 2; ++i) {
+    const int kk = 4 * grp + i;
+    const uint64_t bdesc = umma_desc_sw128(b_addr + kk * 2048, kBoxBytes, 1024);
+    umma_ts(d_tmem, a_buf + 64 * grp + 8 * i, bdesc, idesc, (first && i == 0) ? 0u : 1u);
+  }
+}
+
 __device__ __forceinline__ void load64(uint32_t taddr, float (&x)[kCols]) {
   uint32_t raw[2][32];
   tmem_ld32(taddr, raw[0]);
@@ -420,14 +433,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* st_empty = kv_full + 4;  // [2]
   uint64_t* s_full = kv_full + 6;
   uint64_t* dp_full = kv_full + 7;
-  uint64_t* p_ready = kv_full + 8;   // [2 groups]
-  uint64_t* ds_ready = kv_full + 10;  // [2 groups]
-  uint64_t* s_free = kv_full + 12;
-  uint64_t* dp_free = kv_full + 13;
-  uint64_t* acc_full = kv_full + 14;
-  uint64_t* acc_free = kv_full + 15;
-  uint64_t* mma_done = kv_full + 16;
-  int32_t* s_items = reinterpret_cast<int32_t*>(kv_full + 17);  // [kItemRing]
+  uint64_t* p_ready = kv_full + 8;    // [2 groups][2 halves of the group's 64 query columns]
+  uint64_t* ds_ready = kv_full + 12;  // [2 groups]
+  uint64_t* s_free = kv_full + 14;
+  uint64_t* dp_free = kv_full + 15;
+  uint64_t* acc_full = kv_full + 16;
+  uint64_t* acc_free = kv_full + 17;
+  uint64_t* mma_done = kv_full + 18;
+  int32_t* s_items = reinterpret_cast<int32_t*>(kv_full + 19);  // [kItemRing]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(s_items + kItemRing);
 
   const int64_t n_items = (int64_t)a.batch * a.hkv * a.nq;
@@ -445,7 +458,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < 2; ++s) {
       mbar_init(&st_full[s], 1);
       mbar_init(&st_empty[s], 1);
-      mbar_init(&p_ready[s], 4);
+      mbar_init(&p_ready[2 * s], 4);
+      mbar_init(&p_ready[2 * s + 1], 4);
       mbar_init(&ds_ready[s], 4);
     }
     mbar_init(s_full, 1);
@@ -603,15 +617,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = false;
             break;
           }
+          // each group publishes its P in two halves of 32 query columns: the dV products of
+          // a half go out as soon as it is in
 #pragma unroll
           for (int gr = 0; gr < kGroups; ++gr) {
-            if (!mbar_wait(&p_ready[gr], ph, a.status)) {
-              ok = false;
-              break;
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+              if (!mbar_wait(&p_ready[2 * gr + hf], ph, a.status)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+              mma_tmem_a_half(tmem + kKColDV, tmem + kKColS, do_addr + st * kTileBytes, gr, hf,
+                              j == 0 && gr == 0);
             }
-            tc_fence_after();
-            mma_tmem_a(tmem + kKColDV, tmem + kKColS, do_addr + st * kTileBytes, gr,
-                       j == 0 && gr == 0);
+            if (!ok) break;
           }
           if (!ok) break;
           umma_commit(s_free);
@@ -688,26 +708,32 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const float4* nl = reinterpret_cast<const float4*>(sNL + st * kT + cs0);
         const float4* nd4 = reinterpret_cast<const float4*>(sND + st * kT + cs0);
-        uint32_t pk[kCols / 2];
+        // P over this group's own columns, published in two halves of 32 query columns so
+        // that the first half's dV products overlap the second half's exponentials
 #pragma unroll
-        for (int i = 0; i < kCols / 4; ++i) {
-          const float4 l = nl[i];
-          const float2 e0 = unpack_f32x2(
-              ffma2(pack_f32x2(x[4 * i], x[4 * i + 1]), sl2x2, pack_f32x2(l.x, l.y)));
-          const float2 e1 = unpack_f32x2(
-              ffma2(pack_f32x2(x[4 * i + 2], x[4 * i + 3]), sl2x2, pack_f32x2(l.z, l.w)));
-          x[4 * i] = fast_exp2(e0.x);
-          x[4 * i + 1] = fast_exp2(e0.y);
-          x[4 * i + 2] = fast_exp2(e1.x);
-          x[4 * i + 3] = fast_exp2(e1.y);
-          pk[2 * i] = cvt_bf16x2(x[4 * i], x[4 * i + 1]);
-          pk[2 * i + 1] = cvt_bf16x2(x[4 * i + 2], x[4 * i + 3]);
+        for (int hf = 0; hf < 2; ++hf) {
+          uint32_t pk[kCols / 4];
+#pragma unroll
+          for (int ii = 0; ii < kCols / 8; ++ii) {
+            const int i = hf * (kCols / 8) + ii;
+            const float4 l = nl[i];
+            const float2 e0 = unpack_f32x2(
+                ffma2(pack_f32x2(x[4 * i], x[4 * i + 1]), sl2x2, pack_f32x2(l.x, l.y)));
+            const float2 e1 = unpack_f32x2(
+                ffma2(pack_f32x2(x[4 * i + 2], x[4 * i + 3]), sl2x2, pack_f32x2(l.z, l.w)));
+            x[4 * i] = fast_exp2(e0.x);
+            x[4 * i + 1] = fast_exp2(e0.y);
+            x[4 * i + 2] = fast_exp2(e1.x);
+            x[4 * i + 3] = fast_exp2(e1.y);
+            pk[2 * ii] = cvt_bf16x2(x[4 * i], x[4 * i + 1]);
+            pk[2 * ii + 1] = cvt_bf16x2(x[4 * i + 2], x[4 * i + 3]);
+          }
+          tmem_st16(lane_base + kKColS + cs0 + 16 * hf, pk);
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&p_ready[2 * wg + hf]);
         }
-        tmem_st32(lane_base + kKColS + cs0, pk);  // over this group's own columns
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&p_ready[wg]);
         ok = ok && __all_sync(0xffffffffu, mbar_wait(dp_full, ph, a.status));
         if (!ok) continue;
         tc_fence_after();
