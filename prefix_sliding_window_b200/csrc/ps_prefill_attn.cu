@@ -126,8 +126,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* v_full = k_empty + kKStages;             // [kVStages]
   uint64_t* v_empty = v_full + kVStages;             // [kVStages]
   uint64_t* s_full = v_empty + kVStages;             // [2]
-  uint64_t* p_ready = s_full + 2;                    // [2 buffers][kGroups]
-  uint64_t* pv_done = p_ready + 2 * kGroups;          // [2]: PV of tile g -> g & 1
+  uint64_t* p_ready = s_full + 2;                    // [2 buffers][kGroups][2 halves]
+  uint64_t* pv_done = p_ready + 4 * kGroups;          // [2]: PV of tile g -> g & 1
   uint64_t* o_free = pv_done + 2;
   uint64_t* mma_done = o_free + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
@@ -159,7 +159,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&s_full[s], 1);
-      for (int g = 0; g < kGroups; ++g) mbar_init(&p_ready[s * kGroups + g], 4);
+      for (int g = 0; g < kGroups; ++g) {
+        mbar_init(&p_ready[(s * kGroups + g) * 2], 4);
+        mbar_init(&p_ready[(s * kGroups + g) * 2 + 1], 4);
+      }
     }
     mbar_init(&pv_done[0], 1);
     mbar_init(&pv_done[1], 1);
@@ -314,17 +317,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           const uint32_t vb = v_addr + vs * kTileBytes;
-          // group gr's keys [64gr, 64gr+64) accumulate into its own O_gr, as soon as its P is in
+          // group gr's keys [64gr, 64gr+64) accumulate into its own O_gr, 32 keys at a time
+          // as soon as that half of its P is in
 #pragma unroll
-          for (int gr = 0; gr < kGroups; ++gr) {
-            if (!mbar_wait(&p_ready[s * kGroups + gr], static_cast<uint32_t>((g >> 1) & 1),
-                           a.status)) {
+          for (int gh = 0; gh < 2 * kGroups; ++gh) {
+            const int gr = gh >> 1, hf = gh & 1;
+            if (!mbar_wait(&p_ready[(s * kGroups + gr) * 2 + hf],
+                           static_cast<uint32_t>((g >> 1) & 1), a.status)) {
               ok = false;
               break;
             }
             tc_fence_after();
 #pragma unroll
-            for (int kk = 4 * gr; kk < 4 * gr + 4; ++kk) {
+            for (int kk = 4 * gr + 2 * hf; kk < 4 * gr + 2 * hf + 2; ++kk) {
               // B = V[16 keys][128 d]: MN-major, 64-column halves 16 KB apart (LBO), 8-key
               // groups 1024 B apart (SBO); 16 keys = 2048 B per step.
               // A = P_gr: group gr wrote its bf16 pairs over the first 32 of its own 64 S
@@ -467,25 +472,32 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float ms = (m == -INFINITY) ? 0.f : m * sl2;
         const uint64_t nms2 = pack_f32x2(-ms, -ms);
         uint64_t acc0 = pack_f32x2(0.f, 0.f), acc1 = acc0;
-        uint32_t pk[kCols / 2];
+        // P over this group's own S columns (the other group may not have read its scores),
+        // published in two halves of 32 keys: the PV products of the first half run while
+        // the second half's exponentials are formed
 #pragma unroll
-        for (int i = 0; i < kCols / 2; ++i) {
-          const float2 e = unpack_f32x2(ffma2(pack_f32x2(x[2 * i], x[2 * i + 1]), sl2x2, nms2));
-          const float p0 = fast_exp2(e.x), p1 = fast_exp2(e.y);
-          if (i & 1)
-            acc1 = fadd2(acc1, pack_f32x2(p0, p1));
-          else
-            acc0 = fadd2(acc0, pack_f32x2(p0, p1));
-          pk[i] = cvt_bf16x2(p0, p1);
+        for (int hf = 0; hf < 2; ++hf) {
+          uint32_t pk[kCols / 4];
+#pragma unroll
+          for (int ii = 0; ii < kCols / 4; ++ii) {
+            const int i = hf * (kCols / 4) + ii;
+            const float2 e =
+                unpack_f32x2(ffma2(pack_f32x2(x[2 * i], x[2 * i + 1]), sl2x2, nms2));
+            const float p0 = fast_exp2(e.x), p1 = fast_exp2(e.y);
+            if (i & 1)
+              acc1 = fadd2(acc1, pack_f32x2(p0, p1));
+            else
+              acc0 = fadd2(acc0, pack_f32x2(p0, p1));
+            pk[ii] = cvt_bf16x2(p0, p1);
+          }
+          tmem_st16(lane_base + col_s(s) + cs0 + 16 * hf, pk);
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&p_ready[(s * kGroups + wg) * 2 + hf]);
         }
-        // P over this group's own S columns: the other group may not have read its scores
-        tmem_st32(lane_base + col_s(s) + cs0, pk);
         const float2 a0 = unpack_f32x2(acc0), a1 = unpack_f32x2(acc1);
         l += (a0.x + a0.y) + (a1.x + a1.y);
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&p_ready[s * kGroups + wg]);
       }
       // ---------------------------------------------------------- epilogue of the item
       fetch_item(it + gridDim.x);
