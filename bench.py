@@ -1152,9 +1152,12 @@ def run_reference(args, world, rank):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total_t / args.steps * 1e3, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "impl": "reference",
-        "config": {"workload": WORKLOAD, "batch_per_gpu": wl.batch, "n_q_heads": wl.n_q_heads,
-                   "n_kv_heads": wl.n_kv_heads, "head_dim": D, "l_prefix": wl.l_prefix,
-                   "window": wl.window, "positions": f"U[{wl.pos_lo},{wl.pos_hi}]"},
+        "config": {"workload": WORKLOAD, "batch_per_gpu": wl.batch, "global_batch": wl.batch * world,
+                   "n_q_heads": wl.n_q_heads, "n_kv_heads": wl.n_kv_heads, "head_dim": D,
+                   "l_prefix": wl.l_prefix, "window": wl.window,
+                   "positions": f"U[{wl.pos_lo},{wl.pos_hi}]", "layers": 1,
+                   "step": "one decode step (append with Continue-PE RoPE + decode), float64 oracle",
+                   "parallelism": f"dp{world} (independent sequences, no collective)"},
         "cpu_baseline": {"value": round(value, 3), "unit": UNIT, "cores": _blas_threads(),
                          "kind": "oracle",
                          "sample": f"{per_step} sequence per step of {WORKLOAD}, float64 numpy"},
