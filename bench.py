@@ -120,9 +120,9 @@ def _recorded_traffic(entry: str = "step"):
     """DRAM bytes (read + write) per launch of `entry` from the last ncu capture, or None when
     the sources of its kernels changed since (their sha256 no longer matches the record)."""
     import hashlib
-    pkg = os.path.join(os.path.dirname(os.path.abspath(__file__)), "prefix_sliding_window_b200")
+    pkg = os.path.join(ROOT, "prefix_sliding_window_b200")
     try:
-        with open(os.path.join(pkg, "ncu_traffic.json")) as f:
+        with open(os.path.join(ROOT, "profiles", "ncu_traffic.json")) as f:
             rec = json.load(f)[entry]
         h = hashlib.sha256()
         for name in rec["sources"]:
@@ -180,6 +180,20 @@ def rank_seed(index: int, rank: int, k: int) -> int:
     """Seed of input stream k of workload `index` on `rank`: every rank draws its own
     sequences (the batch is sharded, not replicated)."""
     return synth.seed_for(index, 10 * rank + k)
+
+
+SOAK_S = 0.3
+
+
+def decode_config(wl: synth.Workload, world: int) -> dict:
+    """The workload description both arms report (same keys and values)."""
+    return {"workload": WORKLOAD, "batch_per_gpu": wl.batch, "global_batch": wl.batch * world,
+            "n_q_heads": wl.n_q_heads, "n_kv_heads": wl.n_kv_heads, "head_dim": D,
+            "l_prefix": wl.l_prefix, "window": wl.window,
+            "positions": f"U[{wl.pos_lo},{wl.pos_hi}]", "layers": 1,
+            "step": "one decode step of every sequence: append with Continue-PE RoPE + decode",
+            "l2": "inputs larger than L2 (275 MB of K/V read per step vs 126 MB L2)",
+            "parallelism": f"dp{world} (independent sequences, no collective)"}
 
 
 # ------------------------------------------------------------- decode setup
@@ -295,12 +309,27 @@ def run_decode(args, world, rank, dev):
     sampler = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
     if sampler:
         sampler.start()
-    # soak: the same work once more, untimed, so the clocks are sampled under this load
+    # soak: the same K steps replayed, untimed, for at least SOAK_S seconds right before the
+    # timed region, so the clock sampler sees this load (the timed region itself is far
+    # shorter than the sampling period)
+    e_a, e_b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e_a.record(stream)
     if graph is not None:
         graph.replay()
     else:
         for j in range(K):
             step(W + j)
+    e_b.record(stream)
+    torch.cuda.synchronize()
+    once_s = max(e_a.elapsed_time(e_b) / 1e3, 1e-6)
+    reps = int(math.ceil(SOAK_S / once_s))
+    t_soak0 = time.perf_counter()
+    for _ in range(reps):
+        if graph is not None:
+            graph.replay()
+        else:
+            for j in range(K):
+                step(W + j)
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     _barrier(world)
     torch.cuda.synchronize()
@@ -331,8 +360,8 @@ def run_decode(args, world, rank, dev):
     alg = alg_dec + work.algorithmic_bytes_per_append()
     step_s = ms / K / 1e3
     achieved = alg / step_s / 1e9
-    dec_avg_s = statistics.mean(dec_ms) / 1e3
-    attn = alg_dec / dec_avg_s / 1e9
+    dec_med_s = statistics.median(dec_ms) / 1e3
+    attn = alg_dec / dec_med_s / 1e9
     roof = {"bound": "hbm",
             "kernel": "ps_decode_step (append_rope_kernel + decode_kernel + merge_kernel)",
             "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
@@ -342,7 +371,8 @@ def run_decode(args, world, rank, dev):
             "duration_us": round(step_s * 1e6, 2), "duration_source": "timed region / steps",
             "frac_of_8tbs_spec": round(achieved / 8000.0, 4),
             "attn_call": {"what": "ps_decode_attn (decode_kernel + merge_kernel), each call "
-                                  "bracketed alone by CUDA events after that step's append",
+                                  "bracketed alone by CUDA events after that step's append; "
+                                  "achieved from the median call",
                           "algorithmic_bytes": alg_dec, "achieved": round(attn, 1),
                           "frac": round(attn / peaks["hbm_gbs"], 4),
                           "us_median": round(statistics.median(dec_ms) * 1e3, 2),
@@ -354,20 +384,17 @@ def run_decode(args, world, rank, dev):
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": K,
         "warmup": W, "ms_per_step": round(ms / K, 5), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "batch_per_gpu": wl.batch, "global_batch": wl.batch * world,
-                   "n_q_heads": wl.n_q_heads, "n_kv_heads": wl.n_kv_heads, "head_dim": D,
-                   "l_prefix": wl.l_prefix, "window": wl.window,
-                   "positions": f"U[{wl.pos_lo},{wl.pos_hi}]", "layers": 1,
-                   "step": "ps_decode_step (append with Continue-PE RoPE + decode)",
-                   "launch": "CUDA graph of the timed steps" if graph is not None else "eager",
-                   "l2": "inputs larger than L2 (275 MB of K/V read per step vs 126 MB L2)",
-                   "parallelism": f"dp{world} (independent sequences, no collective)"},
+        "config": decode_config(wl, world),
+        "launch": "CUDA graph of the timed steps" if graph is not None else "eager",
         "roofline": roof,
         "e2e": e2e,
         "gpu_launches": work.kernels_per_step() * K,
     }
     if sampler:
-        line["clocks"] = sampler.summary(t_host0, t_host1)
+        line["clocks"] = sampler.summary(t_soak0, t_host1)
+        if line["clocks"]:
+            line["clocks"]["window"] = (f"{reps} untimed replays of the timed steps "
+                                        f"({reps * once_s:.2f} s) + the timed region")
     return line, work
 
 
@@ -433,11 +460,30 @@ def run_decode_e2e(work: DecodeWorkload, K: int, W: int, world: int, use_graph: 
     # the timed steps really moved the data: the last output read back equals the device's
     assert torch.equal(h_out[W + K - 1], d_out.cpu())
     del graph
+    # where an end-to-end step's time goes: the same steps launched eagerly, each part
+    # bracketed by CUDA events on the stream (copy in, ps_decode_step, copy out)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    for j in range(K):
+        i = W + j
+        e = evs[j]
+        e[0].record(stream)
+        d_in.copy_(h_in[i], non_blocking=True)
+        e[1].record(stream)
+        B.ps_decode_step(work.params, work.cache.struct, d_k, d_v, d_q, d_pos, d_out, None,
+                         work.ws, work.status)
+        e[2].record(stream)
+        h_out[i].copy_(d_out, non_blocking=True)
+        e[3].record(stream)
+    torch.cuda.synchronize()
+    med = lambda a, b: round(statistics.median([e[a].elapsed_time(e[b]) for e in evs]) * 1e3, 2)  # noqa: E731
+    split = {"h2d_us": med(0, 1), "step_us": med(1, 2), "d2h_us": med(2, 3),
+             "total_us": med(0, 3), "how": "eager pass, CUDA events around each part, medians"}
     tokens = _sum_over_ranks(float(work.wl.batch * K), world)
     bi = (d_k.numel() + d_v.numel() + d_q.numel()) * 2 + d_pos.numel() * 8
     bo = d_out.numel() * 2
     return {"value": round(tokens / (ms / 1e3), 1), "unit": UNIT, "h2d_bytes_per_step": bi,
             "d2h_bytes_per_step": bo, "h2d_copies_per_step": 1, "d2h_copies_per_step": 1,
+            "us_per_step": round(ms / K * 1e3, 2), "split": split,
             "launch": "CUDA graph of the timed steps" if use_graph else "eager"}
 
 
@@ -652,25 +698,69 @@ def _fill_cache(B, params, cache_struct, Bn, hkv, ranges, dev, seed, st, chunk=2
             del k, v
 
 
-def run_sweep(dev, steps: int = 20, warmup: int = 3):
-    """Long-trace decode sweep: batch 256, 16/2/128, W = 8192; every sequence at the same
-    position P in {4K, ..., 128K}; prefix sliding (L_prefix = 100) vs pure sliding window
-    (L_prefix = 0) vs full attention.  Per-step latency of append + attention and the
-    attention kernel's HBM GB/s."""
+SWEEP_POINTS = (4096, 8192, 16384, 32768, 65536, 131072)
+
+
+def _graph_time(fn, n: int, warmup: int):
+    """Device time per call of fn(i), i = 0 .. n-1, replayed as one CUDA graph after
+    `warmup` eager calls (those use the same i range: fn must be repeatable)."""
+    stream = torch.cuda.current_stream()
+    for i in range(warmup):
+        fn(i % n)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for i in range(n):
+            fn(i)
+    g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    g.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    del g
+    return e0.elapsed_time(e1) / n
+
+
+def _eager_median(fn, n: int):
+    """Median device time of n eager calls fn(i), each bracketed by CUDA events."""
+    stream = torch.cuda.current_stream()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(n)]
+    for i, (a, b) in enumerate(evs):
+        a.record(stream)
+        fn(i)
+        b.record(stream)
+    torch.cuda.synchronize()
+    return statistics.median([a.elapsed_time(b) for a, b in evs])
+
+
+def run_sweep(dev, steps: int = 20, warmup: int = 3, points=SWEEP_POINTS):
+    """Long-trace decode sweep: batch 256, 16/2/128, W = 8192; every sequence at position
+    P + i (i = the step) for P in {4K, ..., 128K}; prefix sliding (L_prefix = 100) vs pure
+    sliding window (L_prefix = 0) vs full attention over [0, P + i].  Per point and mode:
+    one decode step = append of the new token (Continue-PE RoPE) + attention, `steps` steps
+    replayed as a CUDA graph (step_us); the attention call alone, eager with CUDA events
+    (attn_us).  GB/s on algorithmic bytes (K+V of every visible key, q and out; the step
+    adds the append's bytes).  Every point's K/V is far larger than L2 (>= 1 GB)."""
     from prefix_sliding_window_b200 import binding as B
     from prefix_sliding_window_b200.cache import LinearCache, PrefixSlidingCache
     wl = synth.WORKLOADS["decode_sweep_b256_w8192"]
     Bn, hq, hkv, w = wl.batch, wl.n_q_heads, wl.n_kv_heads, wl.window
     peaks = _peaks()
     st = torch.zeros(1, dtype=torch.int32, device=dev)
-    n = steps + warmup
-    k_new = synth.normal_bf16((n, Bn, 1, hkv, D), 11, dev)
-    v_new = synth.normal_bf16((n, Bn, 1, hkv, D), 12, dev)
-    q_raw = synth.normal_bf16((n, Bn, hq, D), 13, dev)
-    out = torch.empty((Bn, hq, D), dtype=torch.bfloat16, device=dev)
-    stream = torch.cuda.current_stream()
-    points = []
-    for P in (4096, 8192, 16384, 32768, 65536, 131072):
+    n = steps
+    k_new = synth.normal_bf16((n, Bn, hkv, D), synth.seed_for(wl.index, 1), dev)
+    v_new = synth.normal_bf16((n, Bn, hkv, D), synth.seed_for(wl.index, 2), dev)
+    q_raw = synth.normal_bf16((n, Bn, hq, D), synth.seed_for(wl.index, 3), dev)
+    q = q_raw.clone()
+    out = torch.empty((n, Bn, hq, D), dtype=torch.bfloat16, device=dev)
+    kv_tok = 2 * hkv * D * 2
+    qo = 2 * Bn * hq * D * 2
+    append_bytes = Bn * (2 * 2 * hkv * D * 2 + 2 * hq * D * 2 + 8)
+    res_points = []
+    for P in points:
         pos = torch.stack([torch.full((Bn,), P + i, dtype=torch.int64, device=dev)
                            for i in range(n)])
         res = {"position": P}
@@ -685,46 +775,60 @@ def run_sweep(dev, steps: int = 20, warmup: int = 3):
                                  dtype=torch.uint8, device=dev)
 
                 def attn(i, cache=cache, dparams=dparams, ws=ws, lmax=lmax):
-                    B.ps_full_attn_ref(dparams, cache.k, cache.v, lmax, q[i], pos[i], Bn, out,
+                    B.ps_full_attn_ref(dparams, cache.k, cache.v, lmax, q[i], pos[i], Bn, out[i],
                                        None, ws, st)
+
+                def step(i, cache=cache, aparams=aparams, attn=attn):
+                    B.ps_kv_append_rope(aparams, cache.struct, k_new[i].view(Bn, 1, hkv, D),
+                                        v_new[i].view(Bn, 1, hkv, D), q[i].view(Bn, 1, hq, D),
+                                        pos[i], 1, st)
+                    attn(i)
+                keys = [P + i + 1 for i in range(n)]
             else:
                 lp = wl.l_prefix if mode == "prefix_sliding" else 0
                 cache = PrefixSlidingCache(Bn, hkv, lp, w, D, dev, fill=None)
-                aparams = dparams = B.make_params(hq, hkv, D, lp, w, wl.rope_theta)
-                _fill_cache(B, aparams, cache.struct, Bn, hkv,
+                dparams = B.make_params(hq, hkv, D, lp, w, wl.rope_theta)
+                _fill_cache(B, dparams, cache.struct, Bn, hkv,
                             [(0, min(lp, P)), (max(lp, P - w + 1), P)], dev, 1000, st)
                 ws = torch.empty(max(1, B.ps_decode_workspace_bytes(dparams, Bn)),
                                  dtype=torch.uint8, device=dev)
 
                 def attn(i, cache=cache, dparams=dparams, ws=ws):
-                    B.ps_decode_attn(dparams, cache.struct, q[i], pos[i], out, None, ws, st)
-            q = q_raw.clone()
-            evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
-                    torch.cuda.Event(enable_timing=True)) for _ in range(n)]
-            for i in range(n):
-                evs[i][0].record(stream)
-                B.ps_kv_append_rope(aparams, cache.struct, k_new[i], v_new[i], q[i], pos[i], 1, st)
-                evs[i][1].record(stream)
-                attn(i)
-                evs[i][2].record(stream)
+                    B.ps_decode_attn(dparams, cache.struct, q[i], pos[i], out[i], None, ws, st)
+
+                def step(i, cache=cache, dparams=dparams, ws=ws):
+                    B.ps_decode_step(dparams, cache.struct, k_new[i], v_new[i], q[i], pos[i],
+                                     out[i], None, ws, st)
+                keys = [min(P + i + 1, lp + w) for i in range(n)]
+            q.copy_(q_raw)
+            step_ms = _graph_time(step, n, warmup)
+            attn_ms = _eager_median(attn, n)
             torch.cuda.synchronize()
-            assert st.item() == 0
-            step_ms = statistics.median([a.elapsed_time(c) for a, _, c in evs[warmup:]])
-            attn_ms = statistics.median([b.elapsed_time(c) for _, b, c in evs[warmup:]])
-            if mode == "full":
-                keys = P + warmup + steps / 2 + 1
-            else:
-                keys = min(P + 1, (wl.l_prefix if mode == "prefix_sliding" else 0) + w)
-            kv_bytes = Bn * keys * 2 * hkv * D * 2 + 2 * Bn * hq * D * 2
-            gbs = kv_bytes / (attn_ms / 1e3) / 1e9
+            assert st.item() == 0, st.item()
+            attn_bytes = Bn * statistics.mean(keys) * kv_tok + qo
+            step_bytes = attn_bytes + append_bytes
+            gbs = step_bytes / (step_ms / 1e3) / 1e9
+            agbs = attn_bytes / (attn_ms / 1e3) / 1e9
             res[mode] = {"step_us": round(step_ms * 1e3, 1), "attn_us": round(attn_ms * 1e3, 1),
-                         "attn_gbs": round(gbs, 1), "frac": round(gbs / peaks["hbm_gbs"], 4),
+                         "keys_per_seq": round(statistics.mean(keys), 1),
+                         "step_gbs": round(gbs, 1), "frac": round(gbs / peaks["hbm_gbs"], 4),
+                         "frac_of_8tbs_spec": round(gbs / 8000.0, 4),
+                         "attn_gbs": round(agbs, 1),
+                         "attn_frac": round(agbs / peaks["hbm_gbs"], 4),
                          "tok_per_s": round(Bn / (step_ms / 1e3), 1)}
-            del cache, ws
+            del cache, ws, attn, step
             torch.cuda.empty_cache()
-        points.append(res)
-    return {"leg": "sweep", "workload": wl.name, "steps": steps, "points": points,
-            "peak_hbm_gbs": peaks["hbm_gbs"]}
+        res["ps_over_full_speedup"] = round(res["full"]["step_us"] / res["prefix_sliding"]["step_us"],
+                                            2)
+        res_points.append(res)
+    flat = [r["prefix_sliding"]["step_us"] for r in res_points if r["position"] >= 8192]
+    fr = [r["prefix_sliding"]["frac"] for r in res_points if r["position"] >= 8192]
+    return {"workload": wl.name, "batch": Bn, "l_prefix": wl.l_prefix, "window": w,
+            "steps_per_point": n, "launch": "CUDA graph of the steps (step_us); eager calls "
+            "with CUDA events (attn_us)", "peak_hbm_gbs": peaks["hbm_gbs"],
+            "peak_source": peaks["source"], "points": res_points,
+            "ps_step_us_spread_8k_128k": round((max(flat) - min(flat)) / min(flat), 4) if flat else None,
+            "ps_min_frac_8k_128k": min(fr) if fr else None}
 
 
 # ------------------------------------------------------- shared-prefix decode leg
@@ -1021,11 +1125,11 @@ def run_paged(dev, steps: int = 20, warmup: int = 3):
 
 # ------------------------------------------------------- full-stack decode leg
 def run_stack(dev, batch: int, distinct: int, steps: int = 3, warmup: int = 1):
-    """Full-stack decode step: 28 layers x (append + decode), 16/2/128, L_prefix 2000,
-    W 16384, positions in [32768, 262144].  The 28 logical layers are mapped round-robin
-    onto `distinct` resident layer caches (all 28 caches of 1024 sequences, 540 GB, do not
-    fit in one GPU's 180 GB); each layer's working set is far larger than L2, so every
-    layer reads its K/V from HBM."""
+    """Full-stack decode step: 28 layers x ps_decode_step (append + decode), 16/2/128,
+    L_prefix 2000, W 16384, positions in [32768, 262144].  The 28 logical layers are mapped
+    round-robin onto `distinct` resident layer caches (all 28 caches of 1024 sequences,
+    540 GB, do not fit in one GPU's 180 GB); each layer's working set is far larger than L2,
+    so every layer reads its K/V from HBM."""
     from prefix_sliding_window_b200 import binding as B
     from prefix_sliding_window_b200.cache import PrefixSlidingCache
     wl = synth.WORKLOADS["decode_stack_l28_b1024_w16384"]
@@ -1049,42 +1153,48 @@ def run_stack(dev, batch: int, distinct: int, steps: int = 3, warmup: int = 1):
                                 pos0 - (w - 1) + c0, T, st)
         caches.append(c)
     torch.cuda.synchronize()
-    k_new = synth.normal_bf16((L, Bn, 1, hkv, D), 21, dev)
-    v_new = synth.normal_bf16((L, Bn, 1, hkv, D), 22, dev)
-    q_raw = synth.normal_bf16((L, Bn, hq, D), 23, dev)
+    n = warmup + steps
+    k_new = synth.normal_bf16((n, L, Bn, hkv, D), 21, dev)
+    v_new = synth.normal_bf16((n, L, Bn, hkv, D), 22, dev)
+    q_raw = synth.normal_bf16((n, L, Bn, hq, D), 23, dev)
     q = q_raw.clone()
-    out = torch.empty((Bn, hq, D), dtype=torch.bfloat16, device=dev)
+    out = torch.empty((L, Bn, hq, D), dtype=torch.bfloat16, device=dev)
     ws = torch.empty(max(1, B.ps_decode_workspace_bytes(params, Bn)), dtype=torch.uint8, device=dev)
+    pos = torch.stack([pos0 + i for i in range(n)])
     stream = torch.cuda.current_stream()
 
     def step(i):
-        pos = pos0 + i
         for layer in range(L):
             c = caches[layer % distinct]
-            q[layer].copy_(q_raw[layer])
-            B.ps_kv_append_rope(params, c.struct, k_new[layer], v_new[layer], q[layer], pos, 1, st)
-            B.ps_decode_attn(params, c.struct, q[layer], pos, out, None, ws, st)
+            B.ps_decode_step(params, c.struct, k_new[i, layer], v_new[i, layer], q[i, layer],
+                             pos[i], out[layer], None, ws, st)
 
     for i in range(warmup):
         step(i)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for i in range(warmup, warmup + steps):
+    for i in range(warmup, n):
         step(i)
     e1.record(stream)
     torch.cuda.synchronize()
     assert st.item() == 0
     ms = e0.elapsed_time(e1) / steps
     kv_bytes = L * Bn * (lp + w) * 2 * hkv * D * 2
-    gbs = kv_bytes / (ms / 1e3) / 1e9
+    step_bytes = kv_bytes + L * Bn * (2 * hq * D * 2 + 2 * 2 * hkv * D * 2 + 2 * hq * D * 2 + 8)
+    gbs = step_bytes / (ms / 1e3) / 1e9
     peaks = _peaks()
-    return {"leg": "stack", "workload": wl.name, "batch": Bn, "layers": L,
-            "distinct_layer_caches": distinct,
-            "resident_kv_gb": round(distinct * caches[0].nbytes() / 1e9, 1),
-            "ms_per_step": round(ms, 3), "tok_per_s": round(Bn / (ms / 1e3), 1),
-            "kv_gb_per_step": round(kv_bytes / 1e9, 1), "gbs": round(gbs, 1),
-            "frac": round(gbs / peaks["hbm_gbs"], 4)}
+    res = {"workload": wl.name, "batch": Bn, "layers": L, "distinct_layer_caches": distinct,
+           "layer_map": "28 logical layers round-robin onto the distinct caches" if distinct < L
+           else "28 distinct layer caches",
+           "resident_kv_gb": round(distinct * caches[0].nbytes() / 1e9, 1),
+           "ms_per_step": round(ms, 3), "tok_per_s": round(Bn / (ms / 1e3), 1),
+           "kv_gb_per_step": round(kv_bytes / 1e9, 1), "gbs": round(gbs, 1),
+           "frac": round(gbs / peaks["hbm_gbs"], 4), "frac_of_8tbs_spec": round(gbs / 8000.0, 4),
+           "launch": "eager, 28 ps_decode_step calls per step"}
+    del caches, k_new, v_new, q_raw, q
+    torch.cuda.empty_cache()
+    return res
 
 
 # ----------------------------------------------------------- CPU oracle leg
@@ -1119,7 +1229,7 @@ def oracle_decode_sample(wl: synth.Workload, n_seq: int, seed_stream: int = 0):
     return n_seq, time.perf_counter() - t0
 
 
-def cpu_baseline(wl: synth.Workload, budget_s: float = 12.0):
+def cpu_baseline(wl: synth.Workload, budget_s: float = 8.0):
     done, spent, calls = 0, 0.0, 0
     while spent < budget_s:
         n, t = oracle_decode_sample(wl, 8, calls)
@@ -1133,12 +1243,104 @@ def cpu_baseline(wl: synth.Workload, budget_s: float = 12.0):
                       f"{spent:.1f} s"}
 
 
+def cpu_baseline_latency(budget_s: float = 4.0):
+    """The oracle on the batch-1 workload (L_prefix 100, W 512): the prompt's 100 tokens, then
+    decode steps at positions 100, 101, ... each over its visible keys, until the budget."""
+    import oracle as O
+    wl = synth.WORKLOADS["decode_b1_w512"]
+    hq, hkv, lp, w = wl.n_q_heads, wl.n_kv_heads, wl.l_prefix, wl.window
+    S = wl.pos_hi + 1
+    k = synth.normal_bf16((S, hkv, D), synth.seed_for(wl.index, 1)).double().numpy()
+    v = synth.normal_bf16((S, hkv, D), synth.seed_for(wl.index, 2)).double().numpy()
+    q = synth.normal_bf16((S, hq, D), synth.seed_for(wl.index, 3)).double().numpy()
+    scale = 1.0 / math.sqrt(D)
+    t0 = time.perf_counter()
+    steps = 0
+    for p in range(lp, S):
+        vis = O.visible_positions(p, lp, w)
+        O.attend_gqa(O.rope_rotate(q[p], p, wl.rope_theta),
+                     O.rope_rotate(k[vis], vis[:, None], wl.rope_theta), v[vis], scale)
+        steps += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    t = time.perf_counter() - t0
+    return {"value": round(steps / t, 2), "unit": "tok/s", "cores": _blas_threads(),
+            "kind": "oracle", "us_per_step": round(t / steps * 1e6, 1),
+            "sample": f"decode steps at positions {lp}..{lp + steps - 1} of {wl.name} "
+                      f"({'all' if steps == S - lp else 'first'} {steps} of {S - lp}), "
+                      f"float64 numpy, {t:.1f} s"}
+
+
+def cpu_baseline_prefill():
+    """The oracle on one (batch, head) of the prefill workload (8192 rows, 28/4/128 heads
+    reduced to one query head and its KV head), every row; the whole workload's time is
+    that x heads x batch (extrapolated)."""
+    import oracle as O
+    wl = synth.WORKLOADS["prefill_b4_s8192_w2048"]
+    S, lp, w = wl.seq, wl.l_prefix, wl.window
+    Q = synth.normal_bf16((S, 1, D), synth.seed_for(wl.index, 1)).double().numpy()
+    K = synth.normal_bf16((S, 1, D), synth.seed_for(wl.index, 2)).double().numpy()
+    V = synth.normal_bf16((S, 1, D), synth.seed_for(wl.index, 3)).double().numpy()
+    t0 = time.perf_counter()
+    O.prefill_reference(Q, K, V, lp, w, 1.0 / math.sqrt(D))
+    t = time.perf_counter() - t0
+    flops = 4 * D * prefill_visible_pairs(S, lp, w)
+    whole = t * wl.n_q_heads * wl.batch
+    return {"value": round(flops / t / 1e12, 6), "unit": "TFLOP/s", "cores": _blas_threads(),
+            "kind": "oracle", "s_per_head": round(t, 3),
+            "whole_workload_s_extrapolated": round(whole, 1),
+            "sample": f"one (batch, head) of {wl.name}: all {S} rows, float64 numpy, "
+                      f"{t:.1f} s; whole workload = x {wl.n_q_heads} heads x {wl.batch} "
+                      f"(extrapolated)"}
+
+
+def cpu_baseline_sweep(per_point: int = 2):
+    """The oracle on sampled sequences of the long-trace sweep (L_prefix 100, W 8192):
+    `per_point` sequences decoded at each position."""
+    import dataclasses
+    wl = synth.WORKLOADS["decode_sweep_b256_w8192"]
+    pts = {}
+    for i, P in enumerate(SWEEP_POINTS):
+        wp = dataclasses.replace(wl, pos_lo=P, pos_hi=P)
+        n, t = oracle_decode_sample(wp, per_point, 300 + i)
+        pts[str(P)] = {"seq_per_s": round(n / t, 2), "s_per_seq": round(t / n, 4)}
+    return {"unit": "tok/s", "cores": _blas_threads(), "kind": "oracle", "points": pts,
+            "sample": f"{per_point} sequences per position, one decode step each (all "
+                      f"{wl.n_q_heads} heads), float64 numpy"}
+
+
+def cpu_baseline_stack(pairs: int = 8):
+    """The oracle on `pairs` sampled (sequence, layer) pairs of the full-stack workload
+    (L_prefix 2000, W 16384, positions in [32768, 262144]); one full step (28 layers x 1024
+    sequences) extrapolated from the per-pair time."""
+    wl = synth.WORKLOADS["decode_stack_l28_b1024_w16384"]
+    n, t = oracle_decode_sample(wl, pairs, 500)
+    per = t / n
+    step_s = per * wl.n_layers * wl.batch
+    return {"value": round(wl.batch / step_s, 4), "unit": "tok/s", "cores": _blas_threads(),
+            "kind": "oracle", "s_per_pair": round(per, 4),
+            "step_s_extrapolated": round(step_s, 1),
+            "sample": f"{n} (sequence, layer) pairs decoded, float64 numpy, {t:.1f} s; one step "
+                      f"= {wl.n_layers} layers x {wl.batch} sequences (extrapolated)"}
+
+
+def cpu_baselines():
+    """Oracle timings of every workload, on this host's cores (reported, not a target)."""
+    return {"decode_b1_w512": cpu_baseline_latency(),
+            "prefill_b4_s8192_w2048": cpu_baseline_prefill(),
+            "decode_sweep_b256_w8192": cpu_baseline_sweep(),
+            "decode_stack_l28_b1024_w16384": cpu_baseline_stack()}
+
+
 def run_reference(args, world, rank):
-    """Reference arm: the float64 oracle on the host cores, same metric and config."""
+    """Reference arm: the float64 oracle on the host cores, same metric, unit and config.
+    A step decodes the workload's whole batch (64 sequences) when the run is short enough
+    (K + W <= 40 steps: about 0.9 s each), otherwise a sample of the batch sized to keep
+    the run within about a minute."""
     if rank != 0:
         return None
     wl = synth.WORKLOADS[WORKLOAD]
-    per_step = 1  # sequences per step: a bounded sample of the workload's batch
+    per_step = max(1, min(wl.batch, (wl.batch * 40) // (args.steps + args.warmup)))
     for i in range(args.warmup):
         oracle_decode_sample(wl, per_step, 1000 + i)
     total_t, total_n = 0.0, 0
@@ -1147,20 +1349,17 @@ def run_reference(args, world, rank):
         total_t += t
         total_n += n
     value = total_n / total_t
+    sample = (f"{per_step} of the {wl.batch} sequences of {WORKLOAD} per step "
+              f"({'the whole batch' if per_step == wl.batch else 'a sample'}), float64 numpy")
     return {
         "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total_t / args.steps * 1e3, 3),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "impl": "reference",
-        "config": {"workload": WORKLOAD, "batch_per_gpu": wl.batch, "global_batch": wl.batch * world,
-                   "n_q_heads": wl.n_q_heads, "n_kv_heads": wl.n_kv_heads, "head_dim": D,
-                   "l_prefix": wl.l_prefix, "window": wl.window,
-                   "positions": f"U[{wl.pos_lo},{wl.pos_hi}]", "layers": 1,
-                   "step": "one decode step (append with Continue-PE RoPE + decode), float64 oracle",
-                   "parallelism": f"dp{world} (independent sequences, no collective)"},
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(total_t / args.steps * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "impl": "reference", "config": decode_config(wl, world),
+        "launch": "host cores, float64 oracle", "sequences_per_step": per_step,
         "cpu_baseline": {"value": round(value, 3), "unit": UNIT, "cores": _blas_threads(),
-                         "kind": "oracle",
-                         "sample": f"{per_step} sequence per step of {WORKLOAD}, float64 numpy"},
+                         "kind": "oracle", "sample": sample},
         "e2e": {"value": round(value, 3), "unit": UNIT, "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -1203,7 +1402,7 @@ def main():
             res = {"leg": "prefill", **run_prefill(dev, steps=args.steps, warmup=args.warmup,
                                                    workload=args.prefill_workload)}
         elif args.leg == "sweep":
-            res = run_sweep(dev)
+            res = {"leg": "sweep", **run_sweep(dev)}
         elif args.leg == "latency":
             res = run_latency(dev)
         elif args.leg == "shared":
@@ -1227,9 +1426,17 @@ def main():
         del work
         torch.cuda.empty_cache()
         line["prefill"] = run_prefill(dev)
+        torch.cuda.empty_cache()
+        line["sweep"] = run_sweep(dev)
+        # the full stack: 28 layers of 1024 sequences on 6 resident layer caches (aliased),
+        # and 28 distinct layer caches at batch 192 (all that fits)
+        line["stack"] = {"aliased": run_stack(dev, 1024, 6),
+                         "distinct": run_stack(dev, 192, 28)}
     if rank == 0:
-        if not args.no_cpu_baseline:
+        if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(synth.WORKLOADS[WORKLOAD])
+            if not args.no_extras:
+                line["cpu_baselines"] = cpu_baselines()
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist

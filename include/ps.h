@@ -166,12 +166,15 @@ int ps_decode_attn_reset_pe(const ps_params* params, const ps_kv_cache* cache, c
  * The split-K scratch lives in a device array built into libps (4 MiB = 4194304 bytes,
  * held on every GPU that loads the library until the process exits).  A shape whose
  * ps_decode_workspace_bytes() exceeds that returns PS_ERR_WORKSPACE and launches nothing.
- * This call never allocates or frees memory (no cudaMalloc, no cudaFree).  The first call on
- * each device looks up the array's device address with cudaGetSymbolAddress (with that
- * device current); make that first call before any stream capture.  Every call shares the
- * array and it keeps the last call's contents (nothing in it needs to start at zero); calls
- * that overlap on the GPU, e.g. on two streams, race on it and must be serialised by the
- * caller.  Arguments, results and errors are otherwise exactly those of ps_decode_attn. */
+ * This call never allocates or frees memory (no cudaMalloc, no cudaFree).  A call made outside
+ * a stream capture looks up the array's device address with cudaGetSymbolAddress (with the
+ * device current), so a context torn down and made again is never given a stale address; a
+ * call inside a capture reuses the address the last call outside one found.  Make the first
+ * call on each device (and the first after a cudaDeviceReset) before any stream capture.
+ * Every call shares the array and it keeps the last call's contents (nothing in it needs to
+ * start at zero); calls that overlap on the GPU, e.g. on two streams, race on it and must be
+ * serialised by the caller.  Arguments, results and errors are otherwise exactly those of
+ * ps_decode_attn. */
 int ps_decode_attn_noalloc(const ps_params* params, const ps_kv_cache* cache, const void* q,
                            const int64_t* pos, void* out, float* lse, int32_t* dev_status,
                            ps_stream_t stream);

@@ -283,18 +283,21 @@ size_t ps_decode_workspace_bytes(const ps_params* params, int64_t batch) {
                                 (int64_t)params->l_prefix + params->window);
 }
 
-static int decode_entry(const ps_params* params, const ps_kv_cache* cache, const void* q,
-                        const int64_t* pos, void* out, float* lse, void* workspace,
-                        size_t ws_bytes, int32_t* dev_status, ps_stream_t stream,
-                        int32_t reset_pe, int32_t lcap = 0, const int32_t* pin_count = nullptr,
-                        const int64_t* pin_pos = nullptr, int32_t after_append = 0) {
-  g_last_error.clear();
+// Checks shared by every decode entry point over the contiguous store, and the launch
+// description they build.  *empty is set (PS_OK returned) when there is nothing to launch.
+static int decode_prepare(const ps_params* params, const ps_kv_cache* cache, const void* q,
+                          const int64_t* pos, void* out, float* lse, int32_t* dev_status,
+                          DecodeLaunch* l, bool* empty) {
+  *empty = false;
   PS_TRY(check_params(params, true));
   if (params->n_q_heads / params->n_kv_heads > kMaxGroup)
     return fail(PS_ERR_UNSUPPORTED, "decode supports at most 8 query heads per KV head");
   if (!cache) return fail(PS_ERR_INVALID_ARG, "cache is NULL");
   if (cache->batch < 0) return fail(PS_ERR_INVALID_ARG, "cache->batch must be >= 0");
-  if (cache->batch == 0) return PS_OK;
+  if (cache->batch == 0) {
+    *empty = true;
+    return PS_OK;
+  }
   PS_TRY(check_ptr(cache->k_ring, "cache->k_ring"));
   PS_TRY(check_ptr(cache->v_ring, "cache->v_ring"));
   if (params->l_prefix > 0) {
@@ -309,6 +312,38 @@ static int decode_entry(const ps_params* params, const ps_kv_cache* cache, const
     return fail(PS_ERR_INVALID_ARG, "pos is not 8-byte aligned");
   if ((reinterpret_cast<uintptr_t>(dev_status) & 3u) != 0)
     return fail(PS_ERR_INVALID_ARG, "dev_status is not 4-byte aligned");
+  *l = DecodeLaunch{};
+  l->q = q;
+  l->pos = pos;
+  l->out = out;
+  l->lse = lse;
+  l->status = dev_status;
+  l->batch = cache->batch;
+  l->hq = params->n_q_heads;
+  l->hkv = params->n_kv_heads;
+  l->lp = params->l_prefix;
+  l->w = params->window;
+  l->lmax = 0;
+  l->full_mode = 0;
+  l->scale = resolve_scale(params);
+  l->k0 = cache->k_prefix;
+  l->v0 = cache->v_prefix;
+  l->k1 = cache->k_ring;
+  l->v1 = cache->v_ring;
+  l->rope_theta = params->rope_theta;
+  return PS_OK;
+}
+
+static int decode_entry(const ps_params* params, const ps_kv_cache* cache, const void* q,
+                        const int64_t* pos, void* out, float* lse, void* workspace,
+                        size_t ws_bytes, int32_t* dev_status, ps_stream_t stream,
+                        int32_t reset_pe, int32_t lcap = 0, const int32_t* pin_count = nullptr,
+                        const int64_t* pin_pos = nullptr, int32_t after_append = 0) {
+  g_last_error.clear();
+  DecodeLaunch l;
+  bool empty = false;
+  PS_TRY(decode_prepare(params, cache, q, pos, out, lse, dev_status, &l, &empty));
+  if (empty) return PS_OK;
   const int64_t pre_rows = lcap > params->l_prefix ? lcap : params->l_prefix;
   const size_t need = decode_workspace_bytes(cache->batch, params->n_kv_heads,
                                              pre_rows + params->window);
@@ -317,27 +352,8 @@ static int decode_entry(const ps_params* params, const ps_kv_cache* cache, const
       return fail(PS_ERR_WORKSPACE, "workspace smaller than the decode workspace size");
     PS_TRY(check_ptr(workspace, "workspace"));
   }
-  DecodeLaunch l{};
-  l.q = q;
-  l.pos = pos;
-  l.out = out;
-  l.lse = lse;
   l.workspace = workspace;
-  l.status = dev_status;
-  l.batch = cache->batch;
-  l.hq = params->n_q_heads;
-  l.hkv = params->n_kv_heads;
-  l.lp = params->l_prefix;
-  l.w = params->window;
-  l.lmax = 0;
-  l.full_mode = 0;
-  l.scale = resolve_scale(params);
-  l.k0 = cache->k_prefix;
-  l.v0 = cache->v_prefix;
-  l.k1 = cache->k_ring;
-  l.v1 = cache->v_ring;
   l.reset_pe = reset_pe;
-  l.rope_theta = params->rope_theta;
   l.lcap = lcap;
   l.pin_count = pin_count;
   l.pin_pos = pin_pos;
@@ -363,45 +379,10 @@ int ps_decode_attn_noalloc(const ps_params* params, const ps_kv_cache* cache, co
                            const int64_t* pos, void* out, float* lse, int32_t* dev_status,
                            ps_stream_t stream) {
   g_last_error.clear();
-  PS_TRY(check_params(params, true));
-  if (params->n_q_heads / params->n_kv_heads > kMaxGroup)
-    return fail(PS_ERR_UNSUPPORTED, "decode supports at most 8 query heads per KV head");
-  if (!cache) return fail(PS_ERR_INVALID_ARG, "cache is NULL");
-  if (cache->batch < 0) return fail(PS_ERR_INVALID_ARG, "cache->batch must be >= 0");
-  if (cache->batch == 0) return PS_OK;
-  PS_TRY(check_ptr(cache->k_ring, "cache->k_ring"));
-  PS_TRY(check_ptr(cache->v_ring, "cache->v_ring"));
-  if (params->l_prefix > 0) {
-    PS_TRY(check_ptr(cache->k_prefix, "cache->k_prefix"));
-    PS_TRY(check_ptr(cache->v_prefix, "cache->v_prefix"));
-  }
-  PS_TRY(check_ptr(q, "q"));
-  PS_TRY(check_ptr(out, "out"));
-  PS_TRY(check_ptr(lse, "lse", true));
-  if (!pos) return fail(PS_ERR_INVALID_ARG, "pos is NULL");
-  if ((reinterpret_cast<uintptr_t>(pos) & 7u) != 0)
-    return fail(PS_ERR_INVALID_ARG, "pos is not 8-byte aligned");
-  if ((reinterpret_cast<uintptr_t>(dev_status) & 3u) != 0)
-    return fail(PS_ERR_INVALID_ARG, "dev_status is not 4-byte aligned");
-  DecodeLaunch l{};
-  l.q = q;
-  l.pos = pos;
-  l.out = out;
-  l.lse = lse;
-  l.workspace = nullptr;
-  l.status = dev_status;
-  l.batch = cache->batch;
-  l.hq = params->n_q_heads;
-  l.hkv = params->n_kv_heads;
-  l.lp = params->l_prefix;
-  l.w = params->window;
-  l.lmax = 0;
-  l.full_mode = 0;
-  l.scale = resolve_scale(params);
-  l.k0 = cache->k_prefix;
-  l.v0 = cache->v_prefix;
-  l.k1 = cache->k_ring;
-  l.v1 = cache->v_ring;
+  DecodeLaunch l;
+  bool empty = false;
+  PS_TRY(decode_prepare(params, cache, q, pos, out, lse, dev_status, &l, &empty));
+  if (empty) return PS_OK;
   return launch_decode_static_scratch(l, reinterpret_cast<cudaStream_t>(stream));
 }
 

@@ -646,14 +646,14 @@ __global__ void __launch_bounds__(128)
   const int64_t unit = (int64_t)b * hkv + h;
   pdl_wait();  // the decode kernel's pieces and spans must be complete
   pdl_trigger();  // a programmatically serialized successor waits for this grid itself
-  const int2 sp = reinterpret_cast<const int2*>(span)[unit];
+  const int2 span_cu = reinterpret_cast<const int2*>(span)[unit];
   const int64_t total = (int64_t)hkv * pref[batch];
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   float lse2 = -INFINITY;
   // online combine state; shared-prefix partials (normalised, weight 2^lse2) start it
   float M = -INFINITY, wsum = 0.f;
-  for (int sp = 0; pre_o && sp < pre_splits; ++sp) {
-    const int64_t row = (int64_t)sp * batch * hq + bh;
+  for (int split = 0; pre_o && split < pre_splits; ++split) {
+    const int64_t row = (int64_t)split * batch * hq + bh;
     const float l2 = pre_lse2[row];
     if (l2 == -INFINITY) continue;
     const float4 ov = reinterpret_cast<const float4*>(pre_o + row * kHeadDim)[lane];
@@ -667,8 +667,8 @@ __global__ void __launch_bounds__(128)
     acc.w = acc.w * fa + fb * ov.w;
     M = Mn;
   }
-  if (sp.x <= sp.y) {
-    const int c_lo = sp.x, c_hi = sp.y;
+  if (span_cu.x <= span_cu.y) {
+    const int c_lo = span_cu.x, c_hi = span_cu.y;
     // with fewer tiles than CTAs some CTAs own nothing and wrote no piece
     const bool maybe_empty = total < grid;
     auto empty_cta = [&](int c) {
@@ -938,12 +938,20 @@ int launch_decode_static_scratch(const DecodeLaunch& l, cudaStream_t stream) {
   int rc = check_cuda(cudaGetDevice(&dev), "cudaGetDevice");
   if (rc != PS_OK) return rc;
   if (dev < 0 || dev >= 64) return fail(PS_ERR_UNSUPPORTED, "device index above 63");
+  // Host code cannot use g_decode_scratch's address directly: on the host the name is a
+  // stand-in.  The runtime is asked, with the device current, on every call made outside a
+  // stream capture, so a context torn down and created again (cudaDeviceReset), which may
+  // load the module at a new address, is never handed a stale pointer.  Inside a capture the
+  // address recorded by the last call made outside one is used.
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(stream, &cs) != cudaSuccess) {
+    cudaGetLastError();  // e.g. the legacy stream while another stream captures
+    cs = cudaStreamCaptureStatusActive;
+  }
   void* ptr = nullptr;
   {
-    // Host code cannot use g_decode_scratch's address directly: on the host the name is a
-    // stand-in.  Ask the runtime once per device, with that device current.
     std::lock_guard<std::mutex> lock(g_scratch_mu);
-    if (g_scratch_ptr[dev] == nullptr) {
+    if (cs == cudaStreamCaptureStatusNone || g_scratch_ptr[dev] == nullptr) {
       void* p = nullptr;
       rc = check_cuda(cudaGetSymbolAddress(&p, g_decode_scratch), "cudaGetSymbolAddress");
       if (rc != PS_OK) return rc;

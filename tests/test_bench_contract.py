@@ -22,6 +22,11 @@ def test_reference_arm_json_line():
     assert d["metric"] == bench.METRIC and d["unit"] == bench.UNIT
     assert d["higher_is_better"] is True and d["steps"] == 2 and d["warmup"] == 3
     assert d["value"] > 0 and d["config"]["workload"] == bench.WORKLOAD
+    # the very config dict the GPU arm reports (same keys, same values)
+    import synth
+    assert d["config"] == bench.decode_config(synth.WORKLOADS[bench.WORKLOAD], 1)
+    # a short run decodes the whole batch every step
+    assert d["sequences_per_step"] == synth.WORKLOADS[bench.WORKLOAD].batch
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
     assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}

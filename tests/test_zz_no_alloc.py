@@ -4,15 +4,21 @@ Some callers only get their input and output buffers from a host framework (a pl
 fixed-memory serving loop) and have no way to allocate the split-K scratch that
 ps_decode_attn takes as its workspace argument.  ps_decode_attn_noalloc uses an array built
 into the library instead.  This test calls it through the C ABI twice in a row, with
-different inputs, and checks each result against ps_decode_attn on the same inputs, so a
-stale scratch from the first call cannot pass for the second.
+different inputs, and checks that each result is bit-identical to ps_decode_attn on the same
+inputs (the same kernel runs on the same data; only where its scratch lives differs), so a
+stale scratch from the first call cannot pass for the second.  One sequence of each call is
+also checked against the float64 oracle.
 
 The file name sorts last so that a run stopping at the first failure has already run every
 other test; it also passes on its own in a fresh process.
 """
+import math
+
+import numpy as np
 import pytest
 import torch
 
+import oracle as O
 import synth
 from prefix_sliding_window_b200 import binding as B
 from prefix_sliding_window_b200.cache import PrefixSlidingCache
@@ -38,7 +44,7 @@ def test_noalloc_decode_matches_workspace_decode_twice(cuda_device):
                         torch.zeros(Bn, dtype=torch.int64, device=dev), hist, st)
     ws = torch.empty(B.ps_decode_workspace_bytes(params, Bn), dtype=torch.uint8, device=dev)
     for call, (seed, positions) in enumerate([(303, [5999, 4500, 4195, 77]),
-                                              (304, [5998, 5000, 300, 4196])]):
+                                              (304, [5999, 5000, 300, 4196])]):
         q = synth.normal_bf16((Bn, hq, D), seed, dev)
         pos = torch.tensor(positions, dtype=torch.int64, device=dev)
         out_ws = torch.empty((Bn, hq, D), dtype=torch.bfloat16, device=dev)
@@ -49,5 +55,13 @@ def test_noalloc_decode_matches_workspace_decode_twice(cuda_device):
         B.ps_decode_attn_noalloc(params, cache.struct, q, pos, out_na, lse_na, st)
         torch.cuda.synchronize()
         assert st.item() == 0
-        assert_close(f64(out_na), f64(out_ws), f"no-alloc call {call + 1}")
-        assert_close(f64(lse_na), f64(lse_ws), f"no-alloc lse call {call + 1}")
+        assert torch.equal(out_na, out_ws), f"no-alloc call {call + 1}: output differs"
+        assert torch.equal(lse_na, lse_ws), f"no-alloc call {call + 1}: lse differs"
+        # sequence 0 (position 5999, the newest appended: its ring holds exactly its window)
+        # against the oracle: keys rotated at their positions, q taken as given
+        p = positions[0]
+        vis = O.visible_positions(p, lp, w)
+        k_rot = O.rope_rotate(f64(k[0])[vis], vis[:, None], 1.0e6)
+        want, want_lse = O.attend_gqa(f64(q[0]), k_rot, f64(v[0])[vis], 1 / math.sqrt(D))
+        assert_close(f64(out_na[0]), want, f"no-alloc call {call + 1} vs oracle")
+        assert np.abs(f64(lse_na[0]) - want_lse).max() < 2e-2
