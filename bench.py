@@ -5,7 +5,8 @@ Default workload: steady-state batched decode on one layer (batch 64, 16 query /
 heads, head_dim 128, bf16, L_prefix = 100, W = 4096, positions drawn in [8192, 131072],
 KV prefilled with RoPE at every absolute position).  One step = one decode step of the
 whole batch through ps_decode_step: the new token's append (Continue-PE RoPE of k and q,
-ring write), then split-K decode + merge.  Prints ONE JSON line on rank 0.
+ring write) folded into the split-K decode, then the merge.  Prints ONE JSON line on
+rank 0.
 
   python bench.py [--gpus N --steps K --warmup W] [--impl reference]
 
@@ -240,7 +241,9 @@ class DecodeWorkload:
         torch.cuda.synchronize()
 
     def kernels_per_step(self) -> int:
-        return 2 + (1 if self.splits_used else 0)
+        """ps_decode_step launches the decode kernel (append folded in) and, when the batch
+        is split across CTAs (stream-K), the merge kernel."""
+        return 1 + (1 if self.splits_used else 0)
 
     def append(self, i):
         B = self.B
@@ -363,7 +366,7 @@ def run_decode(args, world, rank, dev):
     dec_med_s = statistics.median(dec_ms) / 1e3
     attn = alg_dec / dec_med_s / 1e9
     roof = {"bound": "hbm",
-            "kernel": "ps_decode_step (append_rope_kernel + decode_kernel + merge_kernel)",
+            "kernel": "ps_decode_step (decode_kernel with the append folded in + merge_kernel)",
             "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
             "frac": round(achieved / peaks["hbm_gbs"], 4),
             "traffic": args.traffic if args.traffic is not None else _recorded_traffic("step"),
@@ -398,11 +401,50 @@ def run_decode(args, world, rank, dev):
     return line, work
 
 
+class MappedHostBuffer:
+    """Pinned host memory mapped into the device address space (cudaHostAlloc with
+    cudaHostAllocMapped); device_ptr() is the address kernels write through, host() a uint8
+    CPU tensor over the same bytes."""
+
+    def __init__(self, nbytes: int):
+        from cuda.bindings import runtime as cudart
+        self._rt = cudart
+        err, self.hp = cudart.cudaHostAlloc(nbytes, cudart.cudaHostAllocMapped)
+        if err != cudart.cudaError_t.cudaSuccess:
+            raise RuntimeError(f"cudaHostAlloc: {err}")
+        err, self.dp = cudart.cudaHostGetDevicePointer(self.hp, 0)
+        if err != cudart.cudaError_t.cudaSuccess:
+            raise RuntimeError(f"cudaHostGetDevicePointer: {err}")
+        self.nbytes = nbytes
+
+    def device_view(self, offset: int):
+        ptr = self.dp + offset
+
+        class _P:
+            def data_ptr(self):
+                return ptr
+        return _P()
+
+    def host(self) -> torch.Tensor:
+        import ctypes
+        arr = (ctypes.c_uint8 * self.nbytes).from_address(self.hp)
+        return torch.frombuffer(arr, dtype=torch.uint8)
+
+    def __del__(self):
+        try:
+            self._rt.cudaFreeHost(self.hp)
+        except Exception:
+            pass
+
+
 def run_decode_e2e(work: DecodeWorkload, K: int, W: int, world: int, use_graph: bool = True):
-    """Same metric through the C ABI with host buffers: every step copies its inputs
-    (q, k_new, v_new, pos: packed in one pinned host buffer, so one DMA) host->device and
-    reads out device->host, in stream order: step i+1's inputs are copied after step i's
-    output has been read back, as a decode loop whose next inputs depend on it would."""
+    """Same metric through the C ABI with host buffers: every step copies its inputs (q,
+    k_new, v_new, pos: packed in one pinned host buffer, so one DMA) host->device, and
+    ps_decode_step writes that step's output straight into pinned host memory mapped into the
+    device's address space (the merge kernel's stores cross PCIe; no second copy).  In stream
+    order: step i+1's inputs are copied after step i's output has been written, as a decode
+    loop whose next inputs depend on it would.  The same steps with a device->host DMA of the
+    output instead are reported beside it (dma_out)."""
     B = work.B
     dev = work.dev
     n = K + W
@@ -424,43 +466,57 @@ def run_decode_e2e(work: DecodeWorkload, K: int, W: int, world: int, use_graph: 
         return d_in[offs[name]:offs[name] + nb].view(like.dtype).view(like.shape)
     d_k, d_v = view("k", work.k_new[0]), view("v", work.v_new[0])
     d_q, d_pos = view("q", work.q[0]), view("pos", work.pos[0])
+    out_bytes = work.out[0].numel() * 2
+    h_map = MappedHostBuffer(n * out_bytes)
     h_out = torch.empty((n,) + tuple(work.out.shape[1:]), dtype=torch.bfloat16).pin_memory()
     d_out = torch.empty_like(work.out[0])
     stream = torch.cuda.current_stream()
 
-    def step(i):
+    def step_mapped(i):
+        d_in.copy_(h_in[i], non_blocking=True)
+        B.ps_decode_step(work.params, work.cache.struct, d_k, d_v, d_q, d_pos,
+                         h_map.device_view(i * out_bytes), None, work.ws, work.status)
+
+    def step_dma(i):
         d_in.copy_(h_in[i], non_blocking=True)
         B.ps_decode_step(work.params, work.cache.struct, d_k, d_v, d_q, d_pos, d_out, None,
                          work.ws, work.status)
         h_out[i].copy_(d_out, non_blocking=True)
 
-    for i in range(W):
-        step(i)
-    torch.cuda.synchronize()
-    graph = None
-    if use_graph:
-        # the same K steps (copy in, step, copy out, in stream order) as one CUDA graph
-        graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph):
+    def timed(step):
+        for i in range(W):
+            step(i)
+        torch.cuda.synchronize()
+        graph = None
+        if use_graph:
+            # the K steps (copy in, step, output to the host, in stream order) as one graph
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph):
+                for j in range(K):
+                    step(W + j)
+            torch.cuda.synchronize()
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        _barrier(world)
+        ev0.record(stream)
+        if graph is not None:
+            graph.replay()
+        else:
             for j in range(K):
                 step(W + j)
+        ev1.record(stream)
         torch.cuda.synchronize()
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    _barrier(world)
-    ev0.record(stream)
-    if graph is not None:
-        graph.replay()
-    else:
-        for j in range(K):
-            step(W + j)
-    ev1.record(stream)
-    torch.cuda.synchronize()
-    ms = _max_over_ranks(ev0.elapsed_time(ev1), world)
-    assert work.status.item() == 0, f"device status {work.status.item()}"
-    # the timed steps really moved the data: the last output read back equals the device's
-    assert torch.equal(h_out[W + K - 1], d_out.cpu())
-    del graph
-    # where an end-to-end step's time goes: the same steps launched eagerly, each part
+        assert work.status.item() == 0, f"device status {work.status.item()}"
+        del graph
+        return _max_over_ranks(ev0.elapsed_time(ev1), world)
+
+    ms = timed(step_mapped)
+    # the timed steps really moved the data: the last output on the host equals the device
+    # run's output of the same step
+    last = h_map.host()[(n - 1) * out_bytes:n * out_bytes].view(torch.bfloat16)
+    assert torch.equal(last.view(work.out[0].shape), work.out[n - 1].cpu())
+    ms_dma = timed(step_dma)
+    assert torch.equal(h_out[n - 1], work.out[n - 1].cpu())
+    # where an end-to-end step's time goes: the DMA variant launched eagerly, each part
     # bracketed by CUDA events on the stream (copy in, ps_decode_step, copy out)
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
     for j in range(K):
@@ -477,13 +533,20 @@ def run_decode_e2e(work: DecodeWorkload, K: int, W: int, world: int, use_graph: 
     torch.cuda.synchronize()
     med = lambda a, b: round(statistics.median([e[a].elapsed_time(e[b]) for e in evs]) * 1e3, 2)  # noqa: E731
     split = {"h2d_us": med(0, 1), "step_us": med(1, 2), "d2h_us": med(2, 3),
-             "total_us": med(0, 3), "how": "eager pass, CUDA events around each part, medians"}
+             "total_us": med(0, 3), "how": "DMA variant, eager, CUDA events around each part, "
+             "medians"}
     tokens = _sum_over_ranks(float(work.wl.batch * K), world)
     bi = (d_k.numel() + d_v.numel() + d_q.numel()) * 2 + d_pos.numel() * 8
     bo = d_out.numel() * 2
+    del h_map
     return {"value": round(tokens / (ms / 1e3), 1), "unit": UNIT, "h2d_bytes_per_step": bi,
-            "d2h_bytes_per_step": bo, "h2d_copies_per_step": 1, "d2h_copies_per_step": 1,
-            "us_per_step": round(ms / K * 1e3, 2), "split": split,
+            "d2h_bytes_per_step": bo, "h2d_copies_per_step": 1,
+            "d2h": "out written by ps_decode_step into mapped pinned host memory",
+            "us_per_step": round(ms / K * 1e3, 2),
+            "dma_out": {"value": round(tokens / (ms_dma / 1e3), 1),
+                        "us_per_step": round(ms_dma / K * 1e3, 2),
+                        "d2h": "one cudaMemcpyAsync of out per step"},
+            "split": split,
             "launch": "CUDA graph of the timed steps" if use_graph else "eager"}
 
 

@@ -38,8 +38,8 @@ __device__ __forceinline__ void rotate8(const uint4& x1, const uint4& x2, const 
     const float2 v = __bfloat1622float2(bb[e]);
     const float c0 = cs[2 * e], c1 = cs[2 * e + 1];
     const float s0 = sn[2 * e], s1 = sn[2 * e + 1];
-    o1[e] = __floats2bfloat162_rn(u.x * c0 - v.x * s0, u.y * c1 - v.y * s1);
-    o2[e] = __floats2bfloat162_rn(v.x * c0 + u.x * s0, v.y * c1 + u.y * s1);
+    o1[e] = __floats2bfloat162_rn(rope_lo(u.x, v.x, c0, s0), rope_lo(u.y, v.y, c1, s1));
+    o2[e] = __floats2bfloat162_rn(rope_hi(u.x, v.x, c0, s0), rope_hi(u.y, v.y, c1, s1));
   }
 }
 
@@ -128,16 +128,9 @@ __global__ void __launch_bounds__(kAppendThreads) append_rope_kernel(const Appen
   if (threadIdx.x < n_items) load(threadIdx.x, x1, x2);
 
   if (threadIdx.x < kHalf) {
-    // angle = p * inv_f[i] in float64, reduced to [-pi, pi] by subtracting k * 2*pi with
-    // 2*pi split in two parts (Cody-Waite): the first has 24 significant bits, so k * part1
-    // is exact for |k| < 2^29; the second carries the rest of 2*pi in double precision.
-    // The remainder is small, so the fp32 sincosf of it is accurate to ~1e-7.
-    const double ang = double(p) * a.inv_freq[threadIdx.x];
-    const double k = rint(ang * 0.15915494309189535);
-    double red = fma(-k, 6.2831854820251465, ang);
-    red = fma(-k, -1.748455600074497e-07, red);
+    // angle = p * inv_f[i], formed and reduced modulo 2 pi in float64 (rope_cos_sin)
     float sf, cf;
-    sincosf(static_cast<float>(red), &sf, &cf);
+    rope_cos_sin(double(p), a.inv_freq[threadIdx.x], &cf, &sf);
     s_cos[threadIdx.x] = cf;
     s_sin[threadIdx.x] = sf;
   }

@@ -25,6 +25,11 @@
 //    P^T goes from the accumulator layout to the operand layout with movmatrix; softmax is
 //    online, in base 2, with warp-shuffle max reductions;
 //  * the four warps' (m, l, O) states are merged through shared memory.
+// ps_decode_step runs the same kernel with the one-token append folded in (kFused): the
+// consumers rotate the raw query at its position themselves, and the warp whose 16 keys
+// include the sequence's newest row writes the rotated new key and the new value over that
+// row of the shared-memory tile before reading it, and stores them in the cache.  No separate
+// append kernel runs, so the decode streams from its first cycle.
 #include <cuda_bf16.h>
 #include <math.h>
 
@@ -51,6 +56,12 @@ constexpr int kMinTilesPerCta = 4;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
+// decode_kernel modes (a template parameter: each mode's extra registers stay out of the
+// others)
+constexpr int kPlain = 0;  // ps_decode_attn and its variants
+constexpr int kReset = 1;  // Reset PE: prefix tiles see the query at its Reset-PE id
+constexpr int kFused = 2;  // ps_decode_step: the one-token append folded in
+
 // shared memory: stages | barriers (2 x STAGES) | flush area [2][32 lanes][36] | prefix
 constexpr size_t kFlushFloats = 2 * 32 * 36;
 constexpr size_t smem_bytes(int stages) {
@@ -75,12 +86,17 @@ struct DecodeArgs {
   float scale_log2;
   int32_t skip_prefix;     // shared-prefix decode: window rows only
   // Reset PE: prefix tiles use the query rotated by delta = L_prefix + |window| - 1 - p
-  // more (its Reset-PE id); inv_freq = theta^(-2i/D) in float64
+  // more (its Reset-PE id); inv_freq = theta^(-2i/D) in float64 (also used by kFused)
   int32_t reset_pe;
-  // launched right after a one-token append at pos (ps_decode_step): only the tile holding
-  // each sequence's newest row and the rotated q depend on that kernel, so everything else
-  // may stream before the programmatic wait
-  int32_t after_append;
+  // kFused: raw new key / value [batch, Hkv, D] of the token at pos, and the stores their
+  // rotated key and value go to (prefix rows [batch, Hkv, lp, D], ring [batch, Hkv, W, D]);
+  // q holds the raw query and receives the rotated one
+  const __nv_bfloat16* k_new;
+  const __nv_bfloat16* v_new;
+  __nv_bfloat16* k_pre;
+  __nv_bfloat16* v_pre;
+  __nv_bfloat16* k_ring;
+  __nv_bfloat16* v_ring;
   // paged store: K/V of every (sequence, KV head) in 64-row blocks of one pool
   // [n_blocks][Hkv][64][D]; logical block i of sequence b is table[b * table_stride + i]
   // (prefix blocks first, then W / 64 ring blocks)
@@ -216,10 +232,14 @@ __device__ __forceinline__ void store_state(float* dst, float m0, float m1, floa
   dst[35] = l1;
 }
 
-// RESET: Reset-PE mode (prefix tiles see the query at its renumbered id).  A template
-// flag, not a run-time one, so the plain decode carries none of its registers.
-template <int STAGES, bool RESET>
-__global__ void __launch_bounds__(kThreads)
+// MODE: kPlain, kReset (prefix tiles see the query at its renumbered id) or kFused (the
+// one-token append folded in).  A template parameter, not a run-time flag, so the plain
+// decode carries none of the other modes' registers.
+// Two CTAs of 5 warps per SM need at most 168 registers per thread (10 warps on 4 SMSPs: 3
+// warps x 168 x 32 fit one SMSP's 16K registers); the bound keeps every mode there, and the
+// stream-K grid is sized for two per SM.
+template <int STAGES, int MODE>
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
     decode_kernel(const __grid_constant__ CUtensorMap mk0, const __grid_constant__ CUtensorMap mv0,
                   const __grid_constant__ CUtensorMap mk1, const __grid_constant__ CUtensorMap mv1,
                   const DecodeArgs a) {
@@ -247,8 +267,8 @@ __global__ void __launch_bounds__(kThreads)
     prefetch_tensormap(&mv1);
   }
   // launched with programmatic serialization: everything above overlapped the previous
-  // kernel (usually the append); positions, q and the cache are read only after this
-  if (!a.after_append) pdl_wait();
+  // kernel; positions, q and the cache are read only after this
+  pdl_wait();
   pdl_trigger();  // the merge may be scheduled now; it waits for this grid to finish
 
   // ---------------------------------------------------------------- work range
@@ -317,7 +337,6 @@ __global__ void __launch_bounds__(kThreads)
     if (lane == 0 && ntiles > 0) {
       const uint64_t pol = l2_policy_evict_first();
       int issued = 0;
-      bool waited = !a.after_append;
       TileWalker pw = wk;
       for (int i = 0; i < ntiles; ++i, ++pw.t) {
         if (pw.t >= pw.pu1) pw.next_unit(a, pref);
@@ -325,16 +344,6 @@ __global__ void __launch_bounds__(kThreads)
         const uint32_t ph = (i / STAGES) & 1;
         if (i >= STAGES && !mbar_wait(&empty[s], ph ^ 1, a.status)) break;
         const DecodeTile d = tiling_tile(pw.tiling, static_cast<int32_t>(pw.t - pw.pu));
-        if (!waited) {
-          // the newest row of sequence b: prefix row p, or ring slot (p - Lp) mod W
-          const int64_t p = a.pos[pw.b];
-          const bool pre = a.full_mode || p < a.lp;
-          const int64_t row = pre ? p : (p - a.lp) % a.w;
-          if (d.map_id == (pre ? 0 : 1) && row >= d.row0 + d.lo && row < d.row0 + d.hi) {
-            pdl_wait();
-            waited = true;
-          }
-        }
         const CUtensorMap* mk = d.map_id ? &mk1 : &mk0;
         const CUtensorMap* mv = d.map_id ? &mv1 : &mv0;
         const int unit = pw.b * a.hkv + pw.h;
@@ -379,30 +388,22 @@ __global__ void __launch_bounds__(kThreads)
     float m0, m1, l0, l1;
     uint32_t qf[8][2];
     uint32_t qp[8][2];  // Reset PE: the query at its Reset-PE id, for prefix tiles
-    // qp = R_delta qf (rotate-half RoPE composes: R_a R_b = R_(a+b)).  This lane's pairs are
-    // (d, d + 64) for d = 16 ks + 2 qq + {0, 1, 8, 9}, ks < 4: fragments ks and ks + 4.
-    // delta * inv_freq is formed and reduced modulo 2 pi in float64, as in the append.
-    auto rotate_prefix_q = [&](int64_t p) {
-      const int64_t n = p + 1;
-      int64_t ws = n - a.w;
-      if (ws < a.lp) ws = a.lp;
-      const int64_t delta = (int64_t)a.lp - ws;  // <= 0; 0 while nothing is evicted
-      // This lane forms the angles of frequencies d = lane and lane + 32; every lane then
-      // reads the 16 it needs (each is needed by the 8 lanes of one qq) with shuffles.
+    // dst = R_shift src on this lane's fragments (rotate-half RoPE composes: R_a R_b =
+    // R_(a+b)).  This lane's pairs are (d, d + 64) for d = 16 ks + 8 r + 2 qq + {0, 1},
+    // ks < 4: fragments ks and ks + 4.  The lane forms the angles of frequencies d = lane and
+    // lane + 32 (rope_cos_sin: float64, reduced modulo 2 pi, as in the append); every lane
+    // then reads the 16 it needs with shuffles (each is needed by the 8 lanes of one qq).
+    // src and dst may be the same array.
+    auto rope_frag = [&](const uint32_t (&src)[8][2], int64_t shift, uint32_t (&dst)[8][2]) {
       float cw[2], sw[2];
 #pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {
-        const double ang = double(delta) * a.inv_freq[lane + 32 * hf];
-        const double k = rint(ang * 0.15915494309189535);
-        double red = fma(-k, 6.2831854820251465, ang);
-        red = fma(-k, -1.748455600074497e-07, red);
-        sincosf(static_cast<float>(red), &sw[hf], &cw[hf]);
-      }
+      for (int hf = 0; hf < 2; ++hf)
+        rope_cos_sin(double(shift), a.inv_freq[lane + 32 * hf], &cw[hf], &sw[hf]);
 #pragma unroll
       for (int ks = 0; ks < 4; ++ks) {
 #pragma unroll
         for (int r = 0; r < 2; ++r) {
-          const uint32_t lo = qf[ks][r], hi = qf[ks + 4][r];
+          const uint32_t lo = src[ks][r], hi = src[ks + 4][r];
           const float2 x1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&lo));
           const float2 x2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&hi));
           float c[2], sn[2];
@@ -412,10 +413,68 @@ __global__ void __launch_bounds__(kThreads)
             c[e] = __shfl_sync(0xffffffffu, cw[ks >> 1], d & 31);
             sn[e] = __shfl_sync(0xffffffffu, sw[ks >> 1], d & 31);
           }
-          qp[ks][r] = pack_bf16x2(x1.x * c[0] - x2.x * sn[0], x1.y * c[1] - x2.y * sn[1]);
-          qp[ks + 4][r] = pack_bf16x2(x2.x * c[0] + x1.x * sn[0], x2.y * c[1] + x1.y * sn[1]);
+          dst[ks][r] = pack_bf16x2(rope_lo(x1.x, x2.x, c[0], sn[0]), rope_lo(x1.y, x2.y, c[1], sn[1]));
+          dst[ks + 4][r] =
+              pack_bf16x2(rope_hi(x1.x, x2.x, c[0], sn[0]), rope_hi(x1.y, x2.y, c[1], sn[1]));
         }
       }
+    };
+    // Reset PE: prefix tiles see the query at its Reset-PE id L_prefix + |window| - 1, i.e.
+    // rotated by delta = L_prefix - max(L_prefix, p + 1 - W) <= 0 more (0 while nothing is
+    // evicted)
+    auto rotate_prefix_q = [&](int64_t p) {
+      int64_t ws = p + 1 - a.w;
+      if (ws < a.lp) ws = a.lp;
+      rope_frag(qf, (int64_t)a.lp - ws, qp);
+    };
+    // kFused state.  The current unit's query (qf), new key and new value arrive raw and are
+    // rotated at the unit's position p; those of the next unit are loaded when the current
+    // unit begins and rotated one tile later, while the warp would otherwise wait for TMA,
+    // so a unit switch costs no global-load or trigonometry latency.
+    int32_t new_map = -1;  // where the unit's newest row lives: prefix row p (map 0) or
+    int64_t new_row = 0;   // ring slot (p - L_prefix) mod W (map 1)
+    uint32_t nk_lo = 0, nk_hi = 0;      // new key pairs (2l, 2l+1) and (2l+64, 2l+65)
+    uint2 nv = make_uint2(0u, 0u);      // new value dims 4l .. 4l+3
+    // Rotates raw key pairs (2 lane, 2 lane + 1) with partners (+64) at position p.
+    auto rope_key_pairs = [&](uint32_t& lo, uint32_t& hi, int64_t p) {
+      const float2 x1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&lo));
+      const float2 x2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&hi));
+      float c0, s0, c1, s1;
+      rope_cos_sin(double(p), a.inv_freq[2 * lane], &c0, &s0);
+      rope_cos_sin(double(p), a.inv_freq[2 * lane + 1], &c1, &s1);
+      lo = pack_bf16x2(rope_lo(x1.x, x2.x, c0, s0), rope_lo(x1.y, x2.y, c1, s1));
+      hi = pack_bf16x2(rope_hi(x1.x, x2.x, c0, s0), rope_hi(x1.y, x2.y, c1, s1));
+    };
+    auto load_new_kv = [&](int b, int h, uint32_t& lo, uint32_t& hi, uint2& v) {
+      const int64_t kvrow = (int64_t)b * a.hkv + h;
+      const __nv_bfloat16* kn = a.k_new + kvrow * kHeadDim;
+      lo = *reinterpret_cast<const uint32_t*>(kn + 2 * lane);
+      hi = *reinterpret_cast<const uint32_t*>(kn + 64 + 2 * lane);
+      v = *reinterpret_cast<const uint2*>(a.v_new + kvrow * kHeadDim + 4 * lane);
+    };
+    auto set_newest_row = [&](int64_t p) {
+      new_map = p < a.lp ? 0 : 1;
+      new_row = p < a.lp ? p : (p - a.lp) % a.w;
+    };
+    // The warp whose 16 keys include the newest row writes the rotated new key and the new
+    // value over that row of the shared-memory tile (128-byte swizzle: K in two 64-column
+    // boxes, then V) and stores both in the cache.
+    auto patch_newest_row = [&](int stage, int r, int b, int h, int64_t p) {
+      uint8_t* kt = smem + stage * kStageBytes;
+      const uint32_t ko = swz(r, lane >> 2) + (lane & 3) * 4;
+      *reinterpret_cast<uint32_t*>(kt + ko) = nk_lo;
+      *reinterpret_cast<uint32_t*>(kt + kBoxBytes + ko) = nk_hi;
+      *reinterpret_cast<uint2*>(kt + kTileBytes + (lane >> 4) * kBoxBytes +
+                                swz(r, (lane & 15) >> 1) + (lane & 1) * 8) = nv;
+      const int64_t kvrow = (int64_t)b * a.hkv + h;
+      const bool pre = p < a.lp;
+      const int64_t grow = kvrow * (pre ? a.lp : a.w) + (pre ? p : (p - a.lp) % a.w);
+      __nv_bfloat16* kd = (pre ? a.k_pre : a.k_ring) + grow * kHeadDim;
+      __nv_bfloat16* vd = (pre ? a.v_pre : a.v_ring) + grow * kHeadDim;
+      *reinterpret_cast<uint32_t*>(kd + 2 * lane) = nk_lo;
+      *reinterpret_cast<uint32_t*>(kd + 64 + 2 * lane) = nk_hi;
+      *reinterpret_cast<uint2*>(vd + 4 * lane) = nv;
+      __syncwarp();
     };
     auto reset = [&]() {
       m0 = m1 = -INFINITY;
@@ -501,6 +560,10 @@ __global__ void __launch_bounds__(kThreads)
     reset();
     TileWalker cw = wk;
     uint32_t qn[8][2];  // q of the next unit, prefetched
+    int64_t pn = 0;     // its position
+    uint32_t nk_lo_n = 0, nk_hi_n = 0;  // kFused: its new key (raw, then rotated) and value
+    uint2 nv_n = make_uint2(0u, 0u);
+    bool next_raw = false;  // kFused: the next unit's q and key are loaded, not yet rotated
     auto prefetch_next_q = [&](const TileWalker& w) {
       if (w.pu1 < w.t_end) {
         TileWalker nx = w;
@@ -517,14 +580,35 @@ __global__ void __launch_bounds__(kThreads)
 #pragma unroll
           for (int ks = 0; ks < 8; ++ks) qn[ks][0] = qn[ks][1] = 0u;
         }
+        if (MODE != kPlain) pn = a.pos[nx.b];
+        if (MODE == kFused) {
+          load_new_kv(nx.b, nx.h, nk_lo_n, nk_hi_n, nv_n);
+          next_raw = true;
+        }
       }
     };
-    if (a.after_append) pdl_wait();  // q is rotated by the append just before
+    // kFused: rotate the prefetched next unit's q and new key (warp-uniform: shuffles inside)
+    auto rotate_next = [&]() {
+      if (MODE == kFused && next_raw) {
+        rope_frag(qn, pn, qn);
+        rope_key_pairs(nk_lo_n, nk_hi_n, pn);
+        next_raw = false;
+      }
+    };
+    int64_t unit_p = 0;  // position of the current unit's query
     if (ntiles > 0) {
       load_q(cw.b, cw.h);
-      if (RESET) rotate_prefix_q(a.pos[cw.b]);
+      if (MODE != kPlain) unit_p = a.pos[cw.b];
+      if (MODE == kFused) load_new_kv(cw.b, cw.h, nk_lo, nk_hi, nv);
       note_span(cw, cw.t, (cw.pu1 < wk.t_end ? cw.pu1 : wk.t_end) - 1);
       prefetch_next_q(cw);
+      if (MODE == kReset) rotate_prefix_q(unit_p);
+      if (MODE == kFused) {
+        // the first unit's raw q and key: rotated while the first tiles are in flight
+        rope_frag(qf, unit_p, qf);
+        rope_key_pairs(nk_lo, nk_hi, unit_p);
+        set_newest_row(unit_p);
+      }
     }
     bool alive = true;
     for (int i = 0; i < ntiles; ++i, ++cw.t) {
@@ -532,12 +616,20 @@ __global__ void __launch_bounds__(kThreads)
         flush_unit(cw.b, cw.h);
         cw.next_unit(a, pref);
         reset();
+        rotate_next();  // only if no tile of the previous unit had time to do it
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
           qf[ks][0] = qn[ks][0];
           qf[ks][1] = qn[ks][1];
         }
-        if (RESET) rotate_prefix_q(a.pos[cw.b]);
+        if (MODE != kPlain) unit_p = pn;
+        if (MODE == kFused) {
+          nk_lo = nk_lo_n;
+          nk_hi = nk_hi_n;
+          nv = nv_n;
+          set_newest_row(unit_p);
+        }
+        if (MODE == kReset) rotate_prefix_q(unit_p);
         note_span(cw, cw.t, (cw.pu1 < wk.t_end ? cw.pu1 : wk.t_end) - 1);
         prefetch_next_q(cw);
       }
@@ -547,6 +639,14 @@ __global__ void __launch_bounds__(kThreads)
         alive = false;
       if (!alive) continue;  // keep the flush barriers in step with the other warps
       const DecodeTile d = tiling_tile(cw.tiling, static_cast<int32_t>(cw.t - cw.pu));
+      bool patched = false;
+      if (MODE == kFused) {
+        const int64_t r = new_row - d.row0;  // the newest row's place in this tile
+        if (d.map_id == new_map && r >= d.lo && r < d.hi && (r >> 4) == warp) {
+          patch_newest_row(s, static_cast<int>(r), cw.b, cw.h, unit_p);
+          patched = true;
+        }
+      }
       const uint32_t kbase = smem_u32(smem + s * kStageBytes);
       const uint32_t vbase = kbase + kTileBytes;
 
@@ -558,7 +658,7 @@ __global__ void __launch_bounds__(kThreads)
             kbase + (ks >> 2) * kBoxBytes + swz(arow, ((ks & 3) << 1) + achunk);
         ldmatrix_x4(addr, a0, a1, a2, a3);
         // Reset PE: prefix tiles (map 0) see the query at its Reset-PE id
-        const bool pre_q = RESET && d.map_id == 0;
+        const bool pre_q = MODE == kReset && d.map_id == 0;
         mma_bf16_16816(sc, a0, a1, a2, a3, pre_q ? qp[ks][0] : qf[ks][0],
                        pre_q ? qp[ks][1] : qf[ks][1]);
       }
@@ -615,8 +715,14 @@ __global__ void __launch_bounds__(kThreads)
       } else {
         pv(0xffffffffu, 0xffffffffu);
       }
+      // the patched row was written through the generic proxy: order it before the next
+      // TMA write into this stage
+      if (MODE == kFused && patched) fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[s]);
+      // off the unit switch, and late enough in the unit that the next unit's loads (issued
+      // when this unit began) have landed
+      if (cw.t + 2 >= cw.pu1) rotate_next();
     }
     if (ntiles > 0) {
       flush_unit(cw.b, cw.h);
@@ -745,14 +851,24 @@ int occupancy_per_sm() {
   if (cached[dev] == 0) {
     int occ = 0;
     const size_t sb = smem_bytes(kStages);
-    cudaFuncSetAttribute(decode_kernel<kStages, false>,
+    cudaFuncSetAttribute(decode_kernel<kStages, kPlain>,
                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sb);
-    cudaFuncSetAttribute(decode_kernel<kStages, true>,
+    cudaFuncSetAttribute(decode_kernel<kStages, kReset>,
                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sb);
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, decode_kernel<kStages, false>,
+    cudaFuncSetAttribute(decode_kernel<kStages, kFused>,
+                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sb);
+    // the grid must fit in one wave of whichever mode is launched: take the smallest
+    int o[3] = {0, 0, 0};
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o[0], decode_kernel<kStages, kPlain>,
                                                       kThreads, sb) != cudaSuccess ||
-        occ < 1)
-      occ = 1;
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o[1], decode_kernel<kStages, kReset>,
+                                                      kThreads, sb) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o[2], decode_kernel<kStages, kFused>,
+                                                      kThreads, sb) != cudaSuccess)
+      o[0] = o[1] = o[2] = 1;
+    occ = o[0] < o[1] ? o[0] : o[1];
+    if (o[2] < occ) occ = o[2];
+    if (occ < 1) occ = 1;
     cached[dev] = occ < kCtasPerSm ? occ : kCtasPerSm;
   }
   return cached[dev];
@@ -865,7 +981,13 @@ int launch_decode(const DecodeLaunch& l, cudaStream_t stream) {
   a.scale_log2 = l.scale * kLog2e;
   a.skip_prefix = l.skip_prefix;
   a.reset_pe = l.reset_pe;
-  a.after_append = l.after_append;
+  const bool fused = l.k_new != nullptr;
+  a.k_new = static_cast<const __nv_bfloat16*>(l.k_new);
+  a.v_new = static_cast<const __nv_bfloat16*>(l.v_new);
+  a.k_pre = static_cast<__nv_bfloat16*>(const_cast<void*>(l.k0));
+  a.v_pre = static_cast<__nv_bfloat16*>(const_cast<void*>(l.v0));
+  a.k_ring = static_cast<__nv_bfloat16*>(const_cast<void*>(l.k1));
+  a.v_ring = static_cast<__nv_bfloat16*>(const_cast<void*>(l.v1));
   a.paged = l.paged;
   a.table = l.table;
   a.table_stride = l.table_stride;
@@ -875,7 +997,7 @@ int launch_decode(const DecodeLaunch& l, cudaStream_t stream) {
   a.pin_pos = l.pin_pos;
   a.pin_cap = (l.lcap > l.lp) ? l.lcap - l.lp : 0;
   for (int i = 0; i < kHeadDim / 2; ++i)
-    a.inv_freq[i] = l.reset_pe ? pow(l.rope_theta, -2.0 * i / double(kHeadDim)) : 0.0;
+    a.inv_freq[i] = (l.reset_pe || fused) ? pow(l.rope_theta, -2.0 * i / double(kHeadDim)) : 0.0;
   const int32_t pre_splits = l.pre_o ? (l.pre_splits > 0 ? l.pre_splits : 1) : 0;
 
   const size_t sb = smem_bytes(kStages);
@@ -884,10 +1006,10 @@ int launch_decode(const DecodeLaunch& l, cudaStream_t stream) {
   if (grid <= 0) return PS_OK;
   if (grid > 0x7fffffff || l.batch > 0x7fffffff)
     return fail(PS_ERR_UNSUPPORTED, "decode grid too large");
-  int rc = check_cuda(launch_pdl(a.reset_pe ? decode_kernel<kStages, true>
-                                            : decode_kernel<kStages, false>,
-                                 dim3(static_cast<unsigned>(grid)), dim3(kThreads), sb, stream,
-                                 mk0, mv0, mk1, mv1, a),
+  auto kern = a.reset_pe ? decode_kernel<kStages, kReset>
+                         : (fused ? decode_kernel<kStages, kFused> : decode_kernel<kStages, kPlain>);
+  int rc = check_cuda(launch_pdl(kern, dim3(static_cast<unsigned>(grid)), dim3(kThreads), sb,
+                                 stream, mk0, mv0, mk1, mv1, a),
                       "decode_kernel launch");
   if (rc != PS_OK) return rc;
   if (l.before_merge) {

@@ -4,10 +4,12 @@ The forward runs first through the C ABI (its bf16 output and fp32 lse are what 
 keeps); the backward then gets dO.  Every row of dQ and every key row of dK, dV is checked
 on small shapes (ragged tails, W = 1, no prefix, dense causal, prefix longer than a tile,
 GQA groups 2, 7 and 8); at the full truncated-backprop size, sampled rows and keys.
-Bar: |got - ref| <= 2e-2 * max(1, rms of the reference row) per element and rel_rms <= 5e-3
-per tensor (P and dS are rounded to bf16 before the products, so an element's error scales
-with its row's terms; gradients exceed 1, where a bf16 step is larger than 2e-2); the element
-bar is widened by max(1, scale * sqrt(D)) for a softmax scale above the default.
+Bar: |got - ref| <= bar * max(1, rms of the reference row) per element and rel_rms <= 5e-3
+per tensor, with bar = max(2e-2, 1.25 x the same measure of the rounding model of the
+kernels (tests/bwd_model.py) on the same inputs).  P and dS are rounded to bf16 before the
+products, so an element's error scales with its row's terms; gradients exceed 1, where a
+bf16 step is larger than 2e-2; at a softmax scale above the default, peakier P makes dS
+larger and the model's error exceeds 2e-2 by itself.
 """
 import math
 
@@ -18,6 +20,7 @@ import torch
 import oracle as O
 import synth
 from prefix_sliding_window_b200 import binding as B
+from tests import bwd_model as M
 from tests.gpu_util import assert_close_grad, f64
 
 pytestmark = pytest.mark.gpu
@@ -50,12 +53,12 @@ def _forward_backward(dev, Bn, S, hq, hkv, lp, w, seed, scale=0.0):
 def _check_all(inputs, grads, lp, w, scale):
     q, k, v, do = (f64(t) for t in inputs)
     dq, dk, dv = (f64(t) for t in grads)
-    gain = max(1.0, scale * math.sqrt(D))
     for b in range(q.shape[0]):
         wq, wk, wv = O.prefill_backward_reference(q[b], k[b], v[b], do[b], lp, w, scale)
-        assert_close_grad(dq[b], wq, f"dq b={b}", score_gain=gain)
-        assert_close_grad(dk[b], wk, f"dk b={b}", score_gain=gain)
-        assert_close_grad(dv[b], wv, f"dv b={b}", score_gain=gain)
+        _, mq, mk, mv = M.forward_backward(q[b], k[b], v[b], do[b], lp, w, scale)
+        assert_close_grad(dq[b], wq, f"dq b={b}", model_err=M.scaled_error(mq, wq))
+        assert_close_grad(dk[b], wk, f"dk b={b}", model_err=M.scaled_error(mk, wk))
+        assert_close_grad(dv[b], wv, f"dv b={b}", model_err=M.scaled_error(mv, wv))
 
 
 @pytest.mark.parametrize("S,lp,w,hq,hkv", [(520, 16, 200, 4, 2), (300, 0, 64, 4, 2),
