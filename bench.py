@@ -5,8 +5,7 @@ Default workload: steady-state batched decode on one layer (batch 64, 16 query /
 heads, head_dim 128, bf16, L_prefix = 100, W = 4096, positions drawn in [8192, 131072],
 KV prefilled with RoPE at every absolute position).  One step = one decode step of the
 whole batch through ps_decode_step: the new token's append (Continue-PE RoPE of k and q,
-ring write) folded into the split-K decode, then the merge.  Prints ONE JSON line on
-rank 0.
+ring write), then split-K decode + merge.  Prints ONE JSON line on rank 0.
 
   python bench.py [--gpus N --steps K --warmup W] [--impl reference]
 
@@ -241,9 +240,9 @@ class DecodeWorkload:
         torch.cuda.synchronize()
 
     def kernels_per_step(self) -> int:
-        """ps_decode_step launches the decode kernel (append folded in) and, when the batch
-        is split across CTAs (stream-K), the merge kernel."""
-        return 1 + (1 if self.splits_used else 0)
+        """ps_decode_step launches the append, the decode and, when the batch is split across
+        CTAs (stream-K), the merge."""
+        return 2 + (1 if self.splits_used else 0)
 
     def append(self, i):
         B = self.B
@@ -333,6 +332,10 @@ def run_decode(args, world, rank, dev):
         else:
             for j in range(K):
                 step(W + j)
+    # ps_decode_step rotates q in place, so every replay above rotated the same q again:
+    # the timed steps start from the unrotated q (the work is the same either way; the last
+    # output is then the one the end-to-end run below must reproduce)
+    work.q.copy_(work.q_raw)
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     _barrier(world)
     torch.cuda.synchronize()
@@ -366,7 +369,7 @@ def run_decode(args, world, rank, dev):
     dec_med_s = statistics.median(dec_ms) / 1e3
     attn = alg_dec / dec_med_s / 1e9
     roof = {"bound": "hbm",
-            "kernel": "ps_decode_step (decode_kernel with the append folded in + merge_kernel)",
+            "kernel": "ps_decode_step (append_rope_kernel + decode_kernel + merge_kernel)",
             "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
             "frac": round(achieved / peaks["hbm_gbs"], 4),
             "traffic": args.traffic if args.traffic is not None else _recorded_traffic("step"),
@@ -381,7 +384,7 @@ def run_decode(args, world, rank, dev):
                           "us_median": round(statistics.median(dec_ms) * 1e3, 2),
                           "us_p10": round(float(np.percentile(dec_ms, 10)) * 1e3, 2),
                           "us_p90": round(float(np.percentile(dec_ms, 90)) * 1e3, 2),
-                          "traffic": _recorded_traffic("decode_kernel")}}
+                          "traffic": _recorded_traffic("attn_call")}}
     e2e = run_decode_e2e(work, K, W, world, use_graph=not args.no_graph)
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": K,

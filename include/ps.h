@@ -128,21 +128,18 @@ int ps_decode_attn(const ps_params* params, const ps_kv_cache* cache, const void
                    const int64_t* pos, void* out, float* lse, void* workspace, size_t ws_bytes,
                    int32_t* dev_status, ps_stream_t stream);
 
-/* One whole decode step: the append of one token per sequence at pos[b] (its key rotated
- * with Continue-PE RoPE and stored, its value stored, as ps_kv_append_rope does), then
- * ps_decode_attn at the same pos with the query rotated at pos.  Source: §核心机制 and §位置编码
- * (append with Continue PE, then attend the visible keys).  The append runs inside the
- * decode kernel: its consumer warps rotate the query themselves, and the warp that reads the
- * new row's tile writes the rotated key and the value over that row in shared memory and in
- * the cache.  Results (out, lse and the cache) are bit-identical to ps_kv_append_rope
- * followed by ps_decode_attn.
+/* One whole decode step: ps_kv_append_rope of one token per sequence at pos[b] (q rotated
+ * in place), then ps_decode_attn at the same pos.  Source: §核心机制 and §位置编码 (append
+ * with Continue PE, then attend the visible keys).  Results equal the two calls made one
+ * after the other; because the library knows the append wrote exactly the newest row of
+ * every sequence, the decode streams every other key tile while the append is still
+ * running and waits for it only before that row and q.
  *   k_new, v_new : device bf16 [batch, Hkv, D], raw keys and values of the new token.
- *   q            : device bf16 [batch, Hq, D], raw (un-rotated) query; read only.
+ *   q_inout      : device bf16 [batch, Hq, D], raw query; rotated at pos in place.
  * Other arguments, errors and the workspace (ps_decode_workspace_bytes) as ps_decode_attn;
- * a linear cache (ring NULL) is not accepted.  A position < 0 sets PS_DEV_BAD_POS and leaves
- * that sequence's cache untouched. */
+ * a linear cache (ring NULL) is not accepted. */
 int ps_decode_step(const ps_params* params, const ps_kv_cache* cache, const void* k_new,
-                   const void* v_new, const void* q, const int64_t* pos, void* out, float* lse,
+                   const void* v_new, void* q_inout, const int64_t* pos, void* out, float* lse,
                    void* workspace, size_t ws_bytes, int32_t* dev_status, ps_stream_t stream);
 
 /* One decode step under Reset PE, from the same Continue-PE cache ps_kv_append_rope fills.

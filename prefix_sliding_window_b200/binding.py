@@ -218,13 +218,12 @@ def ps_decode_attn_paged(params: PsParams, k_pool, v_pool, block_table, batch: i
     _check(rc, "ps_decode_attn_paged")
 
 
-def ps_decode_step(params: PsParams, cache: PsKVCache, k_new, v_new, q, pos, out,
+def ps_decode_step(params: PsParams, cache: PsKVCache, k_new, v_new, q_inout, pos, out,
                    lse=None, workspace=None, dev_status=None, stream=None) -> None:
-    """Append one token per sequence at pos, then decode at pos (q: the raw query, read
-    only; it is rotated inside the kernel)."""
+    """Append one token per sequence at pos (q rotated in place), then decode at pos."""
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     rc = load().ps_decode_step(ctypes.byref(params), ctypes.byref(cache), _ptr(k_new),
-                               _ptr(v_new), _ptr(q), _ptr(pos), _ptr(out), _ptr(lse),
+                               _ptr(v_new), _ptr(q_inout), _ptr(pos), _ptr(out), _ptr(lse),
                                _ptr(workspace), ws_bytes, _ptr(dev_status), _stream(stream))
     _check(rc, "ps_decode_step")
 

@@ -338,8 +338,7 @@ static int decode_entry(const ps_params* params, const ps_kv_cache* cache, const
                         const int64_t* pos, void* out, float* lse, void* workspace,
                         size_t ws_bytes, int32_t* dev_status, ps_stream_t stream,
                         int32_t reset_pe, int32_t lcap = 0, const int32_t* pin_count = nullptr,
-                        const int64_t* pin_pos = nullptr, const void* k_new = nullptr,
-                        const void* v_new = nullptr) {
+                        const int64_t* pin_pos = nullptr, int32_t after_append = 0) {
   g_last_error.clear();
   DecodeLaunch l;
   bool empty = false;
@@ -358,8 +357,7 @@ static int decode_entry(const ps_params* params, const ps_kv_cache* cache, const
   l.lcap = lcap;
   l.pin_count = pin_count;
   l.pin_pos = pin_pos;
-  l.k_new = k_new;
-  l.v_new = v_new;
+  l.after_append = after_append;
   return launch_decode(l, reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -745,18 +743,25 @@ int ps_decode_attn_pinned(const ps_params* params, const ps_kv_cache* cache,
 }
 
 int ps_decode_step(const ps_params* params, const ps_kv_cache* cache, const void* k_new,
-                   const void* v_new, const void* q, const int64_t* pos, void* out, float* lse,
+                   const void* v_new, void* q_inout, const int64_t* pos, void* out, float* lse,
                    void* workspace, size_t ws_bytes, int32_t* dev_status, ps_stream_t stream) {
-  // One kernel (plus the split-K merge): the decode rotates the raw query and the new key at
-  // pos itself, patches the new row into the tile it streams and writes it to the store.
   g_last_error.clear();
-  PS_TRY(check_ptr(q, "q"));
-  PS_TRY(check_ptr(k_new, "k_new"));
-  PS_TRY(check_ptr(v_new, "v_new"));
-  if (cache && cache->batch > 0 && cache->k_ring == nullptr)
+  PS_TRY(check_ptr(q_inout, "q_inout"));
+  // validate the decode half first, so that nothing is launched on a bad call
+  if (!params) return fail(PS_ERR_INVALID_ARG, "params is NULL");
+  PS_TRY(check_params(params, true));
+  if (params->n_q_heads / params->n_kv_heads > kMaxGroup)
+    return fail(PS_ERR_UNSUPPORTED, "decode supports at most 8 query heads per KV head");
+  if (!cache) return fail(PS_ERR_INVALID_ARG, "cache is NULL");
+  if (cache->batch > 0 && cache->k_ring == nullptr)
     return fail(PS_ERR_INVALID_ARG, "ps_decode_step needs a ring cache");
-  return decode_entry(params, cache, q, pos, out, lse, workspace, ws_bytes, dev_status, stream,
-                      0, 0, nullptr, nullptr, k_new, v_new);
+  const size_t need = decode_workspace_bytes(cache->batch, params->n_kv_heads,
+                                             (int64_t)params->l_prefix + params->window);
+  if (need > 0 && (!workspace || ws_bytes < need))
+    return fail(PS_ERR_WORKSPACE, "workspace smaller than ps_decode_workspace_bytes()");
+  PS_TRY(ps_kv_append_rope(params, cache, k_new, v_new, q_inout, pos, 1, dev_status, stream));
+  return decode_entry(params, cache, q_inout, pos, out, lse, workspace, ws_bytes, dev_status,
+                      stream, 0, 0, nullptr, nullptr, 1);
 }
 
 // ---------------------------------------------------------------- paged store

@@ -129,10 +129,9 @@ __global__ void __launch_bounds__(kAppendThreads) append_rope_kernel(const Appen
 
   if (threadIdx.x < kHalf) {
     // angle = p * inv_f[i], formed and reduced modulo 2 pi in float64 (rope_cos_sin)
-    float sf, cf;
-    rope_cos_sin(double(p), a.inv_freq[threadIdx.x], &cf, &sf);
-    s_cos[threadIdx.x] = cf;
-    s_sin[threadIdx.x] = sf;
+    const float2 cs = rope_cos_sin(double(p), a.inv_freq[threadIdx.x]);
+    s_cos[threadIdx.x] = cs.x;
+    s_sin[threadIdx.x] = cs.y;
   }
   __syncthreads();
 

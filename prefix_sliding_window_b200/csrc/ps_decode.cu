@@ -25,11 +25,6 @@
 //    P^T goes from the accumulator layout to the operand layout with movmatrix; softmax is
 //    online, in base 2, with warp-shuffle max reductions;
 //  * the four warps' (m, l, O) states are merged through shared memory.
-// ps_decode_step runs the same kernel with the one-token append folded in (kFused): the
-// consumers rotate the raw query at its position themselves, and the warp whose 16 keys
-// include the sequence's newest row writes the rotated new key and the new value over that
-// row of the shared-memory tile before reading it, and stores them in the cache.  No separate
-// append kernel runs, so the decode streams from its first cycle.
 #include <cuda_bf16.h>
 #include <math.h>
 
@@ -60,7 +55,6 @@ constexpr float kLn2 = 0.6931471805599453f;
 // others)
 constexpr int kPlain = 0;  // ps_decode_attn and its variants
 constexpr int kReset = 1;  // Reset PE: prefix tiles see the query at its Reset-PE id
-constexpr int kFused = 2;  // ps_decode_step: the one-token append folded in
 
 // shared memory: stages | barriers (2 x STAGES) | flush area [2][32 lanes][36] | prefix
 constexpr size_t kFlushFloats = 2 * 32 * 36;
@@ -76,8 +70,6 @@ struct DecodeArgs {
   float* lse;
   float* ws_o;      // stream-K: [slots, 8, D] normalised partial outputs
   float* ws_lse;    // stream-K: [slots, 8] base-2 lse of each partial
-  int32_t* ws_pref; // stream-K: [batch + 1] tiles-per-sequence prefix
-  int32_t* ws_span; // stream-K: [units][2] first and last CTA holding a piece of the unit
   int32_t* status;
   int32_t batch, hq, hkv, group;
   int32_t lp, w, dim0;
@@ -86,17 +78,12 @@ struct DecodeArgs {
   float scale_log2;
   int32_t skip_prefix;     // shared-prefix decode: window rows only
   // Reset PE: prefix tiles use the query rotated by delta = L_prefix + |window| - 1 - p
-  // more (its Reset-PE id); inv_freq = theta^(-2i/D) in float64 (also used by kFused)
+  // more (its Reset-PE id); inv_freq = theta^(-2i/D) in float64
   int32_t reset_pe;
-  // kFused: raw new key / value [batch, Hkv, D] of the token at pos, and the stores their
-  // rotated key and value go to (prefix rows [batch, Hkv, lp, D], ring [batch, Hkv, W, D]);
-  // q holds the raw query and receives the rotated one
-  const __nv_bfloat16* k_new;
-  const __nv_bfloat16* v_new;
-  __nv_bfloat16* k_pre;
-  __nv_bfloat16* v_pre;
-  __nv_bfloat16* k_ring;
-  __nv_bfloat16* v_ring;
+  // launched right after a one-token append at pos (ps_decode_step): only the tile holding
+  // each sequence's newest row and the rotated q depend on that kernel, so everything else
+  // may stream before the programmatic wait
+  int32_t after_append;
   // paged store: K/V of every (sequence, KV head) in 64-row blocks of one pool
   // [n_blocks][Hkv][64][D]; logical block i of sequence b is table[b * table_stride + i]
   // (prefix blocks first, then W / 64 ring blocks)
@@ -232,11 +219,10 @@ __device__ __forceinline__ void store_state(float* dst, float m0, float m1, floa
   dst[35] = l1;
 }
 
-// MODE: kPlain, kReset (prefix tiles see the query at its renumbered id) or kFused (the
-// one-token append folded in).  A template parameter, not a run-time flag, so the plain
-// decode carries none of the other modes' registers.
+// MODE: kPlain or kReset (prefix tiles see the query at its renumbered id).  A template
+// parameter, not a run-time flag, so the plain decode carries none of Reset PE's registers.
 // Two CTAs of 5 warps per SM need at most 168 registers per thread (10 warps on 4 SMSPs: 3
-// warps x 168 x 32 fit one SMSP's 16K registers); the bound keeps every mode there, and the
+// warps x 168 x 32 fit one SMSP's 16K registers); the bound keeps both modes there, and the
 // stream-K grid is sized for two per SM.
 template <int STAGES, int MODE>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
@@ -267,8 +253,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     prefetch_tensormap(&mv1);
   }
   // launched with programmatic serialization: everything above overlapped the previous
-  // kernel; positions, q and the cache are read only after this
-  pdl_wait();
+  // kernel (usually the append); positions, q and the cache are read only after this
+  if (!a.after_append) pdl_wait();
   pdl_trigger();  // the merge may be scheduled now; it waits for this grid to finish
 
   // ---------------------------------------------------------------- work range
@@ -279,14 +265,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       const int64_t p = a.pos[b];
       const int32_t cnt = tiling_of(a, b, p).total;
       pref[b + 1] = cnt;
-      if (blockIdx.x == 0 && cnt == 0) {
-        if (bad_position(a, p) && a.status)
-          atomicOr(a.status, p < 0 ? PS_DEV_BAD_POS : PS_DEV_POS_RANGE);
-        for (int h = 0; h < a.hkv; ++h) {  // an empty span: no pieces to merge
-          a.ws_span[2 * (b * a.hkv + h)] = 1;
-          a.ws_span[2 * (b * a.hkv + h) + 1] = 0;
-        }
-      }
+      if (blockIdx.x == 0 && cnt == 0 && bad_position(a, p) && a.status)
+        atomicOr(a.status, p < 0 ? PS_DEV_BAD_POS : PS_DEV_POS_RANGE);
     }
     if (threadIdx.x == 0) pref[0] = 0;
     __syncthreads();
@@ -305,8 +285,6 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       }
     }
     __syncthreads();
-    if (blockIdx.x == 0)
-      for (int i = threadIdx.x; i <= a.batch; i += kThreads) a.ws_pref[i] = pref[i];
     const int64_t total = (int64_t)a.hkv * pref[a.batch];
     const int64_t t0 = total * blockIdx.x / gridDim.x;
     const int64_t t1 = total * (blockIdx.x + 1) / gridDim.x;
@@ -337,6 +315,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     if (lane == 0 && ntiles > 0) {
       const uint64_t pol = l2_policy_evict_first();
       int issued = 0;
+      bool waited = !a.after_append;
       TileWalker pw = wk;
       for (int i = 0; i < ntiles; ++i, ++pw.t) {
         if (pw.t >= pw.pu1) pw.next_unit(a, pref);
@@ -344,6 +323,16 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         const uint32_t ph = (i / STAGES) & 1;
         if (i >= STAGES && !mbar_wait(&empty[s], ph ^ 1, a.status)) break;
         const DecodeTile d = tiling_tile(pw.tiling, static_cast<int32_t>(pw.t - pw.pu));
+        if (!waited) {
+          // the newest row of sequence b: prefix row p, or ring slot (p - Lp) mod W
+          const int64_t p = a.pos[pw.b];
+          const bool pre = a.full_mode || p < a.lp;
+          const int64_t row = pre ? p : (p - a.lp) % a.w;
+          if (d.map_id == (pre ? 0 : 1) && row >= d.row0 + d.lo && row < d.row0 + d.hi) {
+            pdl_wait();
+            waited = true;
+          }
+        }
         const CUtensorMap* mk = d.map_id ? &mk1 : &mk0;
         const CUtensorMap* mv = d.map_id ? &mv1 : &mv0;
         const int unit = pw.b * a.hkv + pw.h;
@@ -397,8 +386,11 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     auto rope_frag = [&](const uint32_t (&src)[8][2], int64_t shift, uint32_t (&dst)[8][2]) {
       float cw[2], sw[2];
 #pragma unroll
-      for (int hf = 0; hf < 2; ++hf)
-        rope_cos_sin(double(shift), a.inv_freq[lane + 32 * hf], &cw[hf], &sw[hf]);
+      for (int hf = 0; hf < 2; ++hf) {
+        const float2 cs = rope_cos_sin(double(shift), a.inv_freq[lane + 32 * hf]);
+        cw[hf] = cs.x;
+        sw[hf] = cs.y;
+      }
 #pragma unroll
       for (int ks = 0; ks < 4; ++ks) {
 #pragma unroll
@@ -426,55 +418,6 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       int64_t ws = p + 1 - a.w;
       if (ws < a.lp) ws = a.lp;
       rope_frag(qf, (int64_t)a.lp - ws, qp);
-    };
-    // kFused state.  The current unit's query (qf), new key and new value arrive raw and are
-    // rotated at the unit's position p; those of the next unit are loaded when the current
-    // unit begins and rotated one tile later, while the warp would otherwise wait for TMA,
-    // so a unit switch costs no global-load or trigonometry latency.
-    int32_t new_map = -1;  // where the unit's newest row lives: prefix row p (map 0) or
-    int64_t new_row = 0;   // ring slot (p - L_prefix) mod W (map 1)
-    uint32_t nk_lo = 0, nk_hi = 0;      // new key pairs (2l, 2l+1) and (2l+64, 2l+65)
-    uint2 nv = make_uint2(0u, 0u);      // new value dims 4l .. 4l+3
-    // Rotates raw key pairs (2 lane, 2 lane + 1) with partners (+64) at position p.
-    auto rope_key_pairs = [&](uint32_t& lo, uint32_t& hi, int64_t p) {
-      const float2 x1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&lo));
-      const float2 x2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&hi));
-      float c0, s0, c1, s1;
-      rope_cos_sin(double(p), a.inv_freq[2 * lane], &c0, &s0);
-      rope_cos_sin(double(p), a.inv_freq[2 * lane + 1], &c1, &s1);
-      lo = pack_bf16x2(rope_lo(x1.x, x2.x, c0, s0), rope_lo(x1.y, x2.y, c1, s1));
-      hi = pack_bf16x2(rope_hi(x1.x, x2.x, c0, s0), rope_hi(x1.y, x2.y, c1, s1));
-    };
-    auto load_new_kv = [&](int b, int h, uint32_t& lo, uint32_t& hi, uint2& v) {
-      const int64_t kvrow = (int64_t)b * a.hkv + h;
-      const __nv_bfloat16* kn = a.k_new + kvrow * kHeadDim;
-      lo = *reinterpret_cast<const uint32_t*>(kn + 2 * lane);
-      hi = *reinterpret_cast<const uint32_t*>(kn + 64 + 2 * lane);
-      v = *reinterpret_cast<const uint2*>(a.v_new + kvrow * kHeadDim + 4 * lane);
-    };
-    auto set_newest_row = [&](int64_t p) {
-      new_map = p < a.lp ? 0 : 1;
-      new_row = p < a.lp ? p : (p - a.lp) % a.w;
-    };
-    // The warp whose 16 keys include the newest row writes the rotated new key and the new
-    // value over that row of the shared-memory tile (128-byte swizzle: K in two 64-column
-    // boxes, then V) and stores both in the cache.
-    auto patch_newest_row = [&](int stage, int r, int b, int h, int64_t p) {
-      uint8_t* kt = smem + stage * kStageBytes;
-      const uint32_t ko = swz(r, lane >> 2) + (lane & 3) * 4;
-      *reinterpret_cast<uint32_t*>(kt + ko) = nk_lo;
-      *reinterpret_cast<uint32_t*>(kt + kBoxBytes + ko) = nk_hi;
-      *reinterpret_cast<uint2*>(kt + kTileBytes + (lane >> 4) * kBoxBytes +
-                                swz(r, (lane & 15) >> 1) + (lane & 1) * 8) = nv;
-      const int64_t kvrow = (int64_t)b * a.hkv + h;
-      const bool pre = p < a.lp;
-      const int64_t grow = kvrow * (pre ? a.lp : a.w) + (pre ? p : (p - a.lp) % a.w);
-      __nv_bfloat16* kd = (pre ? a.k_pre : a.k_ring) + grow * kHeadDim;
-      __nv_bfloat16* vd = (pre ? a.v_pre : a.v_ring) + grow * kHeadDim;
-      *reinterpret_cast<uint32_t*>(kd + 2 * lane) = nk_lo;
-      *reinterpret_cast<uint32_t*>(kd + 64 + 2 * lane) = nk_hi;
-      *reinterpret_cast<uint2*>(vd + 4 * lane) = nv;
-      __syncwarp();
     };
     auto reset = [&]() {
       m0 = m1 = -INFINITY;
@@ -548,22 +491,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       named_bar_sync(1, kConsumerThreads);  // the flush area is free again
     };
 
-    // A unit's first tile is owned by exactly one CTA and so is its last: those CTAs
-    // record themselves, so the merge finds the pieces without any division.
-    auto note_span = [&](const TileWalker& w, int64_t t_first, int64_t t_last) {
-      if (a.streamk && threadIdx.x == 0) {
-        const int unit = w.b * a.hkv + w.h;
-        if (t_first == w.pu) a.ws_span[2 * unit] = blockIdx.x;
-        if (t_last == w.pu1 - 1) a.ws_span[2 * unit + 1] = blockIdx.x;
-      }
-    };
     reset();
     TileWalker cw = wk;
     uint32_t qn[8][2];  // q of the next unit, prefetched
-    int64_t pn = 0;     // its position
-    uint32_t nk_lo_n = 0, nk_hi_n = 0;  // kFused: its new key (raw, then rotated) and value
-    uint2 nv_n = make_uint2(0u, 0u);
-    bool next_raw = false;  // kFused: the next unit's q and key are loaded, not yet rotated
     auto prefetch_next_q = [&](const TileWalker& w) {
       if (w.pu1 < w.t_end) {
         TileWalker nx = w;
@@ -580,35 +510,13 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 #pragma unroll
           for (int ks = 0; ks < 8; ++ks) qn[ks][0] = qn[ks][1] = 0u;
         }
-        if (MODE != kPlain) pn = a.pos[nx.b];
-        if (MODE == kFused) {
-          load_new_kv(nx.b, nx.h, nk_lo_n, nk_hi_n, nv_n);
-          next_raw = true;
-        }
       }
     };
-    // kFused: rotate the prefetched next unit's q and new key (warp-uniform: shuffles inside)
-    auto rotate_next = [&]() {
-      if (MODE == kFused && next_raw) {
-        rope_frag(qn, pn, qn);
-        rope_key_pairs(nk_lo_n, nk_hi_n, pn);
-        next_raw = false;
-      }
-    };
-    int64_t unit_p = 0;  // position of the current unit's query
+    if (a.after_append) pdl_wait();  // q is rotated by the append just before
     if (ntiles > 0) {
       load_q(cw.b, cw.h);
-      if (MODE != kPlain) unit_p = a.pos[cw.b];
-      if (MODE == kFused) load_new_kv(cw.b, cw.h, nk_lo, nk_hi, nv);
-      note_span(cw, cw.t, (cw.pu1 < wk.t_end ? cw.pu1 : wk.t_end) - 1);
+      if (MODE == kReset) rotate_prefix_q(a.pos[cw.b]);
       prefetch_next_q(cw);
-      if (MODE == kReset) rotate_prefix_q(unit_p);
-      if (MODE == kFused) {
-        // the first unit's raw q and key: rotated while the first tiles are in flight
-        rope_frag(qf, unit_p, qf);
-        rope_key_pairs(nk_lo, nk_hi, unit_p);
-        set_newest_row(unit_p);
-      }
     }
     bool alive = true;
     for (int i = 0; i < ntiles; ++i, ++cw.t) {
@@ -616,21 +524,12 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         flush_unit(cw.b, cw.h);
         cw.next_unit(a, pref);
         reset();
-        rotate_next();  // only if no tile of the previous unit had time to do it
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
           qf[ks][0] = qn[ks][0];
           qf[ks][1] = qn[ks][1];
         }
-        if (MODE != kPlain) unit_p = pn;
-        if (MODE == kFused) {
-          nk_lo = nk_lo_n;
-          nk_hi = nk_hi_n;
-          nv = nv_n;
-          set_newest_row(unit_p);
-        }
-        if (MODE == kReset) rotate_prefix_q(unit_p);
-        note_span(cw, cw.t, (cw.pu1 < wk.t_end ? cw.pu1 : wk.t_end) - 1);
+        if (MODE == kReset) rotate_prefix_q(a.pos[cw.b]);
         prefetch_next_q(cw);
       }
       const int s = i % STAGES;
@@ -639,14 +538,6 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         alive = false;
       if (!alive) continue;  // keep the flush barriers in step with the other warps
       const DecodeTile d = tiling_tile(cw.tiling, static_cast<int32_t>(cw.t - cw.pu));
-      bool patched = false;
-      if (MODE == kFused) {
-        const int64_t r = new_row - d.row0;  // the newest row's place in this tile
-        if (d.map_id == new_map && r >= d.lo && r < d.hi && (r >> 4) == warp) {
-          patch_newest_row(s, static_cast<int>(r), cw.b, cw.h, unit_p);
-          patched = true;
-        }
-      }
       const uint32_t kbase = smem_u32(smem + s * kStageBytes);
       const uint32_t vbase = kbase + kTileBytes;
 
@@ -715,14 +606,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       } else {
         pv(0xffffffffu, 0xffffffffu);
       }
-      // the patched row was written through the generic proxy: order it before the next
-      // TMA write into this stage
-      if (MODE == kFused && patched) fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[s]);
-      // off the unit switch, and late enough in the unit that the next unit's loads (issued
-      // when this unit began) have landed
-      if (cw.t + 2 >= cw.pu1) rotate_next();
     }
     if (ntiles > 0) {
       flush_unit(cw.b, cw.h);
@@ -735,25 +620,58 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 }
 
 // Combines the stream-K pieces of one (sequence, query head): weights 2^(lse_s - max).
-// Pieces of unit u are the CTAs c in [first, last] recorded by the decode kernel, stored at
-// slot u + c.  One warp per (sequence, query head); lane i owns d = 4i .. 4i+3.
+// CTA c of the decode owned the global tiles [total c / grid, total (c+1) / grid) and stored
+// its piece of unit u at slot u + c.  The merge recomputes that partition itself, from the
+// positions (written before the decode ran), while the decode still runs: only the pieces
+// are read after the programmatic wait.  One warp per (sequence, query head); lane i owns
+// d = 4i .. 4i+3.
 __global__ void __launch_bounds__(128)
-    merge_kernel(const float* __restrict__ ws_o, const float* __restrict__ ws_lse,
-                 const int32_t* __restrict__ pref, const int32_t* __restrict__ span,
-                 __nv_bfloat16* __restrict__ out, float* __restrict__ lse, int32_t batch,
-                 int32_t hq, int32_t hkv, int32_t group, int32_t grid,
+    merge_kernel(const __grid_constant__ DecodeArgs a, int32_t grid,
                  const float* __restrict__ pre_o, const float* __restrict__ pre_lse2,
                  int32_t pre_splits) {
-  const int64_t bh = (int64_t)blockIdx.x * 4 + (threadIdx.x >> 5);
-  if (bh >= (int64_t)batch * hq) return;
+  __shared__ int32_t s_pref[kMaxStreamKSeqs + 1];
+  const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  // tiles per sequence, exactly as the decode counts them, then an inclusive scan
+  for (int i = threadIdx.x; i < a.batch; i += blockDim.x)
+    s_pref[i + 1] = tiling_of(a, i, a.pos[i]).total;
+  if (threadIdx.x == 0) s_pref[0] = 0;
+  __syncthreads();
+  if (warp == 0) {
+    int32_t carry = 0;
+    for (int base = 1; base <= a.batch; base += 32) {
+      const int i = base + lane;
+      int32_t v = i <= a.batch ? s_pref[i] : 0;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int32_t u = __shfl_up_sync(0xffffffffu, v, off);
+        if (lane >= off) v += u;
+      }
+      if (i <= a.batch) s_pref[i] = v + carry;
+      carry += __shfl_sync(0xffffffffu, v, 31);
+    }
+  }
+  __syncthreads();
+  const int64_t bh = (int64_t)blockIdx.x * 4 + warp;
+  if (bh >= (int64_t)a.batch * a.hq) return;
+  const int hq = a.hq, hkv = a.hkv, group = a.group, batch = a.batch;
   const int b = static_cast<int>(bh / hq), head = static_cast<int>(bh % hq);
   const int h = head / group, hh = head % group;
   const int64_t unit = (int64_t)b * hkv + h;
-  pdl_wait();  // the decode kernel's pieces and spans must be complete
+  const int64_t total = (int64_t)hkv * s_pref[batch];
+  const int64_t cnt = s_pref[b + 1] - s_pref[b];
+  // the CTAs holding the unit's first and last tiles: the CTA owning tile t is
+  // ((t + 1) grid - 1) / total
+  int c_lo = 1, c_hi = 0;
+  if (cnt > 0) {
+    const int64_t pu = (int64_t)hkv * s_pref[b] + h * cnt;
+    c_lo = static_cast<int>(((pu + 1) * grid - 1) / total);
+    c_hi = static_cast<int>(((pu + cnt) * grid - 1) / total);
+  }
+  const float* ws_o = a.ws_o;
+  const float* ws_lse = a.ws_lse;
+  pdl_wait();  // the decode kernel's pieces must be complete
   pdl_trigger();  // a programmatically serialized successor waits for this grid itself
-  const int2 span_cu = reinterpret_cast<const int2*>(span)[unit];
-  const int64_t total = (int64_t)hkv * pref[batch];
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   float lse2 = -INFINITY;
   // online combine state; shared-prefix partials (normalised, weight 2^lse2) start it
@@ -773,8 +691,7 @@ __global__ void __launch_bounds__(128)
     acc.w = acc.w * fa + fb * ov.w;
     M = Mn;
   }
-  if (span_cu.x <= span_cu.y) {
-    const int c_lo = span_cu.x, c_hi = span_cu.y;
+  if (c_lo <= c_hi) {
     // with fewer tiles than CTAs some CTAs own nothing and wrote no piece
     const bool maybe_empty = total < grid;
     auto empty_cta = [&](int c) {
@@ -827,8 +744,8 @@ __global__ void __launch_bounds__(128)
   uint2 pk;
   pk.x = pack_bf16x2(acc.x, acc.y);
   pk.y = pack_bf16x2(acc.z, acc.w);
-  reinterpret_cast<uint2*>(out + bh * kHeadDim)[lane] = pk;
-  if (lse && lane == 0) lse[bh] = lse2 * kLn2;
+  reinterpret_cast<uint2*>(a.out + bh * kHeadDim)[lane] = pk;
+  if (a.lse && lane == 0) a.lse[bh] = lse2 * kLn2;
 }
 
 __global__ void visible_ranges_kernel(const int64_t* __restrict__ pos, int64_t batch, int32_t lp,
@@ -855,19 +772,14 @@ int occupancy_per_sm() {
                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sb);
     cudaFuncSetAttribute(decode_kernel<kStages, kReset>,
                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sb);
-    cudaFuncSetAttribute(decode_kernel<kStages, kFused>,
-                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sb);
-    // the grid must fit in one wave of whichever mode is launched: take the smallest
-    int o[3] = {0, 0, 0};
+    // the grid must fit in one wave of whichever mode is launched: take the smaller
+    int o[2] = {0, 0};
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o[0], decode_kernel<kStages, kPlain>,
                                                       kThreads, sb) != cudaSuccess ||
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o[1], decode_kernel<kStages, kReset>,
-                                                      kThreads, sb) != cudaSuccess ||
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o[2], decode_kernel<kStages, kFused>,
                                                       kThreads, sb) != cudaSuccess)
-      o[0] = o[1] = o[2] = 1;
+      o[0] = o[1] = 1;
     occ = o[0] < o[1] ? o[0] : o[1];
-    if (o[2] < occ) occ = o[2];
     if (occ < 1) occ = 1;
     cached[dev] = occ < kCtasPerSm ? occ : kCtasPerSm;
   }
@@ -903,8 +815,7 @@ size_t decode_workspace_bytes(int64_t batch, int32_t hkv, int64_t max_keys, bool
   const size_t slots = size_t(batch * hkv + g) * 8;
   const size_t o_bytes = slots * kHeadDim * sizeof(float);
   const size_t lse_bytes = (slots * sizeof(float) + 255) & ~size_t(255);
-  const size_t pref_bytes = (size_t(batch + 1) * sizeof(int32_t) + 255) & ~size_t(255);
-  return o_bytes + lse_bytes + pref_bytes + size_t(batch * hkv) * 2 * sizeof(int32_t);
+  return o_bytes + lse_bytes;
 }
 
 int launch_decode(const DecodeLaunch& l, cudaStream_t stream) {
@@ -960,13 +871,6 @@ int launch_decode(const DecodeLaunch& l, cudaStream_t stream) {
   const size_t nslots = size_t(units + g) * 8;
   a.ws_o = g ? static_cast<float*>(l.workspace) : nullptr;
   a.ws_lse = g ? a.ws_o + nslots * kHeadDim : nullptr;
-  a.ws_pref = g ? reinterpret_cast<int32_t*>(
-                      reinterpret_cast<char*>(a.ws_lse) +
-                      ((nslots * sizeof(float) + 255) & ~size_t(255)))
-                : nullptr;
-  a.ws_span = g ? a.ws_pref + (((size_t(l.batch + 1) * sizeof(int32_t) + 255) & ~size_t(255)) /
-                                sizeof(int32_t))
-                : nullptr;
   a.status = l.status;
   a.batch = static_cast<int32_t>(l.batch);
   a.hq = l.hq;
@@ -981,13 +885,7 @@ int launch_decode(const DecodeLaunch& l, cudaStream_t stream) {
   a.scale_log2 = l.scale * kLog2e;
   a.skip_prefix = l.skip_prefix;
   a.reset_pe = l.reset_pe;
-  const bool fused = l.k_new != nullptr;
-  a.k_new = static_cast<const __nv_bfloat16*>(l.k_new);
-  a.v_new = static_cast<const __nv_bfloat16*>(l.v_new);
-  a.k_pre = static_cast<__nv_bfloat16*>(const_cast<void*>(l.k0));
-  a.v_pre = static_cast<__nv_bfloat16*>(const_cast<void*>(l.v0));
-  a.k_ring = static_cast<__nv_bfloat16*>(const_cast<void*>(l.k1));
-  a.v_ring = static_cast<__nv_bfloat16*>(const_cast<void*>(l.v1));
+  a.after_append = l.after_append;
   a.paged = l.paged;
   a.table = l.table;
   a.table_stride = l.table_stride;
@@ -997,7 +895,7 @@ int launch_decode(const DecodeLaunch& l, cudaStream_t stream) {
   a.pin_pos = l.pin_pos;
   a.pin_cap = (l.lcap > l.lp) ? l.lcap - l.lp : 0;
   for (int i = 0; i < kHeadDim / 2; ++i)
-    a.inv_freq[i] = (l.reset_pe || fused) ? pow(l.rope_theta, -2.0 * i / double(kHeadDim)) : 0.0;
+    a.inv_freq[i] = l.reset_pe ? pow(l.rope_theta, -2.0 * i / double(kHeadDim)) : 0.0;
   const int32_t pre_splits = l.pre_o ? (l.pre_splits > 0 ? l.pre_splits : 1) : 0;
 
   const size_t sb = smem_bytes(kStages);
@@ -1006,8 +904,7 @@ int launch_decode(const DecodeLaunch& l, cudaStream_t stream) {
   if (grid <= 0) return PS_OK;
   if (grid > 0x7fffffff || l.batch > 0x7fffffff)
     return fail(PS_ERR_UNSUPPORTED, "decode grid too large");
-  auto kern = a.reset_pe ? decode_kernel<kStages, kReset>
-                         : (fused ? decode_kernel<kStages, kFused> : decode_kernel<kStages, kPlain>);
+  auto kern = a.reset_pe ? decode_kernel<kStages, kReset> : decode_kernel<kStages, kPlain>;
   int rc = check_cuda(launch_pdl(kern, dim3(static_cast<unsigned>(grid)), dim3(kThreads), sb,
                                  stream, mk0, mv0, mk1, mv1, a),
                       "decode_kernel launch");
@@ -1019,10 +916,7 @@ int launch_decode(const DecodeLaunch& l, cudaStream_t stream) {
   if (g > 0) {
     rc = check_cuda(
         launch_pdl(merge_kernel, dim3(static_cast<unsigned>((l.batch * l.hq + 3) / 4)), dim3(128),
-                   0, stream, static_cast<const float*>(a.ws_o),
-                   static_cast<const float*>(a.ws_lse), static_cast<const int32_t*>(a.ws_pref),
-                   static_cast<const int32_t*>(a.ws_span), a.out, a.lse, a.batch, l.hq, l.hkv,
-                   group, static_cast<int32_t>(g), l.pre_o, l.pre_lse2, pre_splits),
+                   0, stream, a, static_cast<int32_t>(g), l.pre_o, l.pre_lse2, pre_splits),
         "merge_kernel launch");
   }
   return rc;

@@ -160,13 +160,17 @@ __device__ __forceinline__ float fast_exp2(float x) {
 // double precision); the remainder, within [-pi, pi], goes through fp32 sincosf (accurate to
 // ~1e-7 there).  At p ~ 2^18 an fp32 product alone would be off by ~0.03 rad.  Every kernel
 // that rotates keys or queries uses this function and rope_lo / rope_hi, so a vector rotated
-// by any of them is bit-identical.
-__device__ __forceinline__ void rope_cos_sin(double p, double inv_f, float* c, float* s) {
+// by any of them is bit-identical.  Out of line: sincosf carries a large slow path (for
+// arguments it never gets here), which would otherwise sit inside the callers' hot loops.
+// Returns (cos, sin).
+static __device__ __noinline__ float2 rope_cos_sin(double p, double inv_f) {
   const double ang = p * inv_f;
   const double k = rint(ang * 0.15915494309189535);
   double red = fma(-k, 6.2831854820251465, ang);
   red = fma(-k, -1.748455600074497e-07, red);
-  sincosf(static_cast<float>(red), s, c);
+  float c, s;
+  sincosf(static_cast<float>(red), &s, &c);
+  return make_float2(c, s);
 }
 
 // One rotate-half pair (x1 = x[i], x2 = x[i + D/2]) rotated by (c, s): the first and second
@@ -177,12 +181,6 @@ __device__ __forceinline__ float rope_lo(float x1, float x2, float c, float s) {
 }
 __device__ __forceinline__ float rope_hi(float x1, float x2, float c, float s) {
   return __fadd_rn(__fmul_rn(x2, c), __fmul_rn(x1, s));
-}
-
-// Orders this thread's earlier generic-proxy accesses to shared memory before later
-// async-proxy (TMA) writes to the same bytes.
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 }  // namespace ps

@@ -130,11 +130,8 @@ struct DecodeLaunch {
   int32_t lcap;
   const int32_t* pin_count;
   const int64_t* pin_pos;
-  // ps_decode_step: the one-token append folded into the decode.  k_new / v_new are the raw
-  // key and value [batch, Hkv, D] of the token at pos (NULL: no append); q is then the raw
-  // query, rotated at pos in place.  Contiguous store only (k0/v0 prefix, k1/v1 ring).
-  const void* k_new;
-  const void* v_new;
+  // the previous kernel on the stream is the one-token append at pos (ps_decode_step)
+  int32_t after_append;
   // paged store (k0/v0 = the pool [n_blocks][Hkv][64][D], table [batch][table_stride])
   int32_t paged;
   const int32_t* table;

@@ -415,10 +415,9 @@ def test_prefix_sliding_equals_full_attention_in_warmup(cuda_device):
                                          (160, 100, 256, 0, 4000),         # one CTA per unit
                                          (5, 300, 64, 0, 400)])            # prompt / warm-up
 def test_decode_step_equals_append_then_decode(cuda_device, Bn, lp, w, lo, hi):
-    """ps_decode_step (the append folded into the decode kernel: query and new key rotated
-    there, the new row patched into the streamed tile) is bit-identical to ps_kv_append_rope
-    followed by ps_decode_attn: outputs, lse, status and every row of the cache.  Its query
-    argument is left as it was (raw)."""
+    """ps_decode_step (the decode streams before the append finishes, except the newest row)
+    is bit-identical to ps_kv_append_rope followed by ps_decode_attn: the rotated query,
+    outputs, lse, status and every row of the cache."""
     dev = cuda_device
     hq, hkv = 16, 2
     params = B.make_params(hq, hkv, D, lp, w, THETA)
@@ -453,8 +452,7 @@ def test_decode_step_equals_append_then_decode(cuda_device, Bn, lp, w, lo, hi):
         outs.append((q, out, lse, st.item()))
     (qa, oa, la, sa), (qb, ob, lb, sb) = outs
     assert sa == sb
-    assert torch.equal(oa, ob) and torch.equal(la, lb)
-    assert torch.equal(qb, q_raw)  # read only
+    assert torch.equal(qa, qb) and torch.equal(oa, ob) and torch.equal(la, lb)
     for a, b in ((caches[0].k_ring, caches[1].k_ring), (caches[0].v_ring, caches[1].v_ring)):
         assert torch.equal(a, b)
     if lp:
@@ -464,7 +462,7 @@ def test_decode_step_equals_append_then_decode(cuda_device, Bn, lp, w, lo, hi):
 
 def test_graph_launched_steps_equal_eager_steps(cuda_device):
     """The launch configuration bench.py times: ps_decode_step on the batch-64, W=4096
-    workload replayed as one CUDA graph of 8 steps is bit-identical (out, cache) to the
+    workload replayed as one CUDA graph of 8 steps is bit-identical (q, out, cache) to the
     same 8 steps launched one by one."""
     import bench
     dev = cuda_device

@@ -102,9 +102,9 @@ def _fill_history(params, cache, pos, lp, w, hkv, sample, seed, dev, st, chunk=2
 
 def _step_and_check(params, cache, pos, lp, w, hq, hkv, raw, seed, dev, st):
     """Appends the new token at pos and decodes it twice: ps_kv_append_rope + ps_decode_attn
-    on one copy of the cache, ps_decode_step (append folded into the decode) on another.
-    Outputs, lse and caches must be bit-identical.  Sampled sequences are checked against the
-    oracle on every head and the lse."""
+    on one copy of the cache, ps_decode_step on another.  Rotated queries, outputs, lse and
+    caches must be bit-identical.  Sampled sequences are checked against the oracle on every
+    head and the lse."""
     Bn = pos.numel()
     k_new = synth.normal_bf16((Bn, 1, hkv, D), seed, dev)
     v_new = synth.normal_bf16((Bn, 1, hkv, D), seed + 1, dev)
@@ -127,7 +127,7 @@ def _step_and_check(params, cache, pos, lp, w, hq, hkv, raw, seed, dev, st):
                      pos, out2, lse2, ws, st)
     torch.cuda.synchronize()
     assert st.item() == 0, st.item()
-    assert torch.equal(out1, out2) and torch.equal(lse1, lse2) and torch.equal(q2, q_raw)
+    assert torch.equal(out1, out2) and torch.equal(lse1, lse2) and torch.equal(q1, q2)
     for a, b in ((twin.k_prefix, cache.k_prefix), (twin.v_prefix, cache.v_prefix),
                  (twin.k_ring, cache.k_ring), (twin.v_ring, cache.v_ring)):
         assert torch.equal(a.view(torch.int16), b.view(torch.int16))  # bits, NaN canaries too
@@ -304,5 +304,6 @@ def test_decode_equals_prefill_row(cuda_device, hq, hkv, lp, w, S, rows):
                      q, pos, out_d, None, ws, st)
     torch.cuda.synchronize()
     assert st.item() == 0
+    assert torch.equal(q, q_rot[0, idx])  # the same rotation on both paths
     for b, p in enumerate(rows):
         assert_close(f64(out_d[b]), f64(out_p[0, p]), f"decode vs prefill row {p}")
