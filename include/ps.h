@@ -326,8 +326,13 @@ int ps_masked_prefill_attn(const ps_params* params, const void* q, const void* k
                            int64_t tile_plan_cap, int64_t* n_tiles, void* workspace,
                            size_t ws_bytes, int32_t* dev_status, ps_stream_t stream);
 
-/* Bytes of device workspace ps_masked_prefill_attn_bwd needs: the tile plan, two fp32 row
- * statistics per (batch, head, row) padded to whole 128-row tiles, and a work counter. */
+/* Bytes of device workspace recommended for ps_masked_prefill_attn_bwd over `batch`
+ * sequences: the tile plan, a work counter, and per sequence of one pass two fp32 row
+ * statistics per (head, row) padded to whole 128-row tiles and the bf16 dS^T tile of every
+ * planned (query tile, key tile) pair per head (32 KB each).  The batch runs in passes: one
+ * pass when that store stays within 4 GiB, else passes of as many sequences as fit in 4 GiB
+ * (so the size stops growing with the batch).  The value for batch = 1 is the minimum the
+ * call accepts; a workspace between the two runs passes of as many sequences as it holds. */
 size_t ps_prefill_bwd_workspace_bytes(const ps_params* params, int64_t batch, int64_t seq);
 
 /* Backward of ps_masked_prefill_attn: gradients of the masked attention with respect to
@@ -344,8 +349,9 @@ size_t ps_prefill_bwd_workspace_bytes(const ps_params* params, int64_t batch, in
  *   lse      : device fp32 [batch, Hq, seq], the forward's log-sum-exp (required).
  *   dq       : device bf16 [batch, seq, Hq, D] (written).
  *   dk, dv   : device bf16 [batch, seq, Hkv, D] (written).
- *   workspace, ws_bytes : device scratch of at least ps_prefill_bwd_workspace_bytes(),
- *              256-byte aligned.
+ *   workspace, ws_bytes : device scratch of at least ps_prefill_bwd_workspace_bytes() for
+ *              batch 1, 256-byte aligned; results do not depend on its size (every pass
+ *              covers whole sequences).  Smaller: PS_ERR_WORKSPACE.
  *   dev_status : device int32 or NULL (PS_DEV_TIMEOUT only).
  * Requires seq >= 1, Hq / Hkv integral.  All of q, k, v, out, dout, dq, dk, dv 16-byte
  * aligned.  Outputs are written in full (no accumulation into existing values). */

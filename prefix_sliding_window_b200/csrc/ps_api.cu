@@ -545,10 +545,11 @@ int ps_masked_prefill_attn_bwd(const ps_params* params, const void* q, const voi
   PS_TRY(check_ptr(dv, "dv"));
   if ((reinterpret_cast<uintptr_t>(dev_status) & 3u) != 0)
     return fail(PS_ERR_INVALID_ARG, "dev_status is not 4-byte aligned");
-  const size_t need = prefill_bwd_workspace_bytes(batch, params->n_q_heads, seq,
-                                                  params->l_prefix, params->window);
+  // one sequence per pass at least; more per pass as the workspace allows
+  const size_t need =
+      prefill_bwd_min_workspace_bytes(params->n_q_heads, seq, params->l_prefix, params->window);
   if (!workspace || ws_bytes < need)
-    return fail(PS_ERR_WORKSPACE, "workspace smaller than ps_prefill_bwd_workspace_bytes()");
+    return fail(PS_ERR_WORKSPACE, "workspace smaller than ps_prefill_bwd_workspace_bytes(batch 1)");
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
     return fail(PS_ERR_INVALID_ARG, "workspace is not 256-byte aligned");
   PrefillBwdLaunch l{};
@@ -562,6 +563,7 @@ int ps_masked_prefill_attn_bwd(const ps_params* params, const void* q, const voi
   l.dk = dk;
   l.dv = dv;
   l.workspace = workspace;
+  l.ws_bytes = ws_bytes;
   l.batch = batch;
   l.seq = seq;
   l.hq = params->n_q_heads;

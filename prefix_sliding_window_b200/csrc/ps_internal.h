@@ -202,12 +202,16 @@ struct PrefillBwdLaunch {
   void* dk;
   void* dv;
   void* workspace;
+  size_t ws_bytes;  // sequences run in passes of as many as this workspace holds
   int64_t batch, seq;
   int32_t hq, hkv, lp, w;
   float scale;
   int32_t* status;
 };
+// Recommended workspace: the whole batch in one pass, unless its dS^T store would pass 4 GiB
+// (then passes of fewer sequences).  The minimum holds one sequence.
 size_t prefill_bwd_workspace_bytes(int64_t batch, int32_t hq, int64_t seq, int32_t lp, int32_t w);
+size_t prefill_bwd_min_workspace_bytes(int32_t hq, int64_t seq, int32_t lp, int32_t w);
 int launch_prefill_bwd(const PrefillBwdLaunch& l, cudaStream_t stream);
 
 }  // namespace ps

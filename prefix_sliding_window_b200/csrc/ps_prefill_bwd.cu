@@ -814,7 +814,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 // Workspace: [plan][-lse*log2e rows][-D rows][counter][dS^T tiles of every planned tile,
-// 32 KB each]
+// 32 KB each], for `batch` sequences per pass.
 struct BwdLayout {
   size_t plan, stats, counter, ds, total;
   int64_t n_plan;
@@ -829,6 +829,24 @@ BwdLayout bwd_layout(int64_t batch, int32_t hq, int64_t seq, int32_t lp, int32_t
   L.ds = size_t(batch) * hq * L.n_plan * kT * kT * 2;
   L.total = align256(L.plan) + 2 * L.stats + L.counter + L.ds;
   return L;
+}
+
+// The dS^T store of one pass is kept under this many bytes: a batch whose store would be
+// larger runs in passes of fewer sequences (the workspace stops growing with the batch).
+constexpr size_t kDsPassBytes = size_t(4) << 30;
+
+// Sequences per pass: the most (up to `batch`) whose layout fits `ws_bytes`; 0 if not even
+// one does.
+int64_t bwd_pass_batch(int64_t batch, int32_t hq, int64_t seq, int32_t lp, int32_t w,
+                       size_t ws_bytes) {
+  const BwdLayout one = bwd_layout(1, hq, seq, lp, w);
+  if (one.total > ws_bytes) return 0;
+  int64_t lo = 1, hi = batch;  // largest n in [1, batch] with layout(n) <= ws_bytes
+  while (lo < hi) {
+    const int64_t mid = lo + (hi - lo + 1) / 2;
+    if (bwd_layout(mid, hq, seq, lp, w).total <= ws_bytes) lo = mid; else hi = mid - 1;
+  }
+  return lo;
 }
 
 bool set_smem(const void* fn, size_t bytes, bool* done, const char* what, int* rc) {
@@ -848,24 +866,40 @@ bool set_smem(const void* fn, size_t bytes, bool* done, const char* what, int* r
 }  // namespace
 
 size_t prefill_bwd_workspace_bytes(int64_t batch, int32_t hq, int64_t seq, int32_t lp, int32_t w) {
-  return bwd_layout(batch, hq, seq, lp, w).total;
+  const BwdLayout one = bwd_layout(1, hq, seq, lp, w);
+  int64_t n = batch < 1 ? 1 : batch;
+  const int64_t per_pass = static_cast<int64_t>(kDsPassBytes / (one.ds > 0 ? one.ds : 1));
+  if (n > per_pass) n = per_pass < 1 ? 1 : per_pass;
+  return bwd_layout(n, hq, seq, lp, w).total;
 }
 
-int launch_prefill_bwd(const PrefillBwdLaunch& l, cudaStream_t stream) {
+size_t prefill_bwd_min_workspace_bytes(int32_t hq, int64_t seq, int32_t lp, int32_t w) {
+  return bwd_layout(1, hq, seq, lp, w).total;
+}
+
+namespace {
+
+// One pass over sequences [b0, b0 + nb) of the batch (the plan is already in the workspace).
+int launch_bwd_pass(const PrefillBwdLaunch& l, int64_t b0, int64_t nb, cudaStream_t stream) {
   const int64_t nq = (l.seq + kT - 1) / kT;
   const int64_t s_pad = nq * kT;
-  const BwdLayout L = bwd_layout(l.batch, l.hq, l.seq, l.lp, l.w);
+  const BwdLayout L = bwd_layout(nb, l.hq, l.seq, l.lp, l.w);
   char* ws = static_cast<char*>(l.workspace);
-  const int64_t n_tiles = prefill_plan_tiles(l.seq, l.lp, l.w);
-  int rc = check_cuda(launch_plan(l.seq, l.lp, l.w, n_tiles, ws, nullptr, stream),
-                      "plan_kernel launch");
-  if (rc != PS_OK) return rc;
+  const size_t qrow = size_t(l.seq) * l.hq * kHeadDim * 2;   // bytes per sequence, q-shaped
+  const size_t krow = size_t(l.seq) * l.hkv * kHeadDim * 2;  // k-shaped
+  const char* q = static_cast<const char*>(l.q) + b0 * qrow;
+  const char* k = static_cast<const char*>(l.k) + b0 * krow;
+  const char* v = static_cast<const char*>(l.v) + b0 * krow;
+  const char* out = static_cast<const char*>(l.out) + b0 * qrow;
+  const char* dout = static_cast<const char*>(l.dout) + b0 * qrow;
+  const float* lse = l.lse + b0 * l.hq * l.seq;
+  int rc = PS_OK;
 
   BwdArgs a;
   a.status = l.status;
   a.seq = l.seq;
   a.s_pad = s_pad;
-  a.batch = static_cast<int32_t>(l.batch);
+  a.batch = static_cast<int32_t>(nb);
   a.hq = l.hq;
   a.hkv = l.hkv;
   a.group = l.hq / l.hkv;
@@ -883,30 +917,30 @@ int launch_prefill_bwd(const PrefillBwdLaunch& l, cudaStream_t stream) {
   a.counter = reinterpret_cast<int32_t*>(ws + align256(L.plan) + 2 * L.stats);
   a.ds = reinterpret_cast<__nv_bfloat16*>(ws + align256(L.plan) + 2 * L.stats + L.counter);
   a.n_plan = L.n_plan;
-  a.dq = static_cast<__nv_bfloat16*>(l.dq);
-  a.dk = static_cast<__nv_bfloat16*>(l.dk);
-  a.dv = static_cast<__nv_bfloat16*>(l.dv);
+  a.dq = reinterpret_cast<__nv_bfloat16*>(static_cast<char*>(l.dq) + b0 * qrow);
+  a.dk = reinterpret_cast<__nv_bfloat16*>(static_cast<char*>(l.dk) + b0 * krow);
+  a.dv = reinterpret_cast<__nv_bfloat16*>(static_cast<char*>(l.dv) + b0 * krow);
 
   // row statistics: a grid of a few waves of the SMs, each half-warp striding over rows
   const int64_t sms = sm_count();
-  const int64_t real_rows = l.batch * l.seq * l.hq;
+  const int64_t real_rows = nb * l.seq * l.hq;
   int64_t prep_blocks = (real_rows * 16 + kPrepThreads - 1) / kPrepThreads;
   if (prep_blocks > sms * 16) prep_blocks = sms * 16;
   if (prep_blocks < 1) prep_blocks = 1;
   rc = check_cuda(launch_pdl(bwd_prep_kernel, dim3(static_cast<unsigned>(prep_blocks)),
                              dim3(kPrepThreads), 0, stream,
-                             static_cast<const __nv_bfloat16*>(l.out),
-                             static_cast<const __nv_bfloat16*>(l.dout), l.lse, l.seq, l.hq, s_pad,
-                             l.batch, nl, nd, a.counter),
+                             reinterpret_cast<const __nv_bfloat16*>(out),
+                             reinterpret_cast<const __nv_bfloat16*>(dout), lse, l.seq, l.hq, s_pad,
+                             nb, nl, nd, a.counter),
                   "bwd_prep_kernel launch");
   if (rc != PS_OK) return rc;
 
   CUtensorMap mq, mdo, mk, mv;
-  const uint64_t dq_dims[4] = {kHeadDim, (uint64_t)l.hq, (uint64_t)l.seq, (uint64_t)l.batch};
-  const uint64_t dk_dims[4] = {kHeadDim, (uint64_t)l.hkv, (uint64_t)l.seq, (uint64_t)l.batch};
+  const uint64_t dq_dims[4] = {kHeadDim, (uint64_t)l.hq, (uint64_t)l.seq, (uint64_t)nb};
+  const uint64_t dk_dims[4] = {kHeadDim, (uint64_t)l.hkv, (uint64_t)l.seq, (uint64_t)nb};
   const uint32_t box[4] = {64, 1, 128, 1};
-  if (!make_map_4d(&mq, l.q, dq_dims, box) || !make_map_4d(&mdo, l.dout, dq_dims, box) ||
-      !make_map_4d(&mk, l.k, dk_dims, box) || !make_map_4d(&mv, l.v, dk_dims, box))
+  if (!make_map_4d(&mq, q, dq_dims, box) || !make_map_4d(&mdo, dout, dq_dims, box) ||
+      !make_map_4d(&mk, k, dk_dims, box) || !make_map_4d(&mv, v, dk_dims, box))
     return PS_ERR_CUDA;
 
 
@@ -916,8 +950,8 @@ int launch_prefill_bwd(const PrefillBwdLaunch& l, cudaStream_t stream) {
       !set_smem(reinterpret_cast<const void*>(bwd_dkdv_kernel), kDkdvSmem, kv_attr,
                 "cudaFuncSetAttribute(bwd_dkdv_kernel)", &rc))
     return rc;
-  const int64_t q_items = l.batch * l.hq * nq;
-  const int64_t kv_items = l.batch * l.hkv * nq;
+  const int64_t q_items = nb * l.hq * nq;
+  const int64_t kv_items = nb * l.hkv * nq;
   if (q_items > 0x7fffffffLL) return fail(PS_ERR_UNSUPPORTED, "prefill backward too large");
   // dK, dV (and the dS^T tiles) first, then dQ from the stored tiles
   rc = check_cuda(
@@ -929,6 +963,20 @@ int launch_prefill_bwd(const PrefillBwdLaunch& l, cudaStream_t stream) {
       launch_pdl(bwd_dq_kernel, dim3(static_cast<unsigned>(q_items < sms ? q_items : sms)),
                  dim3(kDqThreads), kDqSmem, stream, mk, a),
       "bwd_dq_kernel launch");
+}
+
+}  // namespace
+
+int launch_prefill_bwd(const PrefillBwdLaunch& l, cudaStream_t stream) {
+  const int64_t nb = bwd_pass_batch(l.batch, l.hq, l.seq, l.lp, l.w, l.ws_bytes);
+  if (nb < 1) return fail(PS_ERR_WORKSPACE, "prefill backward workspace too small");
+  const int64_t n_tiles = prefill_plan_tiles(l.seq, l.lp, l.w);
+  int rc = check_cuda(launch_plan(l.seq, l.lp, l.w, n_tiles, l.workspace, nullptr, stream),
+                      "plan_kernel launch");
+  // passes of nb sequences; each writes its own rows of dq, dk and dv
+  for (int64_t b0 = 0; rc == PS_OK && b0 < l.batch; b0 += nb)
+    rc = launch_bwd_pass(l, b0, l.batch - b0 < nb ? l.batch - b0 : nb, stream);
+  return rc;
 }
 
 }  // namespace ps

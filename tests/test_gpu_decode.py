@@ -413,17 +413,24 @@ def test_prefix_sliding_equals_full_attention_in_warmup(cuda_device):
 
 @pytest.mark.parametrize("Bn,lp,w,lo,hi", [(64, 100, 4096, 8192, 131072),   # stream-K
                                          (160, 100, 256, 0, 4000),         # one CTA per unit
-                                         (5, 300, 64, 0, 400)])            # prompt / warm-up
+                                         (5, 300, 64, 0, 400),             # prompt / warm-up
+                                         (40, 100, 4096, 0, 131072)])      # mixed lengths
 def test_decode_step_equals_append_then_decode(cuda_device, Bn, lp, w, lo, hi):
     """ps_decode_step (the decode streams before the append finishes, except the newest row)
     is bit-identical to ps_kv_append_rope followed by ps_decode_attn: the rotated query,
-    outputs, lse, status and every row of the cache."""
+    outputs, lse, status and every row of the cache.  The mixed batch puts short sequences
+    (one or two tiles, each inside one CTA's share) next to long ones (about seven stream-K
+    pieces each, two rounds of the merge's four-piece combine)."""
     dev = cuda_device
     hq, hkv = 16, 2
     params = B.make_params(hq, hkv, D, lp, w, THETA)
     pos = synth.uniform_positions(Bn, lo, hi, seed=77, device=dev)
     if Bn == 5:
         pos[0] = -3  # a bad position: both paths flag it and write zeros
+    if Bn == 40:
+        short = synth.uniform_positions(Bn, 0, 100, seed=76, device=dev)
+        pos[0::2] = short[0::2]
+        pos[1::2] = pos[1::2].clamp(min=65536)
     caches = []
     for _ in range(2):
         c = PrefixSlidingCache(Bn, hkv, lp, w, D, dev, fill=None)

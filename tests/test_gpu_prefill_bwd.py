@@ -116,3 +116,25 @@ def test_prefill_bwd_truncated_context_full_size(cuda_device):
     assert_close_grad(f64(dq[b][rows][:, hs]), wq, "dq rows")
     assert_close_grad(f64(dk[b][keys][:, kvh:kvh + 1]), wk, "dk keys")
     assert_close_grad(f64(dv[b][keys][:, kvh:kvh + 1]), wv, "dv keys")
+
+
+def test_prefill_bwd_passes_bit_identical(cuda_device):
+    """A workspace smaller than the whole batch needs runs the batch in passes of as many
+    sequences as it holds (one, two, then all three here); every pass covers whole sequences,
+    so the gradients are bit-identical to the one-pass call.  One of the batch-3 sequences is
+    also checked against the oracle."""
+    S, hq, hkv, lp, w = 390, 8, 2, 50, 128
+    params, inputs, grads, (out, lse, wsb, st) = _forward_backward(cuda_device, 3, S, hq, hkv,
+                                                                   lp, w, seed=77)
+    q, k, v, do = inputs
+    sizes = [B.ps_prefill_bwd_workspace_bytes(params, n, S) for n in (1, 2, 3)]
+    assert sizes[0] < sizes[1] < sizes[2] == wsb.numel()
+    for nbytes in sizes[:2] + [sizes[1] + 1000]:
+        ws = torch.empty(nbytes, dtype=torch.uint8, device=cuda_device)
+        again = [torch.full_like(t, float("nan")) for t in grads]
+        B.ps_masked_prefill_attn_bwd(params, q, k, v, out, do, lse, 3, S, *again, ws, st)
+        torch.cuda.synchronize()
+        assert st.item() == 0
+        for g, a in zip(grads, again):
+            assert torch.equal(g.view(torch.int16), a.view(torch.int16))
+    _check_all([t[2:3] for t in inputs], [t[2:3] for t in grads], lp, w, 1 / math.sqrt(D))

@@ -150,12 +150,28 @@ def test_prefill_bwd_host_validation(lib):
     assert f(*args([16, 16, 16, 16, None])) == B.PS_ERR_INVALID_ARG  # dout NULL
     assert f(*args([16, 16, 8, 16, 16])) == B.PS_ERR_INVALID_ARG     # v misaligned
     assert f(*args(ok, grads=(16, None, 16))) == B.PS_ERR_INVALID_ARG
-    assert f(*args(ok, wsb=need - 1)) == B.PS_ERR_WORKSPACE
+    one = B.ps_prefill_bwd_workspace_bytes(p, 1, 8192)       # the minimum: one sequence
+    assert f(*args(ok, wsb=one - 1)) == B.PS_ERR_WORKSPACE
     assert f(*args(ok, ws=None)) == B.PS_ERR_WORKSPACE
     assert f(*args(ok, ws=272)) == B.PS_ERR_INVALID_ARG              # workspace not 256-aligned
     assert f(ctypes.byref(p), *ok, 16, 4, 0, 16, 16, 16, 256, need, None, None) == \
         B.PS_ERR_INVALID_ARG                                          # seq < 1
     assert f(ctypes.byref(p), *ok, 16, 0, 8192, 16, 16, 16, None, 0, None, None) == B.PS_OK
+
+
+def test_prefill_bwd_workspace_stops_growing_with_batch():
+    """The dS^T store (32 KB per planned tile per head) of one pass stays within 4 GiB: at the
+    truncated-backprop shape (28 heads, 8192 tokens, W 2048, 1045 planned tiles per head: 0.96
+    GB per sequence) four sequences fit, so batch 32 takes the workspace of batch 4; below
+    that the size grows with the batch."""
+    p = _params(n_q_heads=28, n_kv_heads=4, l_prefix=256, window=2048)
+    ws = [B.ps_prefill_bwd_workspace_bytes(p, n, 8192) for n in (1, 2, 4, 5, 32, 1000)]
+    per_seq = 28 * 1045 * 128 * 128 * 2
+    assert ws[1] - ws[0] >= per_seq
+    assert ws[2] - ws[1] >= 2 * per_seq
+    assert ws[2] <= 4 * per_seq + (64 << 20)
+    assert ws[3] == ws[4] == ws[5] == ws[2]
+    assert ws[2] - 4 * per_seq < (1 << 30) and 4 * per_seq <= 4 << 30 < 5 * per_seq
 
 
 def test_shared_prefix_host_validation(lib):
