@@ -173,11 +173,38 @@ SharedPrefixLayout shared_prefix_layout(const ps_params* p, int64_t batch, int64
   L.total = L.dec + L.o + L.lse;
   return L;
 }
-// Side stream (one per device, created on first use) on which the shared-prefix pass runs
-// concurrently with the window decode.
+// Process-unique id of the current context (cuCtxGetId), 0 if the driver cannot tell.  The
+// primary context keeps its handle across cudaDeviceReset, but not its id.
+unsigned long long current_context_id() {
+  using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+  using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(p);
+  });
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_current && get_id && get_current(&ctx) == CUDA_SUCCESS && ctx)
+    get_id(ctx, &id);
+  return id;
+}
+
+// Side stream (one per device and context, created on first use) on which the shared-prefix
+// pass runs concurrently with the window decode.  A stream of a context that has since been
+// destroyed (cudaDeviceReset) is abandoned, not reused: its handle is no longer valid.
 cudaStream_t side_stream(int* rc) {
   static std::mutex mu;
   static cudaStream_t streams[64] = {nullptr};
+  static unsigned long long owner[64] = {0};
   int dev = 0;
   *rc = check_cuda(cudaGetDevice(&dev), "cudaGetDevice");
   if (*rc != PS_OK) return nullptr;
@@ -185,11 +212,17 @@ cudaStream_t side_stream(int* rc) {
     *rc = fail(PS_ERR_UNSUPPORTED, "device index above 63");
     return nullptr;
   }
+  // the current context: the caller's device buffers live in it
+  const unsigned long long ctx = current_context_id();
   std::lock_guard<std::mutex> lock(mu);
-  if (!streams[dev]) {
+  if (!streams[dev] || owner[dev] != ctx) {
     *rc = check_cuda(cudaStreamCreateWithFlags(&streams[dev], cudaStreamNonBlocking),
                      "cudaStreamCreateWithFlags");
-    if (*rc != PS_OK) return nullptr;
+    if (*rc != PS_OK) {
+      streams[dev] = nullptr;
+      return nullptr;
+    }
+    owner[dev] = ctx;
   }
   return streams[dev];
 }
