@@ -670,8 +670,12 @@ __global__ void __launch_bounds__(128)
   }
   const float* ws_o = a.ws_o;
   const float* ws_lse = a.ws_lse;
+  // The next kernel (usually the next step's append) may be scheduled at once: every kernel
+  // of this library that can follow this one waits for its predecessor's grid before it
+  // touches memory, and this grid completes only after its own wait below.  That hides the
+  // successor's scheduling behind this merge.
+  pdl_trigger();
   pdl_wait();  // the decode kernel's pieces must be complete
-  pdl_trigger();  // a programmatically serialized successor waits for this grid itself
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   float lse2 = -INFINITY;
   // online combine state; shared-prefix partials (normalised, weight 2^lse2) start it
