@@ -15,7 +15,10 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 B = 128
 CASES = [(1, 0, 1), (129, 7, 1), (300, 100, 64), (1000, 0, 128), (1000, 127, 129),
          (2500, 256, 1000), (4096, 128, 2048), (8192, 256, 2048), (8191, 1000, 5000),
-         (3000, 300, 10000), (640, 129, 127)]
+         (3000, 300, 10000), (640, 129, 127),
+         # L_prefix reaching or passing the sequence's end, tile-edge lengths
+         (129, 134, 12), (1, 6, 129), (127, 127, 256), (129, 129, 2), (128, 128, 1),
+         (256, 256, 129), (675, 489, 128), (129, 1, 256), (255, 127, 215), (509, 129, 129)]
 
 _DRIVER = r"""
 #include <cstdio>
