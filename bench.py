@@ -1442,7 +1442,7 @@ def main():
                     help="launch the timed steps one by one instead of as a CUDA graph")
     ap.add_argument("--leg", default="main", choices=["main", "prefill", "sweep", "stack", "latency",
                                                       "shared", "reset", "pin", "paged"],
-                    help="main: the driver's line; prefill/sweep/stack: one extra workload")
+                    help="main: the default decode line; prefill/sweep/stack: one extra workload")
     ap.add_argument("--prefill-workload", default="prefill_b4_s8192_w2048",
                     choices=[k for k in synth.WORKLOADS if k.startswith("prefill")],
                     help="workload of the prefill leg")

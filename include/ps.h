@@ -42,7 +42,7 @@ typedef struct CUstream_st* ps_stream_t;
 typedef enum {
   PS_OK = 0,
   PS_ERR_INVALID_ARG = -1, /* null pointer, bad size, misaligned pointer            */
-  PS_ERR_UNSUPPORTED = -2, /* shape outside what this build implements              */
+  PS_ERR_UNSUPPORTED = -2, /* shape outside what the library implements              */
   PS_ERR_WORKSPACE = -3,   /* workspace null or smaller than the *_workspace_bytes  */
   PS_ERR_CUDA = -4         /* a CUDA runtime call or kernel launch failed           */
 } ps_status;
@@ -62,7 +62,7 @@ typedef enum {
 typedef struct {
   int32_t n_q_heads;   /* Hq; Hq % Hkv == 0                                          */
   int32_t n_kv_heads;  /* Hkv; GQA: query head h reads KV head h / (Hq / Hkv)        */
-  int32_t head_dim;    /* D; this build supports D == 128 only                       */
+  int32_t head_dim;    /* D; the library supports D == 128 only                       */
   int32_t l_prefix;    /* L_prefix >= 0; 0 gives the pure sliding window            */
   int32_t window;      /* W >= 1                                                    */
   int32_t reserved;    /* must be 0                                                 */

@@ -44,7 +44,7 @@ int check_params(const ps_params* prm, bool need_window) {
   if (prm->reserved != 0 || prm->reserved2 != 0)
     return fail(PS_ERR_INVALID_ARG, "params reserved fields must be 0");
   if (prm->head_dim != kHeadDim)
-    return fail(PS_ERR_UNSUPPORTED, "head_dim must be 128 in this build");
+    return fail(PS_ERR_UNSUPPORTED, "head_dim must be 128 (the only head size this library implements)");
   if (prm->n_q_heads < 1 || prm->n_kv_heads < 1)
     return fail(PS_ERR_INVALID_ARG, "n_q_heads and n_kv_heads must be >= 1");
   if (prm->n_q_heads % prm->n_kv_heads != 0)
@@ -173,8 +173,8 @@ SharedPrefixLayout shared_prefix_layout(const ps_params* p, int64_t batch, int64
   L.total = L.dec + L.o + L.lse;
   return L;
 }
-// Process-unique id of the current context (cuCtxGetId), 0 if the driver cannot tell.  The
-// primary context keeps its handle across cudaDeviceReset, but not its id.
+// Process-unique id of the current context (cuCtxGetId), 0 if the CUDA driver cannot tell.
+// The primary context keeps its handle across cudaDeviceReset, but not its id.
 unsigned long long current_context_id() {
   using CtxGetCurrentFn = CUresult (*)(CUcontext*);
   using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);

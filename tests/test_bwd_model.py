@@ -4,7 +4,7 @@ The model is the oracle's chain rule with the kernels' bf16 rounding points adde
 parity tests of the backward take their element bar from it.  Here: with rounding switched
 off it must reproduce the oracle exactly (so its algebra is the oracle's, not a copy of the
 kernel's), and with rounding on, at the default softmax scale, it stays inside the plain
-spec bar (|err| <= 2e-2 per element, relative to max(1, row rms); rel_rms <= 5e-3).
+floating-point bar (|err| <= 2e-2 per element, relative to max(1, row rms); rel_rms <= 5e-3).
 """
 import math
 

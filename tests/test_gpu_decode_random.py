@@ -7,7 +7,7 @@ cap L_prefix + W, the first eviction, ring wrap-arounds.  Every sequence's histo
 appended through the C ABI (Continue-PE RoPE), then one decode runs, through
 ps_decode_step for even cases (the step appends token p itself) and ps_decode_attn for odd
 ones.  Every output row is compared with the oracle's attention over the visible set at the
-spec bar (max_abs <= 2e-2, rel_rms <= 5e-3), and lse within 2e-2.
+floating-point bar (max_abs <= 2e-2, rel_rms <= 5e-3), and lse within 2e-2.
 """
 import math
 

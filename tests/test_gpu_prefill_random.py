@@ -3,9 +3,10 @@
 Each case draws a sequence length, L_prefix, W and a head grouping (with L_prefix and W
 often on tile boundaries or past the sequence), then checks, against the float64 oracle
 ("Prefix Sliding 完全拆解", §核心机制 eq. A(i) for the mask, §Kernel 实现 for the tile plan):
-the tile plan bit-exact, every output row and lse of the forward (spec bar), and for
-every other case every row of dQ and key of dK, dV of the backward (the bar of
-tests/test_gpu_prefill_bwd.py, derived from the kernels' rounding model).
+the tile plan bit-exact, every output row and lse of the forward (max_abs <= 2e-2,
+rel_rms <= 5e-3), and for every other case every row of dQ and key of dK, dV of the
+backward (the bar of tests/test_gpu_prefill_bwd.py, derived from the kernels' rounding
+model).
 """
 import math
 
