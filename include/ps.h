@@ -369,6 +369,16 @@ int ps_masked_prefill_attn_bwd(const ps_params* params, const void* q, const voi
 int ps_decode_visible_ranges(const ps_params* params, const int64_t* pos, int64_t batch,
                              int32_t* ranges_out, ps_stream_t stream);
 
+/* Diagnostic of the bounded waits every kernel uses (the pages have no counterpart): one
+ * CTA waits, with the library's own wait, on a shared-memory barrier phase that nothing
+ * completes.  After the wait limit (about one second) the wait gives up, the kernel ORs
+ * PS_DEV_TIMEOUT into *dev_status and returns, so the stream moves on and the context stays
+ * usable.  Lets a test check on the device that a stalled wait ends with a status, not a
+ * hang.
+ *   dev_status : device int32, 4-byte aligned (required).
+ * Asynchronous on `stream`; about one second of device time. */
+int ps_check_wait_timeout(int32_t* dev_status, ps_stream_t stream);
+
 /* Thread-local description of the last host-side failure of this thread ("" if none). */
 const char* ps_last_error(void);
 

@@ -112,6 +112,7 @@ _SIGS = {
                                              c_void_p, c_void_p]),
     "ps_decode_visible_ranges": (c_int32, [POINTER(PsParams), c_void_p, c_int64, c_void_p,
                                            c_void_p]),
+    "ps_check_wait_timeout": (c_int32, [c_void_p, c_void_p]),
     "ps_last_error": (c_char_p, []),
     "ps_version": (c_char_p, []),
 }
@@ -354,6 +355,11 @@ def ps_decode_visible_ranges(params: PsParams, pos, batch: int, ranges_out, stre
     rc = load().ps_decode_visible_ranges(ctypes.byref(params), _ptr(pos), int(batch),
                                          _ptr(ranges_out), _stream(stream))
     _check(rc, "ps_decode_visible_ranges")
+
+
+def ps_check_wait_timeout(dev_status, stream=None) -> None:
+    rc = load().ps_check_wait_timeout(_ptr(dev_status), _stream(stream))
+    _check(rc, "ps_check_wait_timeout")
 
 
 def ps_version() -> str:

@@ -13,6 +13,11 @@
 #include "ps_ranges.cuh"
 
 namespace ps {
+// ps_diag.cu: one CTA whose bounded wait runs out (ps_check_wait_timeout).
+cudaError_t launch_wait_timeout(int32_t* status, cudaStream_t stream);
+}  // namespace ps
+
+namespace ps {
 
 namespace {
 thread_local std::string g_last_error;
@@ -481,6 +486,14 @@ int ps_decode_visible_ranges(const ps_params* params, const int64_t* pos, int64_
   return check_cuda(launch_visible_ranges(pos, batch, params->l_prefix, params->window,
                                           ranges_out, reinterpret_cast<cudaStream_t>(stream)),
                     "visible_ranges_kernel launch");
+}
+
+int ps_check_wait_timeout(int32_t* dev_status, ps_stream_t stream) {
+  g_last_error.clear();
+  if (!dev_status || (reinterpret_cast<uintptr_t>(dev_status) & 3u) != 0)
+    return fail(PS_ERR_INVALID_ARG, "dev_status is NULL or not 4-byte aligned");
+  return check_cuda(launch_wait_timeout(dev_status, reinterpret_cast<cudaStream_t>(stream)),
+                    "wait_timeout_kernel launch");
 }
 
 int ps_prefill_tile_geometry(int32_t* bq, int32_t* bk) {

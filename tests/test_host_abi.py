@@ -252,3 +252,10 @@ def test_paged_host_validation(lib):
     assert app(T=0) == B.PS_ERR_INVALID_ARG
     assert app(pos0=None) == B.PS_ERR_INVALID_ARG
     assert app(pos0=12) == B.PS_ERR_INVALID_ARG         # not 8-byte aligned
+
+
+def test_wait_timeout_diagnostic_host_validation(lib):
+    """The wait diagnostic needs a status word: NULL or misaligned is refused before any
+    launch."""
+    assert lib.ps_check_wait_timeout(None, None) == B.PS_ERR_INVALID_ARG
+    assert lib.ps_check_wait_timeout(2, None) == B.PS_ERR_INVALID_ARG
