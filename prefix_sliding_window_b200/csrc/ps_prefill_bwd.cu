@@ -103,8 +103,8 @@ __device__ __forceinline__ void mma_kmajor(uint32_t d_tmem, uint32_t a_addr, uin
 }
 
 // D += A * B[rows 64 grp .. 64 grp + 63] for one softmax group: A = the group's bf16 pairs in
-// TMEM (written over the first 32 of its own 64 columns, buffer column 64 grp, 8 columns per
-// 16 rows of B), B = smem [128 rows][128 cols] MN-major.
+// TMEM (32 columns from a_buf + 64 grp, 8 columns per 16 rows of B), B = smem [128 rows][128
+// cols] MN-major.
 __device__ __forceinline__ void mma_tmem_a(uint32_t d_tmem, uint32_t a_buf, uint32_t b_addr,
                                            int grp, bool first) {
   constexpr uint32_t idesc = umma_idesc_bf16(128, 128, true);
@@ -385,9 +385,15 @@ __global__ void __launch_bounds__(kDqThreads, 1)
 }
 
 // ------------------------------------------------------------------ dK, dV
-// TMEM: S^T [0,128), dP^T [128,256), dV [256,384), dK [384,512).
-constexpr uint32_t kKColS = 0;
-constexpr uint32_t kKColDP = 128;
+// TMEM: two 128-column score buffers T0 [0,128) and T1 [128,256), dV [256,384), dK
+// [384,512).  Pair g forms S^T in T[g & 1] and dP^T in T[(g + 1) & 1].  The softmax warps
+// load S^T, write P^T (bf16) over the first 32 of their group's 64 columns of the same buffer
+// and, once they have loaded dP^T, dS^T (bf16) over the other 32; so T[(g + 1) & 1] is free
+// for S^T of pair g + 1 as soon as dP^T is in registers, and T[g & 1] takes dP^T of pair
+// g + 1 once the dV and dK products have read P^T and dS^T.  The next pair's scores thus no
+// longer wait for this pair's dV products.
+constexpr uint32_t kKColT = 0;    // T0; T1 = kKColT + 128
+constexpr uint32_t kKColDsOff = 32;  // dS^T: 32 columns after P^T in the group's slice
 constexpr uint32_t kKColDV = 256;
 constexpr uint32_t kKColDK = 384;
 constexpr int kStatBytes = kT * 4;  // one tile of -lse*log2e (or -D)
@@ -435,8 +441,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* dp_full = kv_full + 7;
   uint64_t* p_ready = kv_full + 8;    // [2 groups][2 halves of the group's 64 query columns]
   uint64_t* ds_ready = kv_full + 12;  // [2 groups]
-  uint64_t* s_free = kv_full + 14;
-  uint64_t* dp_free = kv_full + 15;
+  uint64_t* dp_loaded = kv_full + 14;  // softmax warps: dP^T of the pair is in registers
+  uint64_t* pd_free = kv_full + 15;    // the pair's dV and dK products have read P^T, dS^T
   uint64_t* acc_full = kv_full + 16;
   uint64_t* acc_free = kv_full + 17;
   uint64_t* mma_done = kv_full + 18;
@@ -464,8 +470,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(s_full, 1);
     mbar_init(dp_full, 1);
-    mbar_init(s_free, 1);
-    mbar_init(dp_free, 1);
+    mbar_init(dp_loaded, kSoftmaxWarps);
+    mbar_init(pd_free, 1);
     mbar_init(acc_full, 1);
     mbar_init(acc_free, kSoftmaxWarps);
     mbar_init(mma_done, 2);
@@ -576,19 +582,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int st = static_cast<int>(g & 1);
           const uint32_t prev = static_cast<uint32_t>((g - 1) & 1);
           if (!mbar_wait(&st_full[st], static_cast<uint32_t>((g >> 1) & 1), a.status) ||
-              (g >= 1 && !mbar_wait(s_free, prev, a.status))) {
+              (g >= 1 && !mbar_wait(dp_loaded, prev, a.status))) {
             ok = false;
             break;
           }
           tc_fence_after();
-          mma_kmajor(tmem + kKColS, k_addr, q_addr + st * kTileBytes);
+          // S^T into T[g & 1], which held dP^T of pair g - 1
+          mma_kmajor(tmem + kKColT + 128 * st, k_addr, q_addr + st * kTileBytes);
           umma_commit(s_full);
-          if (g >= 1 && !mbar_wait(dp_free, prev, a.status)) {
+          if (g >= 1 && !mbar_wait(pd_free, prev, a.status)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          mma_kmajor(tmem + kKColDP, v_addr, do_addr + st * kTileBytes);
+          // dP^T into T[(g + 1) & 1], which held P^T and dS^T of pair g - 1
+          mma_kmajor(tmem + kKColT + 128 * (st ^ 1), v_addr, do_addr + st * kTileBytes);
           umma_commit(dp_full);
         }
         if (!ok) break;
@@ -628,13 +636,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 break;
               }
               tc_fence_after();
-              mma_tmem_a_half(tmem + kKColDV, tmem + kKColS, do_addr + st * kTileBytes, gr, hf,
-                              j == 0 && gr == 0);
+              mma_tmem_a_half(tmem + kKColDV, tmem + kKColT + 128 * st,
+                              do_addr + st * kTileBytes, gr, hf, j == 0 && gr == 0);
             }
             if (!ok) break;
           }
           if (!ok) break;
-          umma_commit(s_free);
 #pragma unroll
           for (int gr = 0; gr < kGroups; ++gr) {
             if (!mbar_wait(&ds_ready[gr], ph, a.status)) {
@@ -642,11 +649,12 @@ __global__ void __launch_bounds__(kThreads, 1)
               break;
             }
             tc_fence_after();
-            mma_tmem_a(tmem + kKColDK, tmem + kKColDP, q_addr + st * kTileBytes, gr,
+            mma_tmem_a(tmem + kKColDK, tmem + kKColT + 128 * st + kKColDsOff,
+                       q_addr + st * kTileBytes, gr,
                        j == 0 && gr == 0);
           }
           if (!ok) break;
-          umma_commit(dp_free);
+          umma_commit(pd_free);
           umma_commit(&st_empty[st]);
         }
         if (!ok) break;
@@ -699,7 +707,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) continue;
         tc_fence_after();
         float x[kCols];
-        load64(lane_base + kKColS + cs0, x);
+        const uint32_t t_s = lane_base + kKColT + 128 * st;         // S^T, then P^T, dS^T
+        const uint32_t t_dp = lane_base + kKColT + 128 * (st ^ 1);  // dP^T
+        load64(t_s + cs0, x);
         if (flag == PS_TILE_PARTIAL) {
           const uint64_t vis = span_bits(kr, vis_end, (int64_t)qt * kT + cs0);
 #pragma unroll
@@ -728,7 +738,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             pk[2 * ii] = cvt_bf16x2(x[4 * i], x[4 * i + 1]);
             pk[2 * ii + 1] = cvt_bf16x2(x[4 * i + 2], x[4 * i + 3]);
           }
-          tmem_st16(lane_base + kKColS + cs0 + 16 * hf, pk);
+          tmem_st16(t_s + cs0 + 16 * hf, pk);
           tmem_wait_st();
           tc_fence_before();
           __syncwarp();
@@ -740,8 +750,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
           uint32_t raw[32];
-          tmem_ld32(lane_base + kKColDP + cs0 + 32 * c, raw);
+          tmem_ld32(t_dp + cs0 + 32 * c, raw);
           tmem_wait_ld();
+          if (c == 1) {
+            // dP^T is in registers: its buffer can take the next pair's S^T
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(dp_loaded);
+          }
           uint32_t dk[16];
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
@@ -759,7 +775,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             dk[2 * i] = cvt_bf16x2(v0.x, v0.y);
             dk[2 * i + 1] = cvt_bf16x2(v1.x, v1.y);
           }
-          tmem_st16(lane_base + kKColDP + cs0 + 16 * c, dk);
+          tmem_st16(t_s + cs0 + kKColDsOff + 16 * c, dk);
 #pragma unroll
           for (int v = 0; v < 4; ++v) {
             const int chunk = (cs0 >> 3) + 4 * c + v;  // query cols [8 chunk, 8 chunk + 8)
