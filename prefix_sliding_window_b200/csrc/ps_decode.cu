@@ -161,7 +161,9 @@ struct TileWalker {
     }
     b = lo;
     const int64_t cnt = pref[b + 1] - pref[b];
-    h = static_cast<int32_t>((t0 - (int64_t)a.hkv * pref[b]) / cnt);
+    const int64_t off = t0 - (int64_t)a.hkv * pref[b];  // < hkv * cnt
+    h = static_cast<int32_t>(off < (int64_t(1) << 32) ? uint32_t(off) / uint32_t(cnt)
+                                                       : off / cnt);
     t = t0;
     enter_unit(a, pref);
   }
@@ -290,8 +292,16 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     }
     __syncthreads();
     const int64_t total = (int64_t)a.hkv * pref[a.batch];
-    const int64_t t0 = total * blockIdx.x / gridDim.x;
-    const int64_t t1 = total * (blockIdx.x + 1) / gridDim.x;
+    // this CTA's share [total c / G, total (c + 1) / G), in 32 bits when total G fits
+    int64_t t0, t1;
+    if (total * gridDim.x < (int64_t(1) << 32)) {
+      const uint32_t tt = static_cast<uint32_t>(total);
+      t0 = (tt * blockIdx.x) / gridDim.x;
+      t1 = (tt * (blockIdx.x + 1)) / gridDim.x;
+    } else {
+      t0 = total * blockIdx.x / gridDim.x;
+      t1 = total * (blockIdx.x + 1) / gridDim.x;
+    }
     wk.t_end = t1;
     if (t0 < t1) {
       wk.seek(a, pref, t0);
@@ -331,7 +341,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
           // the newest row of sequence b: prefix row p, or ring slot (p - Lp) mod W
           const int64_t p = a.pos[pw.b];
           const bool pre = a.full_mode || p < a.lp;
-          const int64_t row = pre ? p : (p - a.lp) % a.w;
+          const int64_t row = pre ? p : mod_nonneg(p - a.lp, a.w);
           if (d.map_id == (pre ? 0 : 1) && row >= d.row0 + d.lo && row < d.row0 + d.hi) {
             pdl_wait();
             waited = true;

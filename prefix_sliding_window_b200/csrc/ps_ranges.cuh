@@ -32,6 +32,13 @@ struct VisibleRanges {
 // Visible ranges of the query at position p (p >= 0).  Ring slot of position q >= Lp is
 // (q - Lp) mod W.  The window positions [wstart, n) are contiguous, so their slots form
 // at most two runs: [s0, W) and [0, ...).
+// x mod w for x >= 0, w > 0: a 32-bit remainder when x fits (the case in practice), which
+// on the GPU is a few instructions against a long emulated 64-bit division.
+PS_HD int64_t mod_nonneg(int64_t x, int32_t w) {
+  if (x < (int64_t(1) << 32)) return int64_t(uint32_t(x) % uint32_t(w));
+  return x % w;
+}
+
 PS_HD VisibleRanges visible_ranges(int64_t p, int32_t lp, int32_t w) {
   VisibleRanges r;
   const int64_t n = p + 1;
@@ -44,7 +51,7 @@ PS_HD VisibleRanges visible_ranges(int64_t p, int32_t lp, int32_t w) {
     r.seg1_len = 0;
     return r;
   }
-  const int64_t s0 = (wstart - lp) % w;
+  const int64_t s0 = mod_nonneg(wstart - lp, w);
   const int64_t room = w - s0;
   r.seg0_start = static_cast<int32_t>(s0);
   r.seg0_len = static_cast<int32_t>(win < room ? win : room);
