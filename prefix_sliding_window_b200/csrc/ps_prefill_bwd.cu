@@ -17,7 +17,8 @@
 //             atomic counter (a prefix key tile is seen by every later query tile, a window
 //             key tile by about W/128 of them, so static striding would leave SMs idle): per
 //             (query head of the group, query tile), S^T = K Q^T and dP^T = V dO^T into
-//             TMEM, P^T and dS^T as bf16 over them, dV += P^T dO and dK += dS^T Q in TMEM
+//             TMEM, P^T and dS^T as bf16 in the columns that held S^T (two score buffers
+//             swap roles every pair), dV += P^T dO and dK += dS^T Q in TMEM
 //             across the whole group, so no atomics are needed.  It also stores each dS^T
 //             tile (bf16) for the dQ pass.
 //   bwd_dq_kernel - dQ = scale * dS K over the plan: a GEMM reading the stored dS^T tiles as
@@ -390,8 +391,8 @@ __global__ void __launch_bounds__(kDqThreads, 1)
 // load S^T, write P^T (bf16) over the first 32 of their group's 64 columns of the same buffer
 // and, once they have loaded dP^T, dS^T (bf16) over the other 32; so T[(g + 1) & 1] is free
 // for S^T of pair g + 1 as soon as dP^T is in registers, and T[g & 1] takes dP^T of pair
-// g + 1 once the dV and dK products have read P^T and dS^T.  The next pair's scores thus no
-// longer wait for this pair's dV products.
+// g + 1 once the dV and dK products have read P^T and dS^T.  So the next pair's scores wait
+// for this pair's dP^T to be loaded, not for its dV products.
 constexpr uint32_t kKColT = 0;    // T0; T1 = kKColT + 128
 constexpr uint32_t kKColDsOff = 32;  // dS^T: 32 columns after P^T in the group's slice
 constexpr uint32_t kKColDV = 256;
