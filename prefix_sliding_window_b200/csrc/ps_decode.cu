@@ -11,10 +11,11 @@
 // tiles (make_tiling).  Two schedules:
 //  * per-unit: when there are at least as many units as CTA slots (148 SMs x 2), one CTA
 //    per unit, written straight to `out`;
-//  * stream-K: otherwise exactly one wave of CTAs (2 per SM) takes equal contiguous shares
-//    of the global tile sequence (all units' tiles back to back), so every SM streams the
-//    same number of bytes whatever the positions are.  A CTA whose share crosses a unit
-//    boundary flushes a partial (o, lse) per unit piece; merge_kernel combines the pieces.
+//  * stream-K: otherwise one wave of CTAs (up to 2 per SM; a multiple of the unit count when
+//    that fills at least 5/6 of the slots) takes equal contiguous shares of the global tile
+//    sequence (all units' tiles back to back), so every SM streams the same number of bytes
+//    whatever the positions are.  A CTA whose share crosses a unit boundary flushes a partial
+//    (o, lse) per unit piece; merge_kernel combines the pieces.
 // Inside a CTA:
 //  * warp 4 is the producer: one lane issues four 3-D TMA loads per tile (K and V, two
 //    64-column halves each, 128-byte swizzle) into a 3-stage mbarrier ring;
@@ -816,6 +817,14 @@ int64_t streamk_grid(int64_t batch, int32_t hkv, int64_t max_keys, bool force = 
   // forced (prefix partials to fold in) with more units than CTA slots: about one unit per
   // CTA over several waves streams faster than one wave of long shares
   if (g > slots) g = (force && units > slots) ? units : slots;
+  // a full wave: prefer a multiple of the unit count when one fills at least 5/6 of the
+  // slots, so that with equally long units (every sequence past L_prefix + W) each share ends
+  // on a unit boundary and no CTA switches unit mid-stream (batch 32 / 64 / 128 at W 4096:
+  // 1.1-1.8, 0.5-1.6 and 0.5-1.1 us per step faster; with 200 of 296 slots, slower)
+  if (!force && g == slots && units <= slots) {
+    const int64_t ga = units * (slots / units);
+    if (ga * 6 >= slots * 5) g = ga;
+  }
   if (g < 1) g = 1;
   return g;
 }
