@@ -17,61 +17,80 @@ namespace ps {
 namespace {
 constexpr int kPlanThreads = 1024;
 
-// Single-CTA planner: counts tiles per query tile, scans the counts into offsets and writes
-// the entries.  ws_off: [nq + 1] int32; ws_ent: [n_tiles][2] int32 (k_tile, flag);
+// Single-CTA planner (32 warps): the tiles per query tile in closed form, an exclusive scan
+// of those counts into offsets (warp shuffles, then the warp totals), then one warp per query
+// tile writes its entries, 32 candidate key tiles at a time, compacted by a ballot in
+// ascending order.  ws_off: [nq + 1] int32; ws_ent: [n_tiles][2] int32 (k_tile, flag);
 // plan_out (optional): [n_tiles][3] int32 (q_tile, k_tile, flag).
 __global__ void __launch_bounds__(kPlanThreads)
     plan_kernel(int64_t seq, int32_t lp, int32_t w, int32_t* __restrict__ ws_off,
                 int32_t* __restrict__ ws_ent, int32_t* __restrict__ plan_out) {
-  __shared__ int32_t s_scan[kPlanThreads];
+  constexpr int kWarps = kPlanThreads / 32;
+  static_assert(kWarps == 32, "the warp totals are scanned by one warp");
+  __shared__ int32_t s_warp[kWarps];
   __shared__ int32_t s_base;
   pdl_trigger();  // the attention kernel may start its prologue; it waits for this plan
   const int64_t nq = (seq + kPrefillBq - 1) / kPrefillBq;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   if (threadIdx.x == 0) s_base = 0;
   __syncthreads();
   for (int64_t c0 = 0; c0 < nq; c0 += kPlanThreads) {
     const int64_t qt = c0 + threadIdx.x;
-    int32_t cnt = 0;
-    if (qt < nq) cnt = static_cast<int32_t>(qtile_count(qt, seq, lp, w, kPrefillBq, kPrefillBk));
-    s_scan[threadIdx.x] = cnt;
-    __syncthreads();
-    // Hillis-Steele inclusive scan
-    for (int off = 1; off < kPlanThreads; off <<= 1) {
-      const int32_t v = threadIdx.x >= off ? s_scan[threadIdx.x - off] : 0;
-      __syncthreads();
-      s_scan[threadIdx.x] += v;
-      __syncthreads();
+    const int32_t cnt =
+        qt < nq ? static_cast<int32_t>(qtile_count(qt, seq, lp, w, kPrefillBq, kPrefillBk)) : 0;
+    int32_t v = cnt;  // inclusive scan inside the warp
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int32_t u = __shfl_up_sync(0xffffffffu, v, off);
+      if (lane >= off) v += u;
     }
-    const int32_t base = s_base;
-    const int32_t start = base + s_scan[threadIdx.x] - cnt;
-    if (qt < nq) {
-      ws_off[qt] = start;
-      int64_t pe, wsb, we;
-      qtile_candidates(qt, seq, lp, w, kPrefillBq, kPrefillBk, &pe, &wsb, &we);
-      int32_t k = start;
-      const int64_t kt_last = (seq - 1) / kPrefillBk;
-      for (int pass = 0; pass < 2; ++pass) {
-        const int64_t lo = pass == 0 ? 0 : wsb;
-        const int64_t hi = pass == 0 ? (pe - 1 < kt_last ? pe - 1 : kt_last) : we;
-        for (int64_t kt = lo; kt <= hi; ++kt) {
-          const int32_t f = classify_tile(qt, kt, seq, lp, w, kPrefillBq, kPrefillBk);
-          if (!f) continue;
-          ws_ent[2 * k] = static_cast<int32_t>(kt);
-          ws_ent[2 * k + 1] = f;
-          if (plan_out) {
-            plan_out[3 * k] = static_cast<int32_t>(qt);
-            plan_out[3 * k + 1] = static_cast<int32_t>(kt);
-            plan_out[3 * k + 2] = f;
-          }
-          ++k;
-        }
+    if (lane == 31) s_warp[warp] = v;
+    __syncthreads();
+    if (warp == 0) {
+      int32_t t = s_warp[lane];
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int32_t u = __shfl_up_sync(0xffffffffu, t, off);
+        if (lane >= off) t += u;
       }
+      s_warp[lane] = t;  // inclusive totals of warps 0 .. lane
     }
     __syncthreads();
-    if (threadIdx.x == kPlanThreads - 1) s_base = base + s_scan[kPlanThreads - 1];
+    const int32_t base = s_base;
+    if (qt < nq) ws_off[qt] = base + (warp > 0 ? s_warp[warp - 1] : 0) + v - cnt;
+    __syncthreads();
+    if (threadIdx.x == 0) s_base = base + s_warp[kWarps - 1];
     __syncthreads();
   }
   if (threadIdx.x == 0) ws_off[nq] = s_base;
+  __syncthreads();  // the offsets are visible to every warp of the block
+  const int64_t kt_last = (seq - 1) / kPrefillBk;
+  for (int64_t qt = warp; qt < nq; qt += kWarps) {
+    int64_t pe, wsb, we;
+    qtile_candidates(qt, seq, lp, w, kPrefillBq, kPrefillBk, &pe, &wsb, &we);
+    int32_t k = ws_off[qt];
+    for (int pass = 0; pass < 2; ++pass) {
+      const int64_t lo = pass == 0 ? 0 : wsb;
+      const int64_t hi = pass == 0 ? (pe - 1 < kt_last ? pe - 1 : kt_last) : we;
+      for (int64_t k0 = lo; k0 <= hi; k0 += 32) {  // warp-uniform bounds
+        const int64_t kt = k0 + lane;
+        const int32_t f =
+            kt <= hi ? classify_tile(qt, kt, seq, lp, w, kPrefillBq, kPrefillBk) : 0;
+        const unsigned m = __ballot_sync(0xffffffffu, f != 0);
+        if (f) {
+          const int32_t e = k + __popc(m & ((1u << lane) - 1u));
+          ws_ent[2 * e] = static_cast<int32_t>(kt);
+          ws_ent[2 * e + 1] = f;
+          if (plan_out) {
+            plan_out[3 * e] = static_cast<int32_t>(qt);
+            plan_out[3 * e + 1] = static_cast<int32_t>(kt);
+            plan_out[3 * e + 2] = f;
+          }
+        }
+        k += __popc(m);
+      }
+    }
+  }
 }
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
