@@ -104,3 +104,36 @@ def test_tiles_cover_exactly_the_visible_rows(driver, paged):
                         assert lo <= i < hi, (lp, w, p, map_id, row0, lo, hi, i)
         assert len(covered) == len(set(covered)), (lp, w, p)
         assert set(covered) == _expected(lp, w, p), (lp, w, p)
+
+
+def _expected_intervals(lp, w, p):
+    """The same set as _expected, from the two intervals of eq. A(i) (prefix [0, min(p+1,
+    Lp)), window [max(Lp, p+1-W), p]), for positions too large to enumerate every earlier
+    key; test_oracle_pins ties the brute-force set to these intervals at small p."""
+    pre = {(0, k) for k in range(min(p + 1, lp))}
+    win = {(1, (k - lp) % w) for k in range(max(lp, p + 1 - w), p + 1)}
+    return pre | win
+
+
+@pytest.mark.parametrize("paged", [False, True])
+def test_tiles_at_large_positions(driver, paged):
+    """Ring offsets (window start - Lp) on both sides of 2^31 and 2^32 and far past them: the
+    32-bit remainder and its 64-bit fallback in visible_ranges give the visible rows, once
+    each, with the window starting at its oldest key's slot."""
+    ws = [64, 100, 4096] if not paged else [64, 128, 4096]
+    offs = [2 ** 31 - 1, 2 ** 31, 2 ** 32 - 1, 2 ** 32, 2 ** 32 + 1, 2 ** 32 + 63,
+            2 ** 33 + 12345, 2 ** 40 + 7]
+    cases = [(lp, w, lp + w - 1 + x) for lp in (0, 100, 300) for w in ws for x in offs]
+    got = _run(driver, cases, paged)
+    assert len(got) == len(cases)
+    for (lp, w, p), tiles in got.items():
+        covered = []
+        for map_id, row0, lo, hi in tiles:
+            assert 0 <= lo < hi <= TILE, (lp, w, p, row0, lo, hi)
+            covered += [(map_id, row0 + i) for i in range(lo, hi)]
+        assert len(covered) == len(set(covered)), (lp, w, p)
+        assert set(covered) == _expected_intervals(lp, w, p), (lp, w, p)
+        # a full window covers every slot whatever the start, so also check the order: the
+        # window's first covered row is the slot of its oldest key
+        first = next(row0 + lo for map_id, row0, lo, hi in tiles if map_id == 1)
+        assert first == (max(lp, p + 1 - w) - lp) % w, (lp, w, p, first)
