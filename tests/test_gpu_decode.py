@@ -236,6 +236,56 @@ def test_decode_b64_w4096_full_size(cuda_device):
             assert np.abs(got_lse[i, b] - l).max() < 2e-2
 
 
+@pytest.mark.parametrize("Bn", [32, 128])
+def test_decode_equal_lengths_unit_aligned_waves(cuda_device, Bn):
+    """Batch 32 and 128 at W=4096 with every sequence past L_prefix + W: the stream-K wave is
+    then a multiple of the unit count (64 units x 4 CTAs, 256 units x 2), so each CTA streams
+    a whole part of one unit and the merge combines exactly that many pieces.  One decode
+    step through ps_decode_step; 5 sampled sequences checked head by head."""
+    dev = cuda_device
+    wl = synth.WORKLOADS["decode_b64_w4096"]
+    hq, hkv, lp, w = wl.n_q_heads, wl.n_kv_heads, wl.l_prefix, wl.window
+    seed = lambda k: synth.seed_for(20 + Bn, k)  # noqa: E731
+    pos = synth.uniform_positions(Bn, wl.pos_lo, wl.pos_hi, seed(0), dev)
+    k_pre = synth.normal_bf16((Bn, lp, hkv, D), seed(1), dev)
+    v_pre = synth.normal_bf16((Bn, lp, hkv, D), seed(2), dev)
+    k_win = synth.normal_bf16((Bn, w, hkv, D), seed(3), dev)
+    v_win = synth.normal_bf16((Bn, w, hkv, D), seed(4), dev)
+    q_raw = synth.normal_bf16((Bn, hq, D), seed(5), dev)
+    params = B.make_params(hq, hkv, D, lp, w, wl.rope_theta)
+    cache = PrefixSlidingCache(Bn, hkv, lp, w, D, dev, fill=float("nan"))
+    st = _status(dev)
+    B.ps_kv_append_rope(params, cache.struct, k_pre, v_pre, None,
+                        torch.zeros(Bn, dtype=torch.int64, device=dev), lp, st)
+    # window history: positions p - W + 1 .. p - 1; the step appends position p itself
+    B.ps_kv_append_rope(params, cache.struct, k_win[:, :w - 1].contiguous(),
+                        v_win[:, :w - 1].contiguous(), None, pos - (w - 1), w - 1, st)
+    ws = torch.empty(max(1, B.ps_decode_workspace_bytes(params, Bn)), dtype=torch.uint8,
+                     device=dev)
+    q = q_raw.clone()
+    out = torch.empty((Bn, hq, D), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((Bn, hq), dtype=torch.float32, device=dev)
+    B.ps_decode_step(params, cache.struct, k_win[:, w - 1].contiguous(),
+                     v_win[:, w - 1].contiguous(), q, pos, out, lse, ws, st)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    scale = 1 / math.sqrt(D)
+    P = pos.cpu().numpy()
+    kp, vp, kw, vw, qr = f64(k_pre), f64(v_pre), f64(k_win), f64(v_win), f64(q_raw)
+    got, got_lse = f64(out), f64(lse)
+    for b in (0, 1, Bn // 2, Bn - 2, Bn - 1):
+        p = int(P[b])
+        vis = O.visible_positions(p, lp, w)
+        assert len(vis) == lp + w
+        base = p - (w - 1)  # position of k_win[:, 0]
+        kr = np.stack([kp[b, x] if x < lp else kw[b, x - base] for x in vis])
+        vr = np.stack([vp[b, x] if x < lp else vw[b, x - base] for x in vis])
+        k_rot = O.rope_rotate(kr, vis[:, None], THETA)
+        o, l = O.attend_gqa(O.rope_rotate(qr[b], p, THETA), k_rot, vr, scale)
+        assert_close(got[b], o, f"Bn={Bn} b={b}")
+        assert np.abs(got_lse[b] - l).max() < 2e-2
+
+
 @pytest.mark.parametrize("lp,w,positions", [
     (0, 64, [0, 1, 63, 64, 65, 200]),            # pure sliding window
     (7, 1, [0, 6, 7, 8, 50]),                     # window of one
